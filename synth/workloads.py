@@ -63,7 +63,7 @@ class Workload:
     topic_amp: float = 4.0     # |key/value shift along the topic direction|
     topic_gain: float = 9.0    # logits a matching topic adds to a key
     needle_gain: float = 18.0  # logits a head's needle adds for that head
-    needle_query_amp: float = 4.0
+    needle_query_amp: float = 0.0   # 0: sqrt(needle_gain*sqrt(d)), the same size as the key's needle shift
     extra: dict = field(default_factory=dict)
 
     @property
@@ -179,7 +179,8 @@ def generate(w: Workload, device: str = "cpu", n_total: Optional[int] = None) ->
             V[h] += shift
         # needle directions: one per query head, planted once in its KV head's keys
         nu = _unit(randn(Hq, d))
-        lam = w.needle_gain * math.sqrt(d) / w.needle_query_amp
+        kappa = w.needle_query_amp or math.sqrt(w.needle_gain * math.sqrt(d))
+        lam = w.needle_gain * math.sqrt(d) / kappa
         pos = torch.randperm(max(n - 1, 1), generator=g, device=device)[:Hq] + 1
         pos = pos.clamp(max=n - 1)
         for h in range(Hq):
@@ -190,10 +191,10 @@ def generate(w: Workload, device: str = "cpu", n_total: Optional[int] = None) ->
             z = randn(w.batch, Hq, d)
             topic = randint(w.n_topics, (w.batch, Hq))
             kvh = torch.arange(Hq, device=device) // G
-            qs = z + beta * T[kvh[None, :].expand(w.batch, Hq), topic] + w.needle_query_amp * nu[None]
+            qs = z + beta * T[kvh[None, :].expand(w.batch, Hq), topic] + kappa * nu[None]
             sets.append(qs)
         Q = torch.stack(sets)
-        meta.update(topic_beta=beta, needle_lambda=lam, n_topics=w.n_topics,
+        meta.update(topic_beta=beta, needle_lambda=lam, needle_kappa=kappa, n_topics=w.n_topics,
                     n_segments=w.n_segments)
     else:
         raise KeyError(w.gen)

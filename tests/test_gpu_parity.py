@@ -1,0 +1,266 @@
+"""CUDA path vs the fp64 oracle, element by element, at sizes the oracle finishes in seconds.
+
+Every case spans several chunks / tiles and a ragged tail.  Inputs come from
+synth/ (seeded); nothing here feeds a CUDA result into the oracle except the
+stage-wise protocol of parity_helpers (oracle routing on the GPU-stored planes,
+oracle attention on the GPU-kept blocks), whose expected values are still the
+oracle's arithmetic.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.zha_oracle as zo
+from parity_helpers import (assert_close_out, compare_planes, compare_route, f64, oracle_attend_on_sets, p32)
+from synth.workloads import generate, random_tree_case, small_topics, workload
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import tree_indexed_sparse_03_b200 as z
+
+
+class Case:
+    """A tree over the first n tokens of (K, V), with room to append the rest."""
+
+    def __init__(self, K, V, refs, *, block, levels, p, n, group, max_batch=16, capacity=None):
+        self.Kall, self.Vall, self.refs_cpu = K, V, refs
+        Hkv, ntot, d = K.shape
+        self.dtype = "bf16" if K.dtype == torch.bfloat16 else "f32"
+        self.block, self.levels, self.p, self.group = block, levels, p, group
+        cap = capacity or max(ntot, 1)
+        self.cfg = z.make_config(d=d, n_q_heads=Hkv * group, n_kv_heads=Hkv, block=block, levels=levels,
+                                 n_refs=refs.shape[1], p=p, dtype=self.dtype, capacity=cap, max_batch=max_batch)
+        self.Kc = torch.zeros(Hkv, cap, d, dtype=K.dtype, device="cuda")
+        self.Vc = torch.zeros_like(self.Kc)
+        self.Kc[:, :n] = K[:, :n].cuda()
+        self.Vc[:, :n] = V[:, :n].cuda()
+        self.refs = refs.cuda().contiguous()
+        self.tree = z.ZhaTree(self.cfg, self.Kc, self.Vc, self.refs)
+        self.tree.build(n)
+        self.n = n
+
+    def append(self, m):
+        self.tree.append(self.Kall[:, self.n:self.n + m].cuda(), self.Vall[:, self.n:self.n + m].cuda())
+        self.n += m
+
+    def oracle_tree(self, kvh):
+        return zo.build_tree(f64(self.Kall[kvh]), f64(self.refs_cpu[kvh]), self.n, self.block, self.levels)
+
+    def decode(self, Q):
+        O, (kept, cnt), stats = self.tree.decode(Q.cuda(), want_kept=True, want_stats=True)
+        torch.cuda.synchronize()
+        self.tree.status()
+        return O, kept, cnt, stats
+
+
+def check_build(case: Case):
+    for kvh in range(case.Kall.shape[0]):
+        orc = case.oracle_tree(kvh)
+        for level in range(1, case.levels + 1):
+            n_l = case.n // case.block ** level
+            if n_l == 0:
+                continue
+            mu, bias, f = case.tree.level_planes(level)
+            compare_planes(f64(mu[kvh, :n_l]), f64(bias[kvh, :n_l]), f64(f[kvh, :n_l]), orc[level], case.dtype,
+                           f64(case.refs_cpu[kvh]), label=f"kv{kvh} level {level}")
+
+
+def check_decode(case: Case, Q, allow_flagged_frac=0.2):
+    O, kept, cnt, stats = case.decode(Q)
+    rep = compare_route(case.tree, Q, kept, cnt, p32(case.p), case.n, case.block, case.levels, case.group)
+    assert not rep.failures, "\n".join(rep.failures[:5])
+    assert rep.flagged <= allow_flagged_frac * rep.heads + 1, (rep.flagged, rep.heads)
+    ref = oracle_attend_on_sets(case.Kall, case.Vall, Q, kept, cnt, case.n, case.block, case.group)
+    atol = 2e-5 * float(case.Vall[:, :case.n].abs().max()) + 1e-6
+    assert_close_out(O.cpu().numpy(), ref, atol, "attend")
+    # stats agree with the kept sets
+    st = stats.cpu()
+    assert torch.equal(st[..., 1], cnt.cpu().long())
+    return rep, O, kept, cnt
+
+
+# ------------------------------------------------------------------ dense decode
+@pytest.mark.parametrize("dtype,d,hq,hkv,n", [("f32", 64, 1, 1, 4096), ("bf16", 128, 32, 4, 5003),
+                                                ("bf16", 64, 16, 2, 777), ("f32", 128, 4, 2, 130),
+                                                ("bf16", 128, 16, 1, 1), ("bf16", 128, 4, 4, 33)])
+def test_dense_decode(dtype, d, hq, hkv, n):
+    K, V, refs, Q = random_tree_case(7, n_tokens=n, d=d, n_q_heads=hq, n_kv_heads=hkv, n_refs=1, batch=3,
+                                     dtype=dtype)
+    cfg = z.make_config(d=d, n_q_heads=hq, n_kv_heads=hkv, block=4, levels=1, n_refs=1, p=1.0, dtype=dtype,
+                        capacity=n, max_batch=3)
+    dec = z.DenseDecoder(cfg, 3, n)
+    Kc, Vc, Qc = K.cuda(), V.cuda(), Q.cuda()
+    for _ in range(2):  # the scratch must come back zero-filled: run twice
+        O = dec(Kc, Vc, n, Qc)
+        torch.cuda.synchronize()
+        G = hq // hkv
+        ref = np.stack([[zo.dense(f64(K[h // G]), f64(V[h // G]), f64(Q[b, h]), n) for h in range(hq)]
+                        for b in range(3)])
+        # bf16 P in the tensor-core path rounds each softmax weight to 8 bits
+        atol = (2e-2 if dtype == "bf16" else 2e-5) * max(1.0, float(V.abs().max()))
+        assert_close_out(O.cpu().numpy(), ref, atol, f"dense {dtype} d={d} n={n}")
+
+
+# ------------------------------------------------------------------ build
+BUILD_CASES = [
+    # dtype, d, hkv, group, n, block, levels, R
+    ("f32", 64, 1, 1, 4096, 4, 3, 4),
+    ("f32", 128, 2, 2, 1000, 3, 3, 5),
+    ("bf16", 128, 1, 8, 20011, 4, 4, 8),
+    ("bf16", 64, 2, 4, 9000, 8, 2, 1),
+    ("bf16", 128, 1, 2, 5000, 256, 1, 16),
+    ("bf16", 128, 1, 1, 2100, 2, 7, 3),
+    ("f32", 64, 1, 1, 100, 4, 5, 2),
+]
+
+
+@pytest.mark.parametrize("dtype,d,hkv,group,n,block,levels,R", BUILD_CASES)
+def test_build_planes(dtype, d, hkv, group, n, block, levels, R):
+    K, V, refs, _ = random_tree_case(3, n_tokens=n, d=d, n_q_heads=hkv * group, n_kv_heads=hkv, n_refs=R,
+                                     batch=1, dtype=dtype)
+    case = Case(K, V, refs, block=block, levels=levels, p=0.9, n=n, group=group)
+    torch.cuda.synchronize()
+    check_build(case)
+
+
+@pytest.mark.parametrize("dtype,d,hkv,group,n,block,levels,R", BUILD_CASES[:6])
+def test_append_bit_exact(dtype, d, hkv, group, n, block, levels, R):
+    """build(n0) followed by appends of assorted sizes stores the same bits as build(n)."""
+    K, V, refs, _ = random_tree_case(5, n_tokens=n, d=d, n_q_heads=hkv * group, n_kv_heads=hkv, n_refs=R,
+                                     batch=1, dtype=dtype)
+    n0 = n // 3
+    inc = Case(K, V, refs, block=block, levels=levels, p=0.9, n=n0, group=group, capacity=n)
+    sizes = [1, 1, 2, 3, 17, 64, 1, 255, 1000]
+    i = 0
+    while inc.n < n:
+        inc.append(min(sizes[i % len(sizes)], n - inc.n))
+        i += 1
+    full = Case(K, V, refs, block=block, levels=levels, p=0.9, n=n, group=group, capacity=n)
+    torch.cuda.synchronize()
+    for level in range(1, levels + 1):
+        n_l = n // block ** level
+        a = inc.tree.level_planes(level)
+        b = full.tree.level_planes(level)
+        for x, y in zip(a, b):
+            assert torch.equal(x[:, :n_l].cpu(), y[:, :n_l].cpu()), f"level {level} differs"
+
+
+# ------------------------------------------------------------------ route + attend
+def test_tiny_needles_fp32():
+    """The tiny fp32 workload: 1 head, d=64, N=4096, b=4, L=3, R=4, p=0.9, 8 queries with planted needles."""
+    w = workload("tiny4k_fp32")
+    inp = generate(w)
+    case = Case(inp.K, inp.V, inp.refs, block=w.block, levels=w.levels, p=w.p, n=w.n_tokens, group=1,
+                max_batch=w.batch)
+    check_build(case)
+    rep, O, kept, cnt = check_decode(case, inp.Q[0])
+    print(f"tiny: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+
+
+@pytest.mark.parametrize("n,block,levels,R,p,d,G,hkv", [
+    (20011, 4, 4, 8, 0.95, 128, 8, 1),
+    (9000, 8, 2, 1, 0.75, 128, 4, 2),
+    (5000, 256, 1, 16, 0.95, 128, 8, 1),
+    (3001, 3, 5, 4, 0.6, 64, 2, 1),
+])
+def test_topics_route_attend(n, block, levels, R, p, d, G, hkv):
+    w = small_topics(n, d=d, n_q_heads=G * hkv, n_kv_heads=hkv, block=block, levels=levels, n_refs=R, p=p, batch=2)
+    inp = generate(w)
+    case = Case(inp.K, inp.V, inp.refs, block=block, levels=levels, p=p, n=n, group=G)
+    check_build(case)
+    for s in range(3):
+        check_decode(case, inp.Q[s])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_small_trees(seed):
+    rng = np.random.default_rng(seed)
+    block = int(rng.choice([2, 3, 4, 5, 8]))
+    levels = int(rng.integers(1, 5))
+    n = int(rng.integers(1, 3 * block ** (levels + 1) + 50))
+    d = int(rng.choice([64, 128]))
+    dtype = str(rng.choice(["f32", "bf16"]))
+    R = int(rng.choice([1, 2, 4, 16, 32]))
+    G = int(rng.choice([1, 2, 8]))
+    p = float(rng.choice([0.3, 0.75, 0.9, 0.99, 1.0]))
+    K, V, refs, Q = random_tree_case(100 + seed, n_tokens=n, d=d, n_q_heads=G, n_kv_heads=1, n_refs=R, batch=3,
+                                     dtype=dtype, key_scale=float(rng.choice([0.3, 1.0, 2.0])))
+    case = Case(K, V, refs, block=block, levels=levels, p=p, n=n, group=G)
+    check_build(case)
+    check_decode(case, Q)
+
+
+# ------------------------------------------------------------------ special cases
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 17])
+def test_short_contexts(n):
+    """Fewer tokens than a block, one block, ragged: the attended set is sink + kept blocks + tail."""
+    K, V, refs, Q = random_tree_case(9, n_tokens=n, d=128, n_q_heads=8, n_kv_heads=1, n_refs=4, batch=2,
+                                     dtype="bf16")
+    case = Case(K, V, refs, block=4, levels=2, p=0.9, n=n, group=8)
+    check_decode(case, Q)
+
+
+def test_p1_equals_dense():
+    K, V, refs, Q = random_tree_case(11, n_tokens=7777, d=128, n_q_heads=16, n_kv_heads=2, n_refs=4, batch=2,
+                                     dtype="bf16")
+    case = Case(K, V, refs, block=4, levels=4, p=1.0, n=7777, group=8)
+    O, kept, cnt, _ = case.decode(Q)
+    assert (cnt.cpu() == 7777 // 4).all()
+    ref = np.stack([[zo.dense(f64(K[h // 8]), f64(V[h // 8]), f64(Q[b, h]), 7777) for h in range(16)]
+                    for b in range(2)])
+    assert_close_out(O.cpu().numpy(), ref, 2e-5 * float(V.abs().max()), "p=1 vs dense")
+
+
+def test_exact_ties_lower_start():
+    """Identical keys everywhere: every estimate ties exactly and the lower start tokens are kept."""
+    d = 128
+    k = torch.randn(d, generator=torch.Generator().manual_seed(1))
+    K = k.expand(1, 4096, d).contiguous().to(torch.bfloat16)
+    V = torch.randn(1, 4096, d, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    refs = torch.randn(1, 4, d, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    Q = torch.randn(2, 2, d, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    for p in (0.3, 0.5, 0.9):
+        case = Case(K, V, refs, block=4, levels=3, p=p, n=4096, group=2)
+        rep, *_ = check_decode(case, Q, allow_flagged_frac=0.0)
+        assert rep.exact == rep.heads
+
+
+def test_many_candidates_in_cut_bin():
+    """Near-identical estimates over thousands of candidates exercise the radix fallback of the cut."""
+    d = 64
+    g = torch.Generator().manual_seed(5)
+    K = (torch.randn(1, 1, d, generator=g) + 1e-3 * torch.randn(1, 40000, d, generator=g)).to(torch.float32)
+    V = torch.randn(1, 40000, d, generator=g)
+    refs = torch.randn(1, 2, d, generator=g)
+    Q = torch.randn(1, 1, d, generator=g)
+    case = Case(K, V, refs, block=4, levels=2, p=0.7, n=40000, group=1)
+    check_build(case)
+    check_decode(case, Q)
+
+
+def test_append_then_decode():
+    w = small_topics(6000, d=128, n_q_heads=8, n_kv_heads=1, block=4, levels=3, n_refs=4, p=0.9, batch=1)
+    inp = generate(w, n_total=6000)
+    case = Case(inp.K, inp.V, inp.refs, block=4, levels=3, p=0.9, n=4000, group=8, capacity=6000)
+    for m in (1, 1, 1, 1, 7, 100, 1890):
+        case.append(m)
+        check_decode(case, inp.Q[0])
+    check_build(case)
+
+
+def test_errors():
+    K, V, refs, Q = random_tree_case(1, n_tokens=64, d=64, n_q_heads=2, n_kv_heads=1, n_refs=2, batch=1,
+                                     dtype="f32")
+    case = Case(K, V, refs, block=4, levels=2, p=0.9, n=64, group=2, max_batch=2, capacity=64)
+    with pytest.raises(z.ZhaError) as e:
+        case.tree.append(K[:, :1].cuda(), V[:, :1].cuda())
+    assert e.value.code == z.zha.ZHA_ERR_CAPACITY
+    with pytest.raises(z.ZhaError) as e:
+        case.tree.decode(torch.zeros(3, 2, 64, device="cuda"))
+    assert e.value.code == z.zha.ZHA_ERR_CAPACITY
+    with pytest.raises(z.ZhaError):
+        case.tree.build(65)
+    case.tree.status()

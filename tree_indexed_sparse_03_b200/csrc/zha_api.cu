@@ -1,0 +1,420 @@
+// Host side of the C ABI declared in include/zha.h: validation, buffer
+// layouts, tree bookkeeping and kernel launches.  No device memory is
+// allocated here; every buffer belongs to the caller.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "zha_common.cuh"
+
+namespace zha {
+// kernels (zha_build.cu, zha_decode.cu, zha_dense.cu)
+cudaError_t launch_tree_update(const TreeDev& t, int dtype, int64_t n_old, int64_t n_new, cudaStream_t st);
+cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
+                               cudaStream_t st);
+size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R);
+size_t decode_smem_bytes();
+int usable_cluster(int dtype, int d, int want);
+void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
+}  // namespace zha
+
+#include "zha_args.cuh"
+
+using namespace zha;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* msg) {
+  g_err = msg;
+  return code;
+}
+
+int fail_cuda(cudaError_t e, const char* where) {
+  g_err = std::string(where) + ": " + cudaGetErrorString(e);
+  return ZHA_ERR_CUDA;
+}
+
+struct Layout {
+  int S;                                 // chunk level
+  int64_t cap_nodes[kMaxLevels + 1];
+  int64_t pow_b[kMaxLevels + 1];
+  uint64_t rec_off[kMaxLevels + 1], f_off[kMaxLevels + 1], up_off[kMaxLevels + 1];
+  uint64_t rec_bytes, up_bytes, node_bytes;
+  // scratch
+  uint64_t status_off, ws_off, ws_per_bh, stage_off, scratch_bytes;
+  int64_t cap_sel, cap_list;
+  uint64_t stage_k, stage_v, stage_q, stage_o;
+};
+
+uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+int elem_size(int dtype) { return dtype == ZHA_BF16 ? 2 : 4; }
+
+int validate(const zha_config* c) {
+  if (!c) return fail(ZHA_ERR_INVALID, "config is NULL");
+  if (c->d != 64 && c->d != 128) return fail(ZHA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+  if (c->n_kv_heads < 1 || c->n_q_heads < 1) return fail(ZHA_ERR_INVALID, "head counts must be >= 1");
+  if (c->n_q_heads % c->n_kv_heads) return fail(ZHA_ERR_UNSUPPORTED, "n_q_heads must be a multiple of n_kv_heads");
+  if (c->block < 2) return fail(ZHA_ERR_UNSUPPORTED, "block must be >= 2");
+  if (c->levels < 1 || c->levels > kMaxLevels) return fail(ZHA_ERR_UNSUPPORTED, "levels must be in [1, 20]");
+  if (c->n_refs < 1 || c->n_refs > kMaxRefs) return fail(ZHA_ERR_UNSUPPORTED, "n_refs must be in [1, 32]");
+  if (!(c->p > 0.f) || !(c->p <= 1.f)) return fail(ZHA_ERR_INVALID, "p must be in (0, 1]");
+  if (c->dtype != ZHA_F32 && c->dtype != ZHA_BF16) return fail(ZHA_ERR_UNSUPPORTED, "dtype must be ZHA_F32 or ZHA_BF16");
+  if (c->capacity < 1 || c->capacity >= (int64_t(1) << 31)) return fail(ZHA_ERR_INVALID, "capacity must be in [1, 2^31)");
+  if (c->capacity / c->block >= (int64_t(1) << 27)) return fail(ZHA_ERR_UNSUPPORTED, "capacity / block must be < 2^27");
+  if (c->max_batch < 1 || c->max_batch > 65535) return fail(ZHA_ERR_INVALID, "max_batch must be in [1, 65535]");
+  if (c->n_q_heads > 65535) return fail(ZHA_ERR_UNSUPPORTED, "too many query heads");
+  // block^levels must fit comfortably in int64
+  double span = std::pow(double(c->block), double(c->levels));
+  if (span > 4e18) return fail(ZHA_ERR_UNSUPPORTED, "block^levels too large");
+  return ZHA_OK;
+}
+
+int chunk_level_for(const zha_config* c) {
+  int S = 1;
+  int64_t w = c->block;
+  while (S < c->levels && w * c->block <= 64) {
+    w *= c->block;
+    ++S;
+  }
+  return S;
+}
+
+int make_layout(const zha_config* c, Layout* L) {
+  int rc = validate(c);
+  if (rc) return rc;
+  std::memset(L, 0, sizeof(*L));
+  const int es = elem_size(c->dtype);
+  L->S = chunk_level_for(c);
+  if (chunk_smem_bytes(c->dtype, c->d, c->block, L->S, c->n_refs) > 200 * 1024)
+    return fail(ZHA_ERR_UNSUPPORTED, "block too large for the build kernel's shared memory");
+  L->rec_bytes = uint64_t(c->n_refs) * c->d * es + ((uint64_t(c->n_refs) * 4 + 15) & ~uint64_t(15));
+  L->up_bytes = uint64_t(c->n_refs) * (c->d + 2) * 4;
+  uint64_t off = 0;
+  int64_t pw = 1;
+  L->pow_b[0] = 1;
+  L->cap_nodes[0] = c->capacity;
+  for (int l = 1; l <= c->levels; ++l) {
+    pw *= c->block;
+    L->pow_b[l] = pw;
+    L->cap_nodes[l] = c->capacity / pw;
+    L->rec_off[l] = off;
+    off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * L->rec_bytes);
+    L->f_off[l] = off;
+    off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * c->n_refs * 4);
+  }
+  for (int l = L->S; l < c->levels; ++l) {
+    L->up_off[l] = off;
+    off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * L->up_bytes);
+  }
+  L->node_bytes = off > 0 ? off : 256;
+  // scratch: status word, per (sequence, query head) routing workspace, host-step staging
+  L->status_off = 0;
+  const int64_t n1cap = L->cap_nodes[1] > 0 ? L->cap_nodes[1] : 1;
+  L->cap_sel = n1cap;
+  L->cap_list = n1cap + 64;
+  L->ws_off = 256;
+  L->ws_per_bh = align256(uint64_t(2) * L->cap_sel * 8 + uint64_t(L->cap_list) * 8 + uint64_t(L->cap_list) * 4);
+  uint64_t s = L->ws_off + L->ws_per_bh * uint64_t(c->max_batch) * c->n_q_heads;
+  L->stage_off = s;
+  L->stage_k = s;
+  s = align256(s + uint64_t(c->n_kv_heads) * c->d * es);
+  L->stage_v = s;
+  s = align256(s + uint64_t(c->n_kv_heads) * c->d * es);
+  L->stage_q = s;
+  s = align256(s + uint64_t(c->max_batch) * c->n_q_heads * c->d * es);
+  L->stage_o = s;
+  s = align256(s + uint64_t(c->max_batch) * c->n_q_heads * c->d * 4);
+  L->scratch_bytes = s;
+  return ZHA_OK;
+}
+
+}  // namespace
+
+struct zha_tree {
+  zha_config cfg;
+  Layout L;
+  TreeDev dev;
+  char* scratch;
+  int64_t n;
+  int device;
+};
+
+extern "C" {
+
+const char* zha_last_error(void) { return g_err.c_str(); }
+
+int zha_tree_bytes(const zha_config* cfg, size_t* node_bytes, size_t* scratch_bytes) {
+  Layout L;
+  int rc = make_layout(cfg, &L);
+  if (rc) return rc;
+  if (node_bytes) *node_bytes = L.node_bytes;
+  if (scratch_bytes) *scratch_bytes = L.scratch_bytes;
+  return ZHA_OK;
+}
+
+int zha_tree_layout(const zha_config* cfg, int32_t level, size_t* rec_offset, size_t* f_offset, int64_t* cap_nodes,
+                    size_t* rec_bytes) {
+  Layout L;
+  int rc = make_layout(cfg, &L);
+  if (rc) return rc;
+  if (level < 1 || level > cfg->levels) return fail(ZHA_ERR_INVALID, "level out of range");
+  if (rec_offset) *rec_offset = L.rec_off[level];
+  if (f_offset) *f_offset = L.f_off[level];
+  if (cap_nodes) *cap_nodes = L.cap_nodes[level];
+  if (rec_bytes) *rec_bytes = L.rec_bytes;
+  return ZHA_OK;
+}
+
+int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, void* node_buf, void* scratch,
+                    zha_tree** out) {
+  if (!out) return fail(ZHA_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  Layout L;
+  int rc = make_layout(cfg, &L);
+  if (rc) return rc;
+  if (!K || !V || !refs || !node_buf || !scratch) return fail(ZHA_ERR_INVALID, "a buffer pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(refs)) & 15)
+    return fail(ZHA_ERR_INVALID, "K, V and refs must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(node_buf) | reinterpret_cast<uintptr_t>(scratch)) & 255)
+    return fail(ZHA_ERR_INVALID, "node_buf and scratch must be 256-byte aligned");
+  zha_tree* t = new (std::nothrow) zha_tree;
+  if (!t) return fail(ZHA_ERR_INVALID, "out of host memory");
+  t->cfg = *cfg;
+  t->L = L;
+  t->scratch = static_cast<char*>(scratch);
+  t->n = 0;
+  cudaGetDevice(&t->device);
+  TreeDev& d = t->dev;
+  std::memset(&d, 0, sizeof(d));
+  d.d = cfg->d;
+  d.hq = cfg->n_q_heads;
+  d.hkv = cfg->n_kv_heads;
+  d.group = cfg->n_q_heads / cfg->n_kv_heads;
+  d.block = cfg->block;
+  d.levels = cfg->levels;
+  d.refs = cfg->n_refs;
+  d.chunk_level = L.S;
+  d.capacity = cfg->capacity;
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    d.cap_nodes[l] = L.cap_nodes[l];
+    d.pow_b[l] = L.pow_b[l];
+    d.rec_off[l] = L.rec_off[l];
+    d.f_off[l] = L.f_off[l];
+    d.up_off[l] = L.up_off[l];
+  }
+  d.rec_bytes = L.rec_bytes;
+  d.up_bytes = L.up_bytes;
+  d.nodes = static_cast<char*>(node_buf);
+  d.K = K;
+  d.V = V;
+  d.refsp = refs;
+  d.status = reinterpret_cast<int*>(t->scratch + L.status_off);
+  d.inv_sqrt_d = 1.0f / std::sqrt(float(cfg->d));
+  *out = t;
+  return ZHA_OK;
+}
+
+void zha_tree_destroy(zha_tree* tree) { delete tree; }
+
+int64_t zha_tree_size(const zha_tree* tree) { return tree ? tree->n : -1; }
+
+int zha_tree_build(zha_tree* t, int64_t n, void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (n < 0) return fail(ZHA_ERR_INVALID, "n must be >= 0");
+  if (n > t->cfg.capacity) return fail(ZHA_ERR_CAPACITY, "n exceeds capacity");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(t->scratch, 0, t->L.ws_off, st);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build: clearing the status word");
+  e = launch_tree_update(t->dev, t->cfg.dtype, 0, n, st);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build");
+  t->n = n;
+  return ZHA_OK;
+}
+
+int zha_tree_append(zha_tree* t, const void* K_new, const void* V_new, int64_t m, void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (m < 0) return fail(ZHA_ERR_INVALID, "m must be >= 0");
+  if (m == 0) return ZHA_OK;
+  if (!K_new || !V_new) return fail(ZHA_ERR_INVALID, "K_new / V_new is NULL");
+  if ((reinterpret_cast<uintptr_t>(K_new) | reinterpret_cast<uintptr_t>(V_new)) & 15)
+    return fail(ZHA_ERR_INVALID, "K_new and V_new must be 16-byte aligned");
+  if (t->n + m > t->cfg.capacity) return fail(ZHA_ERR_CAPACITY, "append exceeds capacity");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_append_copy(t->dev, t->cfg.dtype, K_new, V_new, t->n, m, st);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_append: copy");
+  e = launch_tree_update(t->dev, t->cfg.dtype, t->n, t->n + m, st);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_append: update");
+  t->n += m;
+  return ZHA_OK;
+}
+
+static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t* kept, int32_t* kept_cnt,
+                            int64_t* stats, DecodeArgs* a) {
+  std::memset(a, 0, sizeof(*a));
+  a->t = t->dev;
+  a->Q = Q;
+  a->O = O;
+  a->n_tokens = t->n;
+  const int L = t->cfg.levels, b = t->cfg.block;
+  for (int l = 0; l <= L; ++l) a->nl[l] = t->n / t->L.pow_b[l];
+  int64_t roots = a->nl[L];
+  int steps = roots > 0 ? L : 0;
+  for (int l = L - 1; l >= 1; --l) {
+    const int64_t cnt = a->nl[l] - int64_t(b) * a->nl[l + 1];
+    roots += cnt;
+    if (cnt > 0 && steps < l) steps = l;
+  }
+  a->n_roots = int(roots);
+  a->n_steps = steps;
+  a->ws = t->scratch + t->L.ws_off;
+  a->ws_per_bh = t->L.ws_per_bh;
+  a->cap_sel = t->L.cap_sel;
+  a->cap_list = t->L.cap_list;
+  a->kept = kept;
+  a->kept_cnt = kept_cnt;
+  a->stats = stats;
+  a->kept_stride = t->L.cap_nodes[1];
+  const float p = t->cfg.p;
+  if (p >= 1.f) {
+    a->p_all = 1;
+  } else {
+    int ex = 0;
+    const float fr = std::frexp(p, &ex);           // p = fr * 2^ex, fr in [0.5, 1)
+    a->p_mant = uint32_t(std::ldexp(fr, 24));      // exact: fr has 24 significant bits
+    a->p_shift = 24 - ex;
+  }
+  return ZHA_OK;
+}
+
+static int cluster_size_for(const zha_tree* t, int B) {
+  static thread_local int cached[2][2] = {{-1, -1}, {-1, -1}};
+  int& max_cs = cached[t->cfg.dtype == ZHA_BF16][t->cfg.d == 128];
+  if (max_cs < 0) max_cs = usable_cluster(t->cfg.dtype, t->cfg.d, 16);
+  const int64_t heads = int64_t(B) * t->cfg.n_q_heads;
+  int want = heads <= 64 ? 16 : (heads <= 128 ? 8 : 4);
+  if (want > max_cs) want = max_cs;
+  return want;
+}
+
+int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* kept, int32_t* kept_cnt,
+               int64_t* stats, void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (!Q || !O) return fail(ZHA_ERR_INVALID, "Q / O is NULL");
+  if ((kept == nullptr) != (kept_cnt == nullptr)) return fail(ZHA_ERR_INVALID, "kept and kept_cnt go together");
+  if (B < 1) return fail(ZHA_ERR_INVALID, "B must be >= 1");
+  if (B > t->cfg.max_batch) return fail(ZHA_ERR_CAPACITY, "B exceeds max_batch");
+  if (t->n < 1) return fail(ZHA_ERR_INVALID, "decode needs at least one cached token");
+  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)
+    return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
+  DecodeArgs a;
+  fill_decode_args(t, Q, O, kept, kept_cnt, stats, &a);
+  const int cs = cluster_size_for(t, B);
+  if (cs < 1) return fail(ZHA_ERR_CUDA, "no thread-block cluster size fits the decode kernel");
+  cudaError_t e = launch_decode(a, t->cfg.dtype, B, cs, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "zha_decode");
+  return ZHA_OK;
+}
+
+int zha_decode_step_host(zha_tree* t, const void* k_host, const void* v_host, const void* q_host, float* o_host,
+                         int32_t B, void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (!q_host || !o_host) return fail(ZHA_ERR_INVALID, "q_host / o_host is NULL");
+  if ((k_host == nullptr) != (v_host == nullptr)) return fail(ZHA_ERR_INVALID, "k_host and v_host go together");
+  if (B < 1 || B > t->cfg.max_batch) return fail(ZHA_ERR_CAPACITY, "B out of range");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int es = elem_size(t->cfg.dtype);
+  char* sk = t->scratch + t->L.stage_k;
+  char* sv = t->scratch + t->L.stage_v;
+  char* sq = t->scratch + t->L.stage_q;
+  float* so = reinterpret_cast<float*>(t->scratch + t->L.stage_o);
+  const size_t kv_bytes = size_t(t->cfg.n_kv_heads) * t->cfg.d * es;
+  const size_t q_bytes = size_t(B) * t->cfg.n_q_heads * t->cfg.d * es;
+  const size_t o_bytes = size_t(B) * t->cfg.n_q_heads * t->cfg.d * 4;
+  cudaError_t e;
+  if (k_host) {
+    if ((e = cudaMemcpyAsync(sk, k_host, kv_bytes, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+      return fail_cuda(e, "zha_decode_step_host: K copy");
+    if ((e = cudaMemcpyAsync(sv, v_host, kv_bytes, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+      return fail_cuda(e, "zha_decode_step_host: V copy");
+  }
+  if ((e = cudaMemcpyAsync(sq, q_host, q_bytes, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+    return fail_cuda(e, "zha_decode_step_host: Q copy");
+  int rc;
+  if (k_host && (rc = zha_tree_append(t, sk, sv, 1, stream)) != ZHA_OK) return rc;
+  if ((rc = zha_decode(t, sq, so, B, nullptr, nullptr, nullptr, stream)) != ZHA_OK) return rc;
+  if ((e = cudaMemcpyAsync(o_host, so, o_bytes, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return fail_cuda(e, "zha_decode_step_host: O copy");
+  return ZHA_OK;
+}
+
+// Dense-decode scratch: completion counters first (fixed size, from max_batch,
+// so that every call finds them at the same place and zero-filled), then the
+// split partials.
+static uint64_t dense_counter_bytes(const zha_config* cfg) {
+  return align256(uint64_t(cfg->max_batch) * cfg->n_q_heads * 4);
+}
+
+size_t zha_dense_scratch_bytes(const zha_config* cfg, int32_t B, int64_t n) {
+  if (validate(cfg) || B < 1 || n < 1 || B > cfg->max_batch) return 0;
+  int splits;
+  int64_t per;
+  dense_plan(B, cfg->n_kv_heads, n, &splits, &per);
+  const uint64_t part = uint64_t(B) * cfg->n_q_heads * splits * (cfg->d + 2) * 4;
+  return size_t(dense_counter_bytes(cfg) + align256(part));
+}
+
+int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n, const void* Q,
+                     float* O, int32_t B, void* scratch, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!K || !V || !Q || !O || !scratch) return fail(ZHA_ERR_INVALID, "a pointer is NULL");
+  if (n < 1 || ld < n) return fail(ZHA_ERR_INVALID, "need 1 <= n <= ld");
+  if (B < 1) return fail(ZHA_ERR_INVALID, "B must be >= 1");
+  if (B > cfg->max_batch) return fail(ZHA_ERR_CAPACITY, "B exceeds max_batch");
+  if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(Q) |
+       reinterpret_cast<uintptr_t>(O)) & 15)
+    return fail(ZHA_ERR_INVALID, "K, V, Q and O must be 16-byte aligned");
+  DenseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  dense_plan(B, cfg->n_kv_heads, n, &a.splits, &a.per);
+  const uint64_t part = uint64_t(B) * cfg->n_q_heads * a.splits * (cfg->d + 2) * 4;
+  a.K = K;
+  a.V = V;
+  a.Q = Q;
+  a.O = O;
+  (void)part;
+  a.counters = static_cast<int*>(scratch);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(scratch) + dense_counter_bytes(cfg));
+  a.ld = ld;
+  a.n = n;
+  a.hq = cfg->n_q_heads;
+  a.hkv = cfg->n_kv_heads;
+  a.group = cfg->n_q_heads / cfg->n_kv_heads;
+  a.inv_sqrt_d = 1.0f / std::sqrt(float(cfg->d));
+  cudaError_t e = launch_dense(a, cfg->dtype, cfg->d, B, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "zha_dense_decode");
+  return ZHA_OK;
+}
+
+int zha_tree_status(zha_tree* t, void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_status: synchronize");
+  int status = 0;
+  e = cudaMemcpy(&status, t->dev.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_tree_status: read");
+  if (status != 0) {
+    const int zero = 0;
+    cudaMemcpy(t->dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(status, "a kernel raised an error status (capacity bound exceeded)");
+  }
+  return ZHA_OK;
+}
+
+}  // extern "C"

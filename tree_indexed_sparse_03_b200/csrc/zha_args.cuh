@@ -1,0 +1,46 @@
+// Kernel argument blocks shared by the host code (zha_api.cu) and the
+// decode / dense kernels.
+#pragma once
+
+#include "zha_common.cuh"
+
+namespace zha {
+
+struct DecodeArgs {
+  TreeDev t;
+  const void* Q;
+  float* O;
+  int64_t n_tokens;
+  int64_t nl[kMaxLevels + 1];   // complete nodes per level (nl[0] = tokens)
+  int n_roots, n_steps;
+  char* ws;
+  uint64_t ws_per_bh;
+  int64_t cap_sel;              // entries per step buffer
+  int64_t cap_list;             // parent / leaf list entries (all CTAs together)
+  int32_t* kept;
+  int32_t* kept_cnt;
+  int64_t* stats;
+  int64_t kept_stride;
+  uint32_t p_mant;              // p = p_mant * 2^-p_shift  (p < 1)
+  int p_shift;
+  int p_all;                    // p >= 1: keep every candidate
+};
+
+struct DenseArgs {
+  const void* K;
+  const void* V;
+  const void* Q;
+  float* O;
+  float* part;       // [B][Hq][splits][D + 2]
+  int* counters;     // [B][Hq]
+  int64_t ld;        // row stride of K / V in tokens
+  int64_t n;
+  int64_t per;       // keys per split (multiple of 64)
+  int splits, hq, hkv, group;
+  float inv_sqrt_d;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, int B, int cs, cudaStream_t st);
+cudaError_t launch_dense(const DenseArgs& a, int dtype, int d, int B, cudaStream_t st);
+
+}  // namespace zha

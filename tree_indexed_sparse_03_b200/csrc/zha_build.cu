@@ -1,0 +1,382 @@
+// Tree build and append kernels.
+//
+// Method ("Zyphra Hierarchical Attention", Zyphra blog, section "Building the
+// tree"; tanhow.com summary, section "How does ZHA's tree indexer work? /
+// Building the tree"): contiguous blocks of `block` raw keys are summarised at
+// each reference query r_j by the tangent plane of their log attention mass
+// f_B(r_j) = log sum_k exp(r_j.k/sqrt(d)): value f, slope mu_j/sqrt(d) with
+// mu_j the softmax-weighted mean key, intercept b_j = f - r_j.mu_j/sqrt(d).
+// Summaries are merged exactly, `block` children per parent: parent f is the
+// logsumexp of the children's f, parent mu_j the children's mu_j weighted by
+// the softmax of their f(r_j).
+//
+// GPU arithmetic (fp32, fixed order, identical for build and append):
+//   leaf:  s_k = (r_j . k) * (1/sqrt d)      (sequential fma over d)
+//          m = max s, Z = sum exp(s - m), f = m + log Z, w_k = exp(s_k - m) / Z
+//          g = sum_k w_k s_k  (= r_j.mu_j/sqrt d exactly),  mu_j = sum_k w_k k
+//   merge: m = max f_c, Z = sum exp(f_c - m), f = m + log Z, a_c = exp(f_c - m) / Z
+//          g = sum_c a_c g_c,  mu_j = sum_c a_c mu_c
+//   store: mu rounded to the element type, b_j = f - g and f in fp32.
+// Every merge reads its children's unrounded fp32 values.  Levels 1..S (S =
+// chunk level, b^S <= 64 keys, or S = 1 when b > 64) are computed inside one
+// CTA per aligned chunk of b^S keys; the chunk roots (level S) and the levels
+// above are kept in fp32 as well, and levels S+1..L are merged from them by
+// upper_kernel.  An append recomputes the chunks that gain complete leaves
+// and writes only the nodes that became complete, so build(n) followed by
+// append(m) stores exactly the same bits as build(n + m).
+#include "zha_common.cuh"
+
+namespace zha {
+
+constexpr int kBuildThreads = 256;
+
+struct ChunkSmem {
+  int CK, KS, RG, NN;
+  size_t keys, refs, w, mu, fs, gs, total;
+};
+
+template <typename T, int D>
+__host__ __device__ inline ChunkSmem chunk_smem_layout(int block, int chunk_level, int R) {
+  ChunkSmem L;
+  int CK = 1;
+  for (int i = 0; i < chunk_level; ++i) CK *= block;
+  L.CK = CK;
+  L.KS = D + 16 / int(sizeof(T));  // key row stride in elements (16-byte pad)
+  L.RG = R < 4 ? R : 4;
+  int nn = 0, w = CK;
+  for (int l = 1; l <= chunk_level; ++l) { w /= block; nn += w; }
+  L.NN = nn;
+  size_t off = 0;
+  L.keys = off; off += size_t(CK) * L.KS * sizeof(T); off = (off + 15) & ~size_t(15);
+  L.refs = off; off += size_t(R) * (D + 1) * 4;
+  L.w = off;    off += size_t(CK) * L.RG * 4;
+  L.mu = off;   off += size_t(nn) * L.RG * D * 4;
+  L.fs = off;   off += size_t(nn) * L.RG * 4;
+  L.gs = off;   off += size_t(nn) * L.RG * 4;
+  L.total = (off + 15) & ~size_t(15);
+  return L;
+}
+
+// One CTA per (chunk, KV head).  Computes every complete node of levels
+// 1..S inside the chunk and writes those with index >= the previous count.
+template <typename T, int D>
+__global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t n_tokens,
+                                                              int64_t n_old, int64_t chunk0) {
+  using E = Elem<T>;
+  const int h = blockIdx.y;
+  const int64_t chunk = chunk0 + blockIdx.x;
+  const int b = t.block, S = t.chunk_level, R = t.refs;
+  const ChunkSmem L = chunk_smem_layout<T, D>(b, S, R);
+  const int CK = L.CK, KS = L.KS, RG = L.RG;
+  const int64_t n1 = n_tokens / b;
+  const int64_t leaves_per_chunk = CK / b;
+  const int64_t leaf0 = chunk * leaves_per_chunk;
+  const int nleaves = int(min64(leaves_per_chunk, n1 - leaf0));
+  if (nleaves <= 0) return;
+  const int nkeys = nleaves * b;
+  const int64_t key0 = chunk * CK;
+  const int tid = threadIdx.x;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  T* keys = reinterpret_cast<T*>(smem + L.keys);
+  float* refs = reinterpret_cast<float*>(smem + L.refs);
+  float* w = reinterpret_cast<float*>(smem + L.w);
+  float* mu = reinterpret_cast<float*>(smem + L.mu);
+  float* fs = reinterpret_cast<float*>(smem + L.fs);
+  float* gs = reinterpret_cast<float*>(smem + L.gs);
+
+  // Stage the chunk's complete keys (16-byte vectors) and the fp32 refs.
+  {
+    constexpr int VPR = D * sizeof(T) / 16;  // vectors per key row
+    const T* Kh = static_cast<const T*>(t.K) + (size_t(h) * t.capacity + key0) * D;
+    for (int i = tid; i < nkeys * VPR; i += blockDim.x) {
+      const int k = i / VPR, v = i % VPR;
+      uint4 x = ldg_stream(Kh + size_t(k) * D + v * (16 / sizeof(T)));
+      *reinterpret_cast<uint4*>(keys + size_t(k) * KS + v * (16 / sizeof(T))) = x;
+    }
+    const T* Rh = static_cast<const T*>(t.refsp) + size_t(h) * R * D;
+    for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+  }
+  __syncthreads();
+
+  // node slot of (level, index-in-chunk) inside the per-chunk arrays
+  auto slot = [&](int level, int i) {
+    int off = 0, wdt = CK;
+    for (int l = 1; l < level; ++l) { wdt /= b; off += wdt; }
+    return off + i;
+  };
+
+  int64_t pw = 1;
+  for (int j0 = 0; j0 < R; j0 += RG) {
+    const int rg = min(RG, R - j0);
+    // scores s[k][jj]
+    for (int i = tid; i < nkeys * rg; i += blockDim.x) {
+      const int k = i / rg, jj = i % rg;
+      const T* kr = keys + size_t(k) * KS;
+      const float* rr = refs + (j0 + jj) * (D + 1);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < D; ++e) acc = __fmaf_rn(E::to_f(kr[e]), rr[e], acc);
+      w[k * RG + jj] = __fmul_rn(acc, t.inv_sqrt_d);
+    }
+    __syncthreads();
+    // leaf value, projected mean score and softmax weights
+    for (int i = tid; i < nleaves * rg; i += blockDim.x) {
+      const int li = i / rg, jj = i % rg;
+      float* s = w + (li * b) * RG + jj;
+      float m = -INFINITY;
+      for (int k = 0; k < b; ++k) m = fmaxf(m, s[k * RG]);
+      float Z = 0.f;
+      for (int k = 0; k < b; ++k) Z = __fadd_rn(Z, expf(__fsub_rn(s[k * RG], m)));
+      const float f = __fadd_rn(m, logf(Z));
+      float g = 0.f;
+      for (int k = 0; k < b; ++k) {
+        const float wk = __fdiv_rn(expf(__fsub_rn(s[k * RG], m)), Z);
+        g = __fmaf_rn(wk, s[k * RG], g);
+        s[k * RG] = wk;
+      }
+      fs[slot(1, li) * RG + jj] = f;
+      gs[slot(1, li) * RG + jj] = g;
+    }
+    __syncthreads();
+    // leaf slopes mu
+    for (int i = tid; i < nleaves * rg * D; i += blockDim.x) {
+      const int e = i % D, jj = (i / D) % rg, li = i / (D * rg);
+      float acc = 0.f;
+      for (int k = 0; k < b; ++k)
+        acc = __fmaf_rn(w[(li * b + k) * RG + jj], E::to_f(keys[size_t(li * b + k) * KS + e]), acc);
+      mu[(size_t(slot(1, li)) * RG + jj) * D + e] = acc;
+    }
+    __syncthreads();
+    // exact merges of levels 2..S inside the chunk
+    int64_t bl = b;  // b^(level-1)
+    for (int level = 2; level <= S; ++level) {
+      bl *= b;
+      const int64_t per_chunk = CK / bl;
+      const int nval = int(min64(per_chunk, n_tokens / bl - chunk * per_chunk));
+      if (nval > 0) {
+        for (int i = tid; i < nval * rg; i += blockDim.x) {
+          const int ni = i / rg, jj = i % rg;
+          const int c0 = slot(level - 1, ni * b);
+          float m = -INFINITY;
+          for (int c = 0; c < b; ++c) m = fmaxf(m, fs[(c0 + c) * RG + jj]);
+          float Z = 0.f;
+          for (int c = 0; c < b; ++c) Z = __fadd_rn(Z, expf(__fsub_rn(fs[(c0 + c) * RG + jj], m)));
+          const float f = __fadd_rn(m, logf(Z));
+          float g = 0.f;
+          for (int c = 0; c < b; ++c) {
+            const float a = __fdiv_rn(expf(__fsub_rn(fs[(c0 + c) * RG + jj], m)), Z);
+            w[(ni * b + c) * RG + jj] = a;
+            g = __fmaf_rn(a, gs[(c0 + c) * RG + jj], g);
+          }
+          fs[slot(level, ni) * RG + jj] = f;
+          gs[slot(level, ni) * RG + jj] = g;
+        }
+        __syncthreads();
+        for (int i = tid; i < nval * rg * D; i += blockDim.x) {
+          const int e = i % D, jj = (i / D) % rg, ni = i / (D * rg);
+          const int c0 = slot(level - 1, ni * b);
+          float acc = 0.f;
+          for (int c = 0; c < b; ++c)
+            acc = __fmaf_rn(w[(ni * b + c) * RG + jj], mu[(size_t(c0 + c) * RG + jj) * D + e], acc);
+          mu[(size_t(slot(level, ni)) * RG + jj) * D + e] = acc;
+        }
+      }
+      __syncthreads();
+    }
+    // write the nodes that are new in this call
+    pw = 1;
+    for (int level = 1; level <= S; ++level) {
+      pw *= b;
+      const int64_t per_chunk = CK / pw;
+      const int64_t base = chunk * per_chunk;
+      const int nval = int(min64(per_chunk, n_tokens / pw - base));
+      const int64_t first_new = n_old / pw;
+      const bool keep32 = (level == S) && (S < t.levels);
+      for (int i = tid; i < nval * rg * D; i += blockDim.x) {
+        const int e = i % D, jj = (i / D) % rg, ni = i / (D * rg);
+        const int64_t gi = base + ni;
+        if (gi < first_new) continue;
+        const float v = mu[(size_t(slot(level, ni)) * RG + jj) * D + e];
+        T* rec = reinterpret_cast<T*>(t.rec(level, h, gi));
+        rec[size_t(j0 + jj) * D + e] = E::from_f(v);
+        if (keep32) t.up(level, h, gi)[size_t(j0 + jj) * D + e] = v;
+      }
+      for (int i = tid; i < nval * rg; i += blockDim.x) {
+        const int jj = i % rg, ni = i / rg;
+        const int64_t gi = base + ni;
+        if (gi < first_new) continue;
+        const float f = fs[slot(level, ni) * RG + jj];
+        const float g = gs[slot(level, ni) * RG + jj];
+        float* bias = reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T));
+        bias[j0 + jj] = __fsub_rn(f, g);
+        t.fval(level, h, gi)[j0 + jj] = f;
+        if (keep32) {
+          float* u = t.up(level, h, gi);
+          u[size_t(R) * D + j0 + jj] = f;
+          u[size_t(R) * D + R + j0 + jj] = g;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // zero the padding after bias[R] once per new node so records are fully defined
+  {
+    pw = 1;
+    const int pad = int((t.rec_bytes - size_t(R) * D * sizeof(T)) / 4) - R;
+    if (pad > 0) {
+      for (int level = 1; level <= S; ++level) {
+        pw *= b;
+        const int64_t per_chunk = CK / pw, base = chunk * per_chunk;
+        const int nval = int(min64(per_chunk, n_tokens / pw - base));
+        const int64_t first_new = n_old / pw;
+        for (int i = tid; i < nval * pad; i += blockDim.x) {
+          const int64_t gi = base + i / pad;
+          if (gi < first_new) continue;
+          reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T))[R + i % pad] = 0.f;
+        }
+      }
+    }
+  }
+}
+
+// One CTA per (new node, KV head) at a level above the chunk level.
+template <typename T, int D>
+__global__ void __launch_bounds__(kBuildThreads) upper_kernel(TreeDev t, int level, int64_t first) {
+  using E = Elem<T>;
+  const int h = blockIdx.y;
+  const int64_t gi = first + blockIdx.x;
+  const int b = t.block, R = t.refs;
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* a = reinterpret_cast<float*>(smem);  // [b][R]
+  float* fg = a + size_t(b) * R;               // f[R], g[R]
+  const int tid = threadIdx.x;
+  for (int j = tid; j < R; j += blockDim.x) {
+    float m = -INFINITY;
+    for (int c = 0; c < b; ++c) m = fmaxf(m, t.up(level - 1, h, gi * b + c)[size_t(R) * D + j]);
+    float Z = 0.f;
+    for (int c = 0; c < b; ++c)
+      Z = __fadd_rn(Z, expf(__fsub_rn(t.up(level - 1, h, gi * b + c)[size_t(R) * D + j], m)));
+    const float f = __fadd_rn(m, logf(Z));
+    float g = 0.f;
+    for (int c = 0; c < b; ++c) {
+      const float* u = t.up(level - 1, h, gi * b + c);
+      const float ac = __fdiv_rn(expf(__fsub_rn(u[size_t(R) * D + j], m)), Z);
+      a[c * R + j] = ac;
+      g = __fmaf_rn(ac, u[size_t(R) * D + R + j], g);
+    }
+    fg[j] = f;
+    fg[R + j] = g;
+  }
+  __syncthreads();
+  const bool keep32 = level < t.levels;
+  T* rec = reinterpret_cast<T*>(t.rec(level, h, gi));
+  for (int i = tid; i < R * D; i += blockDim.x) {
+    const int j = i / D, e = i % D;
+    float acc = 0.f;
+    for (int c = 0; c < b; ++c) acc = __fmaf_rn(a[c * R + j], t.up(level - 1, h, gi * b + c)[i], acc);
+    rec[i] = E::from_f(acc);
+    if (keep32) t.up(level, h, gi)[i] = acc;
+  }
+  float* bias = reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T));
+  const int padded = int((t.rec_bytes - size_t(R) * D * sizeof(T)) / 4);
+  for (int j = tid; j < padded; j += blockDim.x) bias[j] = j < R ? __fsub_rn(fg[j], fg[R + j]) : 0.f;
+  for (int j = tid; j < R; j += blockDim.x) {
+    t.fval(level, h, gi)[j] = fg[j];
+    if (keep32) {
+      float* u = t.up(level, h, gi);
+      u[size_t(R) * D + j] = fg[j];
+      u[size_t(R) * D + R + j] = fg[R + j];
+    }
+  }
+}
+
+// Copy m new tokens ([Hkv][m][d] rows) into the cache at positions [n, n+m).
+template <typename T, int D>
+__global__ void append_copy_kernel(TreeDev t, const T* Knew, const T* Vnew, int64_t n, int64_t m) {
+  constexpr int VPR = D * sizeof(T) / 16;
+  const int64_t total = int64_t(t.hkv) * m * VPR;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t v = i % VPR, row = i / VPR;
+    const int64_t h = row / m, r = row % m;
+    const size_t src = size_t(row) * D + v * (16 / sizeof(T));
+    const size_t dst = (size_t(h) * t.capacity + n + r) * D + v * (16 / sizeof(T));
+    *reinterpret_cast<uint4*>(static_cast<T*>(t.K) + dst) = *reinterpret_cast<const uint4*>(Knew + src);
+    *reinterpret_cast<uint4*>(static_cast<T*>(t.V) + dst) = *reinterpret_cast<const uint4*>(Vnew + src);
+  }
+}
+
+// ------------------------------------------------------------------ host launchers
+template <typename T, int D>
+static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_new, cudaStream_t st) {
+  const int b = t.block, S = t.chunk_level;
+  const int64_t CK = t.pow_b[S];
+  const int64_t n1_old = n_old / b, n1_new = n_new / b;
+  if (n1_new > n1_old) {
+    const int64_t c0 = (n1_old * b) / CK;
+    const int64_t c1 = (n1_new * b - 1) / CK;
+    const ChunkSmem L = chunk_smem_layout<T, D>(b, S, t.refs);
+    cudaError_t e = cudaFuncSetAttribute(chunk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(L.total));
+    if (e != cudaSuccess) return e;
+    dim3 grid(unsigned(c1 - c0 + 1), unsigned(t.hkv));
+    chunk_kernel<T, D><<<grid, kBuildThreads, L.total, st>>>(t, n_new, n_old, c0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  for (int level = S + 1; level <= t.levels; ++level) {
+    const int64_t a0 = n_old / t.pow_b[level], a1 = n_new / t.pow_b[level];
+    if (a1 <= a0) continue;
+    const size_t sm = (size_t(b) * t.refs + 2 * t.refs) * 4;
+    cudaError_t e = cudaFuncSetAttribute(upper_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+    if (e != cudaSuccess) return e;
+    dim3 grid(unsigned(a1 - a0), unsigned(t.hkv));
+    upper_kernel<T, D><<<grid, kBuildThreads, sm, st>>>(t, level, a0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_tree_update(const TreeDev& t, int dtype, int64_t n_old, int64_t n_new, cudaStream_t st) {
+  if (dtype == ZHA_BF16) {
+    return t.d == 128 ? launch_update_t<__nv_bfloat16, 128>(t, n_old, n_new, st)
+                      : launch_update_t<__nv_bfloat16, 64>(t, n_old, n_new, st);
+  }
+  return t.d == 128 ? launch_update_t<float, 128>(t, n_old, n_new, st) : launch_update_t<float, 64>(t, n_old, n_new, st);
+}
+
+cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
+                               cudaStream_t st) {
+  const int64_t vecs = int64_t(t.hkv) * m * (t.d * (dtype == ZHA_BF16 ? 2 : 4) / 16);
+  const int threads = 256;
+  const unsigned blocks = unsigned(min64((vecs + threads - 1) / threads, 148 * 8));
+  if (blocks == 0) return cudaSuccess;
+  if (dtype == ZHA_BF16) {
+    if (t.d == 128)
+      append_copy_kernel<__nv_bfloat16, 128><<<blocks, threads, 0, st>>>(
+          t, static_cast<const __nv_bfloat16*>(Kn), static_cast<const __nv_bfloat16*>(Vn), n, m);
+    else
+      append_copy_kernel<__nv_bfloat16, 64><<<blocks, threads, 0, st>>>(
+          t, static_cast<const __nv_bfloat16*>(Kn), static_cast<const __nv_bfloat16*>(Vn), n, m);
+  } else {
+    if (t.d == 128)
+      append_copy_kernel<float, 128><<<blocks, threads, 0, st>>>(t, static_cast<const float*>(Kn),
+                                                                  static_cast<const float*>(Vn), n, m);
+    else
+      append_copy_kernel<float, 64><<<blocks, threads, 0, st>>>(t, static_cast<const float*>(Kn),
+                                                                 static_cast<const float*>(Vn), n, m);
+  }
+  return cudaGetLastError();
+}
+
+size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R) {
+  if (dtype == ZHA_BF16)
+    return d == 128 ? chunk_smem_layout<__nv_bfloat16, 128>(block, chunk_level, R).total
+                    : chunk_smem_layout<__nv_bfloat16, 64>(block, chunk_level, R).total;
+  return d == 128 ? chunk_smem_layout<float, 128>(block, chunk_level, R).total
+                  : chunk_smem_layout<float, 64>(block, chunk_level, R).total;
+}
+
+}  // namespace zha

@@ -1,0 +1,114 @@
+// Shared device-side definitions of the ZHA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zha.h"
+
+namespace zha {
+
+constexpr int kMaxLevels = 20;   // b >= 2 and capacity < 2^31 keep L well below this
+constexpr int kMaxRefs = 32;
+
+// ---------------------------------------------------------------- element types
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Elements of type T in one 16-byte vector.
+template <typename T> struct Vec { static constexpr int N = 16 / sizeof(T); };
+
+// Read-only 16-byte global load (no L1 allocation: the cache lines are streamed).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Unpack a 16-byte vector of T into fp32.
+template <typename T> __device__ __forceinline__ void unpack16(const uint4& v, float* out);
+template <> __device__ __forceinline__ void unpack16<float>(const uint4& v, float* out) {
+  out[0] = __uint_as_float(v.x);
+  out[1] = __uint_as_float(v.y);
+  out[2] = __uint_as_float(v.z);
+  out[3] = __uint_as_float(v.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& v, float* out) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = __uint_as_float(w[i] << 16);          // low half: element 2i
+    out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);  // high half: element 2i+1
+  }
+}
+
+// ---------------------------------------------------------------- ordered keys
+// Order-preserving map of fp32 onto uint32 (ascending), and the descending key
+// used to rank routing candidates: a smaller key means a larger estimate.
+__device__ __forceinline__ uint32_t float_to_ordered(float x) {
+  uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ordered_to_float(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ uint32_t desc_key(float e) { return ~float_to_ordered(e); }
+__device__ __forceinline__ float desc_key_value(uint32_t k) { return ordered_to_float(~k); }
+
+// Node codes: level in the top 5 bits, index within the level in the low 27.
+__device__ __forceinline__ uint32_t node_code(int level, uint32_t idx) {
+  return (uint32_t(level) << 27) | idx;
+}
+__device__ __forceinline__ int code_level(uint32_t c) { return int(c >> 27); }
+__device__ __forceinline__ uint32_t code_index(uint32_t c) { return c & 0x07ffffffu; }
+
+// ---------------------------------------------------------------- tree description
+// Everything a kernel needs to address the node storage of one tree.
+struct TreeDev {
+  int d, hq, hkv, group, block, levels, refs, chunk_level;
+  int64_t capacity;
+  int64_t cap_nodes[kMaxLevels + 1];   // node slots per KV head per level
+  int64_t pow_b[kMaxLevels + 1];       // block^level (tokens per node)
+  uint64_t rec_off[kMaxLevels + 1];    // byte offsets in the node buffer
+  uint64_t f_off[kMaxLevels + 1];
+  uint64_t up_off[kMaxLevels + 1];     // fp32 full nodes, levels chunk_level .. levels-1
+  uint64_t rec_bytes;                  // mu[R][d] (element type) + bias[R] fp32, padded to 16 B
+  uint64_t up_bytes;                   // mu[R][d] fp32 + f[R] + g[R]
+  char* nodes;
+  void* K;
+  void* V;
+  const void* refsp;
+  int* status;
+  float inv_sqrt_d;
+
+  __device__ __forceinline__ char* rec(int level, int head, int64_t i) const {
+    return nodes + rec_off[level] + (uint64_t(head) * cap_nodes[level] + i) * rec_bytes;
+  }
+  __device__ __forceinline__ float* fval(int level, int head, int64_t i) const {
+    return reinterpret_cast<float*>(nodes + f_off[level]) +
+           (uint64_t(head) * cap_nodes[level] + i) * refs;
+  }
+  __device__ __forceinline__ float* up(int level, int head, int64_t i) const {
+    return reinterpret_cast<float*>(nodes + up_off[level] + (uint64_t(head) * cap_nodes[level] + i) * up_bytes);
+  }
+};
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ void raise_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace zha
