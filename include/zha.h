@@ -150,10 +150,14 @@ ZHA_API int64_t zha_tree_size(const zha_tree* tree);
  *              order; kept_cnt [B][Hq] int32 receives their number.  Both NULL
  *              or both non-NULL.
  *   stats    - optional [B][Hq][ZHA_STAT_COUNT] int64 counters.
+ *   scored   - optional [B][Hq][scored_cap] int32: the codes (level << 27 | index)
+ *              of every node the head scored, step by step; ZHA_STAT_NODES_SCORED
+ *              gives how many (entries past scored_cap are dropped).  Used to
+ *              count the bytes a decode must read; leave NULL on the hot path.
  * Requires 1 <= B <= max_batch and at least one cached token.
  */
 ZHA_API int zha_decode(const zha_tree* tree, const void* Q, float* O, int32_t B, int32_t* kept,
-               int32_t* kept_cnt, int64_t* stats, void* stream);
+               int32_t* kept_cnt, int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream);
 
 /*
  * zha_decode_step_host: one decode step from host memory - copies the new
@@ -184,6 +188,10 @@ ZHA_API int zha_dense_decode(const zha_config* cfg, const void* K, const void* V
 ZHA_API int zha_tree_status(zha_tree* tree, void* stream);
 
 ZHA_API void zha_tree_destroy(zha_tree* tree);
+
+/* Number of kernels this library has launched in this process (all threads,
+ * all devices) - lets a caller verify which work ran on the GPU. */
+ZHA_API uint64_t zha_launch_count(void);
 
 /* Message for the last failing call on this thread ("" if none). */
 ZHA_API const char* zha_last_error(void);

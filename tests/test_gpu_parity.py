@@ -43,6 +43,7 @@ class Case:
         self.n = n
 
     def append(self, m):
+        assert self.n + m <= self.Kall.shape[1]
         self.tree.append(self.Kall[:, self.n:self.n + m].cuda(), self.Vall[:, self.n:self.n + m].cuda())
         self.n += m
 
@@ -245,7 +246,7 @@ def test_append_then_decode():
     w = small_topics(6000, d=128, n_q_heads=8, n_kv_heads=1, block=4, levels=3, n_refs=4, p=0.9, batch=1)
     inp = generate(w, n_total=6000)
     case = Case(inp.K, inp.V, inp.refs, block=4, levels=3, p=0.9, n=4000, group=8, capacity=6000)
-    for m in (1, 1, 1, 1, 7, 100, 1890):
+    for m in (1, 1, 1, 1, 7, 100, 1889):
         case.append(m)
         check_decode(case, inp.Q[0])
     check_build(case)

@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/zha.h: validation, buffer
 // layouts, tree bookkeeping and kernel launches.  No device memory is
 // allocated here; every buffer belongs to the caller.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -23,6 +24,9 @@ void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
 #include "zha_args.cuh"
 
 using namespace zha;
+
+static std::atomic<uint64_t> g_launches{0};
+void zha::count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
 
 namespace {
 
@@ -148,6 +152,8 @@ extern "C" {
 
 const char* zha_last_error(void) { return g_err.c_str(); }
 
+uint64_t zha_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 int zha_tree_bytes(const zha_config* cfg, size_t* node_bytes, size_t* scratch_bytes) {
   Layout L;
   int rc = make_layout(cfg, &L);
@@ -254,7 +260,7 @@ int zha_tree_append(zha_tree* t, const void* K_new, const void* V_new, int64_t m
 }
 
 static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t* kept, int32_t* kept_cnt,
-                            int64_t* stats, DecodeArgs* a) {
+                            int64_t* stats, int32_t* scored, int64_t scored_cap, DecodeArgs* a) {
   std::memset(a, 0, sizeof(*a));
   a->t = t->dev;
   a->Q = Q;
@@ -278,6 +284,8 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->kept = kept;
   a->kept_cnt = kept_cnt;
   a->stats = stats;
+  a->scored = scored;
+  a->scored_cap = scored ? scored_cap : 0;
   a->kept_stride = t->L.cap_nodes[1];
   const float p = t->cfg.p;
   if (p >= 1.f) {
@@ -302,17 +310,18 @@ static int cluster_size_for(const zha_tree* t, int B) {
 }
 
 int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* kept, int32_t* kept_cnt,
-               int64_t* stats, void* stream) {
+               int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream) {
   if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
   if (!Q || !O) return fail(ZHA_ERR_INVALID, "Q / O is NULL");
   if ((kept == nullptr) != (kept_cnt == nullptr)) return fail(ZHA_ERR_INVALID, "kept and kept_cnt go together");
   if (B < 1) return fail(ZHA_ERR_INVALID, "B must be >= 1");
   if (B > t->cfg.max_batch) return fail(ZHA_ERR_CAPACITY, "B exceeds max_batch");
   if (t->n < 1) return fail(ZHA_ERR_INVALID, "decode needs at least one cached token");
+  if (scored && scored_cap < 1) return fail(ZHA_ERR_INVALID, "scored needs scored_cap >= 1");
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)
     return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
   DecodeArgs a;
-  fill_decode_args(t, Q, O, kept, kept_cnt, stats, &a);
+  fill_decode_args(t, Q, O, kept, kept_cnt, stats, scored, scored_cap, &a);
   const int cs = cluster_size_for(t, B);
   if (cs < 1) return fail(ZHA_ERR_CUDA, "no thread-block cluster size fits the decode kernel");
   cudaError_t e = launch_decode(a, t->cfg.dtype, B, cs, static_cast<cudaStream_t>(stream));
@@ -346,7 +355,7 @@ int zha_decode_step_host(zha_tree* t, const void* k_host, const void* v_host, co
     return fail_cuda(e, "zha_decode_step_host: Q copy");
   int rc;
   if (k_host && (rc = zha_tree_append(t, sk, sv, 1, stream)) != ZHA_OK) return rc;
-  if ((rc = zha_decode(t, sq, so, B, nullptr, nullptr, nullptr, stream)) != ZHA_OK) return rc;
+  if ((rc = zha_decode(t, sq, so, B, nullptr, nullptr, nullptr, nullptr, 0, stream)) != ZHA_OK) return rc;
   if ((e = cudaMemcpyAsync(o_host, so, o_bytes, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
     return fail_cuda(e, "zha_decode_step_host: O copy");
   return ZHA_OK;

@@ -20,6 +20,8 @@ struct DecodeArgs {
   int32_t* kept;
   int32_t* kept_cnt;
   int64_t* stats;
+  int32_t* scored;
+  int64_t scored_cap;
   int64_t kept_stride;
   uint32_t p_mant;              // p = p_mant * 2^-p_shift  (p < 1)
   int p_shift;
@@ -39,6 +41,9 @@ struct DenseArgs {
   int splits, hq, hkv, group;
   float inv_sqrt_d;
 };
+
+// kernels launched by this library (incremented by every launcher)
+void count_launches(int n);
 
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, int B, int cs, cudaStream_t st);
 cudaError_t launch_dense(const DenseArgs& a, int dtype, int d, int B, cudaStream_t st);

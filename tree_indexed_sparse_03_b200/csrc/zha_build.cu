@@ -24,7 +24,7 @@
 // upper_kernel.  An append recomputes the chunks that gain complete leaves
 // and writes only the nodes that became complete, so build(n) followed by
 // append(m) stores exactly the same bits as build(n + m).
-#include "zha_common.cuh"
+#include "zha_args.cuh"
 
 namespace zha {
 
@@ -321,6 +321,7 @@ static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_ne
                                          int(L.total));
     if (e != cudaSuccess) return e;
     dim3 grid(unsigned(c1 - c0 + 1), unsigned(t.hkv));
+    count_launches(1);
     chunk_kernel<T, D><<<grid, kBuildThreads, L.total, st>>>(t, n_new, n_old, c0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -332,6 +333,7 @@ static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_ne
     cudaError_t e = cudaFuncSetAttribute(upper_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
     if (e != cudaSuccess) return e;
     dim3 grid(unsigned(a1 - a0), unsigned(t.hkv));
+    count_launches(1);
     upper_kernel<T, D><<<grid, kBuildThreads, sm, st>>>(t, level, a0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -353,6 +355,7 @@ cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, cons
   const int threads = 256;
   const unsigned blocks = unsigned(min64((vecs + threads - 1) / threads, 148 * 8));
   if (blocks == 0) return cudaSuccess;
+  count_launches(1);
   if (dtype == ZHA_BF16) {
     if (t.d == 128)
       append_copy_kernel<__nv_bfloat16, 128><<<blocks, threads, 0, st>>>(

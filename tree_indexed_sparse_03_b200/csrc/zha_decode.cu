@@ -425,7 +425,6 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_kernel(DecodeArgs a) {
     cluster.sync();
     if (n_cand == 0) continue;   // uniform across the cluster
     ++steps_taken;
-    scored += n_cand;
 
     // ---- select (identical in every CTA of the cluster)
     const bool cached = n_cand <= kSelSmem;
@@ -436,6 +435,12 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_kernel(DecodeArgs a) {
       }
       __syncthreads();
     }
+    if (a.scored && r == 0) {
+      int32_t* out = a.scored + (size_t(bb) * a.t.hq + h) * a.scored_cap;
+      for (int64_t i = tid; i < n_cand; i += kDecThreads)
+        if (scored + i < a.scored_cap) out[scored + i] = int32_t(load_entry(S, i, cached, sm).code);
+    }
+    scored += n_cand;
     const unsigned long long cut = select_cut(a, S, n_cand, cached, sm);
 
     // ---- ranks of the kept entries in canonical order
@@ -642,6 +647,7 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, int B, int cs, cudaStrea
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  count_launches(1);
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

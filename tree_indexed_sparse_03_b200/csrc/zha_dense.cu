@@ -338,6 +338,7 @@ bool dense_uses_mma(int dtype, int group) { return dtype == ZHA_BF16 && group <=
 
 cudaError_t launch_dense(const DenseArgs& a0, int dtype, int d, int B, cudaStream_t st) {
   DenseArgs a = a0;
+  count_launches(1);
   if (dense_uses_mma(dtype, a.group)) {
     dim3 grid(unsigned(a.splits), unsigned(a.hkv), unsigned(B));
     if (d == 128) dense_mma_kernel<128><<<grid, kDenseThreads, 0, st>>>(a);

@@ -35,7 +35,7 @@ _SIGS = {
     "zha_tree_append": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p]),
     "zha_tree_size": (_c.c_int64, [_c.c_void_p]),
     "zha_decode": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_void_p,
-                              _c.c_void_p, _c.c_void_p]),
+                              _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p]),
     "zha_decode_step_host": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                         _c.c_int32, _c.c_void_p]),
     "zha_dense_scratch_bytes": (_c.c_size_t, [_c.c_void_p, _c.c_int32, _c.c_int64]),
@@ -44,6 +44,7 @@ _SIGS = {
     "zha_tree_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "zha_tree_destroy": (None, [_c.c_void_p]),
     "zha_last_error": (_c.c_char_p, []),
+    "zha_launch_count": (_c.c_uint64, []),
 }
 
 _lib = None
@@ -160,7 +161,7 @@ class ZhaTree:
         _check(lib().zha_tree_append(self._h, K_new.data_ptr(), V_new.data_ptr(), m, _stream(stream)))
 
     def decode(self, Q: torch.Tensor, *, want_kept: bool = False, want_stats: bool = False, out=None,
-               stream=None):
+               scored_cap: int = 0, stream=None):
         """Decode queries Q [B, Hq, d].  Returns O [B, Hq, d] fp32 (and kept lists / stats when asked)."""
         B = Q.shape[0]
         Q = Q.contiguous()
@@ -173,15 +174,20 @@ class ZhaTree:
             cnt = torch.zeros(B, self.cfg.n_q_heads, dtype=torch.int32, device=Q.device)
         if want_stats:
             stats = torch.zeros(B, self.cfg.n_q_heads, STAT_COUNT, dtype=torch.int64, device=Q.device)
+        scored = None
+        if scored_cap > 0:
+            scored = torch.full((B, self.cfg.n_q_heads, scored_cap), -1, dtype=torch.int32, device=Q.device)
         _check(lib().zha_decode(self._h, Q.data_ptr(), O.data_ptr(), B, _ptr(kept), _ptr(cnt), _ptr(stats),
-                                _stream(stream)))
-        if not (want_kept or want_stats):
+                                _ptr(scored), scored_cap, _stream(stream)))
+        if not (want_kept or want_stats or scored is not None):
             return O
         res = [O]
         if want_kept:
             res.append((kept, cnt))
         if want_stats:
             res.append(stats)
+        if scored is not None:
+            res.append(scored)
         return tuple(res)
 
     def decode_step_host(self, k_host: Optional[torch.Tensor], v_host: Optional[torch.Tensor], q_host: torch.Tensor,
@@ -208,6 +214,11 @@ class ZhaTree:
         f = self.nodes[lay.f_offset: lay.f_offset + n * c.n_refs * 4].view(torch.float32).view(
             c.n_kv_heads, lay.cap_nodes, c.n_refs)
         return mu, bias, f
+
+
+def launch_count() -> int:
+    """Kernels libzha.so has launched in this process."""
+    return int(lib().zha_launch_count())
 
 
 def dense_scratch_bytes(cfg: ZhaConfig, B: int, n: int) -> int:
