@@ -265,3 +265,24 @@ def test_errors():
     with pytest.raises(z.ZhaError):
         case.tree.build(65)
     case.tree.status()
+
+
+def test_barrier_timeout_is_reported_and_recoverable(monkeypatch):
+    """A grid-barrier wait that runs out returns ZHA_ERR_TIMEOUT through the status word; the context stays usable.
+
+    ZHA_SPIN_LIMIT=1 (read when a tree is created) makes every waiting CTA give up at once; the kernel
+    then returns without touching memory beyond its bounds-checked workspace.
+    """
+    K, V, refs, Q = random_tree_case(21, n_tokens=3000, d=128, n_q_heads=8, n_kv_heads=1, n_refs=4, batch=2,
+                                     dtype="bf16")
+    monkeypatch.setenv("ZHA_SPIN_LIMIT", "1")
+    bad = Case(K, V, refs, block=4, levels=3, p=0.9, n=3000, group=8)
+    monkeypatch.delenv("ZHA_SPIN_LIMIT")
+    bad.tree.decode(Q.cuda())
+    torch.cuda.synchronize()
+    with pytest.raises(z.ZhaError) as e:
+        bad.tree.status()
+    assert e.value.code == z.zha.ZHA_ERR_TIMEOUT
+    # a tree with the normal spin bound decodes correctly afterwards in the same context
+    good = Case(K, V, refs, block=4, levels=3, p=0.9, n=3000, group=8)
+    check_decode(good, Q)

@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -17,7 +18,9 @@ cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, cons
                                cudaStream_t st);
 size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R);
 size_t decode_smem_bytes();
-int usable_cluster(int dtype, int d, int want);
+size_t decode_head_state_bytes();
+int decode_max_heads();
+int decode_items_per_cta();
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
 }  // namespace zha
 
@@ -49,12 +52,15 @@ struct Layout {
   uint64_t rec_off[kMaxLevels + 1], f_off[kMaxLevels + 1], up_off[kMaxLevels + 1];
   uint64_t rec_bytes, up_bytes, node_bytes;
   // scratch
-  uint64_t status_off, ws_off, ws_per_bh, stage_off, scratch_bytes;
+  uint64_t status_off, bar_off, part_off, part_items, ws_off, ws_per_bh, stage_off, scratch_bytes;
   int64_t cap_sel, cap_list;
   uint64_t stage_k, stage_v, stage_q, stage_o;
 };
 
 uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+constexpr int kMaxDecodeGrid = 256;
+constexpr long long kDefaultSpinLimit = 1ll << 24;  // ~1 s of 40 ns sleeps  // CTAs of the decode launch (one per SM) the scratch is sized for
 
 int elem_size(int dtype) { return dtype == ZHA_BF16 ? 2 : 4; }
 
@@ -71,7 +77,8 @@ int validate(const zha_config* c) {
   if (c->capacity < 1 || c->capacity >= (int64_t(1) << 31)) return fail(ZHA_ERR_INVALID, "capacity must be in [1, 2^31)");
   if (c->capacity / c->block >= (int64_t(1) << 27)) return fail(ZHA_ERR_UNSUPPORTED, "capacity / block must be < 2^27");
   if (c->max_batch < 1 || c->max_batch > 65535) return fail(ZHA_ERR_INVALID, "max_batch must be in [1, 65535]");
-  if (c->n_q_heads > 65535) return fail(ZHA_ERR_UNSUPPORTED, "too many query heads");
+  if (int64_t(c->max_batch) * c->n_q_heads > decode_max_heads())
+    return fail(ZHA_ERR_UNSUPPORTED, "max_batch * n_q_heads must be <= 2048");
   // block^levels must fit comfortably in int64
   double span = std::pow(double(c->block), double(c->levels));
   if (span > 4e18) return fail(ZHA_ERR_UNSUPPORTED, "block^levels too large");
@@ -116,13 +123,19 @@ int make_layout(const zha_config* c, Layout* L) {
     off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * L->up_bytes);
   }
   L->node_bytes = off > 0 ? off : 256;
-  // scratch: status word, per (sequence, query head) routing workspace, host-step staging
+  // scratch: status word and grid barrier, attend partials, per (sequence,
+  // query head) routing workspace, host-step staging
   L->status_off = 0;
+  L->bar_off = 64;
   const int64_t n1cap = L->cap_nodes[1] > 0 ? L->cap_nodes[1] : 1;
   L->cap_sel = n1cap;
   L->cap_list = n1cap + 64;
-  L->ws_off = 256;
-  L->ws_per_bh = align256(uint64_t(2) * L->cap_sel * 8 + uint64_t(L->cap_list) * 8 + uint64_t(L->cap_list) * 4);
+  const uint64_t nheads = uint64_t(c->max_batch) * c->n_q_heads;
+  L->part_off = 256;
+  L->part_items = uint64_t(kMaxDecodeGrid) * decode_items_per_cta() + nheads + 64;
+  L->ws_off = align256(L->part_off + L->part_items * (c->d + 2) * 4);
+  L->ws_per_bh = align256(uint64_t(2) * L->cap_sel * 8 + uint64_t(L->cap_sel) * 4 + uint64_t(L->cap_list) * 4 +
+                          decode_head_state_bytes());
   uint64_t s = L->ws_off + L->ws_per_bh * uint64_t(c->max_batch) * c->n_q_heads;
   L->stage_off = s;
   L->stage_k = s;
@@ -146,6 +159,7 @@ struct zha_tree {
   char* scratch;
   int64_t n;
   int device;
+  long long spin_limit;  // grid-barrier spin bound of the decode kernel
 };
 
 extern "C" {
@@ -194,6 +208,11 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
   t->L = L;
   t->scratch = static_cast<char*>(scratch);
   t->n = 0;
+  t->spin_limit = kDefaultSpinLimit;
+  if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: force the barrier timeout path
+    const long long x = std::atoll(v);
+    if (x > 0) t->spin_limit = x;
+  }
   cudaGetDevice(&t->device);
   TreeDev& d = t->dev;
   std::memset(&d, 0, sizeof(d));
@@ -234,7 +253,7 @@ int zha_tree_build(zha_tree* t, int64_t n, void* stream) {
   if (n < 0) return fail(ZHA_ERR_INVALID, "n must be >= 0");
   if (n > t->cfg.capacity) return fail(ZHA_ERR_CAPACITY, "n exceeds capacity");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(t->scratch, 0, t->L.ws_off, st);
+  cudaError_t e = cudaMemsetAsync(t->scratch, 0, 256, st);
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build: clearing the status word");
   e = launch_tree_update(t->dev, t->cfg.dtype, 0, n, st);
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build");
@@ -279,6 +298,9 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->n_steps = steps;
   a->ws = t->scratch + t->L.ws_off;
   a->ws_per_bh = t->L.ws_per_bh;
+  a->bar = reinterpret_cast<unsigned int*>(t->scratch + t->L.bar_off);
+  a->attn_part = reinterpret_cast<float*>(t->scratch + t->L.part_off);
+  a->spin_limit = t->spin_limit;
   a->cap_sel = t->L.cap_sel;
   a->cap_list = t->L.cap_list;
   a->kept = kept;
@@ -299,16 +321,6 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   return ZHA_OK;
 }
 
-static int cluster_size_for(const zha_tree* t, int B) {
-  static thread_local int cached[2][2] = {{-1, -1}, {-1, -1}};
-  int& max_cs = cached[t->cfg.dtype == ZHA_BF16][t->cfg.d == 128];
-  if (max_cs < 0) max_cs = usable_cluster(t->cfg.dtype, t->cfg.d, 16);
-  const int64_t heads = int64_t(B) * t->cfg.n_q_heads;
-  int want = heads <= 64 ? 16 : (heads <= 128 ? 8 : 4);
-  if (want > max_cs) want = max_cs;
-  return want;
-}
-
 int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* kept, int32_t* kept_cnt,
                int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream) {
   if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
@@ -322,9 +334,8 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
     return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
   DecodeArgs a;
   fill_decode_args(t, Q, O, kept, kept_cnt, stats, scored, scored_cap, &a);
-  const int cs = cluster_size_for(t, B);
-  if (cs < 1) return fail(ZHA_ERR_CUDA, "no thread-block cluster size fits the decode kernel");
-  cudaError_t e = launch_decode(a, t->cfg.dtype, B, cs, static_cast<cudaStream_t>(stream));
+  a.nheads = B * t->cfg.n_q_heads;
+  cudaError_t e = launch_decode(a, t->cfg.dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "zha_decode");
   return ZHA_OK;
 }
@@ -361,20 +372,13 @@ int zha_decode_step_host(zha_tree* t, const void* k_host, const void* v_host, co
   return ZHA_OK;
 }
 
-// Dense-decode scratch: completion counters first (fixed size, from max_batch,
-// so that every call finds them at the same place and zero-filled), then the
-// split partials.
-static uint64_t dense_counter_bytes(const zha_config* cfg) {
-  return align256(uint64_t(cfg->max_batch) * cfg->n_q_heads * 4);
-}
-
 size_t zha_dense_scratch_bytes(const zha_config* cfg, int32_t B, int64_t n) {
   if (validate(cfg) || B < 1 || n < 1 || B > cfg->max_batch) return 0;
   int splits;
   int64_t per;
   dense_plan(B, cfg->n_kv_heads, n, &splits, &per);
   const uint64_t part = uint64_t(B) * cfg->n_q_heads * splits * (cfg->d + 2) * 4;
-  return size_t(dense_counter_bytes(cfg) + align256(part));
+  return size_t(align256(part));
 }
 
 int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n, const void* Q,
@@ -397,8 +401,7 @@ int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_
   a.Q = Q;
   a.O = O;
   (void)part;
-  a.counters = static_cast<int*>(scratch);
-  a.part = reinterpret_cast<float*>(static_cast<char*>(scratch) + dense_counter_bytes(cfg));
+  a.part = static_cast<float*>(scratch);
   a.ld = ld;
   a.n = n;
   a.hq = cfg->n_q_heads;

@@ -8,15 +8,19 @@ namespace zha {
 
 struct DecodeArgs {
   TreeDev t;
-  const void* Q;
-  float* O;
+  const void* Q;                // [nheads][d]: sequence-major, then query head
+  float* O;                     // [nheads][d]
   int64_t n_tokens;
   int64_t nl[kMaxLevels + 1];   // complete nodes per level (nl[0] = tokens)
   int n_roots, n_steps;
-  char* ws;
+  int nheads;                   // sequences x query heads
+  char* ws;                     // per-head workspaces, ws_per_bh bytes each
   uint64_t ws_per_bh;
-  int64_t cap_sel;              // entries per step buffer
-  int64_t cap_list;             // parent / leaf list entries (all CTAs together)
+  int64_t cap_sel;              // entries per step buffer (and kept parents)
+  int64_t cap_list;             // kept leaves per head
+  unsigned int* bar;            // grid barrier: {count, generation}
+  float* attn_part;             // attend partials, (2 + d) floats each
+  long long spin_limit;         // grid-barrier spin bound
   int32_t* kept;
   int32_t* kept_cnt;
   int64_t* stats;
@@ -34,7 +38,6 @@ struct DenseArgs {
   const void* Q;
   float* O;
   float* part;       // [B][Hq][splits][D + 2]
-  int* counters;     // [B][Hq]
   int64_t ld;        // row stride of K / V in tokens
   int64_t n;
   int64_t per;       // keys per split (multiple of 64)
@@ -45,7 +48,7 @@ struct DenseArgs {
 // kernels launched by this library (incremented by every launcher)
 void count_launches(int n);
 
-cudaError_t launch_decode(const DecodeArgs& a, int dtype, int B, int cs, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_dense(const DenseArgs& a, int dtype, int d, int B, cudaStream_t st);
 
 }  // namespace zha

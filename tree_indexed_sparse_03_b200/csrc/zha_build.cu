@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kBuildThreads) upper_kernel(TreeDev t, int lev
   const bool keep32 = level < t.levels;
   T* rec = reinterpret_cast<T*>(t.rec(level, h, gi));
   for (int i = tid; i < R * D; i += blockDim.x) {
-    const int j = i / D, e = i % D;
+    const int j = i / D;
     float acc = 0.f;
     for (int c = 0; c < b; ++c) acc = __fmaf_rn(a[c * R + j], t.up(level - 1, h, gi * b + c)[i], acc);
     rec[i] = E::from_f(acc);

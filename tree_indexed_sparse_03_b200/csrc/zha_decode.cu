@@ -14,31 +14,29 @@
 // mass >= p; ties in e go to the lower start token; tokens after the last
 // complete block (the tail) are always attended.
 //
-// GPU design.  One thread-block cluster of CS CTAs per (sequence, query head);
-// the whole decode of that head is one kernel launch with one cluster barrier
-// per routing step:
-//   score   each CTA scores the candidates it owns (the children of the kept
-//           parents whose rank is = its cluster rank mod CS) with one warp per
-//           node, and writes (descending key of e, node code) at the
-//           candidate's canonical position in the step's global buffer;
-//   barrier
-//   select  every CTA reads the whole buffer and computes the same cut:
-//           masses w = exp(e - max e) as 2^-40 fixed-point integers (exact,
-//           order-independent sums), a 1024-bin histogram of the masses over
-//           (max e - e) in 1/32-logit bins finds the bin holding the cut, and
-//           the few entries of that bin are ordered by (e desc, start asc) to
-//           find the last kept entry;  kept = every entry ordered at or before
-//           it;  each CTA then takes its round-robin share of the kept
-//           parents (next step) and of the kept leaves (attention).
-// After the last step each CTA attends over its share of the kept blocks
-// (plus the sink and tail on the last CTA) with an online softmax, and the
-// partial (max, sum, output) triples are combined in CTA 0's shared memory
-// over distributed shared memory.
-#include <cooperative_groups.h>
-
+// GPU design.  One persistent cooperative launch per decode call; all query
+// heads of all sequences are routed together so that the whole GPU shares
+// the work of the heads whose routing is diffuse.  Phases are separated by a
+// software grid barrier (bounded spin: on timeout the kernel raises
+// ZHA_ERR_TIMEOUT and returns):
+//   score   (all CTAs) the step's candidates of every head form one list;
+//           each warp scores one node at a time (16-byte loads of its planes,
+//           fp32 dot products) and writes (descending key of e, node code) at
+//           the candidate's canonical position in its head's step buffer;
+//   select  (one CTA per head) masses w = exp(e - max e) as 2^-40 fixed-point
+//           integers (exact, order-independent sums); a 1024-bin histogram of
+//           the masses over (max e - e) in 1/32-logit bins, then 1024 sub-bins
+//           of the cut bin, isolate the few entries around the cut, which are
+//           ordered by (e desc, start asc); kept = every entry at or before the
+//           cut.  Kept non-leaf nodes become the next step's parents (their
+//           children, in rank order, are the next candidates); kept leaves are
+//           appended to the head's attend list;
+//   attend  (all CTAs) every head's attended keys (kept blocks, sink, tail)
+//           are cut into chunks; CTAs own contiguous ranges of chunks, warps
+//           run an online softmax per chunk, and each CTA merges its chunks per
+//           head into one partial;
+//   combine (one CTA per head) the partials of each head -> O.
 #include "zha_args.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace zha {
 
@@ -47,34 +45,42 @@ struct Entry {
   uint32_t code;  // node_code(level, index)
 };
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kSelSmem = 4096;   // entries cached in shared memory
+constexpr int kSelCache = 20480;  // entries of one head cached in shared memory by the select
 constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
-constexpr int kMaxCluster = 16;
+constexpr int kMaxHeads = 2048;   // sequences x query heads per call
+constexpr int kItemsPerCta = 256; // attend chunks a CTA owns at most (plus one per head it touches)
+constexpr int kMaxDecodeGrid = 256;  // CTAs per decode launch the scratch is laid out for
 
-constexpr int kLeafSmem = 3840;  // leaf indices cached for the attention phase
-
-struct AttendSmem {
-  uint32_t leaf[kLeafSmem];
-  float grp[kDecWarps * 4][2 + 128];  // per lane-group partials (m, l, o[d])
+struct HeadState {  // per (sequence, query head), written by the head's select CTA
+  long long n_cand;   // candidates of the next step
+  long long n_leaf;   // kept level-1 blocks so far
+  long long scored;   // nodes scored so far
+  int steps;
+  int leaf0;          // leaf block 0 kept (token 0 already attended)
+  long long pad[4];
 };
 
 struct __align__(16) DecSmem {
   union {
-    Entry cache[kSelSmem];            // routing: the step's candidate entries
-    AttendSmem att;                   // attention: this CTA's leaf list + group partials
+    Entry cache[kSelCache];                 // select: the head's entries
+    float part[kSelCache * 2 / (2 + 128)][2 + 128];  // attend: per-chunk partials of this CTA (kPartSlots)
   };
   unsigned long long hist[kBins];
+  long long pref[kMaxHeads + 1];            // per-head prefix of work items
   unsigned long long cut_key[32];
   unsigned long long cut_w[32];
-  float part[kMaxCluster][2 + 128];   // partials received by CTA 0 (m, l, o[d])
   unsigned long long red64[kDecWarps];
   uint32_t red32[kDecWarps * 2];
   unsigned long long bcast64[4];
+  long long bcastll[4];
   int bcast32[8];
+  int fail;
 };
+constexpr int kPartSlots = kSelCache * 2 / (2 + 128);  // attend partials a CTA can hold
+static_assert(kPartSlots >= kItemsPerCta + 32, "attend partial area too small");
 
 __device__ __forceinline__ uint32_t root_code(const DecodeArgs& a, int64_t i) {
   const int L = a.t.levels, b = a.t.block;
@@ -222,15 +228,52 @@ __device__ __forceinline__ Entry load_entry(const Entry* E, int64_t i, bool cach
   return Entry{v.x, v.y};
 }
 
-__device__ __forceinline__ int entry_bin(float m, uint32_t key) {
-  const float x = __fsub_rn(m, desc_key_value(key));
-  const float y = fminf(__fmul_rn(x, kBinScale), float(kBins - 1));
-  return int(y);
+// Distance of an entry below the maximum estimate, in fp32: x = m - e >= 0.
+// Bins over x are monotone in e (fp32 subtraction and power-of-two scaling
+// round monotonically), so every entry of a lower bin precedes every entry of
+// a higher bin in the (e desc, start asc) order, and equal estimates share a
+// bin.  Coarse bins are 1/32 logit wide (kBins of them, the last one open);
+// fine bins split a coarse bin into kBins parts of 1/32768 logit.
+__device__ __forceinline__ float entry_gap(float m, uint32_t key) { return __fsub_rn(m, desc_key_value(key)); }
+__device__ __forceinline__ int coarse_bin(float x) { return int(fminf(__fmul_rn(x, kBinScale), float(kBins - 1))); }
+__device__ __forceinline__ int fine_bin(float x, int cb) {
+  const float y = fminf(__fmul_rn(x, kBinScale * float(kBins)), float(kBins) * float(kBins) - 1.f);
+  return min(int(y) - cb * kBins, kBins - 1);
 }
 
 __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) {
   const float w = expf(__fsub_rn(desc_key_value(key), m));
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
+}
+
+// Over kBins mass bins (shared memory), find the bin where the running mass,
+// starting from `base`, first reaches `target`: returns the bin and the mass
+// before it (all threads).  -1 if no bin does.
+__device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base, unsigned long long target,
+                                            unsigned long long* below_out) {
+  constexpr int BPT = kBins / kDecThreads;
+  const int tid = threadIdx.x;
+  unsigned long long local = 0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) local += sm.hist[tid * BPT + k];
+  unsigned long long total;
+  unsigned long long before = base + block_scan_u64(local, sm.red64, &total);
+  if (tid == 0) sm.bcast32[0] = -1;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    const unsigned long long hb = sm.hist[tid * BPT + k];
+    if (before < target && before + hb >= target) {
+      sm.bcast32[0] = tid * BPT + k;
+      sm.bcast64[0] = before;
+    }
+    before += hb;
+  }
+  __syncthreads();
+  const int bin = sm.bcast32[0];
+  *below_out = sm.bcast64[0];
+  __syncthreads();
+  return bin;
 }
 
 // The cut of one routing step: the largest 64-bit order key (e desc, start
@@ -244,42 +287,47 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
 
+  // coarse histogram of the masses; total mass Z and the target T = ceil(p Z)
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
     const Entry en = load_entry(E, i, cached, sm);
-    atomicAdd(&sm.hist[entry_bin(m, en.key)], entry_mass(m, en.key));
+    atomicAdd(&sm.hist[coarse_bin(entry_gap(m, en.key))], entry_mass(m, en.key));
   }
   __syncthreads();
-  // prefix over the bins (kBins / kDecThreads consecutive bins per thread)
-  constexpr int BPT = kBins / kDecThreads;
-  unsigned long long local = 0;
+  unsigned long long Z = 0;
+  {
+    constexpr int BPT = kBins / kDecThreads;
+    unsigned long long local = 0;
 #pragma unroll
-  for (int k = 0; k < BPT; ++k) local += sm.hist[tid * BPT + k];
-  unsigned long long Z;
-  unsigned long long before = block_scan_u64(local, sm.red64, &Z);
+    for (int k = 0; k < BPT; ++k) local += sm.hist[tid * BPT + k];
+    block_scan_u64(local, sm.red64, &Z);
+  }
   const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);  // keep while mass before < T
-  if (tid == 0) sm.bcast32[0] = -1;
+  unsigned long long below;
+  const int cb = find_cut_bin(sm, 0ull, T, &below);
+  if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
+
+  // fine histogram inside the cut coarse bin
+  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
-#pragma unroll
-  for (int k = 0; k < BPT; ++k) {
-    const unsigned long long hb = sm.hist[tid * BPT + k];
-    if (before < T && before + hb >= T) {
-      sm.bcast32[0] = tid * BPT + k;
-      sm.bcast64[0] = before;
-    }
-    before += hb;
+  for (int64_t i = tid; i < n; i += kDecThreads) {
+    const Entry en = load_entry(E, i, cached, sm);
+    const float x = entry_gap(m, en.key);
+    if (coarse_bin(x) == cb) atomicAdd(&sm.hist[fine_bin(x, cb)], entry_mass(m, en.key));
   }
   __syncthreads();
-  const int cb = sm.bcast32[0];
-  const unsigned long long below = sm.bcast64[0];
-  if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
-  // gather the entries of the cut bin
+  unsigned long long below2;
+  const int fb = find_cut_bin(sm, below, T, &below2);
+  if (fb < 0) return ~0ull;
+
+  // gather the entries of the cut fine bin
   if (tid == 0) sm.bcast32[1] = 0;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
     const Entry en = load_entry(E, i, cached, sm);
-    if (entry_bin(m, en.key) == cb) {
+    const float x = entry_gap(m, en.key);
+    if (coarse_bin(x) == cb && fine_bin(x, cb) == fb) {
       const int s = atomicAdd(&sm.bcast32[1], 1);
       if (s < 32) {
         sm.cut_key[s] = entry_key64(a, en);
@@ -313,7 +361,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
         const unsigned long long y = __shfl_up_sync(0xffffffffu, c, off);
         if (tid >= off) c += y;
       }
-      const unsigned hit = __ballot_sync(0xffffffffu, tid < cnt && below + c >= T);
+      const unsigned hit = __ballot_sync(0xffffffffu, tid < cnt && below2 + c >= T);
       const int first = hit ? __ffs(hit) - 1 : cnt - 1;
       const unsigned long long cut = __shfl_sync(0xffffffffu, k, first);
       if (tid == 0) sm.bcast64[1] = cut;
@@ -321,31 +369,50 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
     __syncthreads();
     return sm.bcast64[1];
   }
-  // Many entries share the cut bin (ties or near-ties): radix select on the
-  // 64-bit order key, 8 bits per pass, over the bin's entries.
-  const unsigned long long target = T - below;  // > 0
-  unsigned long long prefix = 0, acc_below = 0;
+  // Many entries share the cut fine bin (exact ties or near-ties): radix
+  // select on the 64-bit order key, 8 bits per pass, over that bin's entries.
+  unsigned long long prefix = 0, acc_below = below2;
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     for (int i = tid; i < 256; i += kDecThreads) sm.hist[i] = 0ull;
     __syncthreads();
     for (int64_t i = tid; i < n; i += kDecThreads) {
       const Entry en = load_entry(E, i, cached, sm);
-      if (entry_bin(m, en.key) != cb) continue;
+      const float x = entry_gap(m, en.key);
+      if (coarse_bin(x) != cb || fine_bin(x, cb) != fb) continue;
       const unsigned long long k64 = entry_key64(a, en);
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
       atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, en.key));
     }
     __syncthreads();
-    if (tid == 0) {
-      unsigned long long c = acc_below;
-      int digit = 255;
-      for (int dgt = 0; dgt < 256; ++dgt) {
-        if (c + sm.hist[dgt] >= target) { digit = dgt; break; }
-        c += sm.hist[dgt];
+    if (tid < 32) {
+      // warp-parallel search over the 256 digit bins (8 per lane)
+      unsigned long long loc = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) loc += sm.hist[tid * 8 + k];
+      unsigned long long c = loc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, c, off);
+        if (tid >= off) c += y;
       }
-      sm.bcast64[2] = prefix | (uint64_t(digit) << shift);
-      sm.bcast64[3] = c;
+      unsigned long long before = acc_below + c - loc;
+      int digit = -1;
+      unsigned long long dbelow = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const unsigned long long hb = sm.hist[tid * 8 + k];
+        if (digit < 0 && before < T && before + hb >= T) { digit = tid * 8 + k; dbelow = before; }
+        before += hb;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, digit >= 0);
+      const int src = hit ? __ffs(hit) - 1 : 31;
+      const int dg = __shfl_sync(0xffffffffu, hit ? digit : 255, src);
+      const unsigned long long db = __shfl_sync(0xffffffffu, dbelow, src);
+      if (tid == 0) {
+        sm.bcast64[2] = prefix | (uint64_t(dg) << shift);
+        sm.bcast64[3] = hit ? db : acc_below;
+      }
     }
     __syncthreads();
     prefix = sm.bcast64[2];
@@ -355,340 +422,491 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   return prefix;
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, 3) decode_kernel(DecodeArgs a) {
-  using E = Elem<T>;
-  constexpr int EPC = 16 / sizeof(T);
-  constexpr int CPR = D * sizeof(T) / 16;
-  constexpr int KPW = 32 / CPR;  // keys per warp pass in the attention loop
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CS = int(cluster.num_blocks());
-  const int r = int(cluster.block_rank());
-  const int h = blockIdx.y, bb = blockIdx.z;
-  const int kvh = h / a.t.group;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int b = a.t.block;
 
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
-
-  char* ws = a.ws + uint64_t(bb * a.t.hq + h) * a.ws_per_bh;
-  Entry* sel[2] = {reinterpret_cast<Entry*>(ws), reinterpret_cast<Entry*>(ws) + a.cap_sel};
-  const int64_t per_cta = a.cap_list / CS;
-  uint2* my_par = reinterpret_cast<uint2*>(ws + 2 * a.cap_sel * sizeof(Entry)) + r * per_cta;
-  uint32_t* my_leaf = reinterpret_cast<uint32_t*>(ws + 2 * a.cap_sel * sizeof(Entry) + a.cap_list * 8) + r * per_cta;
-
-  // the lane's slice of q (fp32)
-  float qs[EPC];
-  {
-    const T* q = static_cast<const T*>(a.Q) + (size_t(bb) * a.t.hq + h) * D + (lane % CPR) * EPC;
-    const uint4 v = *reinterpret_cast<const uint4*>(q);
-    unpack16<T>(v, qs);
-  }
-
-  // distributed shared memory of CTA 0 is written at the end: make sure every
-  // CTA of the cluster has started when no routing step provides a barrier
-  if (a.n_steps == 0) cluster.sync();
-
-  int64_t n_cand = a.n_roots;
-  int64_t my_npar = 0;          // parents this CTA expands in the next step
-  int64_t leafbase = 0;         // kept leaves so far (all CTAs)
-  int64_t scored = 0;
-  bool leaf0 = false;
-  int steps_taken = 0;
-
-  for (int step = 0; step < a.n_steps; ++step) {
-    Entry* S = sel[step & 1];
-    // ---- score the candidates this CTA owns
-    if (step == 0) {
-      for (int64_t i = r + int64_t(CS) * wid; i < n_cand; i += int64_t(CS) * kDecWarps) {
-        const uint32_t code = root_code(a, i);
-        const float e = score_node<T, D>(a.t, kvh, code, qs, lane);
-        if (lane == 0) S[i] = Entry{desc_key(e), code};
-      }
+// Software grid barrier over all CTAs of the cooperative launch.  Returns
+// true (for every thread of the CTA) if the wait gave up.
+__device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    sm.fail = 0;
+    volatile unsigned int* gen = a.bar + 1;
+    const unsigned int g = *gen;
+    __threadfence();
+    const unsigned int arrived = atomicAdd(a.bar, 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(a.bar, 0u);
+      __threadfence();
+      atomicAdd(a.bar + 1, 1u);
     } else {
-      const int64_t items = my_npar * b;
-      for (int64_t u = wid; u < items; u += kDecWarps) {
-        const uint2 pr = __ldcg(my_par + u / b);
-        const int c = int(u % b);
-        const uint32_t pc = pr.x;
-        const uint32_t code = node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(c));
-        const float e = score_node<T, D>(a.t, kvh, code, qs, lane);
-        const int64_t pos = int64_t(pr.y) * b + c;
-        if (lane == 0) {
-          if (pos < a.cap_sel) S[pos] = Entry{desc_key(e), code};
-          else raise_status(a.t.status, ZHA_ERR_CAPACITY);
+      long long it = 0;
+      while (*gen == g) {
+        if (++it > a.spin_limit) {
+          sm.fail = 1;
+          raise_status(a.t.status, ZHA_ERR_TIMEOUT);
+          break;
         }
+        __nanosleep(40);
       }
     }
     __threadfence();
-    cluster.sync();
-    if (n_cand == 0) continue;   // uniform across the cluster
-    ++steps_taken;
+  }
+  __syncthreads();
+  return sm.fail != 0;
+}
 
-    // ---- select (identical in every CTA of the cluster)
-    const bool cached = n_cand <= kSelSmem;
-    if (cached) {
-      for (int64_t i = tid; i < n_cand; i += kDecThreads) {
-        const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
-        sm.cache[i] = Entry{v.x, v.y};
+// Inclusive prefix of per-head counts into sm.pref[1..nh] (pref[0] = 0); all threads.
+__device__ __forceinline__ long long build_prefix(DecSmem& sm, int nh) {
+  // counts are in sm.pref[1..nh]; scan them in place, chunk by chunk
+  long long carry = 0;
+  for (int base = 0; base < nh; base += kDecThreads) {
+    const int i = base + threadIdx.x;
+    const unsigned long long v = i < nh ? (unsigned long long)sm.pref[1 + i] : 0ull;
+    unsigned long long tot;
+    const unsigned long long ex = block_scan_u64(v, sm.red64, &tot);
+    if (i < nh) sm.pref[1 + i] = carry + (long long)(ex + v);
+    carry += (long long)tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) sm.pref[0] = 0;
+  __syncthreads();
+  return carry;
+}
+
+// Head owning work item i: the largest h with pref[h] <= i.
+__device__ __forceinline__ int owner_of(const DecSmem& sm, int nh, long long i) {
+  int lo = 0, hi = nh - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sm.pref[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ bool valid_code(const DecodeArgs& a, uint32_t code) {
+  const int l = code_level(code);
+  return l >= 1 && l <= a.t.levels && int64_t(code_index(code)) < a.nl[l];
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
+  constexpr int EPC = 16 / sizeof(T);
+  constexpr int CPR = D * sizeof(T) / 16;
+  constexpr int KPW = 32 / CPR;  // keys per warp pass in the attention loop
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nh = a.nheads;
+  const int b = a.t.block;
+  const long long gwarp = (long long)blockIdx.x * kDecWarps + wid;
+  const long long nwarps = (long long)gridDim.x * kDecWarps;
+  auto ws = [&](int h) { return a.ws + uint64_t(h) * a.ws_per_bh; };
+  auto sel = [&](int h, int step) { return reinterpret_cast<Entry*>(ws(h)) + (step & 1) * a.cap_sel; };
+  auto par = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 2 * a.cap_sel * sizeof(Entry)); };
+  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 2 * a.cap_sel * sizeof(Entry) + a.cap_sel * 4); };
+  auto hstate = [&](int h) {
+    return reinterpret_cast<HeadState*>(ws(h) + 2 * a.cap_sel * sizeof(Entry) + a.cap_sel * 4 + a.cap_list * 4);
+  };
+  auto q_slice = [&](int h, float* qs) {
+    const T* q = static_cast<const T*>(a.Q) + size_t(h) * D + (lane % CPR) * EPC;
+    unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
+  };
+
+  for (int step = 0; step < a.n_steps; ++step) {
+    // ---------------- score (all CTAs)
+    for (int i = tid; i < nh; i += kDecThreads) {
+      long long c = a.n_roots;
+      if (step > 0) c = min64(max64(__ldcg(&hstate(i)->n_cand), 0), a.cap_sel);
+      sm.pref[1 + i] = c;
+    }
+    __syncthreads();
+    const long long total = build_prefix(sm, nh);
+    for (long long it = gwarp; it < total; it += nwarps) {
+      const int h = owner_of(sm, nh, it);
+      const long long pos = it - sm.pref[h];
+      uint32_t code;
+      if (step == 0) {
+        code = root_code(a, pos);
+      } else {
+        const uint32_t pc = __ldcg(par(h) + pos / b);
+        code = node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(pos % b));
+        if (code_level(pc) < 2 || !valid_code(a, pc) || !valid_code(a, code)) {
+          if (lane == 0) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+          continue;
+        }
+      }
+      float qs[EPC];
+      q_slice(h, qs);
+      const int kvh = (h % a.t.hq) / a.t.group;
+      const float e = score_node<T, D>(a.t, kvh, code, qs, lane);
+      if (lane == 0) sel(h, step)[pos] = Entry{desc_key(e), code};
+    }
+    if (grid_sync(a, sm)) return;
+
+    // ---------------- select (one CTA per head)
+    for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+      const long long n = sm.pref[h + 1] - sm.pref[h];
+      HeadState* hs = hstate(h);
+      long long n_leaf0 = 0, scored0 = 0;
+      int leaf0 = 0, steps0 = 0;
+      if (step > 0) {
+        n_leaf0 = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
+        scored0 = __ldcg(&hs->scored);
+        leaf0 = __ldcg(&hs->leaf0);
+        steps0 = __ldcg(&hs->steps);
+      }
+      if (n == 0) {
+        if (tid == 0) {
+          hs->n_cand = 0;
+          hs->n_leaf = n_leaf0;
+          hs->scored = scored0;
+          hs->leaf0 = leaf0;
+          hs->steps = steps0;
+        }
+        continue;
+      }
+      const Entry* S = sel(h, step);
+      const bool cached = n <= kSelCache;
+      __syncthreads();
+      if (cached) {
+        for (long long i = tid; i < n; i += kDecThreads) {
+          const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
+          sm.cache[i] = Entry{v.x, v.y};
+        }
+        __syncthreads();
+      }
+      if (a.scored) {
+        int32_t* out = a.scored + size_t(h) * a.scored_cap;
+        for (long long i = tid; i < n; i += kDecThreads)
+          if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(load_entry(S, i, cached, sm).code);
+      }
+      const unsigned long long cut = select_cut(a, S, n, cached, sm);
+      // ranks of the kept entries in canonical order
+      const long long per_thr = (n + kDecThreads - 1) / kDecThreads;
+      const long long lo = min64(n, tid * per_thr), hi = min64(n, lo + per_thr);
+      uint32_t nleaf = 0, npar = 0;
+      for (long long i = lo; i < hi; ++i) {
+        const Entry en = load_entry(S, i, cached, sm);
+        if (entry_key64(a, en) <= cut) {
+          if (code_level(en.code) == 1) ++nleaf; else ++npar;
+        }
+      }
+      uint32_t tot_leaf, tot_par;
+      uint32_t leaf_rank = block_scan_u32(nleaf, sm.red32, &tot_leaf);
+      uint32_t par_rank = block_scan_u32(npar, sm.red32, &tot_par);
+      int my_leaf0 = 0;
+      for (long long i = lo; i < hi; ++i) {
+        const Entry en = load_entry(S, i, cached, sm);
+        if (entry_key64(a, en) > cut) continue;
+        if (code_level(en.code) == 1) {
+          const long long g = n_leaf0 + leaf_rank++;
+          if (code_index(en.code) == 0) my_leaf0 = 1;
+          if (g < a.cap_list) leaves(h)[g] = code_index(en.code);
+          else raise_status(a.t.status, ZHA_ERR_CAPACITY);
+          if (a.kept && g < a.kept_stride) a.kept[size_t(h) * a.kept_stride + g] = int32_t(code_index(en.code));
+        } else {
+          const uint32_t pr = par_rank++;
+          if (pr < a.cap_sel) par(h)[pr] = en.code;
+        }
+      }
+      my_leaf0 = __syncthreads_or(my_leaf0);
+      if (tid == 0) {
+        long long nc = (long long)tot_par * b;
+        if (nc > a.cap_sel) {
+          raise_status(a.t.status, ZHA_ERR_CAPACITY);
+          nc = 0;
+        }
+        hs->n_cand = nc;
+        hs->n_leaf = min64(n_leaf0 + tot_leaf, a.cap_list);
+        hs->scored = scored0 + n;
+        hs->leaf0 = leaf0 | my_leaf0;
+        hs->steps = steps0 + 1;
       }
       __syncthreads();
     }
-    if (a.scored && r == 0) {
-      int32_t* out = a.scored + (size_t(bb) * a.t.hq + h) * a.scored_cap;
-      for (int64_t i = tid; i < n_cand; i += kDecThreads)
-        if (scored + i < a.scored_cap) out[scored + i] = int32_t(load_entry(S, i, cached, sm).code);
-    }
-    scored += n_cand;
-    const unsigned long long cut = select_cut(a, S, n_cand, cached, sm);
-
-    // ---- ranks of the kept entries in canonical order
-    const int64_t per_thr = (n_cand + kDecThreads - 1) / kDecThreads;
-    const int64_t lo = min64(n_cand, tid * per_thr), hi = min64(n_cand, lo + per_thr);
-    uint32_t nleaf = 0, npar = 0;
-    for (int64_t i = lo; i < hi; ++i) {
-      const Entry en = load_entry(S, i, cached, sm);
-      if (entry_key64(a, en) <= cut) {
-        if (code_level(en.code) == 1) ++nleaf; else ++npar;
-      }
-    }
-    uint32_t tot_leaf, tot_par;
-    uint32_t leaf_rank = block_scan_u32(nleaf, sm.red32, &tot_leaf);
-    uint32_t par_rank = block_scan_u32(npar, sm.red32, &tot_par);
-    for (int64_t i = lo; i < hi; ++i) {
-      const Entry en = load_entry(S, i, cached, sm);
-      if (entry_key64(a, en) > cut) continue;
-      if (code_level(en.code) == 1) {
-        const int64_t g = leafbase + leaf_rank++;
-        if (code_index(en.code) == 0) leaf0 = true;
-        if (g % CS == r) {
-          const int64_t slot = g / CS;
-          if (slot < per_cta) my_leaf[slot] = code_index(en.code);
-          else raise_status(a.t.status, ZHA_ERR_CAPACITY);
-        }
-        if (a.kept && r == 0 && g < a.kept_stride)
-          a.kept[(size_t(bb) * a.t.hq + h) * a.kept_stride + g] = int32_t(code_index(en.code));
-      } else {
-        const uint32_t pr = par_rank++;
-        if (int(pr % CS) == r) {
-          const int64_t slot = pr / CS;
-          if (slot < per_cta) my_par[slot] = make_uint2(en.code, pr);
-          else raise_status(a.t.status, ZHA_ERR_CAPACITY);
-        }
-      }
-    }
-    // every CTA learns whether leaf 0 was kept (a leaf-0 entry may sit in another thread's range)
-    leaf0 = __syncthreads_or(leaf0);
-    leafbase += tot_leaf;
-    my_npar = min64((int64_t(tot_par) > r) ? (int64_t(tot_par) - r + CS - 1) / CS : 0, per_cta);
-    n_cand = int64_t(tot_par) * b;
-    if (n_cand > a.cap_sel) {
-      raise_status(a.t.status, ZHA_ERR_CAPACITY);
-      n_cand = a.cap_sel;
-      my_npar = 0;
-    }
+    if (grid_sync(a, sm)) return;
   }
 
-  // ---- attention over this CTA's share of the attended tokens
-  const int64_t n1 = a.nl[1];
-  const int64_t my_nleaf = (leafbase > r) ? (leafbase - r + CS - 1) / CS : 0;
-  const int64_t my_leaf_keys = min64(my_nleaf, per_cta) * b;
-  int64_t extra0 = 0, extra_cnt = 0;  // [extra0, extra0+extra_cnt) after an optional sink
-  bool sink = false;
-  if (r == CS - 1) {
-    sink = (n1 > 0) && !leaf0;
-    extra0 = n1 * b;
-    extra_cnt = a.n_tokens - n1 * b;
+  // ---------------- attend (all CTAs)
+  const long long n1 = a.nl[1];
+  const long long tail = a.n_tokens - n1 * b;
+  // keys per head: kept blocks x b + sink (when block 0 is not kept) + tail
+  for (int i = tid; i < nh; i += kDecThreads) {
+    long long nl = 0;
+    int l0 = 0;
+    if (a.n_steps > 0) {
+      nl = min64(max64(__ldcg(&hstate(i)->n_leaf), 0), a.cap_list);
+      l0 = __ldcg(&hstate(i)->leaf0);
+    }
+    sm.pref[1 + i] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
   }
-  const int64_t total = my_leaf_keys + (sink ? 1 : 0) + extra_cnt;
-  // cache this CTA's leaf list in shared memory (the entry cache is free now)
-  uint32_t* leaf_s = sm.att.leaf;
-  const int64_t nls = min64(my_leaf_keys / b, int64_t(kLeafSmem));
   __syncthreads();
-  for (int64_t i = tid; i < nls; i += kDecThreads) leaf_s[i] = __ldcg(my_leaf + i);
+  const long long total_keys = build_prefix(sm, nh);
+  // chunk size: at least 32 keys, large enough that a CTA owns <= kItemsPerCta chunks (+1 per head)
+  long long chunk = (total_keys + (long long)gridDim.x * kItemsPerCta - 1) / ((long long)gridDim.x * kItemsPerCta);
+  chunk = max64(32, chunk);
+  // items per head = ceil(keys / chunk) (sm.pref becomes the item prefix; key
+  // counts are recomputed from the head state where needed)
+  for (int i = tid; i < nh; i += kDecThreads) {
+    long long nl = 0;
+    int l0 = 0;
+    if (a.n_steps > 0) {
+      nl = min64(max64(__ldcg(&hstate(i)->n_leaf), 0), a.cap_list);
+      l0 = __ldcg(&hstate(i)->leaf0);
+    }
+    const long long kh = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
+    sm.pref[1 + i] = (kh + chunk - 1) / chunk;
+  }
   __syncthreads();
-
-  const T* Kh = static_cast<const T*>(a.t.K) + size_t(kvh) * a.t.capacity * D;
-  const T* Vh = static_cast<const T*>(a.t.V) + size_t(kvh) * a.t.capacity * D;
-  const int sub = lane / CPR, cl = lane % CPR;
-  float m_run = -INFINITY, l_run = 0.f;
-  float o[EPC];
+  const long long total_items = build_prefix(sm, nh);
+  const long long c0 = (long long)blockIdx.x * total_items / gridDim.x;
+  const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kPartSlots);
+  if (tid == 0 && (long long)(blockIdx.x + 1) * total_items / gridDim.x > c1) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+  {
+    const int sub = lane / CPR, cl = lane % CPR;
+    constexpr int kU = 4;
+    for (long long it = c0 + wid; it < c1; it += kDecWarps) {
+      const int h = owner_of(sm, nh, it);
+      const long long ci = it - sm.pref[h];
+      const int kvh = (h % a.t.hq) / a.t.group;
+      long long nl = 0;
+      int l0 = 0;
+      if (a.n_steps > 0) {
+        nl = min64(max64(__ldcg(&hstate(h)->n_leaf), 0), a.cap_list);
+        l0 = __ldcg(&hstate(h)->leaf0);
+      }
+      const bool sink = (n1 > 0) && !l0;
+      const long long leaf_keys = nl * b;
+      const long long kh = leaf_keys + (sink ? 1 : 0) + tail;
+      const long long k0 = ci * chunk, k1 = min64(kh, k0 + chunk);
+      float qs[EPC];
+      q_slice(h, qs);
+      const T* Kh = static_cast<const T*>(a.t.K) + size_t(kvh) * a.t.capacity * D;
+      const T* Vh = static_cast<const T*>(a.t.V) + size_t(kvh) * a.t.capacity * D;
+      const uint32_t* lv = leaves(h);
+      float m_run = -INFINITY, l_run = 0.f, o[EPC];
 #pragma unroll
-  for (int i = 0; i < EPC; ++i) o[i] = 0.f;
-  constexpr int kU = 4;
-  const int64_t gstride = int64_t(kDecWarps) * KPW;
-  // the loop bound is warp-uniform (wb); lane groups differ only through `ok`
-  for (int64_t wb = int64_t(wid) * KPW; wb < total; wb += gstride * kU) {
-    uint4 kv[kU], vv[kU];
-    bool ok[kU];
+      for (int i = 0; i < EPC; ++i) o[i] = 0.f;
+      for (long long wb = k0; wb < k1; wb += (long long)KPW * kU) {
+        uint4 kv[kU], vv[kU];
+        bool ok[kU];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t idx = wb + sub + u * gstride;
-      ok[u] = idx < total;
-      if (ok[u]) {
-        int64_t tok;
-        if (idx < my_leaf_keys) {
-          const int64_t li = idx / b;
-          const uint32_t leaf = li < nls ? leaf_s[li] : __ldcg(my_leaf + li);
-          tok = int64_t(leaf) * b + idx % b;
-        } else {
-          int64_t x = idx - my_leaf_keys;
-          if (sink) {
-            if (x == 0) tok = 0;
-            else tok = extra0 + x - 1;
-          } else {
-            tok = extra0 + x;
+        for (int u = 0; u < kU; ++u) {
+          const long long idx = wb + (long long)u * KPW + sub;
+          ok[u] = idx < k1;
+          if (ok[u]) {
+            long long tok;
+            if (idx < leaf_keys) {
+              const uint32_t leaf = __ldcg(lv + idx / b);
+              tok = int64_t(leaf) * b + idx % b;
+            } else if (sink && idx == leaf_keys) {
+              tok = 0;
+            } else {
+              tok = n1 * b + (idx - leaf_keys - (sink ? 1 : 0));
+            }
+            if (tok < 0 || tok >= a.n_tokens) {  // a corrupted leaf index: skip it
+              ok[u] = false;
+              raise_status(a.t.status, ZHA_ERR_CAPACITY);
+              continue;
+            }
+            kv[u] = ldg_stream(Kh + size_t(tok) * D + cl * EPC);
+            vv[u] = ldg_stream(Vh + size_t(tok) * D + cl * EPC);
           }
         }
-        kv[u] = ldg_stream(Kh + size_t(tok) * D + cl * EPC);
-        vv[u] = ldg_stream(Vh + size_t(tok) * D + cl * EPC);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          float kx[EPC];
+          float s = 0.f;
+          if (ok[u]) {
+            unpack16<T>(kv[u], kx);
+#pragma unroll
+            for (int i = 0; i < EPC; ++i) s = fmaf(kx[i], qs[i], s);
+          }
+#pragma unroll
+          for (int off = CPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+          if (ok[u]) {
+            s *= a.t.inv_sqrt_d;
+            const float mn = fmaxf(m_run, s);
+            const float sc = expf(m_run - mn);
+            const float pk = expf(s - mn);
+            l_run = l_run * sc + pk;
+            float vx[EPC];
+            unpack16<T>(vv[u], vx);
+#pragma unroll
+            for (int i = 0; i < EPC; ++i) o[i] = fmaf(pk, vx[i], o[i] * sc);
+            m_run = mn;
+          }
+        }
       }
-    }
+      // merge the KPW lane groups of the warp (lanes l, l+CPR, ... hold the same d-range)
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      float kx[EPC];
-      float s = 0.f;
-      if (ok[u]) {
-        unpack16<T>(kv[u], kx);
+      for (int off = CPR; off < 32; off <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m_run, off);
+        const float lo2 = __shfl_xor_sync(0xffffffffu, l_run, off);
+        const float mn = fmaxf(m_run, mo);
+        const float sa = m_run == -INFINITY ? 0.f : expf(m_run - mn);
+        const float sb = mo == -INFINITY ? 0.f : expf(mo - mn);
 #pragma unroll
-        for (int i = 0; i < EPC; ++i) s = fmaf(kx[i], qs[i], s);
-      }
-#pragma unroll
-      for (int off = CPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      if (ok[u]) {
-        s *= a.t.inv_sqrt_d;
-        const float mn = fmaxf(m_run, s);
-        const float sc = expf(m_run - mn);
-        const float pk = expf(s - mn);
-        l_run = l_run * sc + pk;
-        float vx[EPC];
-        unpack16<T>(vv[u], vx);
-#pragma unroll
-        for (int i = 0; i < EPC; ++i) o[i] = fmaf(pk, vx[i], o[i] * sc);
+        for (int i = 0; i < EPC; ++i) {
+          const float oo = __shfl_xor_sync(0xffffffffu, o[i], off);
+          o[i] = o[i] * sa + oo * sb;
+        }
+        l_run = l_run * sa + lo2 * sb;
         m_run = mn;
       }
-    }
-  }
-  // lane-group partials -> shared memory
-  const int grp = wid * KPW + sub;
-  if (cl == 0) {
-    sm.att.grp[grp][0] = m_run;
-    sm.att.grp[grp][1] = l_run;
-  }
-#pragma unroll
-  for (int i = 0; i < EPC; ++i) sm.att.grp[grp][2 + cl * EPC + i] = o[i];
-  __syncthreads();
-  // CTA partial: combine the groups in a fixed order; send it to CTA 0
-  float* dst = cluster.map_shared_rank(&sm.part[0][0], 0) + r * (2 + 128);
-  {
-    float M = -INFINITY;
-    for (int g = 0; g < kDecWarps * KPW; ++g) M = fmaxf(M, sm.att.grp[g][0]);
-    for (int e = tid; e < D + 1; e += kDecThreads) {
-      float acc = 0.f;
-      for (int g = 0; g < kDecWarps * KPW; ++g) {
-        const float mg = sm.att.grp[g][0];
-        if (mg == -INFINITY) continue;
-        const float sc = expf(mg - M);
-        acc = fmaf(sc, e == 0 ? sm.att.grp[g][1] : sm.att.grp[g][1 + e], acc);
+      float* P = sm.part[it - c0];
+      if (lane == 0) {
+        P[0] = m_run;
+        P[1] = l_run;
       }
-      dst[1 + e] = acc;   // dst[1] = l, dst[2 + i] = o[i]
+      if (lane < CPR) {
+#pragma unroll
+        for (int i = 0; i < EPC; ++i) P[2 + cl * EPC + i] = o[i];
+      }
     }
-    if (tid == 0) dst[0] = M;
   }
-  cluster.sync();
-  if (r == 0) {
+  __syncthreads();
+  // merge this CTA's chunks per head segment; one partial per segment, stored at
+  // the global slot of the segment's first chunk
+  for (long long seg = c0 + wid; seg < c1; seg += kDecWarps) {
+    const int h = owner_of(sm, nh, seg);
+    if (seg != c0 && seg != sm.pref[h]) continue;  // not the first chunk of a segment
+    const long long send = min64(c1, sm.pref[h + 1]);
     float M = -INFINITY;
-    for (int c = 0; c < CS; ++c) M = fmaxf(M, sm.part[c][0]);
-    float lsum = 0.f;
-    for (int c = 0; c < CS; ++c)
-      if (sm.part[c][0] != -INFINITY) lsum = fmaf(expf(sm.part[c][0] - M), sm.part[c][1], lsum);
-    const float inv = 1.f / lsum;
-    float* out = a.O + (size_t(bb) * a.t.hq + h) * D;
-    for (int e = tid; e < D; e += kDecThreads) {
-      float acc = 0.f;
-      for (int c = 0; c < CS; ++c)
-        if (sm.part[c][0] != -INFINITY) acc = fmaf(expf(sm.part[c][0] - M), sm.part[c][2 + e], acc);
-      out[e] = acc * inv;
+    for (long long j = seg; j < send; ++j) M = fmaxf(M, sm.part[j - c0][0]);
+    float L = 0.f;
+    float acc[(D + 31) / 32];
+#pragma unroll
+    for (int q = 0; q < (D + 31) / 32; ++q) acc[q] = 0.f;
+    for (long long j = seg; j < send; ++j) {
+      const float mj = sm.part[j - c0][0];
+      if (mj == -INFINITY) continue;
+      const float sc = expf(mj - M);
+      L = fmaf(sc, sm.part[j - c0][1], L);
+#pragma unroll
+      for (int q = 0; q < (D + 31) / 32; ++q)
+        if (q * 32 + lane < D) acc[q] = fmaf(sc, sm.part[j - c0][2 + q * 32 + lane], acc[q]);
+    }
+    float* G = a.attn_part + size_t(seg) * (2 + D);
+    if (lane == 0) {
+      G[0] = M;
+      G[1] = L;
+    }
+#pragma unroll
+    for (int q = 0; q < (D + 31) / 32; ++q)
+      if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
+  }
+  if (grid_sync(a, sm)) return;
+
+  // ---------------- combine (one CTA per head)
+  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+    const long long p0 = sm.pref[h], p1 = sm.pref[h + 1];
+    // partial slots: one per CTA whose chunk range meets [p0, p1), at max(p0, range start)
+    float M = -INFINITY;
+    auto range_start = [&](long long c) { return (c * total_items) / (long long)gridDim.x; };
+    long long cfirst = (p0 * gridDim.x) / max64(total_items, 1);
+    while (cfirst > 0 && range_start(cfirst) > p0) --cfirst;
+    while (cfirst + 1 < gridDim.x && range_start(cfirst + 1) <= p0) ++cfirst;
+    for (long long c = cfirst + tid; c < gridDim.x; c += kDecThreads) {
+      const long long cs = max64(p0, range_start(c));
+      if (cs >= p1) break;
+      if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
+      M = fmaxf(M, __ldcg(a.attn_part + size_t(cs) * (2 + D)));
+    }
+    // block max
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) sm.red32[wid] = __float_as_uint(M);
+    __syncthreads();
+    M = -INFINITY;
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, __uint_as_float(sm.red32[w]));
+    __syncthreads();
+    float L = 0.f, acc = 0.f;
+    const int e = tid % D, part = tid / D;  // NP threads per output element
+    constexpr int NP = kDecThreads / D;
+    float Lp = 0.f;
+    for (long long c = cfirst + part; c < gridDim.x; c += NP) {
+      const long long cs = max64(p0, range_start(c));
+      if (cs >= p1) break;
+      if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
+      const float* G = a.attn_part + size_t(cs) * (2 + D);
+      const float mg = __ldcg(G);
+      if (mg == -INFINITY) continue;
+      const float sc = expf(mg - M);
+      Lp = fmaf(sc, __ldcg(G + 1), Lp);
+      acc = fmaf(sc, __ldcg(G + 2 + e), acc);
+    }
+    float* red = reinterpret_cast<float*>(sm.hist);  // [NP][D] + [NP]
+    red[part * D + e] = acc;
+    if (e == 0) red[NP * D + part] = Lp;
+    __syncthreads();
+    if (part == 0) {
+      for (int q = 1; q < NP; ++q) acc += red[q * D + e];
+      for (int q = 0; q < NP; ++q) L += red[NP * D + q];
+      a.O[size_t(h) * D + e] = acc / L;
     }
     if (tid == 0) {
-      if (a.kept_cnt) a.kept_cnt[bb * a.t.hq + h] = int32_t(leafbase);
+      long long nl = 0, scored = 0;
+      int l0 = 0, steps = 0;
+      if (a.n_steps > 0) {
+        nl = __ldcg(&hstate(h)->n_leaf);
+        l0 = __ldcg(&hstate(h)->leaf0);
+        scored = __ldcg(&hstate(h)->scored);
+        steps = __ldcg(&hstate(h)->steps);
+      }
+      if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
       if (a.stats) {
-        int64_t* st = a.stats + (size_t(bb) * a.t.hq + h) * ZHA_STAT_COUNT;
+        int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
         st[ZHA_STAT_NODES_SCORED] = scored;
-        st[ZHA_STAT_LEAVES_KEPT] = leafbase;
-        st[ZHA_STAT_KEYS] = leafbase * b + ((n1 > 0 && !leaf0) ? 1 : 0) + (a.n_tokens - n1 * b);
-        st[ZHA_STAT_STEPS] = steps_taken;
+        st[ZHA_STAT_LEAVES_KEPT] = nl;
+        st[ZHA_STAT_KEYS] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
+        st[ZHA_STAT_STEPS] = steps;
       }
     }
+    __syncthreads();
   }
 }
 
 // ------------------------------------------------------------------ host launcher
 template <typename T, int D>
-static cudaError_t launch_decode_t(const DecodeArgs& a, int B, int cs, cudaStream_t st) {
-  auto kern = decode_kernel<T, D>;
-  const size_t smem = sizeof(DecSmem);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(cs), unsigned(a.t.hq), unsigned(B));
-  cfg.blockDim = dim3(kDecThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(cs);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  count_launches(1);
-  return cudaLaunchKernelEx(&cfg, kern, a);
-}
-
-// Largest usable cluster size <= want (a power of two) for this kernel.
-template <typename T, int D>
-static int usable_cluster_t(int want) {
+static int grid_size_t() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
   auto kern = decode_kernel<T, D>;
   const size_t smem = sizeof(DecSmem);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  for (int cs = want; cs >= 1; cs >>= 1) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(cs), 1, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(cs);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess && nclusters > 0) return cs;
+  int per_sm = 0, dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) != cudaSuccess) {
     cudaGetLastError();
+    return 0;
   }
-  return 0;
+  cached = per_sm * sms;
+  return cached;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, int dtype, int B, int cs, cudaStream_t st) {
+template <typename T, int D>
+static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
+  auto kern = decode_kernel<T, D>;
+  int grid = grid_size_t<T, D>();
+  if (grid < 1) return cudaErrorLaunchOutOfResources;
+  if (grid > kMaxDecodeGrid) grid = kMaxDecodeGrid;  // the scratch's attend partials are sized for this
+  DecodeArgs args = a;
+  void* params[] = {&args};
+  count_launches(1);
+  return cudaLaunchCooperativeKernel((const void*)kern, dim3(unsigned(grid)), dim3(kDecThreads), params,
+                                     sizeof(DecSmem), st);
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
   if (dtype == ZHA_BF16)
-    return a.t.d == 128 ? launch_decode_t<__nv_bfloat16, 128>(a, B, cs, st)
-                        : launch_decode_t<__nv_bfloat16, 64>(a, B, cs, st);
-  return a.t.d == 128 ? launch_decode_t<float, 128>(a, B, cs, st) : launch_decode_t<float, 64>(a, B, cs, st);
-}
-
-int usable_cluster(int dtype, int d, int want) {
-  if (dtype == ZHA_BF16) return d == 128 ? usable_cluster_t<__nv_bfloat16, 128>(want) : usable_cluster_t<__nv_bfloat16, 64>(want);
-  return d == 128 ? usable_cluster_t<float, 128>(want) : usable_cluster_t<float, 64>(want);
+    return a.t.d == 128 ? launch_decode_t<__nv_bfloat16, 128>(a, st) : launch_decode_t<__nv_bfloat16, 64>(a, st);
+  return a.t.d == 128 ? launch_decode_t<float, 128>(a, st) : launch_decode_t<float, 64>(a, st);
 }
 
 size_t decode_smem_bytes() { return sizeof(DecSmem); }
+size_t decode_head_state_bytes() { return sizeof(HeadState); }
+int decode_max_heads() { return kMaxHeads; }
+int decode_items_per_cta() { return kItemsPerCta; }
 
 }  // namespace zha

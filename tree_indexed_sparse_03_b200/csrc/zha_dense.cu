@@ -4,8 +4,8 @@
 // Split-KV flash decode.  The key range of each (sequence, KV head) is split
 // into `splits` contiguous ranges, one CTA each; a CTA keeps an online softmax
 // (running max, running sum, running output) per query head and writes one
-// partial per head.  The last CTA of a (sequence, KV head) to finish (an
-// atomic counter, no waiting) combines the partials and resets the counter.
+// partial per head.  A second kernel (one CTA per query head and sequence)
+// combines the partials.
 //
 // bf16 path: one CTA serves the whole GQA group (<= 8 query heads) so every
 // K/V byte is read once for all of them.  Per 16-key tile a warp computes
@@ -49,45 +49,47 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
   return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
 }
 
-// Combine the split partials of `nheads` query heads (the caller is the last CTA).
+// Combine the split partials of one query head: one CTA per (head, sequence).
+// o = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s with M = max_s m_s.
 template <int D>
-__device__ void combine_partials(const DenseArgs& a, int bb, int h0, int nheads) {
-  for (int hh = 0; hh < nheads; ++hh) {
-    const int h = h0 + hh;
-    const float* P = a.part + (size_t(bb) * a.hq + h) * a.splits * (D + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(P + size_t(s) * (D + 2)));
-    float l = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
-      const float ms = __ldcg(P + size_t(s) * (D + 2));
-      if (ms != -INFINITY) l = fmaf(expf(ms - M), __ldcg(P + size_t(s) * (D + 2) + 1), l);
-    }
-    const float inv = 1.f / l;
-    for (int e = threadIdx.x; e < D; e += blockDim.x) {
-      float acc = 0.f;
-      for (int s = 0; s < a.splits; ++s) {
-        const float ms = __ldcg(P + size_t(s) * (D + 2));
-        if (ms != -INFINITY) acc = fmaf(expf(ms - M), __ldcg(P + size_t(s) * (D + 2) + 2 + e), acc);
-      }
-      a.O[(size_t(bb) * a.hq + h) * D + e] = acc * inv;
-    }
-  }
-}
-
-// Signal completion of this CTA's partials; the last CTA of the group combines.
-template <int D>
-__device__ void finish_split(const DenseArgs& a, int bb, int counter_idx, int h0, int nheads, int* flag) {
-  __threadfence();
+__global__ void __launch_bounds__(256) dense_combine_kernel(DenseArgs a) {
+  constexpr int NP = 256 / D;  // threads per output element
+  const int h = blockIdx.x, bb = blockIdx.y, tid = threadIdx.x;
+  const float* P = a.part + (size_t(bb) * a.hq + h) * a.splits * (D + 2);
+  extern __shared__ float csm[];  // scale[splits], then red[NP][D]
+  float* scale = csm;
+  float* red = csm + a.splits;
+  __shared__ float wred[8];
+  float m = -INFINITY;
+  for (int s = tid; s < a.splits; s += blockDim.x) m = fmaxf(m, __ldcg(P + size_t(s) * (D + 2)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((tid & 31) == 0) wred[tid >> 5] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.counters + counter_idx, 1);
-    *flag = (prev == a.splits - 1);
-  }
+  float M = -INFINITY;
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, wred[w]);
   __syncthreads();
-  if (*flag) {
-    __threadfence();
-    combine_partials<D>(a, bb, h0, nheads);
-    if (threadIdx.x == 0) a.counters[counter_idx] = 0;
+  float l = 0.f;
+  for (int s = tid; s < a.splits; s += blockDim.x) {
+    const float ms = __ldcg(P + size_t(s) * (D + 2));
+    const float sc = ms == -INFINITY ? 0.f : expf(ms - M);
+    scale[s] = sc;
+    l = fmaf(sc, __ldcg(P + size_t(s) * (D + 2) + 1), l);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+  if ((tid & 31) == 0) wred[tid >> 5] = l;
+  __syncthreads();
+  float L = 0.f;
+  for (int w = 0; w < 8; ++w) L += wred[w];
+  const int e = tid % D, part = tid / D;
+  float acc = 0.f;
+  for (int s = part; s < a.splits; s += NP) acc = fmaf(scale[s], __ldcg(P + size_t(s) * (D + 2) + 2 + e), acc);
+  red[part * D + e] = acc;
+  __syncthreads();
+  if (part == 0) {
+    for (int q = 1; q < NP; ++q) acc += red[q * D + e];
+    a.O[(size_t(bb) * a.hq + h) * D + e] = acc / L;
   }
 }
 
@@ -246,8 +248,6 @@ __global__ void __launch_bounds__(kDenseThreads) dense_mma_kernel(DenseArgs a) {
     }
     a.part[((size_t(bb) * a.hq + kvh * a.group + hh) * a.splits + split) * (D + 2) + e] = val;
   }
-  __shared__ int flag;
-  finish_split<D>(a, bb, bb * a.hkv + kvh, kvh * a.group, a.group, &flag);
 }
 
 // ------------------------------------------------------------------ CUDA-core path (fp32, any group)
@@ -315,13 +315,11 @@ __global__ void __launch_bounds__(256) dense_scalar_kernel(DenseArgs a) {
     }
     a.part[((size_t(bb) * a.hq + h) * a.splits + split) * (D + 2) + e] = val;
   }
-  __shared__ int flag;
-  finish_split<D>(a, bb, bb * a.hq + h, h, 1, &flag);
 }
 
 // ------------------------------------------------------------------ host side
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per) {
-  const int target = 148 * 4;
+  const int target = 148 * 4;  // four CTAs per SM
   int64_t s = (target + int64_t(B) * hkv - 1) / (int64_t(B) * hkv);
   const int64_t max_s = (n + 63) / 64;
   if (s > max_s) s = max_s;
@@ -338,7 +336,7 @@ bool dense_uses_mma(int dtype, int group) { return dtype == ZHA_BF16 && group <=
 
 cudaError_t launch_dense(const DenseArgs& a0, int dtype, int d, int B, cudaStream_t st) {
   DenseArgs a = a0;
-  count_launches(1);
+  count_launches(2);
   if (dense_uses_mma(dtype, a.group)) {
     dim3 grid(unsigned(a.splits), unsigned(a.hkv), unsigned(B));
     if (d == 128) dense_mma_kernel<128><<<grid, kDenseThreads, 0, st>>>(a);
@@ -353,6 +351,12 @@ cudaError_t launch_dense(const DenseArgs& a0, int dtype, int d, int B, cudaStrea
       else dense_scalar_kernel<float, 64><<<grid, 256, 0, st>>>(a);
     }
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t sm = (size_t(a.splits) + 256) * sizeof(float);
+  dim3 cgrid(unsigned(a.hq), unsigned(B));
+  if (d == 128) dense_combine_kernel<128><<<cgrid, 256, sm, st>>>(a);
+  else dense_combine_kernel<64><<<cgrid, 256, sm, st>>>(a);
   return cudaGetLastError();
 }
 
