@@ -355,7 +355,7 @@ def run_zha(args, world, rank, local):
     # dense decode at the same context length (the comparator)
     dense = z.DenseDecoder(cfg, w.batch, tree.size, device=dev)
     dense_ms = []
-    for i in range(args.dense_steps + 3):
+    for i in range(args.dense_steps + 3 if args.dense_steps > 0 else 0):
         flush.zero_()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -395,9 +395,9 @@ def run_zha(args, world, rank, local):
         "p90_us": round(float(np.percentile(step_ms, 90)) * 1000, 3),
         "decode_us": round(dec_mean * 1000, 3),
         "append_us": round(statistics.mean(app_ms) * 1000, 3),
-        "dense_us": round(statistics.mean(dense_ms) * 1000, 3),
-        "speedup_vs_dense": round(statistics.mean(dense_ms) / step_ms_mean, 3),
-        "dense_gbs": round(dense_bytes / (statistics.mean(dense_ms) * 1e-3) / 1e9, 1),
+        "dense_us": round(statistics.mean(dense_ms) * 1000, 3) if dense_ms else None,
+        "speedup_vs_dense": round(statistics.mean(dense_ms) / step_ms_mean, 3) if dense_ms else None,
+        "dense_gbs": round(dense_bytes / (statistics.mean(dense_ms) * 1e-3) / 1e9, 1) if dense_ms else None,
         "build_ms": round(build_ms, 3),
         "keys_per_head": round(statistics.mean(keys_ph), 1),
         "keys_frac": round(statistics.mean(keys_ph) / n_final, 6),
@@ -408,8 +408,8 @@ def run_zha(args, world, rank, local):
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_8tbs": round(achieved / 8000.0, 4), "traffic": None},
         "clocks": clk.summary(),
-        "e2e": {"value": round(statistics.mean(e2e_ms) * 1000, 3), "unit": "us", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": ({"value": round(statistics.mean(e2e_ms) * 1000, 3), "unit": "us", "h2d_bytes_per_step": h2d,
+                 "d2h_bytes_per_step": d2h} if e2e_ms else None),
         "gpu_launches": launches,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

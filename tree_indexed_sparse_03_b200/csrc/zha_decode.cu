@@ -454,6 +454,15 @@ __device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm) {
   return sm.fail != 0;
 }
 
+// Phase timestamp (profiling builds pass a buffer of 32 slots per CTA).
+__device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
+  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 32) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.phase_ns[blockIdx.x * 32 + slot] = t;
+  }
+}
+
 // Inclusive prefix of per-head counts into sm.pref[1..nh] (pref[0] = 0); all threads.
 __device__ __forceinline__ long long build_prefix(DecSmem& sm, int nh) {
   // counts are in sm.pref[1..nh]; scan them in place, chunk by chunk
@@ -511,6 +520,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
   };
 
+  stamp(a, 0);
   for (int step = 0; step < a.n_steps; ++step) {
     // ---------------- score (all CTAs)
     for (int i = tid; i < nh; i += kDecThreads) {
@@ -540,7 +550,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       const float e = score_node<T, D>(a.t, kvh, code, qs, lane);
       if (lane == 0) sel(h, step)[pos] = Entry{desc_key(e), code};
     }
+    stamp(a, 1 + 4 * step);
     if (grid_sync(a, sm)) return;
+    stamp(a, 2 + 4 * step);
 
     // ---------------- select (one CTA per head)
     for (int h = blockIdx.x; h < nh; h += gridDim.x) {
@@ -623,7 +635,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       }
       __syncthreads();
     }
+    stamp(a, 3 + 4 * step);
     if (grid_sync(a, sm)) return;
+    stamp(a, 4 + 4 * step);
   }
 
   // ---------------- attend (all CTAs)
@@ -765,6 +779,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
+  stamp(a, 26);
   // merge this CTA's chunks per head segment; one partial per segment, stored at
   // the global slot of the segment's first chunk
   for (long long seg = c0 + wid; seg < c1; seg += kDecWarps) {
@@ -795,7 +810,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     for (int q = 0; q < (D + 31) / 32; ++q)
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
   }
+  stamp(a, 27);
   if (grid_sync(a, sm)) return;
+  stamp(a, 28);
 
   // ---------------- combine (one CTA per head)
   for (int h = blockIdx.x; h < nh; h += gridDim.x) {
@@ -864,6 +881,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     }
     __syncthreads();
   }
+  stamp(a, 29);
 }
 
 // ------------------------------------------------------------------ host launcher
