@@ -154,7 +154,9 @@ ZHA_API int64_t zha_tree_size(const zha_tree* tree);
  *              of every node the head scored, step by step; ZHA_STAT_NODES_SCORED
  *              gives how many (entries past scored_cap are dropped).  Used to
  *              count the bytes a decode must read; leave NULL on the hot path.
- * Requires 1 <= B <= max_batch and at least one cached token.
+ * Requires 1 <= B <= max_batch and at least one cached token.  The call
+ * launches one cooperative kernel (every SM takes part); calls on one tree
+ * share its scratch and must be issued in order on one stream.
  */
 ZHA_API int zha_decode(const zha_tree* tree, const void* Q, float* O, int32_t B, int32_t* kept,
                int32_t* kept_cnt, int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream);

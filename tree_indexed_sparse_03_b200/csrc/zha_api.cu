@@ -21,6 +21,8 @@ size_t decode_smem_bytes();
 size_t decode_head_state_bytes();
 int decode_max_heads();
 int decode_items_per_cta();
+int decode_max_grid();
+int decode_grid(int dtype, int d);
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
 }  // namespace zha
 
@@ -66,7 +68,6 @@ struct Layout {
 
 uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
-constexpr int kMaxDecodeGrid = 256;
 constexpr long long kDefaultSpinLimit = 1ll << 24;  // ~1 s of 40 ns sleeps  // CTAs of the decode launch (one per SM) the scratch is sized for
 
 int elem_size(int dtype) { return dtype == ZHA_BF16 ? 2 : 4; }
@@ -85,7 +86,7 @@ int validate(const zha_config* c) {
   if (c->capacity / c->block >= (int64_t(1) << 27)) return fail(ZHA_ERR_UNSUPPORTED, "capacity / block must be < 2^27");
   if (c->max_batch < 1 || c->max_batch > 65535) return fail(ZHA_ERR_INVALID, "max_batch must be in [1, 65535]");
   if (int64_t(c->max_batch) * c->n_q_heads > decode_max_heads())
-    return fail(ZHA_ERR_UNSUPPORTED, "max_batch * n_q_heads must be <= 2048");
+    return fail(ZHA_ERR_UNSUPPORTED, "max_batch * n_q_heads must be <= 1024");
   // block^levels must fit comfortably in int64
   double span = std::pow(double(c->block), double(c->levels));
   if (span > 4e18) return fail(ZHA_ERR_UNSUPPORTED, "block^levels too large");
@@ -139,9 +140,10 @@ int make_layout(const zha_config* c, Layout* L) {
   L->cap_list = n1cap + 64;
   const uint64_t nheads = uint64_t(c->max_batch) * c->n_q_heads;
   L->part_off = 256;
-  L->part_items = uint64_t(kMaxDecodeGrid) * decode_items_per_cta() + nheads + 64;
+  L->part_items = uint64_t(decode_max_grid()) * decode_items_per_cta() + nheads + 64;
   L->ws_off = align256(L->part_off + L->part_items * (c->d + 2) * 4);
-  L->ws_per_bh = align256(uint64_t(2) * L->cap_sel * 8 + uint64_t(L->cap_sel) * 4 + uint64_t(L->cap_list) * 4 +
+  // step entries (key, code), next candidates (codes), kept leaves, head state
+  L->ws_per_bh = align256(uint64_t(L->cap_sel) * 8 + uint64_t(L->cap_sel) * 4 + uint64_t(L->cap_list) * 4 +
                           decode_head_state_bytes());
   uint64_t s = L->ws_off + L->ws_per_bh * uint64_t(c->max_batch) * c->n_q_heads;
   L->stage_off = s;
@@ -167,6 +169,7 @@ struct zha_tree {
   int64_t n;
   int device;
   long long spin_limit;  // grid-barrier spin bound of the decode kernel
+  unsigned long long bar_count;  // arrivals the decode kernels have made on the grid barrier so far
 };
 
 extern "C" {
@@ -216,6 +219,7 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
   t->scratch = static_cast<char*>(scratch);
   t->n = 0;
   t->spin_limit = kDefaultSpinLimit;
+  t->bar_count = 0;
   if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: force the barrier timeout path
     const long long x = std::atoll(v);
     if (x > 0) t->spin_limit = x;
@@ -265,6 +269,7 @@ int zha_tree_build(zha_tree* t, int64_t n, void* stream) {
   e = launch_tree_update(t->dev, t->cfg.dtype, 0, n, st);
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build");
   t->n = n;
+  t->bar_count = 0;
   return ZHA_OK;
 }
 
@@ -305,7 +310,8 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->n_steps = steps;
   a->ws = t->scratch + t->L.ws_off;
   a->ws_per_bh = t->L.ws_per_bh;
-  a->bar = reinterpret_cast<unsigned int*>(t->scratch + t->L.bar_off);
+  a->bar = reinterpret_cast<unsigned long long*>(t->scratch + t->L.bar_off);
+  a->bar_base = t->bar_count;
   a->attn_part = reinterpret_cast<float*>(t->scratch + t->L.part_off);
   a->spin_limit = t->spin_limit;
 #ifdef ZHA_PHASE_TIMING
@@ -345,8 +351,12 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
   DecodeArgs a;
   fill_decode_args(t, Q, O, kept, kept_cnt, stats, scored, scored_cap, &a);
   a.nheads = B * t->cfg.n_q_heads;
+  const int grid = decode_grid(t->cfg.dtype, t->cfg.d);
+  if (grid < 1) return fail(ZHA_ERR_CUDA, "the decode kernel does not fit on this device");
   cudaError_t e = launch_decode(a, t->cfg.dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "zha_decode");
+  // every CTA arrives once per barrier: two per routing step and one after attention
+  const_cast<zha_tree*>(t)->bar_count += uint64_t(2 * a.n_steps + 1) * uint64_t(grid);
   return ZHA_OK;
 }
 

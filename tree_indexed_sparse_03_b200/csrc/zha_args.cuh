@@ -18,7 +18,8 @@ struct DecodeArgs {
   uint64_t ws_per_bh;
   int64_t cap_sel;              // entries per step buffer (and kept parents)
   int64_t cap_list;             // kept leaves per head
-  unsigned int* bar;            // grid barrier: {count, generation}
+  unsigned long long* bar;      // grid barrier arrival counter (only grows)
+  unsigned long long bar_base;  // its value when this launch starts
   float* attn_part;             // attend partials, (2 + d) floats each
   long long spin_limit;         // grid-barrier spin bound
   int32_t* kept;

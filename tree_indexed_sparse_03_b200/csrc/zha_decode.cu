@@ -17,20 +17,22 @@
 // GPU design.  One persistent cooperative launch per decode call; all query
 // heads of all sequences are routed together so that the whole GPU shares
 // the work of the heads whose routing is diffuse.  Phases are separated by a
-// software grid barrier (bounded spin: on timeout the kernel raises
-// ZHA_ERR_TIMEOUT and returns):
-//   score   (all CTAs) the step's candidates of every head form one list;
-//           each warp scores one node at a time (16-byte loads of its planes,
-//           fp32 dot products) and writes (descending key of e, node code) at
-//           the candidate's canonical position in its head's step buffer;
+// software grid barrier (a monotonic arrival counter; bounded spin: on
+// timeout the kernel raises ZHA_ERR_TIMEOUT and returns):
+//   score   (all CTAs) the step's candidates of every head form one list that
+//           is cut into contiguous per-warp ranges; each warp streams the node
+//           records of its range through a ring of shared-memory slots with
+//           cp.async (several records in flight per warp), computes the
+//           estimates in fp32 and writes (descending key of e, node code) at
+//           the candidate's position in its head's step buffer;
 //   select  (one CTA per head) masses w = exp(e - max e) as 2^-40 fixed-point
 //           integers (exact, order-independent sums); a 1024-bin histogram of
 //           the masses over (max e - e) in 1/32-logit bins, then 1024 sub-bins
 //           of the cut bin, isolate the few entries around the cut, which are
 //           ordered by (e desc, start asc); kept = every entry at or before the
-//           cut.  Kept non-leaf nodes become the next step's parents (their
-//           children, in rank order, are the next candidates); kept leaves are
-//           appended to the head's attend list;
+//           cut.  The children of the kept non-leaf nodes, in rank order, are
+//           written as the next step's candidates; kept leaves are appended to
+//           the head's attend list;
 //   attend  (all CTAs) every head's attended keys (kept blocks, sink, tail)
 //           are cut into chunks; CTAs own contiguous ranges of chunks, warps
 //           run an online softmax per chunk, and each CTA merges its chunks per
@@ -47,12 +49,17 @@ struct Entry {
 
 constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kSelCache = 20480;  // entries of one head cached in shared memory by the select
+constexpr int kUnionBytes = 200 * 1024;            // select cache / score rings / attend partials
+constexpr int kCache8 = kUnionBytes / 8;           // entries cached with their codes
+constexpr int kCache4 = kUnionBytes / 4;           // entries cached as keys only
 constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
-constexpr int kMaxHeads = 2048;   // sequences x query heads per call
-constexpr int kItemsPerCta = 256; // attend chunks a CTA owns at most (plus one per head it touches)
-constexpr int kMaxDecodeGrid = 256;  // CTAs per decode launch the scratch is laid out for
+constexpr int kMaxHeads = 1024;                    // sequences x query heads per call
+constexpr int kItemsPerCta = 256;                  // attend chunks a CTA owns at most (plus one per head)
+constexpr int kMaxDecodeGrid = 256;                // CTAs per decode launch the scratch is laid out for
+constexpr int kPartSlots = kUnionBytes / ((2 + 128) * 4);  // attend partials a CTA can hold
+constexpr int kMaxSlots = 8;                       // score ring slots per warp
+static_assert(kPartSlots >= kItemsPerCta + 32, "attend partial area too small");
 
 struct HeadState {  // per (sequence, query head), written by the head's select CTA
   long long n_cand;   // candidates of the next step
@@ -64,10 +71,7 @@ struct HeadState {  // per (sequence, query head), written by the head's select 
 };
 
 struct __align__(16) DecSmem {
-  union {
-    Entry cache[kSelCache];                 // select: the head's entries
-    float part[kSelCache * 2 / (2 + 128)][2 + 128];  // attend: per-chunk partials of this CTA (kPartSlots)
-  };
+  unsigned char u[kUnionBytes];
   unsigned long long hist[kBins];
   long long pref[kMaxHeads + 1];            // per-head prefix of work items
   unsigned long long cut_key[32];
@@ -75,12 +79,26 @@ struct __align__(16) DecSmem {
   unsigned long long red64[kDecWarps];
   uint32_t red32[kDecWarps * 2];
   unsigned long long bcast64[4];
-  long long bcastll[4];
   int bcast32[8];
   int fail;
 };
-constexpr int kPartSlots = kSelCache * 2 / (2 + 128);  // attend partials a CTA can hold
-static_assert(kPartSlots >= kItemsPerCta + 32, "attend partial area too small");
+
+// The step's entries of one head, read from shared memory when they fit.
+struct SelView {
+  const Entry* g;     // global step buffer
+  const Entry* ce;    // cached entries (mode 1)
+  const uint32_t* ck; // cached keys (mode 2)
+  int mode;           // 0: global, 1: entries cached, 2: keys cached
+  __device__ __forceinline__ uint32_t key(int64_t i) const {
+    if (mode == 1) return ce[i].key;
+    if (mode == 2) return ck[i];
+    return __ldcg(reinterpret_cast<const unsigned int*>(g + i));
+  }
+  __device__ __forceinline__ uint32_t code(int64_t i) const {
+    if (mode == 1) return ce[i].code;
+    return __ldcg(reinterpret_cast<const unsigned int*>(g + i) + 1);
+  }
+};
 
 __device__ __forceinline__ uint32_t root_code(const DecodeArgs& a, int64_t i) {
   const int L = a.t.levels, b = a.t.block;
@@ -222,12 +240,6 @@ __device__ __forceinline__ uint32_t block_min_u32(uint32_t v, uint32_t* red) {
   return m;
 }
 
-__device__ __forceinline__ Entry load_entry(const Entry* E, int64_t i, bool cached, const DecSmem& sm) {
-  if (cached) return sm.cache[i];
-  const uint2 v = __ldcg(reinterpret_cast<const uint2*>(E + i));
-  return Entry{v.x, v.y};
-}
-
 // Distance of an entry below the maximum estimate, in fp32: x = m - e >= 0.
 // Bins over x are monotone in e (fp32 subtraction and power-of-two scaling
 // round monotonically), so every entry of a lower bin precedes every entry of
@@ -276,13 +288,13 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
   return bin;
 }
 
+
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  Every thread returns the same value.
-__device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, int64_t n, bool cached,
-                                         DecSmem& sm) {
+__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, DecSmem& sm) {
   const int tid = threadIdx.x;
   uint32_t kmin = 0xffffffffu;
-  for (int64_t i = tid; i < n; i += kDecThreads) kmin = min(kmin, load_entry(E, i, cached, sm).key);
+  for (int64_t i = tid; i < n; i += kDecThreads) kmin = min(kmin, E.key(i));
   kmin = block_min_u32(kmin, sm.red32);
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
@@ -291,8 +303,8 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
-    const Entry en = load_entry(E, i, cached, sm);
-    atomicAdd(&sm.hist[coarse_bin(entry_gap(m, en.key))], entry_mass(m, en.key));
+    const uint32_t k = E.key(i);
+    atomicAdd(&sm.hist[coarse_bin(entry_gap(m, k))], entry_mass(m, k));
   }
   __syncthreads();
   unsigned long long Z = 0;
@@ -312,9 +324,9 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
-    const Entry en = load_entry(E, i, cached, sm);
-    const float x = entry_gap(m, en.key);
-    if (coarse_bin(x) == cb) atomicAdd(&sm.hist[fine_bin(x, cb)], entry_mass(m, en.key));
+    const uint32_t k = E.key(i);
+    const float x = entry_gap(m, k);
+    if (coarse_bin(x) == cb) atomicAdd(&sm.hist[fine_bin(x, cb)], entry_mass(m, k));
   }
   __syncthreads();
   unsigned long long below2;
@@ -325,13 +337,13 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   if (tid == 0) sm.bcast32[1] = 0;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
-    const Entry en = load_entry(E, i, cached, sm);
-    const float x = entry_gap(m, en.key);
+    const uint32_t k = E.key(i);
+    const float x = entry_gap(m, k);
     if (coarse_bin(x) == cb && fine_bin(x, cb) == fb) {
       const int s = atomicAdd(&sm.bcast32[1], 1);
       if (s < 32) {
-        sm.cut_key[s] = entry_key64(a, en);
-        sm.cut_w[s] = entry_mass(m, en.key);
+        sm.cut_key[s] = entry_key64(a, Entry{k, E.code(i)});
+        sm.cut_w[s] = entry_mass(m, k);
       }
     }
   }
@@ -377,12 +389,12 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
     for (int i = tid; i < 256; i += kDecThreads) sm.hist[i] = 0ull;
     __syncthreads();
     for (int64_t i = tid; i < n; i += kDecThreads) {
-      const Entry en = load_entry(E, i, cached, sm);
-      const float x = entry_gap(m, en.key);
+      const uint32_t k = E.key(i);
+      const float x = entry_gap(m, k);
       if (coarse_bin(x) != cb || fine_bin(x, cb) != fb) continue;
-      const unsigned long long k64 = entry_key64(a, en);
+      const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
-      atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, en.key));
+      atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, k));
     }
     __syncthreads();
     if (tid < 32) {
@@ -422,33 +434,29 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const Entry* E, in
   return prefix;
 }
 
-
-// Software grid barrier over all CTAs of the cooperative launch.  Returns
-// true (for every thread of the CTA) if the wait gave up.
-__device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm) {
+// Grid barrier over all CTAs of the cooperative launch: a 64-bit arrival
+// counter that only grows; barrier k of a launch completes when it reaches
+// base + k * gridDim.x (the host tracks the base).  Returns true for every
+// thread of the CTA if the wait gave up.
+__device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm, unsigned long long& target) {
+  target += gridDim.x;
   __syncthreads();
   if (threadIdx.x == 0) {
     sm.fail = 0;
-    volatile unsigned int* gen = a.bar + 1;
-    const unsigned int g = *gen;
     __threadfence();
-    const unsigned int arrived = atomicAdd(a.bar, 1u);
-    if (arrived == gridDim.x - 1) {
-      atomicExch(a.bar, 0u);
-      __threadfence();
-      atomicAdd(a.bar + 1, 1u);
-    } else {
-      long long it = 0;
-      while (*gen == g) {
-        if (++it > a.spin_limit) {
-          sm.fail = 1;
-          raise_status(a.t.status, ZHA_ERR_TIMEOUT);
-          break;
-        }
-        __nanosleep(40);
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(a.bar) : "memory");
+    long long it = 0;
+    while (true) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.bar) : "memory");
+      if (v >= target) break;
+      if (++it > a.spin_limit) {
+        sm.fail = 1;
+        raise_status(a.t.status, ZHA_ERR_TIMEOUT);
+        break;
       }
+      __nanosleep(20);
     }
-    __threadfence();
   }
   __syncthreads();
   return sm.fail != 0;
@@ -463,9 +471,8 @@ __device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
   }
 }
 
-// Inclusive prefix of per-head counts into sm.pref[1..nh] (pref[0] = 0); all threads.
+// Inclusive prefix of per-head counts held in sm.pref[1..nh] (pref[0] = 0); returns the total.
 __device__ __forceinline__ long long build_prefix(DecSmem& sm, int nh) {
-  // counts are in sm.pref[1..nh]; scan them in place, chunk by chunk
   long long carry = 0;
   for (int base = 0; base < nh; base += kDecThreads) {
     const int i = base + threadIdx.x;
@@ -496,6 +503,55 @@ __device__ __forceinline__ bool valid_code(const DecodeArgs& a, uint32_t code) {
   return l >= 1 && l <= a.t.levels && int64_t(code_index(code)) < a.nl[l];
 }
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most `pending` of this thread's newest groups are still in flight
+__device__ __forceinline__ void cp_async_wait(int pending) {
+  switch (pending) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
+}
+
+// Estimate of a node whose record sits in shared memory (whole warp; the
+// lane's q slice covers elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR).
+template <typename T, int D>
+__device__ __forceinline__ float score_record_smem(const unsigned char* rec, int R, float inv_sqrt_d,
+                                                   const float* qs, int lane) {
+  constexpr int EPC = 16 / sizeof(T);
+  constexpr int CPR = D * sizeof(T) / 16;
+  constexpr int RPI = 32 / CPR;
+  const float* bias = reinterpret_cast<const float*>(rec + size_t(R) * D * sizeof(T));
+  const int sub = lane / CPR, cl = lane % CPR;
+  float best = -INFINITY;
+  for (int j0 = 0; j0 < R; j0 += RPI) {
+    const int j = j0 + sub;
+    float part = 0.f;
+    if (j < R) {
+      const uint4 v = *reinterpret_cast<const uint4*>(rec + (size_t(j) * CPR + cl) * 16);
+      float x[EPC];
+      unpack16<T>(v, x);
+#pragma unroll
+      for (int i = 0; i < EPC; ++i) part = fmaf(x[i], qs[i], part);
+    }
+#pragma unroll
+    for (int off = CPR / 2; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (j < R) best = fmaxf(best, fmaf(part, inv_sqrt_d, bias[j]));
+  }
+#pragma unroll
+  for (int off = 16; off >= CPR; off >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+  return best;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   constexpr int EPC = 16 / sizeof(T);
@@ -506,19 +562,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int nh = a.nheads;
   const int b = a.t.block;
+  const int R = a.t.refs;
   const long long gwarp = (long long)blockIdx.x * kDecWarps + wid;
   const long long nwarps = (long long)gridDim.x * kDecWarps;
+  unsigned long long bar_target = a.bar_base;
   auto ws = [&](int h) { return a.ws + uint64_t(h) * a.ws_per_bh; };
-  auto sel = [&](int h, int step) { return reinterpret_cast<Entry*>(ws(h)) + (step & 1) * a.cap_sel; };
-  auto par = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 2 * a.cap_sel * sizeof(Entry)); };
-  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 2 * a.cap_sel * sizeof(Entry) + a.cap_sel * 4); };
+  auto sel = [&](int h) { return reinterpret_cast<Entry*>(ws(h)); };
+  auto cand = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + a.cap_sel * sizeof(Entry)); };
+  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + a.cap_sel * (sizeof(Entry) + 4)); };
   auto hstate = [&](int h) {
-    return reinterpret_cast<HeadState*>(ws(h) + 2 * a.cap_sel * sizeof(Entry) + a.cap_sel * 4 + a.cap_list * 4);
+    return reinterpret_cast<HeadState*>(ws(h) + a.cap_sel * (sizeof(Entry) + 4) + a.cap_list * 4);
   };
   auto q_slice = [&](int h, float* qs) {
     const T* q = static_cast<const T*>(a.Q) + size_t(h) * D + (lane % CPR) * EPC;
     unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
   };
+  const int rec_bytes = int(a.t.rec_bytes);
+  const int rec_chunks = rec_bytes / 16;
+  const int nslot = max(1, min(kMaxSlots, (kUnionBytes / kDecWarps) / rec_bytes));
+  unsigned char* ring = sm.u + size_t(wid) * nslot * rec_bytes;
 
   stamp(a, 0);
   for (int step = 0; step < a.n_steps; ++step) {
@@ -530,28 +592,67 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     }
     __syncthreads();
     const long long total = build_prefix(sm, nh);
-    for (long long it = gwarp; it < total; it += nwarps) {
-      const int h = owner_of(sm, nh, it);
-      const long long pos = it - sm.pref[h];
-      uint32_t code;
-      if (step == 0) {
-        code = root_code(a, pos);
-      } else {
-        const uint32_t pc = __ldcg(par(h) + pos / b);
-        code = node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(pos % b));
-        if (code_level(pc) < 2 || !valid_code(a, pc) || !valid_code(a, code)) {
-          if (lane == 0) raise_status(a.t.status, ZHA_ERR_CAPACITY);
-          continue;
+    {
+      const long long i0 = gwarp * total / nwarps, i1 = (gwarp + 1) * total / nwarps;
+      const long long cnt = i1 - i0;
+      // codes of the next 32 items, one per lane
+      uint32_t code_reg = 0;
+      int head_reg = 0;
+      auto fetch_codes = [&](long long k0) {
+        const long long it = i0 + k0 + lane;
+        code_reg = 0;
+        head_reg = 0;
+        if (k0 + lane < cnt) {
+          const int h = owner_of(sm, nh, it);
+          const long long pos = it - sm.pref[h];
+          uint32_t code = step == 0 ? root_code(a, pos) : __ldcg(cand(h) + pos);
+          if (!valid_code(a, code)) {
+            raise_status(a.t.status, ZHA_ERR_CAPACITY);
+            code = 0;  // marks an item to skip
+          }
+          code_reg = code;
+          head_reg = h;
         }
-      }
+      };
+      long long issued = 0, done = 0;
+      int qhead = -1;
       float qs[EPC];
-      q_slice(h, qs);
-      const int kvh = (h % a.t.hq) / a.t.group;
-      const float e = score_node<T, D>(a.t, kvh, code, qs, lane);
-      if (lane == 0) sel(h, step)[pos] = Entry{desc_key(e), code};
+      if (cnt > 0) fetch_codes(0);
+      while (done < cnt) {
+        // keep up to nslot records in flight
+        while (issued < cnt && issued - done < nslot && (issued >> 5) == (done >> 5)) {
+          const uint32_t code = __shfl_sync(0xffffffffu, code_reg, int(issued & 31));
+          const int h = __shfl_sync(0xffffffffu, head_reg, int(issued & 31));
+          unsigned char* slot = ring + size_t(issued % nslot) * rec_bytes;
+          if (code != 0) {
+            const int kvh = (h % a.t.hq) / a.t.group;
+            const unsigned char* src =
+                reinterpret_cast<const unsigned char*>(a.t.rec(code_level(code), kvh, code_index(code)));
+            for (int c = lane; c < rec_chunks; c += 32) cp_async16(slot + c * 16, src + c * 16);
+          }
+          cp_async_commit();
+          ++issued;
+        }
+        cp_async_wait(int(issued - done - 1));
+        __syncwarp();
+        const uint32_t code = __shfl_sync(0xffffffffu, code_reg, int(done & 31));
+        const int h = __shfl_sync(0xffffffffu, head_reg, int(done & 31));
+        if (code != 0) {
+          if (h != qhead) {
+            q_slice(h, qs);
+            qhead = h;
+          }
+          const float e = score_record_smem<T, D>(ring + size_t(done % nslot) * rec_bytes, R, a.t.inv_sqrt_d, qs,
+                                                  lane);
+          if (lane == 0) sel(h)[i0 + done - sm.pref[h]] = Entry{desc_key(e), code};
+        }
+        __syncwarp();
+        ++done;
+        if ((done & 31) == 0 && done < cnt) fetch_codes(done);
+      }
     }
     stamp(a, 1 + 4 * step);
-    if (grid_sync(a, sm)) return;
+    if (grid_sync(a, sm, bar_target)) return;
     stamp(a, 2 + 4 * step);
 
     // ---------------- select (one CTA per head)
@@ -576,30 +677,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         }
         continue;
       }
-      const Entry* S = sel(h, step);
-      const bool cached = n <= kSelCache;
+      const Entry* S = sel(h);
+      SelView E;
+      E.g = S;
+      E.ce = reinterpret_cast<const Entry*>(sm.u);
+      E.ck = reinterpret_cast<const uint32_t*>(sm.u);
+      E.mode = n <= kCache8 ? 1 : (n <= kCache4 ? 2 : 0);
       __syncthreads();
-      if (cached) {
+      if (E.mode == 1) {
+        Entry* ce = reinterpret_cast<Entry*>(sm.u);
         for (long long i = tid; i < n; i += kDecThreads) {
           const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
-          sm.cache[i] = Entry{v.x, v.y};
+          ce[i] = Entry{v.x, v.y};
         }
-        __syncthreads();
+      } else if (E.mode == 2) {
+        uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
+        for (long long i = tid; i < n; i += kDecThreads) ck[i] = __ldcg(reinterpret_cast<const unsigned int*>(S + i));
       }
+      __syncthreads();
       if (a.scored) {
         int32_t* out = a.scored + size_t(h) * a.scored_cap;
         for (long long i = tid; i < n; i += kDecThreads)
-          if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(load_entry(S, i, cached, sm).code);
+          if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
       }
-      const unsigned long long cut = select_cut(a, S, n, cached, sm);
-      // ranks of the kept entries in canonical order
+      const unsigned long long cut = select_cut(a, E, n, sm);
+      const uint32_t cut32 = uint32_t(cut >> 32);
+      // ranks of the kept entries in canonical order (contiguous range per thread)
       const long long per_thr = (n + kDecThreads - 1) / kDecThreads;
       const long long lo = min64(n, tid * per_thr), hi = min64(n, lo + per_thr);
+      auto kept_entry = [&](long long i, uint32_t& code) {
+        const uint32_t k = E.key(i);
+        if (k > cut32) return false;
+        code = E.code(i);
+        return k < cut32 || entry_key64(a, Entry{k, code}) <= cut;
+      };
       uint32_t nleaf = 0, npar = 0;
       for (long long i = lo; i < hi; ++i) {
-        const Entry en = load_entry(S, i, cached, sm);
-        if (entry_key64(a, en) <= cut) {
-          if (code_level(en.code) == 1) ++nleaf; else ++npar;
+        uint32_t code;
+        if (kept_entry(i, code)) {
+          if (code_level(code) == 1) ++nleaf; else ++npar;
         }
       }
       uint32_t tot_leaf, tot_par;
@@ -607,17 +723,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       uint32_t par_rank = block_scan_u32(npar, sm.red32, &tot_par);
       int my_leaf0 = 0;
       for (long long i = lo; i < hi; ++i) {
-        const Entry en = load_entry(S, i, cached, sm);
-        if (entry_key64(a, en) > cut) continue;
-        if (code_level(en.code) == 1) {
+        uint32_t code;
+        if (!kept_entry(i, code)) continue;
+        if (code_level(code) == 1) {
           const long long g = n_leaf0 + leaf_rank++;
-          if (code_index(en.code) == 0) my_leaf0 = 1;
-          if (g < a.cap_list) leaves(h)[g] = code_index(en.code);
+          if (code_index(code) == 0) my_leaf0 = 1;
+          if (g < a.cap_list) leaves(h)[g] = code_index(code);
           else raise_status(a.t.status, ZHA_ERR_CAPACITY);
-          if (a.kept && g < a.kept_stride) a.kept[size_t(h) * a.kept_stride + g] = int32_t(code_index(en.code));
+          if (a.kept && g < a.kept_stride) a.kept[size_t(h) * a.kept_stride + g] = int32_t(code_index(code));
         } else {
-          const uint32_t pr = par_rank++;
-          if (pr < a.cap_sel) par(h)[pr] = en.code;
+          const long long pr = par_rank++;
+          const uint32_t cl = code_level(code) - 1, ci = code_index(code) * uint32_t(b);
+          if ((pr + 1) * b <= a.cap_sel) {
+            for (int c = 0; c < b; ++c) cand(h)[pr * b + c] = node_code(cl, ci + uint32_t(c));
+          }
         }
       }
       my_leaf0 = __syncthreads_or(my_leaf0);
@@ -636,67 +755,65 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       __syncthreads();
     }
     stamp(a, 3 + 4 * step);
-    if (grid_sync(a, sm)) return;
+    if (grid_sync(a, sm, bar_target)) return;
     stamp(a, 4 + 4 * step);
   }
 
   // ---------------- attend (all CTAs)
   const long long n1 = a.nl[1];
   const long long tail = a.n_tokens - n1 * b;
-  // keys per head: kept blocks x b + sink (when block 0 is not kept) + tail
-  for (int i = tid; i < nh; i += kDecThreads) {
-    long long nl = 0;
+  auto head_keys = [&](int h, long long& nl, bool& sink) {
+    nl = 0;
     int l0 = 0;
     if (a.n_steps > 0) {
-      nl = min64(max64(__ldcg(&hstate(i)->n_leaf), 0), a.cap_list);
-      l0 = __ldcg(&hstate(i)->leaf0);
+      nl = min64(max64(__ldcg(&hstate(h)->n_leaf), 0), a.cap_list);
+      l0 = __ldcg(&hstate(h)->leaf0);
     }
-    sm.pref[1 + i] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
+    sink = (n1 > 0) && !l0;
+    return nl * b + (sink ? 1 : 0) + tail;
+  };
+  for (int i = tid; i < nh; i += kDecThreads) {
+    long long nl;
+    bool sink;
+    sm.pref[1 + i] = head_keys(i, nl, sink);
   }
   __syncthreads();
   const long long total_keys = build_prefix(sm, nh);
   // chunk size: at least 32 keys, large enough that a CTA owns <= kItemsPerCta chunks (+1 per head)
   long long chunk = (total_keys + (long long)gridDim.x * kItemsPerCta - 1) / ((long long)gridDim.x * kItemsPerCta);
   chunk = max64(32, chunk);
-  // items per head = ceil(keys / chunk) (sm.pref becomes the item prefix; key
-  // counts are recomputed from the head state where needed)
   for (int i = tid; i < nh; i += kDecThreads) {
-    long long nl = 0;
-    int l0 = 0;
-    if (a.n_steps > 0) {
-      nl = min64(max64(__ldcg(&hstate(i)->n_leaf), 0), a.cap_list);
-      l0 = __ldcg(&hstate(i)->leaf0);
-    }
-    const long long kh = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
-    sm.pref[1 + i] = (kh + chunk - 1) / chunk;
+    long long nl;
+    bool sink;
+    sm.pref[1 + i] = (head_keys(i, nl, sink) + chunk - 1) / chunk;
   }
   __syncthreads();
   const long long total_items = build_prefix(sm, nh);
   const long long c0 = (long long)blockIdx.x * total_items / gridDim.x;
   const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kPartSlots);
   if (tid == 0 && (long long)(blockIdx.x + 1) * total_items / gridDim.x > c1) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+  float (*part)[2 + 128] = reinterpret_cast<float (*)[2 + 128]>(sm.u);
   {
     const int sub = lane / CPR, cl = lane % CPR;
-    constexpr int kU = 4;
+    constexpr int kU = 8;
     for (long long it = c0 + wid; it < c1; it += kDecWarps) {
       const int h = owner_of(sm, nh, it);
       const long long ci = it - sm.pref[h];
       const int kvh = (h % a.t.hq) / a.t.group;
-      long long nl = 0;
-      int l0 = 0;
-      if (a.n_steps > 0) {
-        nl = min64(max64(__ldcg(&hstate(h)->n_leaf), 0), a.cap_list);
-        l0 = __ldcg(&hstate(h)->leaf0);
-      }
-      const bool sink = (n1 > 0) && !l0;
+      long long nl;
+      bool sink;
+      const long long kh = head_keys(h, nl, sink);
       const long long leaf_keys = nl * b;
-      const long long kh = leaf_keys + (sink ? 1 : 0) + tail;
       const long long k0 = ci * chunk, k1 = min64(kh, k0 + chunk);
       float qs[EPC];
       q_slice(h, qs);
       const T* Kh = static_cast<const T*>(a.t.K) + size_t(kvh) * a.t.capacity * D;
       const T* Vh = static_cast<const T*>(a.t.V) + size_t(kvh) * a.t.capacity * D;
       const uint32_t* lv = leaves(h);
+      // leaf indices of the chunk's first 32 blocks, one per lane
+      const long long lf0 = k0 / b;
+      uint32_t leaf_reg = 0;
+      if (lf0 + lane < nl) leaf_reg = __ldcg(lv + lf0 + lane);
       float m_run = -INFINITY, l_run = 0.f, o[EPC];
 #pragma unroll
       for (int i = 0; i < EPC; ++i) o[i] = 0.f;
@@ -707,21 +824,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         for (int u = 0; u < kU; ++u) {
           const long long idx = wb + (long long)u * KPW + sub;
           ok[u] = idx < k1;
+          long long tok = 0;
+          const long long li = idx / b;
+          // every lane takes part in the shuffle; only leaf keys use the value
+          const uint32_t lr = __shfl_sync(0xffffffffu, leaf_reg, int((li - lf0) & 31));
+          if (idx < leaf_keys) {
+            const uint32_t leaf = (li - lf0 < 32) ? lr : __ldcg(lv + li);
+            tok = int64_t(leaf) * b + idx % b;
+          } else if (sink && idx == leaf_keys) {
+            tok = 0;
+          } else {
+            tok = n1 * b + (idx - leaf_keys - (sink ? 1 : 0));
+          }
+          if (ok[u] && (tok < 0 || tok >= a.n_tokens)) {  // a corrupted leaf index: skip it
+            ok[u] = false;
+            raise_status(a.t.status, ZHA_ERR_CAPACITY);
+          }
           if (ok[u]) {
-            long long tok;
-            if (idx < leaf_keys) {
-              const uint32_t leaf = __ldcg(lv + idx / b);
-              tok = int64_t(leaf) * b + idx % b;
-            } else if (sink && idx == leaf_keys) {
-              tok = 0;
-            } else {
-              tok = n1 * b + (idx - leaf_keys - (sink ? 1 : 0));
-            }
-            if (tok < 0 || tok >= a.n_tokens) {  // a corrupted leaf index: skip it
-              ok[u] = false;
-              raise_status(a.t.status, ZHA_ERR_CAPACITY);
-              continue;
-            }
             kv[u] = ldg_stream(Kh + size_t(tok) * D + cl * EPC);
             vv[u] = ldg_stream(Vh + size_t(tok) * D + cl * EPC);
           }
@@ -767,7 +886,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         l_run = l_run * sa + lo2 * sb;
         m_run = mn;
       }
-      float* P = sm.part[it - c0];
+      float* P = part[it - c0];
       if (lane == 0) {
         P[0] = m_run;
         P[1] = l_run;
@@ -787,19 +906,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     if (seg != c0 && seg != sm.pref[h]) continue;  // not the first chunk of a segment
     const long long send = min64(c1, sm.pref[h + 1]);
     float M = -INFINITY;
-    for (long long j = seg; j < send; ++j) M = fmaxf(M, sm.part[j - c0][0]);
+    for (long long j = seg; j < send; ++j) M = fmaxf(M, part[j - c0][0]);
     float L = 0.f;
     float acc[(D + 31) / 32];
 #pragma unroll
     for (int q = 0; q < (D + 31) / 32; ++q) acc[q] = 0.f;
     for (long long j = seg; j < send; ++j) {
-      const float mj = sm.part[j - c0][0];
+      const float mj = part[j - c0][0];
       if (mj == -INFINITY) continue;
       const float sc = expf(mj - M);
-      L = fmaf(sc, sm.part[j - c0][1], L);
+      L = fmaf(sc, part[j - c0][1], L);
 #pragma unroll
       for (int q = 0; q < (D + 31) / 32; ++q)
-        if (q * 32 + lane < D) acc[q] = fmaf(sc, sm.part[j - c0][2 + q * 32 + lane], acc[q]);
+        if (q * 32 + lane < D) acc[q] = fmaf(sc, part[j - c0][2 + q * 32 + lane], acc[q]);
     }
     float* G = a.attn_part + size_t(seg) * (2 + D);
     if (lane == 0) {
@@ -811,7 +930,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
   }
   stamp(a, 27);
-  if (grid_sync(a, sm)) return;
+  if (grid_sync(a, sm, bar_target)) return;
   stamp(a, 28);
 
   // ---------------- combine (one CTA per head)
@@ -829,7 +948,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
       M = fmaxf(M, __ldcg(a.attn_part + size_t(cs) * (2 + D)));
     }
-    // block max
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     if (lane == 0) sm.red32[wid] = __float_as_uint(M);
@@ -838,10 +956,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, __uint_as_float(sm.red32[w]));
     __syncthreads();
     float L = 0.f, acc = 0.f;
-    const int e = tid % D, part = tid / D;  // NP threads per output element
+    const int e = tid % D, prt = tid / D;  // NP threads per output element
     constexpr int NP = kDecThreads / D;
     float Lp = 0.f;
-    for (long long c = cfirst + part; c < gridDim.x; c += NP) {
+    for (long long c = cfirst + prt; c < gridDim.x; c += NP) {
       const long long cs = max64(p0, range_start(c));
       if (cs >= p1) break;
       if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
@@ -853,10 +971,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       acc = fmaf(sc, __ldcg(G + 2 + e), acc);
     }
     float* red = reinterpret_cast<float*>(sm.hist);  // [NP][D] + [NP]
-    red[part * D + e] = acc;
-    if (e == 0) red[NP * D + part] = Lp;
+    red[prt * D + e] = acc;
+    if (e == 0) red[NP * D + prt] = Lp;
     __syncthreads();
-    if (part == 0) {
+    if (prt == 0) {
       for (int q = 1; q < NP; ++q) acc += red[q * D + e];
       for (int q = 0; q < NP; ++q) L += red[NP * D + q];
       a.O[size_t(h) * D + e] = acc / L;
@@ -899,16 +1017,15 @@ static int grid_size_t() {
     cudaGetLastError();
     return 0;
   }
-  cached = per_sm * sms;
+  cached = min(per_sm * sms, kMaxDecodeGrid);
   return cached;
 }
 
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   auto kern = decode_kernel<T, D>;
-  int grid = grid_size_t<T, D>();
+  const int grid = grid_size_t<T, D>();
   if (grid < 1) return cudaErrorLaunchOutOfResources;
-  if (grid > kMaxDecodeGrid) grid = kMaxDecodeGrid;  // the scratch's attend partials are sized for this
   DecodeArgs args = a;
   void* params[] = {&args};
   count_launches(1);
@@ -922,9 +1039,15 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
   return a.t.d == 128 ? launch_decode_t<float, 128>(a, st) : launch_decode_t<float, 64>(a, st);
 }
 
+int decode_grid(int dtype, int d) {
+  if (dtype == ZHA_BF16) return d == 128 ? grid_size_t<__nv_bfloat16, 128>() : grid_size_t<__nv_bfloat16, 64>();
+  return d == 128 ? grid_size_t<float, 128>() : grid_size_t<float, 64>();
+}
+
 size_t decode_smem_bytes() { return sizeof(DecSmem); }
 size_t decode_head_state_bytes() { return sizeof(HeadState); }
 int decode_max_heads() { return kMaxHeads; }
 int decode_items_per_cta() { return kItemsPerCta; }
+int decode_max_grid() { return kMaxDecodeGrid; }
 
 }  // namespace zha
