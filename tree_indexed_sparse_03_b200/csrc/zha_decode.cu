@@ -73,6 +73,7 @@ struct HeadState {  // per (sequence, query head), written by the head's select 
 struct __align__(16) DecSmem {
   unsigned char u[kUnionBytes];
   unsigned long long hist[kBins];
+  unsigned int cnt[kBins];                  // entries per coarse bin
   long long pref[kMaxHeads + 1];            // per-head prefix of work items
   unsigned long long cut_key[32];
   unsigned long long cut_w[32];
@@ -258,6 +259,18 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
 }
 
+// Add masses to shared-memory histogram bins, one atomic per distinct bin in
+// the warp: lanes with the same bin sum their masses first (split into two
+// 20-bit halves so that 32 of them fit a 32-bit reduction).  Every lane of the
+// warp must call it; bin < 0 means "nothing to add".
+__device__ __forceinline__ void hist_add_warp(unsigned long long* hist, int bin, unsigned long long w) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xfffffull));
+  const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 20));
+  if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1)
+    atomicAdd(&hist[bin], (unsigned long long)lo + ((unsigned long long)hi << 20));
+}
+
 // Over kBins mass bins (shared memory), find the bin where the running mass,
 // starting from `base`, first reaches `target`: returns the bin and the mass
 // before it (all threads).  -1 if no bin does.
@@ -299,12 +312,23 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
 
-  // coarse histogram of the masses; total mass Z and the target T = ceil(p Z)
-  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
+  // coarse histogram of the masses (and counts); total mass Z and the target T = ceil(p Z)
+  for (int i = tid; i < kBins; i += kDecThreads) {
+    sm.hist[i] = 0ull;
+    sm.cnt[i] = 0u;
+  }
   __syncthreads();
-  for (int64_t i = tid; i < n; i += kDecThreads) {
-    const uint32_t k = E.key(i);
-    atomicAdd(&sm.hist[coarse_bin(entry_gap(m, k))], entry_mass(m, k));
+  for (int64_t base = tid - (tid & 31); base < n; base += kDecThreads) {  // warp-uniform trip count
+    const int64_t i = base + (tid & 31);
+    int bin = -1;
+    unsigned long long w = 0;
+    if (i < n) {
+      const uint32_t k = E.key(i);
+      bin = coarse_bin(entry_gap(m, k));
+      w = entry_mass(m, k);
+      atomicAdd(&sm.cnt[bin], 1u);
+    }
+    hist_add_warp(sm.hist, bin, w);
   }
   __syncthreads();
   unsigned long long Z = 0;
@@ -320,18 +344,32 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
 
-  // fine histogram inside the cut coarse bin
-  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
-  __syncthreads();
-  for (int64_t i = tid; i < n; i += kDecThreads) {
-    const uint32_t k = E.key(i);
-    const float x = entry_gap(m, k);
-    if (coarse_bin(x) == cb) atomicAdd(&sm.hist[fine_bin(x, cb)], entry_mass(m, k));
+  // fine histogram inside the cut coarse bin, unless that bin is small already
+  const bool use_fine = sm.cnt[cb] > 32u;
+  int fb = 0;
+  unsigned long long below2 = below;
+  if (use_fine) {
+    for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
+    __syncthreads();
+    for (int64_t base = tid - (tid & 31); base < n; base += kDecThreads) {
+      const int64_t i = base + (tid & 31);
+      int bin = -1;
+      unsigned long long w = 0;
+      if (i < n) {
+        const uint32_t k = E.key(i);
+        const float x = entry_gap(m, k);
+        if (coarse_bin(x) == cb) {
+          bin = fine_bin(x, cb);
+          w = entry_mass(m, k);
+        }
+      }
+      hist_add_warp(sm.hist, bin, w);
+    }
+    __syncthreads();
+    fb = find_cut_bin(sm, below, T, &below2);
+    if (fb < 0) return ~0ull;
   }
-  __syncthreads();
-  unsigned long long below2;
-  const int fb = find_cut_bin(sm, below, T, &below2);
-  if (fb < 0) return ~0ull;
+  auto in_cut = [&](float x) { return coarse_bin(x) == cb && (!use_fine || fine_bin(x, cb) == fb); };
 
   // gather the entries of the cut fine bin
   if (tid == 0) sm.bcast32[1] = 0;
@@ -339,7 +377,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   for (int64_t i = tid; i < n; i += kDecThreads) {
     const uint32_t k = E.key(i);
     const float x = entry_gap(m, k);
-    if (coarse_bin(x) == cb && fine_bin(x, cb) == fb) {
+    if (in_cut(x)) {
       const int s = atomicAdd(&sm.bcast32[1], 1);
       if (s < 32) {
         sm.cut_key[s] = entry_key64(a, Entry{k, E.code(i)});
@@ -391,7 +429,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     for (int64_t i = tid; i < n; i += kDecThreads) {
       const uint32_t k = E.key(i);
       const float x = entry_gap(m, k);
-      if (coarse_bin(x) != cb || fine_bin(x, cb) != fb) continue;
+      if (!in_cut(x)) continue;
       const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
       atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, k));
@@ -462,12 +500,12 @@ __device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm, unsi
   return sm.fail != 0;
 }
 
-// Phase timestamp (profiling builds pass a buffer of 32 slots per CTA).
+// Phase timestamp (profiling builds pass a buffer of 64 slots per CTA).
 __device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
-  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 32) {
+  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 64) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    a.phase_ns[blockIdx.x * 32 + slot] = t;
+    a.phase_ns[blockIdx.x * 64 + slot] = t;
   }
 }
 
@@ -633,15 +671,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           cp_async_commit();
           ++issued;
         }
-        cp_async_wait(int(issued - done - 1));
-        __syncwarp();
         const uint32_t code = __shfl_sync(0xffffffffu, code_reg, int(done & 31));
         const int h = __shfl_sync(0xffffffffu, head_reg, int(done & 31));
+        if (code != 0 && h != qhead) {  // load the head's query while the record is in flight
+          q_slice(h, qs);
+          qhead = h;
+        }
+        cp_async_wait(int(issued - done - 1));
+        __syncwarp();
         if (code != 0) {
-          if (h != qhead) {
-            q_slice(h, qs);
-            qhead = h;
-          }
           const float e = score_record_smem<T, D>(ring + size_t(done % nslot) * rec_bytes, R, a.t.inv_sqrt_d, qs,
                                                   lane);
           if (lane == 0) sel(h)[i0 + done - sm.pref[h]] = Entry{desc_key(e), code};
@@ -700,7 +738,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         for (long long i = tid; i < n; i += kDecThreads)
           if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
       }
+      stamp(a, 32 + 3 * step);
       const unsigned long long cut = select_cut(a, E, n, sm);
+      stamp(a, 33 + 3 * step);
       const uint32_t cut32 = uint32_t(cut >> 32);
       // ranks of the kept entries in canonical order (contiguous range per thread)
       const long long per_thr = (n + kDecThreads - 1) / kDecThreads;
@@ -789,6 +829,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
   const long long total_items = build_prefix(sm, nh);
+  stamp(a, 60);
   const long long c0 = (long long)blockIdx.x * total_items / gridDim.x;
   const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kPartSlots);
   if (tid == 0 && (long long)(blockIdx.x + 1) * total_items / gridDim.x > c1) raise_status(a.t.status, ZHA_ERR_CAPACITY);
@@ -964,11 +1005,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       if (cs >= p1) break;
       if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
       const float* G = a.attn_part + size_t(cs) * (2 + D);
-      const float mg = __ldcg(G);
-      if (mg == -INFINITY) continue;
-      const float sc = expf(mg - M);
-      Lp = fmaf(sc, __ldcg(G + 1), Lp);
-      acc = fmaf(sc, __ldcg(G + 2 + e), acc);
+      const float mg = __ldcg(G), lg = __ldcg(G + 1), og = __ldcg(G + 2 + e);  // independent loads
+      const float sc = mg == -INFINITY ? 0.f : expf(mg - M);
+      Lp = fmaf(sc, lg, Lp);
+      acc = fmaf(sc, og, acc);
     }
     float* red = reinterpret_cast<float*>(sm.hist);  // [NP][D] + [NP]
     red[prt * D + e] = acc;
