@@ -259,16 +259,26 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
 }
 
-// Add masses to shared-memory histogram bins, one atomic per distinct bin in
-// the warp: lanes with the same bin sum their masses first (split into two
-// 20-bit halves so that 32 of them fit a 32-bit reduction).  Every lane of the
-// warp must call it; bin < 0 means "nothing to add".
-__device__ __forceinline__ void hist_add_warp(unsigned long long* hist, int bin, unsigned long long w) {
-  const unsigned peers = __match_any_sync(0xffffffffu, bin);
-  const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xfffffull));
-  const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 20));
-  if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1)
-    atomicAdd(&hist[bin], (unsigned long long)lo + ((unsigned long long)hi << 20));
+// Add (count 1, mass w) to shared-memory histogram bin `bin` for every lane of
+// the warp (bin < 0: nothing).  When the whole warp hits one bin - the common
+// case for a diffuse head, whose masses crowd a few bins - the warp sums first
+// and one lane does the atomics; otherwise each lane adds its own.
+__device__ __forceinline__ void hist_add_warp(unsigned long long* hist, unsigned int* cnt, int bin,
+                                              unsigned long long w) {
+  const int b0 = __shfl_sync(0xffffffffu, bin, 0);
+  if (__all_sync(0xffffffffu, bin == b0)) {
+    if (b0 < 0) return;
+    unsigned long long s = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if ((threadIdx.x & 31) == 0) {
+      atomicAdd(&hist[b0], s);
+      if (cnt) atomicAdd(&cnt[b0], 32u);
+    }
+  } else if (bin >= 0) {
+    atomicAdd(&hist[bin], w);
+    if (cnt) atomicAdd(&cnt[bin], 1u);
+  }
 }
 
 // Over kBins mass bins (shared memory), find the bin where the running mass,
@@ -302,6 +312,45 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 }
 
 
+// The cut for at most kDecThreads entries: thread i takes entry i, counts the
+// entries ordered before it (its rank), the masses are placed in rank order
+// and scanned, and the cut is the first entry whose running mass reaches T.
+__device__ unsigned long long select_cut_small(const DecodeArgs& a, const SelView& E, int64_t n, float m,
+                                               DecSmem& sm) {
+  const int tid = threadIdx.x;
+  unsigned long long* k64s = sm.hist;                        // [n] order keys
+  unsigned long long* wr = sm.hist + kDecThreads;            // [n] masses in rank order
+  unsigned long long myk = ~0ull, myw = 0;
+  if (tid < n) {
+    const uint32_t k = E.key(tid);
+    myk = entry_key64(a, Entry{k, E.code(tid)});
+    myw = entry_mass(m, k);
+    k64s[tid] = myk;
+  }
+  __syncthreads();
+  int rank = 0;
+  if (tid < n) {
+    for (int j = 0; j < n; ++j) rank += k64s[j] < myk;
+    wr[rank] = myw;
+  }
+  __syncthreads();
+  const unsigned long long w_sorted = tid < n ? wr[tid] : 0ull;
+  unsigned long long Z;
+  const unsigned long long before = block_scan_u64(w_sorted, sm.red64, &Z);
+  const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);
+  // sorted position of the cut: the first with before + w >= T
+  if (tid == 0) sm.bcast32[2] = int(n) - 1;
+  __syncthreads();
+  if (tid < n && before < T && before + w_sorted >= T) sm.bcast32[2] = tid;
+  __syncthreads();
+  const int cut_pos = sm.bcast32[2];
+  if (tid < n && rank == cut_pos) sm.bcast64[1] = myk;
+  __syncthreads();
+  const unsigned long long cut = sm.bcast64[1];
+  __syncthreads();
+  return cut;
+}
+
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  Every thread returns the same value.
 __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, DecSmem& sm) {
@@ -311,6 +360,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   kmin = block_min_u32(kmin, sm.red32);
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
+  if (n <= kDecThreads) return select_cut_small(a, E, n, m, sm);
 
   // coarse histogram of the masses (and counts); total mass Z and the target T = ceil(p Z)
   for (int i = tid; i < kBins; i += kDecThreads) {
@@ -326,9 +376,8 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
       const uint32_t k = E.key(i);
       bin = coarse_bin(entry_gap(m, k));
       w = entry_mass(m, k);
-      atomicAdd(&sm.cnt[bin], 1u);
     }
-    hist_add_warp(sm.hist, bin, w);
+    hist_add_warp(sm.hist, sm.cnt, bin, w);
   }
   __syncthreads();
   unsigned long long Z = 0;
@@ -363,7 +412,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
           w = entry_mass(m, k);
         }
       }
-      hist_add_warp(sm.hist, bin, w);
+      hist_add_warp(sm.hist, nullptr, bin, w);
     }
     __syncthreads();
     fb = find_cut_bin(sm, below, T, &below2);
