@@ -260,24 +260,33 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
 }
 
 // Add (count 1, mass w) to shared-memory histogram bin `bin` for every lane of
-// the warp (bin < 0: nothing).  When the whole warp hits one bin - the common
-// case for a diffuse head, whose masses crowd a few bins - the warp sums first
-// and one lane does the atomics; otherwise each lane adds its own.
+// the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
+// a bin (siblings sit next to each other in a step's candidate list), so the
+// warp sums each run of equal bins with a segmented scan and the last lane of
+// the run does one atomic.  Every lane of the warp must call it.
 __device__ __forceinline__ void hist_add_warp(unsigned long long* hist, unsigned int* cnt, int bin,
                                               unsigned long long w) {
-  const int b0 = __shfl_sync(0xffffffffu, bin, 0);
-  if (__all_sync(0xffffffffu, bin == b0)) {
-    if (b0 < 0) return;
-    unsigned long long s = w;
+  const int lane = threadIdx.x & 31;
+  const int prev = __shfl_up_sync(0xffffffffu, bin, 1);
+  const bool head = lane == 0 || prev != bin;
+  const unsigned heads = __ballot_sync(0xffffffffu, head);
+  const int start = 31 - __clz(heads & (0xffffffffu >> (31 - lane)));  // first lane of my run
+  unsigned long long s = w;
+  unsigned c = 1;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if ((threadIdx.x & 31) == 0) {
-      atomicAdd(&hist[b0], s);
-      if (cnt) atomicAdd(&cnt[b0], 32u);
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, s, off);
+    const unsigned yc = __shfl_up_sync(0xffffffffu, c, off);
+    if (lane - off >= start) {
+      s += y;
+      c += yc;
     }
-  } else if (bin >= 0) {
-    atomicAdd(&hist[bin], w);
-    if (cnt) atomicAdd(&cnt[bin], 1u);
+  }
+  const int next = __shfl_down_sync(0xffffffffu, bin, 1);
+  const bool tail = lane == 31 || next != bin;
+  if (tail && bin >= 0) {
+    atomicAdd(&hist[bin], s);
+    if (cnt) atomicAdd(&cnt[bin], c);
   }
 }
 
@@ -368,11 +377,13 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     sm.cnt[i] = 0u;
   }
   __syncthreads();
-  for (int64_t base = tid - (tid & 31); base < n; base += kDecThreads) {  // warp-uniform trip count
+  const int64_t wseg = (n + kDecWarps - 1) / kDecWarps;           // entries per warp, contiguous
+  const int64_t wlo = min64(n, (tid >> 5) * wseg), whi = min64(n, wlo + wseg);
+  for (int64_t base = wlo; base < whi; base += 32) {
     const int64_t i = base + (tid & 31);
     int bin = -1;
     unsigned long long w = 0;
-    if (i < n) {
+    if (i < whi) {
       const uint32_t k = E.key(i);
       bin = coarse_bin(entry_gap(m, k));
       w = entry_mass(m, k);
@@ -400,11 +411,11 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   if (use_fine) {
     for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
     __syncthreads();
-    for (int64_t base = tid - (tid & 31); base < n; base += kDecThreads) {
+    for (int64_t base = wlo; base < whi; base += 32) {
       const int64_t i = base + (tid & 31);
       int bin = -1;
       unsigned long long w = 0;
-      if (i < n) {
+      if (i < whi) {
         const uint32_t k = E.key(i);
         const float x = entry_gap(m, k);
         if (coarse_bin(x) == cb) {
@@ -791,42 +802,62 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       const unsigned long long cut = select_cut(a, E, n, sm);
       stamp(a, 33 + 3 * step);
       const uint32_t cut32 = uint32_t(cut >> 32);
-      // ranks of the kept entries in canonical order (contiguous range per thread)
-      const long long per_thr = (n + kDecThreads - 1) / kDecThreads;
-      const long long lo = min64(n, tid * per_thr), hi = min64(n, lo + per_thr);
+      // ranks of the kept entries in canonical order: each warp owns a contiguous
+      // segment, walked 32 entries at a time (coalesced reads and writes)
+      const int64_t wseg = (n + kDecWarps - 1) / kDecWarps;
+      const int64_t wlo = min64(n, wid * wseg), whi = min64(n, wlo + wseg);
       auto kept_entry = [&](long long i, uint32_t& code) {
         const uint32_t k = E.key(i);
         if (k > cut32) return false;
         code = E.code(i);
         return k < cut32 || entry_key64(a, Entry{k, code}) <= cut;
       };
-      uint32_t nleaf = 0, npar = 0;
-      for (long long i = lo; i < hi; ++i) {
-        uint32_t code;
-        if (kept_entry(i, code)) {
-          if (code_level(code) == 1) ++nleaf; else ++npar;
-        }
+      uint32_t wleaf = 0, wpar = 0;
+      for (int64_t base = wlo; base < whi; base += 32) {
+        const int64_t i = base + lane;
+        uint32_t code = 0;
+        const bool kp = i < whi && kept_entry(i, code);
+        wleaf += __popc(__ballot_sync(0xffffffffu, kp && code_level(code) == 1));
+        wpar += __popc(__ballot_sync(0xffffffffu, kp && code_level(code) != 1));
       }
-      uint32_t tot_leaf, tot_par;
-      uint32_t leaf_rank = block_scan_u32(nleaf, sm.red32, &tot_leaf);
-      uint32_t par_rank = block_scan_u32(npar, sm.red32, &tot_par);
+      if (lane == 0) {
+        sm.red32[wid] = wleaf;
+        sm.red32[kDecWarps + wid] = wpar;
+      }
+      __syncthreads();
+      uint32_t leaf_off = 0, par_off = 0, tot_leaf = 0, tot_par = 0;
+      for (int w = 0; w < kDecWarps; ++w) {
+        const uint32_t l = sm.red32[w], q = sm.red32[kDecWarps + w];
+        if (w < wid) { leaf_off += l; par_off += q; }
+        tot_leaf += l;
+        tot_par += q;
+      }
       int my_leaf0 = 0;
-      for (long long i = lo; i < hi; ++i) {
-        uint32_t code;
-        if (!kept_entry(i, code)) continue;
-        if (code_level(code) == 1) {
-          const long long g = n_leaf0 + leaf_rank++;
+      const unsigned below_me = (1u << lane) - 1u;
+      for (int64_t base = wlo; base < whi; base += 32) {
+        const int64_t i = base + lane;
+        uint32_t code = 0;
+        const bool kp = i < whi && kept_entry(i, code);
+        const bool isleaf = kp && code_level(code) == 1;
+        const bool ispar = kp && code_level(code) != 1;
+        const unsigned ml = __ballot_sync(0xffffffffu, isleaf);
+        const unsigned mp = __ballot_sync(0xffffffffu, ispar);
+        if (isleaf) {
+          const long long g = n_leaf0 + leaf_off + __popc(ml & below_me);
           if (code_index(code) == 0) my_leaf0 = 1;
           if (g < a.cap_list) leaves(h)[g] = code_index(code);
           else raise_status(a.t.status, ZHA_ERR_CAPACITY);
           if (a.kept && g < a.kept_stride) a.kept[size_t(h) * a.kept_stride + g] = int32_t(code_index(code));
-        } else {
-          const long long pr = par_rank++;
+        }
+        if (ispar) {
+          const long long pr = par_off + __popc(mp & below_me);
           const uint32_t cl = code_level(code) - 1, ci = code_index(code) * uint32_t(b);
           if ((pr + 1) * b <= a.cap_sel) {
             for (int c = 0; c < b; ++c) cand(h)[pr * b + c] = node_code(cl, ci + uint32_t(c));
           }
         }
+        leaf_off += __popc(ml);
+        par_off += __popc(mp);
       }
       my_leaf0 = __syncthreads_or(my_leaf0);
       if (tid == 0) {
