@@ -185,6 +185,29 @@ ZHA_API size_t zha_dense_scratch_bytes(const zha_config* cfg, int32_t B, int64_t
 ZHA_API int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n,
                      const void* Q, float* O, int32_t B, void* scratch, void* stream);
 
+/*
+ * zha_dense_decode_noalloc: zha_dense_decode for callers that cannot allocate
+ * device memory - a serving loop whose device memory is fixed and
+ * pre-partitioned at start-up (an allocation there can fail or fragment the
+ * pool at the worst moment), or a host framework that owns the whole device
+ * arena and gives plug-ins no allocator.  The pages describe nothing like it;
+ * it is a deployment convenience of this library.
+ *   Same arguments and result as zha_dense_decode, without `scratch`: the
+ *   split partials go to a fixed array of 2^20 floats (4 MiB) that the library
+ *   holds on every device that loads it, until the process exits.
+ *   Requires B * n_q_heads * splits * (d + 2) <= 2^20 (splits as planned for
+ *   zha_dense_scratch_bytes, at most 4 * 148 / (B * n_kv_heads) rounded up);
+ *   larger requests return ZHA_ERR_CAPACITY without launching anything.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   No cudaMalloc, cudaFree or other allocation happens in any call.  Every
+ *   call on a device shares the array and overwrites it: calls whose work
+ *   overlaps on the GPU (other streams, other threads) race and must be
+ *   serialised by the caller.  Nothing in the array needs to start at zero.
+ */
+ZHA_API int zha_dense_decode_noalloc(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n,
+                             const void* Q, float* O, int32_t B, void* stream);
+
 /* Synchronise `stream` and return the tree's device status word (ZHA_OK or a
  * ZHA_ERR_* code raised inside a kernel); clears it. */
 ZHA_API int zha_tree_status(zha_tree* tree, void* stream);

@@ -24,6 +24,8 @@ int decode_items_per_cta();
 int decode_max_grid();
 int decode_grid(int dtype, int d);
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
+size_t dense_static_floats();
+cudaError_t dense_static_scratch(float** out);
 }  // namespace zha
 
 #include "zha_args.cuh"
@@ -430,6 +432,44 @@ int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_
   a.inv_sqrt_d = 1.0f / std::sqrt(float(cfg->d));
   cudaError_t e = launch_dense(a, cfg->dtype, cfg->d, B, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "zha_dense_decode");
+  return ZHA_OK;
+}
+
+// Dense decode for callers that cannot allocate device memory: the split
+// partials go to the library's fixed static array (see zha.h).
+int zha_dense_decode_noalloc(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n,
+                             const void* Q, float* O, int32_t B, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!K || !V || !Q || !O) return fail(ZHA_ERR_INVALID, "a pointer is NULL");
+  if (n < 1 || ld < n) return fail(ZHA_ERR_INVALID, "need 1 <= n <= ld");
+  if (B < 1) return fail(ZHA_ERR_INVALID, "B must be >= 1");
+  if (B > cfg->max_batch) return fail(ZHA_ERR_CAPACITY, "B exceeds max_batch");
+  if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(Q) |
+       reinterpret_cast<uintptr_t>(O)) & 15)
+    return fail(ZHA_ERR_INVALID, "K, V, Q and O must be 16-byte aligned");
+  DenseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  dense_plan(B, cfg->n_kv_heads, n, &a.splits, &a.per);
+  const uint64_t floats = uint64_t(B) * cfg->n_q_heads * a.splits * (cfg->d + 2);
+  if (floats > dense_static_floats())
+    return fail(ZHA_ERR_CAPACITY, "B * n_q_heads * splits * (d + 2) exceeds the fixed scratch of 2^20 floats");
+  float* part = nullptr;
+  cudaError_t e = dense_static_scratch(&part);
+  if (e != cudaSuccess) return fail_cuda(e, "zha_dense_decode_noalloc: looking up the fixed scratch");
+  a.K = K;
+  a.V = V;
+  a.Q = Q;
+  a.O = O;
+  a.part = part;
+  a.ld = ld;
+  a.n = n;
+  a.hq = cfg->n_q_heads;
+  a.hkv = cfg->n_kv_heads;
+  a.group = cfg->n_q_heads / cfg->n_kv_heads;
+  a.inv_sqrt_d = 1.0f / std::sqrt(float(cfg->d));
+  e = launch_dense(a, cfg->dtype, cfg->d, B, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "zha_dense_decode_noalloc");
   return ZHA_OK;
 }
 

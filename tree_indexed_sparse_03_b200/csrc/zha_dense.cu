@@ -18,6 +18,8 @@
 // heads), so the tensor core is used only to keep the FMA pipe from becoming
 // the limit.
 // fp32 path: one CTA per query head, CUDA cores.
+#include <mutex>
+
 #include "zha_args.cuh"
 
 namespace zha {
@@ -315,6 +317,37 @@ __global__ void __launch_bounds__(256) dense_scalar_kernel(DenseArgs a) {
     }
     a.part[((size_t(bb) * a.hq + h) * a.splits + split) * (D + 2) + e] = val;
   }
+}
+
+// ------------------------------------------------------------------ fixed scratch
+// Split partials of zha_dense_decode_noalloc live in this array instead of
+// caller memory: 2^20 floats (4 MiB) on every device that loads the library,
+// held until the process exits.  Every call writes the partials it later
+// reads, so nothing in it has to start at zero.
+constexpr size_t kDenseStaticFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_dense_static_part[kDenseStaticFloats];
+
+size_t dense_static_floats() { return kDenseStaticFloats; }
+
+// Device address of the array on the current device.  A host-side reference
+// to g_dense_static_part is only a stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t dense_static_scratch(float** out) {
+  static std::mutex mu;
+  static float* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_dense_static_part);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 // ------------------------------------------------------------------ host side

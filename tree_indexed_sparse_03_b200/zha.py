@@ -41,6 +41,8 @@ _SIGS = {
     "zha_dense_scratch_bytes": (_c.c_size_t, [_c.c_void_p, _c.c_int32, _c.c_int64]),
     "zha_dense_decode": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p,
                                     _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_void_p]),
+    "zha_dense_decode_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64,
+                                            _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p]),
     "zha_tree_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "zha_tree_destroy": (None, [_c.c_void_p]),
     "zha_last_error": (_c.c_char_p, []),
