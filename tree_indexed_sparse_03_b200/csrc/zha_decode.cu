@@ -259,6 +259,15 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
 }
 
+// Phase timestamp (profiling builds pass a buffer of 128 slots per CTA).
+__device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
+  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 128) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.phase_ns[blockIdx.x * 128 + slot] = t;
+  }
+}
+
 // Add (count 1, mass w) to shared-memory histogram bin `bin` for every lane of
 // the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
 // a bin (siblings sit next to each other in a step's candidate list), so the
@@ -362,11 +371,12 @@ __device__ unsigned long long select_cut_small(const DecodeArgs& a, const SelVie
 
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  Every thread returns the same value.
-__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, DecSmem& sm) {
+__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, DecSmem& sm, int step) {
   const int tid = threadIdx.x;
   uint32_t kmin = 0xffffffffu;
   for (int64_t i = tid; i < n; i += kDecThreads) kmin = min(kmin, E.key(i));
   kmin = block_min_u32(kmin, sm.red32);
+  stamp(a, 64 + 8 * step);
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
   if (n <= kDecThreads) return select_cut_small(a, E, n, m, sm);
@@ -400,6 +410,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     block_scan_u64(local, sm.red64, &Z);
   }
   const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);  // keep while mass before < T
+  stamp(a, 65 + 8 * step);
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
@@ -430,6 +441,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     if (fb < 0) return ~0ull;
   }
   auto in_cut = [&](float x) { return coarse_bin(x) == cb && (!use_fine || fine_bin(x, cb) == fb); };
+  stamp(a, 66 + 8 * step);
 
   // gather the entries of the cut fine bin
   if (tid == 0) sm.bcast32[1] = 0;
@@ -446,6 +458,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     }
   }
   __syncthreads();
+  stamp(a, 67 + 8 * step);
   const int cnt = sm.bcast32[1];
   if (cnt <= 32) {
     if (tid < 32) {
@@ -558,15 +571,6 @@ __device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm, unsi
   }
   __syncthreads();
   return sm.fail != 0;
-}
-
-// Phase timestamp (profiling builds pass a buffer of 64 slots per CTA).
-__device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
-  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 64) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    a.phase_ns[blockIdx.x * 64 + slot] = t;
-  }
 }
 
 // Inclusive prefix of per-head counts held in sm.pref[1..nh] (pref[0] = 0); returns the total.
@@ -799,7 +803,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
       }
       stamp(a, 32 + 3 * step);
-      const unsigned long long cut = select_cut(a, E, n, sm);
+      const unsigned long long cut = select_cut(a, E, n, sm, step);
       stamp(a, 33 + 3 * step);
       const uint32_t cut32 = uint32_t(cut >> 32);
       // ranks of the kept entries in canonical order: each warp owns a contiguous
@@ -825,6 +829,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         sm.red32[kDecWarps + wid] = wpar;
       }
       __syncthreads();
+      stamp(a, 68 + 8 * step);
       uint32_t leaf_off = 0, par_off = 0, tot_leaf = 0, tot_par = 0;
       for (int w = 0; w < kDecWarps; ++w) {
         const uint32_t l = sm.red32[w], q = sm.red32[kDecWarps + w];
@@ -860,6 +865,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         par_off += __popc(mp);
       }
       my_leaf0 = __syncthreads_or(my_leaf0);
+      stamp(a, 69 + 8 * step);
       if (tid == 0) {
         long long nc = (long long)tot_par * b;
         if (nc > a.cap_sel) {
