@@ -371,11 +371,25 @@ __device__ unsigned long long select_cut_small(const DecodeArgs& a, const SelVie
 
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  Every thread returns the same value.
-__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, DecSmem& sm, int step) {
-  const int tid = threadIdx.x;
-  uint32_t kmin = 0xffffffffu;
-  for (int64_t i = tid; i < n; i += kDecThreads) kmin = min(kmin, E.key(i));
-  kmin = block_min_u32(kmin, sm.red32);
+// Smallest key in [lo, 2^32) whose bin (a monotone non-decreasing function of
+// the key over the keys that occur) is >= target; 2^32 if none.  Every thread
+// computes it (32 steps), so no broadcast is needed.
+template <typename BinFn>
+__device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, int target, BinFn bin) {
+  unsigned long long L = lo, H = 0x100000000ull;  // answer in [L, H]
+  while (L < H) {
+    const unsigned long long mid = (L + H) >> 1;
+    if (bin(uint32_t(mid)) >= target) H = mid; else L = mid + 1;
+  }
+  return L;
+}
+
+// The cut of one routing step: the largest 64-bit order key (e desc, start
+// asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
+// Every thread returns the same value.
+__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, uint32_t kmin,
+                                         DecSmem& sm, int step) {
+  const int tid = threadIdx.x, lane = tid & 31;
   stamp(a, 64 + 8 * step);
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
@@ -389,16 +403,23 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   __syncthreads();
   const int64_t wseg = (n + kDecWarps - 1) / kDecWarps;           // entries per warp, contiguous
   const int64_t wlo = min64(n, (tid >> 5) * wseg), whi = min64(n, wlo + wseg);
-  for (int64_t base = wlo; base < whi; base += 32) {
-    const int64_t i = base + (tid & 31);
-    int bin = -1;
-    unsigned long long w = 0;
-    if (i < whi) {
-      const uint32_t k = E.key(i);
-      bin = coarse_bin(entry_gap(m, k));
-      w = entry_mass(m, k);
+  constexpr int U = 4;                                              // groups of 32 in flight per warp
+  for (int64_t base = wlo; base < whi; base += 32 * U) {
+    int bin[U];
+    unsigned long long w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + 32 * u + lane;
+      bin[u] = -1;
+      w[u] = 0;
+      if (i < whi) {
+        const uint32_t k = E.key(i);
+        bin[u] = coarse_bin(entry_gap(m, k));
+        w[u] = entry_mass(m, k);
+      }
     }
-    hist_add_warp(sm.hist, sm.cnt, bin, w);
+#pragma unroll
+    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, sm.cnt, bin[u], w[u]);
   }
   __syncthreads();
   unsigned long long Z = 0;
@@ -414,42 +435,58 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
+  auto cbin = [&](uint32_t k) { return coarse_bin(entry_gap(m, k)); };
+  // keys of coarse bin cb form the contiguous range [klo, khi)
+  const unsigned long long klo = first_key_at_least(kmin, cb, cbin);
+  const unsigned long long khi = cb + 1 < kBins ? first_key_at_least(uint32_t(klo), cb + 1, cbin) : 0x100000000ull;
 
   // fine histogram inside the cut coarse bin, unless that bin is small already
   const bool use_fine = sm.cnt[cb] > 32u;
-  int fb = 0;
+  unsigned long long flo = klo, fhi = khi;  // key range of the entries around the cut
   unsigned long long below2 = below;
   if (use_fine) {
     for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
     __syncthreads();
-    for (int64_t base = wlo; base < whi; base += 32) {
-      const int64_t i = base + (tid & 31);
-      int bin = -1;
-      unsigned long long w = 0;
-      if (i < whi) {
-        const uint32_t k = E.key(i);
-        const float x = entry_gap(m, k);
-        if (coarse_bin(x) == cb) {
-          bin = fine_bin(x, cb);
-          w = entry_mass(m, k);
+    for (int64_t base = wlo; base < whi; base += 32 * U) {
+      int bin[U];
+      unsigned long long w[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = base + 32 * u + lane;
+        bin[u] = -1;
+        w[u] = 0;
+        if (i < whi) {
+          const uint32_t k = E.key(i);
+          if (k >= klo && k < khi) {
+            bin[u] = fine_bin(entry_gap(m, k), cb);
+            w[u] = entry_mass(m, k);
+          }
         }
       }
-      hist_add_warp(sm.hist, nullptr, bin, w);
+#pragma unroll
+      for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, nullptr, bin[u], w[u]);
     }
     __syncthreads();
+    int fb;
     fb = find_cut_bin(sm, below, T, &below2);
     if (fb < 0) return ~0ull;
+    auto fbin = [&](uint32_t k) {
+      const float x = entry_gap(m, k);
+      return coarse_bin(x) > cb ? kBins : fine_bin(x, cb);
+    };
+    flo = first_key_at_least(uint32_t(klo), fb, fbin);
+    fhi = fb + 1 < kBins ? first_key_at_least(uint32_t(flo), fb + 1, fbin) : khi;
+    if (fhi > khi) fhi = khi;
   }
-  auto in_cut = [&](float x) { return coarse_bin(x) == cb && (!use_fine || fine_bin(x, cb) == fb); };
+  auto in_cut = [&](uint32_t k) { return k >= flo && k < fhi; };
   stamp(a, 66 + 8 * step);
 
-  // gather the entries of the cut fine bin
+  // gather the entries around the cut
   if (tid == 0) sm.bcast32[1] = 0;
   __syncthreads();
   for (int64_t i = tid; i < n; i += kDecThreads) {
     const uint32_t k = E.key(i);
-    const float x = entry_gap(m, k);
-    if (in_cut(x)) {
+    if (in_cut(k)) {
       const int s = atomicAdd(&sm.bcast32[1], 1);
       if (s < 32) {
         sm.cut_key[s] = entry_key64(a, Entry{k, E.code(i)});
@@ -501,8 +538,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     __syncthreads();
     for (int64_t i = tid; i < n; i += kDecThreads) {
       const uint32_t k = E.key(i);
-      const float x = entry_gap(m, k);
-      if (!in_cut(x)) continue;
+      if (!in_cut(k)) continue;
       const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
       atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, k));
@@ -786,24 +822,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       E.ck = reinterpret_cast<const uint32_t*>(sm.u);
       E.mode = n <= kCache8 ? 1 : (n <= kCache4 ? 2 : 0);
       __syncthreads();
+      uint32_t kmin = 0xffffffffu;
       if (E.mode == 1) {
         Entry* ce = reinterpret_cast<Entry*>(sm.u);
         for (long long i = tid; i < n; i += kDecThreads) {
           const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
           ce[i] = Entry{v.x, v.y};
+          kmin = min(kmin, v.x);
         }
       } else if (E.mode == 2) {
         uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
-        for (long long i = tid; i < n; i += kDecThreads) ck[i] = __ldcg(reinterpret_cast<const unsigned int*>(S + i));
+        for (long long i = tid; i < n; i += kDecThreads) {
+          const uint32_t k = __ldcg(reinterpret_cast<const unsigned int*>(S + i));
+          ck[i] = k;
+          kmin = min(kmin, k);
+        }
+      } else {
+        for (long long i = tid; i < n; i += kDecThreads) kmin = min(kmin, E.key(i));
       }
-      __syncthreads();
+      kmin = block_min_u32(kmin, sm.red32);  // includes the barrier that publishes the cache
       if (a.scored) {
         int32_t* out = a.scored + size_t(h) * a.scored_cap;
         for (long long i = tid; i < n; i += kDecThreads)
           if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
       }
       stamp(a, 32 + 3 * step);
-      const unsigned long long cut = select_cut(a, E, n, sm, step);
+      const unsigned long long cut = select_cut(a, E, n, kmin, sm, step);
       stamp(a, 33 + 3 * step);
       const uint32_t cut32 = uint32_t(cut >> 32);
       // ranks of the kept entries in canonical order: each warp owns a contiguous
@@ -817,12 +861,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         return k < cut32 || entry_key64(a, Entry{k, code}) <= cut;
       };
       uint32_t wleaf = 0, wpar = 0;
-      for (int64_t base = wlo; base < whi; base += 32) {
-        const int64_t i = base + lane;
-        uint32_t code = 0;
-        const bool kp = i < whi && kept_entry(i, code);
-        wleaf += __popc(__ballot_sync(0xffffffffu, kp && code_level(code) == 1));
-        wpar += __popc(__ballot_sync(0xffffffffu, kp && code_level(code) != 1));
+      for (int64_t base = wlo; base < whi; base += 128) {
+        bool kp[4];
+        uint32_t code[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = base + 32 * u + lane;
+          code[u] = 0;
+          kp[u] = i < whi && kept_entry(i, code[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          wleaf += __popc(__ballot_sync(0xffffffffu, kp[u] && code_level(code[u]) == 1));
+          wpar += __popc(__ballot_sync(0xffffffffu, kp[u] && code_level(code[u]) != 1));
+        }
       }
       if (lane == 0) {
         sm.red32[wid] = wleaf;
