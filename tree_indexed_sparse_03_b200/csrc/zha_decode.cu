@@ -271,31 +271,36 @@ __device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
 // Add (count 1, mass w) to shared-memory histogram bin `bin` for every lane of
 // the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
 // a bin (siblings sit next to each other in a step's candidate list), so the
-// warp sums each run of equal bins with a segmented scan and the last lane of
-// the run does one atomic.  Every lane of the warp must call it.
+// lanes whose bin equals lane 0's or lane 31's are summed with the hardware
+// warp reduction (the 40-bit masses split into 20-bit halves so that 32 of
+// them fit 32 bits) and added by one lane; the remaining lanes add their own.
+// Every lane of the warp must call it.
 __device__ __forceinline__ void hist_add_warp(unsigned long long* hist, unsigned int* cnt, int bin,
                                               unsigned long long w) {
   const int lane = threadIdx.x & 31;
-  const int prev = __shfl_up_sync(0xffffffffu, bin, 1);
-  const bool head = lane == 0 || prev != bin;
-  const unsigned heads = __ballot_sync(0xffffffffu, head);
-  const int start = 31 - __clz(heads & (0xffffffffu >> (31 - lane)));  // first lane of my run
-  unsigned long long s = w;
-  unsigned c = 1;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned long long y = __shfl_up_sync(0xffffffffu, s, off);
-    const unsigned yc = __shfl_up_sync(0xffffffffu, c, off);
-    if (lane - off >= start) {
-      s += y;
-      c += yc;
+  const int b0 = __shfl_sync(0xffffffffu, bin, 0);
+  const int b1 = __shfl_sync(0xffffffffu, bin, 31);
+  const bool in0 = bin == b0, in1 = !in0 && bin == b1;
+  const unsigned lo = unsigned(w & 0xfffffull), hi = unsigned(w >> 20);
+  const unsigned lo0 = __reduce_add_sync(0xffffffffu, in0 ? lo : 0u);
+  const unsigned hi0 = __reduce_add_sync(0xffffffffu, in0 ? hi : 0u);
+  const unsigned c0 = __popc(__ballot_sync(0xffffffffu, in0));
+  if (lane == 0 && b0 >= 0) {
+    atomicAdd(&hist[b0], (unsigned long long)lo0 + ((unsigned long long)hi0 << 20));
+    if (cnt) atomicAdd(&cnt[b0], c0);
+  }
+  if (b1 != b0) {
+    const unsigned lo1 = __reduce_add_sync(0xffffffffu, in1 ? lo : 0u);
+    const unsigned hi1 = __reduce_add_sync(0xffffffffu, in1 ? hi : 0u);
+    const unsigned c1 = __popc(__ballot_sync(0xffffffffu, in1));
+    if (lane == 31 && b1 >= 0) {
+      atomicAdd(&hist[b1], (unsigned long long)lo1 + ((unsigned long long)hi1 << 20));
+      if (cnt) atomicAdd(&cnt[b1], c1);
     }
   }
-  const int next = __shfl_down_sync(0xffffffffu, bin, 1);
-  const bool tail = lane == 31 || next != bin;
-  if (tail && bin >= 0) {
-    atomicAdd(&hist[bin], s);
-    if (cnt) atomicAdd(&cnt[bin], c);
+  if (!in0 && !in1 && bin >= 0) {
+    atomicAdd(&hist[bin], w);
+    if (cnt) atomicAdd(&cnt[bin], 1u);
   }
 }
 
@@ -333,7 +338,7 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 // The cut for at most kDecThreads entries: thread i takes entry i, counts the
 // entries ordered before it (its rank), the masses are placed in rank order
 // and scanned, and the cut is the first entry whose running mass reaches T.
-__device__ unsigned long long select_cut_small(const DecodeArgs& a, const SelView& E, int64_t n, float m,
+__device__ __forceinline__ unsigned long long select_cut_small(const DecodeArgs& a, const SelView& E, int64_t n, float m,
                                                DecSmem& sm) {
   const int tid = threadIdx.x;
   unsigned long long* k64s = sm.hist;                        // [n] order keys
@@ -387,7 +392,7 @@ __device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, in
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
 // Every thread returns the same value.
-__device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, uint32_t kmin,
+__device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, uint32_t kmin,
                                          DecSmem& sm, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
   stamp(a, 64 + 8 * step);
@@ -401,15 +406,16 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
     sm.cnt[i] = 0u;
   }
   __syncthreads();
-  const int64_t wseg = (n + kDecWarps - 1) / kDecWarps;           // entries per warp, contiguous
-  const int64_t wlo = min64(n, (tid >> 5) * wseg), whi = min64(n, wlo + wseg);
+  const int n32 = int(n);
+  const int wseg = (n32 + kDecWarps - 1) / kDecWarps;               // entries per warp, contiguous
+  const int wlo = min(n32, (tid >> 5) * wseg), whi = min(n32, wlo + wseg);
   constexpr int U = 4;                                              // groups of 32 in flight per warp
-  for (int64_t base = wlo; base < whi; base += 32 * U) {
+  for (int base = wlo; base < whi; base += 32 * U) {
     int bin[U];
     unsigned long long w[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t i = base + 32 * u + lane;
+      const int i = base + 32 * u + lane;
       bin[u] = -1;
       w[u] = 0;
       if (i < whi) {
@@ -447,12 +453,12 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   if (use_fine) {
     for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
     __syncthreads();
-    for (int64_t base = wlo; base < whi; base += 32 * U) {
+    for (int base = wlo; base < whi; base += 32 * U) {
       int bin[U];
       unsigned long long w[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int64_t i = base + 32 * u + lane;
+        const int i = base + 32 * u + lane;
         bin[u] = -1;
         w[u] = 0;
         if (i < whi) {
@@ -484,7 +490,7 @@ __device__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, 
   // gather the entries around the cut
   if (tid == 0) sm.bcast32[1] = 0;
   __syncthreads();
-  for (int64_t i = tid; i < n; i += kDecThreads) {
+  for (int i = tid; i < n32; i += kDecThreads) {
     const uint32_t k = E.key(i);
     if (in_cut(k)) {
       const int s = atomicAdd(&sm.bcast32[1], 1);
