@@ -84,19 +84,27 @@ struct __align__(16) DecSmem {
   int fail;
 };
 
-// The step's entries of one head, read from shared memory when they fit.
-struct SelView {
-  const Entry* g;     // global step buffer
-  const Entry* ce;    // cached entries (mode 1)
-  const uint32_t* ck; // cached keys (mode 2)
-  int mode;           // 0: global, 1: entries cached, 2: keys cached
-  __device__ __forceinline__ uint32_t key(int64_t i) const {
-    if (mode == 1) return ce[i].key;
-    if (mode == 2) return ck[i];
-    return __ldcg(reinterpret_cast<const unsigned int*>(g + i));
-  }
+// The step's entries of one head: cached in shared memory with their codes,
+// cached as keys only, or read from the global step buffer.  Three concrete
+// types (no run-time switch) so that every access compiles to one load from
+// the right memory.
+struct ViewSmemEntries {
+  const Entry* ce;
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return ce[i].key; }
+  __device__ __forceinline__ uint32_t code(int64_t i) const { return ce[i].code; }
+};
+struct ViewSmemKeys {
+  const uint32_t* ck;
+  const Entry* g;
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return ck[i]; }
   __device__ __forceinline__ uint32_t code(int64_t i) const {
-    if (mode == 1) return ce[i].code;
+    return __ldcg(reinterpret_cast<const unsigned int*>(g + i) + 1);
+  }
+};
+struct ViewGlobal {
+  const Entry* g;
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return __ldcg(reinterpret_cast<const unsigned int*>(g + i)); }
+  __device__ __forceinline__ uint32_t code(int64_t i) const {
     return __ldcg(reinterpret_cast<const unsigned int*>(g + i) + 1);
   }
 };
@@ -338,7 +346,8 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 // The cut for at most kDecThreads entries: thread i takes entry i, counts the
 // entries ordered before it (its rank), the masses are placed in rank order
 // and scanned, and the cut is the first entry whose running mass reaches T.
-__device__ __forceinline__ unsigned long long select_cut_small(const DecodeArgs& a, const SelView& E, int64_t n, float m,
+template <class View>
+__device__ __forceinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
                                                DecSmem& sm) {
   const int tid = threadIdx.x;
   unsigned long long* k64s = sm.hist;                        // [n] order keys
@@ -392,7 +401,8 @@ __device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, in
 // The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
 // Every thread returns the same value.
-__device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, const SelView& E, int64_t n, uint32_t kmin,
+template <class View>
+__device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, const View& E, int64_t n, uint32_t kmin,
                                          DecSmem& sm, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
   stamp(a, 64 + 8 * step);
@@ -822,21 +832,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         continue;
       }
       const Entry* S = sel(h);
-      SelView E;
-      E.g = S;
-      E.ce = reinterpret_cast<const Entry*>(sm.u);
-      E.ck = reinterpret_cast<const uint32_t*>(sm.u);
-      E.mode = n <= kCache8 ? 1 : (n <= kCache4 ? 2 : 0);
+      const int mode = n <= kCache8 ? 1 : (n <= kCache4 ? 2 : 0);
       __syncthreads();
       uint32_t kmin = 0xffffffffu;
-      if (E.mode == 1) {
+      if (mode == 1) {
         Entry* ce = reinterpret_cast<Entry*>(sm.u);
         for (long long i = tid; i < n; i += kDecThreads) {
           const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
           ce[i] = Entry{v.x, v.y};
           kmin = min(kmin, v.x);
         }
-      } else if (E.mode == 2) {
+      } else if (mode == 2) {
         uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
         for (long long i = tid; i < n; i += kDecThreads) {
           const uint32_t k = __ldcg(reinterpret_cast<const unsigned int*>(S + i));
@@ -844,9 +850,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           kmin = min(kmin, k);
         }
       } else {
-        for (long long i = tid; i < n; i += kDecThreads) kmin = min(kmin, E.key(i));
+        for (long long i = tid; i < n; i += kDecThreads)
+          kmin = min(kmin, __ldcg(reinterpret_cast<const unsigned int*>(S + i)));
       }
       kmin = block_min_u32(kmin, sm.red32);  // includes the barrier that publishes the cache
+      int my_leaf0 = 0;
+      uint32_t tot_leaf = 0, tot_par = 0;
+      auto select_and_rank = [&](const auto& E) {
       if (a.scored) {
         int32_t* out = a.scored + size_t(h) * a.scored_cap;
         for (long long i = tid; i < n; i += kDecThreads)
@@ -888,14 +898,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       }
       __syncthreads();
       stamp(a, 68 + 8 * step);
-      uint32_t leaf_off = 0, par_off = 0, tot_leaf = 0, tot_par = 0;
+      uint32_t leaf_off = 0, par_off = 0;
       for (int w = 0; w < kDecWarps; ++w) {
         const uint32_t l = sm.red32[w], q = sm.red32[kDecWarps + w];
         if (w < wid) { leaf_off += l; par_off += q; }
         tot_leaf += l;
         tot_par += q;
       }
-      int my_leaf0 = 0;
       const unsigned below_me = (1u << lane) - 1u;
       for (int64_t base = wlo; base < whi; base += 32) {
         const int64_t i = base + lane;
@@ -922,6 +931,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         leaf_off += __popc(ml);
         par_off += __popc(mp);
       }
+      };
+      if (mode == 1) select_and_rank(ViewSmemEntries{reinterpret_cast<const Entry*>(sm.u)});
+      else if (mode == 2) select_and_rank(ViewSmemKeys{reinterpret_cast<const uint32_t*>(sm.u), S});
+      else select_and_rank(ViewGlobal{S});
       my_leaf0 = __syncthreads_or(my_leaf0);
       stamp(a, 69 + 8 * step);
       if (tid == 0) {
