@@ -18,7 +18,9 @@ cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, cons
                                cudaStream_t st);
 size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R);
 size_t decode_smem_bytes();
-size_t decode_head_state_bytes();
+size_t decode_flow_bytes(int nheads, int64_t cap_sel);
+uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list);
+int decode_barriers(int n_steps, int n_roots);
 int decode_max_heads();
 int decode_items_per_cta();
 int decode_max_grid();
@@ -63,7 +65,7 @@ struct Layout {
   uint64_t rec_off[kMaxLevels + 1], f_off[kMaxLevels + 1], up_off[kMaxLevels + 1];
   uint64_t rec_bytes, up_bytes, node_bytes;
   // scratch
-  uint64_t status_off, bar_off, part_off, part_items, ws_off, ws_per_bh, stage_off, scratch_bytes;
+  uint64_t status_off, bar_off, part_off, part_items, flow_off, flow_bytes, ws_off, ws_per_bh, stage_off, scratch_bytes;
   int64_t cap_sel, cap_list;
   uint64_t stage_k, stage_v, stage_q, stage_o;
 };
@@ -143,10 +145,11 @@ int make_layout(const zha_config* c, Layout* L) {
   const uint64_t nheads = uint64_t(c->max_batch) * c->n_q_heads;
   L->part_off = 256;
   L->part_items = uint64_t(decode_max_grid()) * decode_items_per_cta() + nheads + 64;
-  L->ws_off = align256(L->part_off + L->part_items * (c->d + 2) * 4);
-  // step entries (key, code), next candidates (codes), kept leaves, head state
-  L->ws_per_bh = align256(uint64_t(L->cap_sel) * 8 + uint64_t(L->cap_sel) * 4 + uint64_t(L->cap_list) * 4 +
-                          decode_head_state_bytes());
+  L->flow_off = align256(L->part_off + L->part_items * (c->d + 2) * 4);
+  // head states and leaf bitmaps, cleared together
+  L->flow_bytes = decode_flow_bytes(int(nheads), L->cap_sel);
+  L->ws_off = align256(L->flow_off + L->flow_bytes);
+  L->ws_per_bh = align256(decode_ws_bytes(L->cap_sel, L->cap_list));
   uint64_t s = L->ws_off + L->ws_per_bh * uint64_t(c->max_batch) * c->n_q_heads;
   L->stage_off = s;
   L->stage_k = s;
@@ -172,6 +175,7 @@ struct zha_tree {
   int device;
   long long spin_limit;  // grid-barrier spin bound of the decode kernel
   unsigned long long bar_count;  // arrivals the decode kernels have made on the grid barrier so far
+  bool flow_dirty;               // the routing flow state must be zeroed before the next decode
 };
 
 extern "C" {
@@ -222,6 +226,7 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
   t->n = 0;
   t->spin_limit = kDefaultSpinLimit;
   t->bar_count = 0;
+  t->flow_dirty = true;
   if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: force the barrier timeout path
     const long long x = std::atoll(v);
     if (x > 0) t->spin_limit = x;
@@ -272,6 +277,7 @@ int zha_tree_build(zha_tree* t, int64_t n, void* stream) {
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build");
   t->n = n;
   t->bar_count = 0;
+  t->flow_dirty = true;
   return ZHA_OK;
 }
 
@@ -312,6 +318,7 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->n_steps = steps;
   a->ws = t->scratch + t->L.ws_off;
   a->ws_per_bh = t->L.ws_per_bh;
+  a->flow = reinterpret_cast<unsigned char*>(t->scratch + t->L.flow_off);
   a->bar = reinterpret_cast<unsigned long long*>(t->scratch + t->L.bar_off);
   a->bar_base = t->bar_count;
   a->attn_part = reinterpret_cast<float*>(t->scratch + t->L.part_off);
@@ -350,15 +357,27 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
   if (scored && scored_cap < 1) return fail(ZHA_ERR_INVALID, "scored needs scored_cap >= 1");
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)
     return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
+  const int grid = decode_grid(t->cfg.dtype, t->cfg.d);
+  if (grid < 1) return fail(ZHA_ERR_CUDA, "the decode kernel does not fit on this device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  zha_tree* tm = const_cast<zha_tree*>(t);
+  if (tm->flow_dirty) {  // first decode of this tree, or the first after an error status
+    cudaError_t e = cudaMemsetAsync(t->scratch + t->L.flow_off, 0, t->L.flow_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->scratch + t->L.bar_off, 0, 8, st);
+    if (e != cudaSuccess) return fail_cuda(e, "zha_decode: clearing the flow state");
+    tm->bar_count = 0;
+    tm->flow_dirty = false;
+  }
   DecodeArgs a;
   fill_decode_args(t, Q, O, kept, kept_cnt, stats, scored, scored_cap, &a);
   a.nheads = B * t->cfg.n_q_heads;
-  const int grid = decode_grid(t->cfg.dtype, t->cfg.d);
-  if (grid < 1) return fail(ZHA_ERR_CUDA, "the decode kernel does not fit on this device");
-  cudaError_t e = launch_decode(a, t->cfg.dtype, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail_cuda(e, "zha_decode");
-  // every CTA arrives once per barrier: two per routing step and one after attention
-  const_cast<zha_tree*>(t)->bar_count += uint64_t(2 * a.n_steps + 1) * uint64_t(grid);
+  cudaError_t e = launch_decode(a, t->cfg.dtype, st);
+  if (e != cudaSuccess) {
+    tm->flow_dirty = true;
+    return fail_cuda(e, "zha_decode");
+  }
+  // every CTA arrives once on each grid barrier of the launch
+  tm->bar_count += uint64_t(decode_barriers(a.n_steps, a.n_roots)) * uint64_t(grid);
   return ZHA_OK;
 }
 
@@ -484,6 +503,7 @@ int zha_tree_status(zha_tree* t, void* stream) {
   if (status != 0) {
     const int zero = 0;
     cudaMemcpy(t->dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    t->flow_dirty = true;  // a kernel that gave up may have left its flow state and barrier mid-way
     return fail(status, "a kernel raised an error status (capacity bound exceeded)");
   }
   return ZHA_OK;

@@ -18,6 +18,7 @@ struct DecodeArgs {
   uint64_t ws_per_bh;
   int64_t cap_sel;              // entries per step buffer (and kept parents)
   int64_t cap_list;             // kept leaves per head
+  unsigned char* flow;          // per-head routing states, then leaf bitmaps (zero between launches)
   unsigned long long* bar;      // grid barrier arrival counter (only grows)
   unsigned long long bar_base;  // its value when this launch starts
   float* attn_part;             // attend partials, (2 + d) floats each

@@ -52,6 +52,15 @@ template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4&
   }
 }
 
+// D (16x8, fp32) += A (16x16, bf16, row) x B (16x8, bf16, col), one warp.
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // ---------------------------------------------------------------- ordered keys
 // Order-preserving map of fp32 onto uint32 (ascending), and the descending key
 // used to rank routing candidates: a smaller key means a larger estimate.

@@ -38,6 +38,8 @@
 //           run an online softmax per chunk, and each CTA merges its chunks per
 //           head into one partial;
 //   combine (one CTA per head) the partials of each head -> O.
+#include <type_traits>
+
 #include "zha_args.cuh"
 
 namespace zha {
@@ -47,34 +49,76 @@ struct Entry {
   uint32_t code;  // node_code(level, index)
 };
 
-constexpr int kDecThreads = 512;
+constexpr int kDecThreads = 512;                   // threads per CTA (one CTA per SM)
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kUnionBytes = 200 * 1024;            // select cache / score rings / attend partials
-constexpr int kCache8 = kUnionBytes / 8;           // entries cached with their codes
-constexpr int kCache4 = kUnionBytes / 4;           // entries cached as keys only
+constexpr int kUnionBytes = 208 * 1024;            // select key cache / score rings / attend partials + prefix
+constexpr int kCacheKeys = kUnionBytes / 4;        // step keys a select caches in shared memory
 constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
 constexpr int kMaxHeads = 1024;                    // sequences x query heads per call
 constexpr int kItemsPerCta = 256;                  // attend chunks a CTA owns at most (plus one per head)
-constexpr int kMaxDecodeGrid = 256;                // CTAs per decode launch the scratch is laid out for
-constexpr int kPartSlots = kUnionBytes / ((2 + 128) * 4);  // attend partials a CTA can hold
+constexpr int kMaxDecodeGrid = 512;                // CTAs per decode launch the scratch is laid out for
+constexpr int kPrefOff = kUnionBytes - (kMaxHeads + 1) * 8;  // per-head prefix (attend), inside the union
+constexpr int kPartSlots = kPrefOff / ((2 + 128) * 4);          // attend partials a CTA can hold
 constexpr int kMaxSlots = 8;                       // score ring slots per warp
-static_assert(kPartSlots >= kItemsPerCta + 32, "attend partial area too small");
+static_assert(kPartSlots >= kItemsPerCta + 16, "attend partial area too small");
 
-struct HeadState {  // per (sequence, query head), written by the head's select CTA
-  long long n_cand;   // candidates of the next step
-  long long n_leaf;   // kept level-1 blocks so far
-  long long scored;   // nodes scored so far
-  int steps;
-  int leaf0;          // leaf block 0 kept (token 0 already attended)
-  long long pad[4];
+struct HeadState {  // per (sequence, query head)
+  long long n[2];          // entries of the step built in each parity buffer (step 0: unused)
+  long long kept;          // entries kept by the last select (units of the next scoring phase)
+  long long scored;        // nodes scored so far
+  long long n_leaf;        // kept level-1 blocks (set when routing ends)
+  unsigned int kinv[2];    // ~(smallest key) of the step built in each parity buffer
+  int ovf[2];              // an estimate of that step lies above its anchor span
+  float anchor;            // histogram anchor of the step being built (max e of the step before)
+  int steps;               // selects done
+  int leaf0;               // leaf block 0 kept (token 0 already attended)
+  int pad_i;
+  long long pad[23];
 };
+static_assert(sizeof(HeadState) == 256, "HeadState layout");
+
+// Per-head routing state and leaf bitmaps live in one scratch region that
+// every decode leaves zeroed for the next (the combine phase clears it).
+
+// 32-bit words of a head's leaf bitmap (one bit per level-1 block), a multiple of 4.
+__host__ __device__ __forceinline__ int64_t decode_bitmap_words(int64_t cap_sel) {
+  return (((cap_sel + 31) / 32) + 3) & ~int64_t(3);
+}
+
+// Loads and stores of the routing flow state.  Stores that publish work are
+// releases at GPU scope and the loads that find it acquires, so that what the
+// publisher wrote before (entries, candidate codes, counters) is visible to
+// whoever takes the work.
+__device__ __forceinline__ int ld_volatile_i(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+__device__ __forceinline__ long long ld_volatile_ll(const long long* p) {
+  return *reinterpret_cast<const volatile long long*>(p);
+}
+__device__ __forceinline__ int ld_acquire_i(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
+  return *reinterpret_cast<const volatile unsigned long long*>(p);
+}
+// After a relaxed load that found published work: orders the reads of that work after it.
+__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void st_release_i(int* p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 struct __align__(16) DecSmem {
   unsigned char u[kUnionBytes];
   unsigned long long hist[kBins];
-  unsigned int cnt[kBins];                  // entries per coarse bin
-  long long pref[kMaxHeads + 1];            // per-head prefix of work items
   unsigned long long cut_key[32];
   unsigned long long cut_w[32];
   unsigned long long red64[kDecWarps];
@@ -82,31 +126,22 @@ struct __align__(16) DecSmem {
   unsigned long long bcast64[4];
   int bcast32[8];
   int fail;
+  int job_h, job_s;           // select CTA: the request being served (-2: exit)
+  unsigned long long mbar[kDecWarps][kMaxSlots];  // scoring warps: one mbarrier per ring slot
+  // per-head prefix of attend work items (lives in the union after routing)
+  __device__ __forceinline__ long long* pref() { return reinterpret_cast<long long*>(u + kPrefOff); }
+  __device__ __forceinline__ const long long* pref() const { return reinterpret_cast<const long long*>(u + kPrefOff); }
 };
 
-// The step's entries of one head: cached in shared memory with their codes,
-// cached as keys only, or read from the global step buffer.  Three concrete
-// types (no run-time switch) so that every access compiles to one load from
-// the right memory.
-struct ViewSmemEntries {
-  const Entry* ce;
-  __device__ __forceinline__ uint32_t key(int64_t i) const { return ce[i].key; }
-  __device__ __forceinline__ uint32_t code(int64_t i) const { return ce[i].code; }
-};
-struct ViewSmemKeys {
-  const uint32_t* ck;
-  const Entry* g;
-  __device__ __forceinline__ uint32_t key(int64_t i) const { return ck[i]; }
-  __device__ __forceinline__ uint32_t code(int64_t i) const {
-    return __ldcg(reinterpret_cast<const unsigned int*>(g + i) + 1);
-  }
-};
-struct ViewGlobal {
-  const Entry* g;
-  __device__ __forceinline__ uint32_t key(int64_t i) const { return __ldcg(reinterpret_cast<const unsigned int*>(g + i)); }
-  __device__ __forceinline__ uint32_t code(int64_t i) const {
-    return __ldcg(reinterpret_cast<const unsigned int*>(g + i) + 1);
-  }
+// The step's entries of one head: keys [0, nc) cached in shared memory, the
+// rest (and every code) read from the global step buffers.
+struct StepView {
+  const uint32_t* ck;  // cached keys
+  int nc;
+  const uint32_t* gk;  // global keys
+  const uint32_t* gc;  // global codes
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return i < nc ? ck[i] : __ldcg(gk + i); }
+  __device__ __forceinline__ uint32_t code(int64_t i) const { return __ldcg(gc + i); }
 };
 
 __device__ __forceinline__ uint32_t root_code(const DecodeArgs& a, int64_t i) {
@@ -276,15 +311,24 @@ __device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
   }
 }
 
-// Add (count 1, mass w) to shared-memory histogram bin `bin` for every lane of
+// Per (head, step) event times for profiling builds (heads < 64, steps < 8).
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void trace_hs(const DecodeArgs& a, int h, int step, int field, unsigned long long v) {
+  if (a.phase_ns != nullptr && h < 64 && step < 8) a.phase_ns[40960 + (h * 8 + step) * 32 + field] = v;
+}
+
+// Add mass w to shared-memory histogram bin `bin` for every lane of
 // the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
 // a bin (siblings sit next to each other in a step's candidate list), so the
 // lanes whose bin equals lane 0's or lane 31's are summed with the hardware
 // warp reduction (the 40-bit masses split into 20-bit halves so that 32 of
 // them fit 32 bits) and added by one lane; the remaining lanes add their own.
 // Every lane of the warp must call it.
-__device__ __forceinline__ void hist_add_warp(unsigned long long* hist, unsigned int* cnt, int bin,
-                                              unsigned long long w) {
+__device__ __forceinline__ void hist_add_warp(unsigned long long* hist, int bin, unsigned long long w) {
   const int lane = threadIdx.x & 31;
   const int b0 = __shfl_sync(0xffffffffu, bin, 0);
   const int b1 = __shfl_sync(0xffffffffu, bin, 31);
@@ -292,24 +336,13 @@ __device__ __forceinline__ void hist_add_warp(unsigned long long* hist, unsigned
   const unsigned lo = unsigned(w & 0xfffffull), hi = unsigned(w >> 20);
   const unsigned lo0 = __reduce_add_sync(0xffffffffu, in0 ? lo : 0u);
   const unsigned hi0 = __reduce_add_sync(0xffffffffu, in0 ? hi : 0u);
-  const unsigned c0 = __popc(__ballot_sync(0xffffffffu, in0));
-  if (lane == 0 && b0 >= 0) {
-    atomicAdd(&hist[b0], (unsigned long long)lo0 + ((unsigned long long)hi0 << 20));
-    if (cnt) atomicAdd(&cnt[b0], c0);
-  }
+  if (lane == 0 && b0 >= 0) atomicAdd(&hist[b0], (unsigned long long)lo0 + ((unsigned long long)hi0 << 20));
   if (b1 != b0) {
     const unsigned lo1 = __reduce_add_sync(0xffffffffu, in1 ? lo : 0u);
     const unsigned hi1 = __reduce_add_sync(0xffffffffu, in1 ? hi : 0u);
-    const unsigned c1 = __popc(__ballot_sync(0xffffffffu, in1));
-    if (lane == 31 && b1 >= 0) {
-      atomicAdd(&hist[b1], (unsigned long long)lo1 + ((unsigned long long)hi1 << 20));
-      if (cnt) atomicAdd(&cnt[b1], c1);
-    }
+    if (lane == 31 && b1 >= 0) atomicAdd(&hist[b1], (unsigned long long)lo1 + ((unsigned long long)hi1 << 20));
   }
-  if (!in0 && !in1 && bin >= 0) {
-    atomicAdd(&hist[bin], w);
-    if (cnt) atomicAdd(&cnt[bin], 1u);
-  }
+  if (!in0 && !in1 && bin >= 0) atomicAdd(&hist[bin], w);
 }
 
 // Over kBins mass bins (shared memory), find the bin where the running mass,
@@ -347,7 +380,7 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 // entries ordered before it (its rank), the masses are placed in rank order
 // and scanned, and the cut is the first entry whose running mass reaches T.
 template <class View>
-__device__ __forceinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
+__device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
                                                DecSmem& sm) {
   const int tid = threadIdx.x;
   unsigned long long* k64s = sm.hist;                        // [n] order keys
@@ -402,19 +435,15 @@ __device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, in
 // asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
 // Every thread returns the same value.
 template <class View>
-__device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, const View& E, int64_t n, uint32_t kmin,
-                                         DecSmem& sm, int step) {
+__device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const View& E, int64_t n, uint32_t kmin,
+                                         DecSmem& sm, int h, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
-  stamp(a, 64 + 8 * step);
   if (a.p_all) return ~0ull;
   const float m = desc_key_value(kmin);
   if (n <= kDecThreads) return select_cut_small(a, E, n, m, sm);
 
   // coarse histogram of the masses (and counts); total mass Z and the target T = ceil(p Z)
-  for (int i = tid; i < kBins; i += kDecThreads) {
-    sm.hist[i] = 0ull;
-    sm.cnt[i] = 0u;
-  }
+  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
   const int n32 = int(n);
   const int wseg = (n32 + kDecWarps - 1) / kDecWarps;               // entries per warp, contiguous
@@ -435,7 +464,7 @@ __device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, co
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, sm.cnt, bin[u], w[u]);
+    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, bin[u], w[u]);
   }
   __syncthreads();
   unsigned long long Z = 0;
@@ -447,7 +476,7 @@ __device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, co
     block_scan_u64(local, sm.red64, &Z);
   }
   const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);  // keep while mass before < T
-  stamp(a, 65 + 8 * step);
+  if (tid == 0) trace_hs(a, h, step, 8, now_ns());
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
@@ -455,47 +484,44 @@ __device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, co
   // keys of coarse bin cb form the contiguous range [klo, khi)
   const unsigned long long klo = first_key_at_least(kmin, cb, cbin);
   const unsigned long long khi = cb + 1 < kBins ? first_key_at_least(uint32_t(klo), cb + 1, cbin) : 0x100000000ull;
+  if (tid == 0) trace_hs(a, h, step, 9, now_ns());
 
-  // fine histogram inside the cut coarse bin, unless that bin is small already
-  const bool use_fine = sm.cnt[cb] > 32u;
-  unsigned long long flo = klo, fhi = khi;  // key range of the entries around the cut
-  unsigned long long below2 = below;
-  if (use_fine) {
-    for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
-    __syncthreads();
-    for (int base = wlo; base < whi; base += 32 * U) {
-      int bin[U];
-      unsigned long long w[U];
+  // fine histogram inside the cut coarse bin: the fine cut bin's key range
+  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
+  __syncthreads();
+  for (int base = wlo; base < whi; base += 32 * U) {
+    int bin[U];
+    unsigned long long w[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = base + 32 * u + lane;
-        bin[u] = -1;
-        w[u] = 0;
-        if (i < whi) {
-          const uint32_t k = E.key(i);
-          if (k >= klo && k < khi) {
-            bin[u] = fine_bin(entry_gap(m, k), cb);
-            w[u] = entry_mass(m, k);
-          }
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      bin[u] = -1;
+      w[u] = 0;
+      if (i < whi) {
+        const uint32_t k = E.key(i);
+        if (k >= klo && k < khi) {
+          bin[u] = fine_bin(entry_gap(m, k), cb);
+          w[u] = entry_mass(m, k);
         }
       }
-#pragma unroll
-      for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, nullptr, bin[u], w[u]);
     }
-    __syncthreads();
-    int fb;
-    fb = find_cut_bin(sm, below, T, &below2);
-    if (fb < 0) return ~0ull;
-    auto fbin = [&](uint32_t k) {
-      const float x = entry_gap(m, k);
-      return coarse_bin(x) > cb ? kBins : fine_bin(x, cb);
-    };
-    flo = first_key_at_least(uint32_t(klo), fb, fbin);
-    fhi = fb + 1 < kBins ? first_key_at_least(uint32_t(flo), fb + 1, fbin) : khi;
-    if (fhi > khi) fhi = khi;
+#pragma unroll
+    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, bin[u], w[u]);
   }
+  __syncthreads();
+  if (tid == 0) trace_hs(a, h, step, 10, now_ns());
+  unsigned long long below2;
+  const int fb = find_cut_bin(sm, below, T, &below2);
+  if (fb < 0) return ~0ull;
+  auto fbin = [&](uint32_t k) {
+    const float x = entry_gap(m, k);
+    return coarse_bin(x) > cb ? kBins : fine_bin(x, cb);
+  };
+  const unsigned long long flo = first_key_at_least(uint32_t(klo), fb, fbin);
+  unsigned long long fhi = fb + 1 < kBins ? first_key_at_least(uint32_t(flo), fb + 1, fbin) : khi;
+  if (fhi > khi) fhi = khi;
   auto in_cut = [&](uint32_t k) { return k >= flo && k < fhi; };
-  stamp(a, 66 + 8 * step);
+  if (tid == 0) trace_hs(a, h, step, 11, now_ns());
 
   // gather the entries around the cut
   if (tid == 0) sm.bcast32[1] = 0;
@@ -511,8 +537,11 @@ __device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, co
     }
   }
   __syncthreads();
-  stamp(a, 67 + 8 * step);
   const int cnt = sm.bcast32[1];
+  if (tid == 0) {
+    trace_hs(a, h, step, 12, now_ns());
+    trace_hs(a, h, step, 13, (unsigned long long)cnt);
+  }
   if (cnt <= 32) {
     if (tid < 32) {
       unsigned long long k = tid < cnt ? sm.cut_key[tid] : ~0ull;
@@ -597,6 +626,289 @@ __device__ __forceinline__ unsigned long long select_cut(const DecodeArgs& a, co
   return prefix;
 }
 
+// ---------------------------------------------------------------- anchored histograms
+// The scoring warps of step s >= 1 add every new entry's mass to a histogram
+// of the head's step, anchored at r = the largest estimate of step s-1 (known
+// before step s is scored): bin floor(32 x) of x = (r - e) + kAnchorSpan (the
+// last bin open), mass exp(-(x - bin/32)) as a 2^-40 fixed-point integer
+// (<= 2^40, exact order-independent sums).  A bin's mass relative to the
+// anchor is its integer sum times anchored_scale(bin).  An estimate above
+// r + kAnchorSpan sets the step's overflow flag; the select then recomputes
+// the masses relative to the step's own max, as it does when r lies more
+// than kAnchorFar above that max (the fixed point would lose the masses).
+constexpr float kAnchorSpan = 8.f;
+constexpr float kAnchorFar = 16.f;
+__device__ __forceinline__ int anchored_bin(float r, uint32_t key, unsigned long long* w, float* t) {
+  const float x = __fadd_rn(__fsub_rn(r, desc_key_value(key)), kAnchorSpan);
+  if (!(x >= 0.f)) return -1;
+  const int b = min(int(__fmul_rn(x, kBinScale)), kBins - 1);
+  const float tt = __fsub_rn(x, __fmul_rn(float(b), 1.f / kBinScale));
+  *t = tt;
+  *w = __float2ull_rn(__fmul_rn(expf(-tt), 1099511627776.0f));  // 2^40
+  return b;
+}
+__device__ __forceinline__ double anchored_scale(int b) {
+  return exp(double(kAnchorSpan) - double(b) / double(kBinScale)) * 0x1p-40;
+}
+// sub-bin of t = x - bin/32 inside its bin: 1024 sub-bins of 1/32768, the last open
+__device__ __forceinline__ int anchored_fine(float t) {
+  return min(int(__fmul_rn(t, kBinScale * float(kBins))), kBins - 1);
+}
+
+// Block-wide exclusive scan of one double per thread, in a fixed order (so
+// that every run gives the same sums); *total = the block total.
+__device__ __forceinline__ double block_scan_f64(double v, double* red, double* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  double x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  double ex = __shfl_up_sync(0xffffffffu, x, 1);
+  if (lane == 0) ex = 0.0;
+  if (lane == 31) red[wid] = x;
+  __syncthreads();
+  double base = 0.0, tot = 0.0;
+  for (int w = 0; w < kDecWarps; ++w) {
+    if (w < wid) base += red[w];
+    tot += red[w];
+  }
+  __syncthreads();
+  *total = tot;
+  return base + ex;
+}
+
+// First of kBins per-thread-blocked bin masses (BPT consecutive bins per
+// thread, exclusive prefix `before`) at which base + running mass reaches T:
+// returns the bin and the mass before it (all threads); -1 if none does.
+__device__ __forceinline__ int find_cut_bin_f64(DecSmem& sm, const double* m, double before, double T,
+                                                double* below_out) {
+  constexpr int BPT = kBins / kDecThreads;
+  const int tid = threadIdx.x;
+  if (tid == 0) sm.bcast32[0] = -1;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    if (before < T && before + m[k] >= T) {
+      sm.bcast32[0] = tid * BPT + k;
+      sm.bcast64[0] = (unsigned long long)__double_as_longlong(before);
+    }
+    before += m[k];
+  }
+  __syncthreads();
+  const int bin = sm.bcast32[0];
+  *below_out = __longlong_as_double((long long)sm.bcast64[0]);
+  __syncthreads();
+  return bin;
+}
+
+// The cut of a step from its anchored histogram (global, kBins sums): the
+// coarse cut bin from the histogram alone, then one pass over the keys for
+// the fine histogram of that bin's members, one more to gather the members of
+// the fine cut bin, which are ordered by (e desc, start asc).  Every thread
+// returns the same value.
+template <class View>
+__device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs& a, const View& E, int64_t n,
+                                                                  float r, const unsigned long long* ghist,
+                                                                  DecSmem& sm, int h, int step) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int BPT = kBins / kDecThreads;
+  double* red = reinterpret_cast<double*>(sm.red64);
+  const double p = ldexp(double(a.p_mant), -a.p_shift);
+  double mb[BPT], loc = 0.0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    const int bin = tid * BPT + k;
+    mb[k] = double(__ldcg(ghist + bin)) * anchored_scale(bin);
+    loc += mb[k];
+  }
+  double Z;
+  const double before = block_scan_f64(loc, red, &Z);
+  const double T = p * Z;
+  double below_c;
+  const int cb = find_cut_bin_f64(sm, mb, before, T, &below_c);
+  if (cb < 0) return ~0ull;  // rounding kept T out of reach: keep everything
+  const double sc = anchored_scale(cb);
+  if (tid == 0) trace_hs(a, h, step, 8, now_ns());
+
+  // fine histogram of the cut bin's members (exact integer masses)
+  for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
+  __syncthreads();
+  const int n32 = int(n);
+  const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
+  const int wlo = min(n32, (tid >> 5) * wseg), whi = min(n32, wlo + wseg);
+  constexpr int U = 4;
+  for (int base = wlo; base < whi; base += 32 * U) {
+    int fb[U];
+    unsigned long long w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      fb[u] = -1;
+      w[u] = 0;
+      if (i < whi) {
+        float t;
+        if (anchored_bin(r, E.key(i), &w[u], &t) == cb) fb[u] = anchored_fine(t);
+        else w[u] = 0;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, fb[u], w[u]);
+  }
+  __syncthreads();
+  double fm[BPT];
+  loc = 0.0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    fm[k] = double(sm.hist[tid * BPT + k]) * sc;
+    loc += fm[k];
+  }
+  double FZ;
+  const double fbefore = block_scan_f64(loc, red, &FZ);
+  double below_f;
+  int fbin = find_cut_bin_f64(sm, fm, below_c + fbefore, T, &below_f);
+  if (fbin < 0) {  // rounding: the sub-bins fell short of T; take the last non-empty one
+    if (tid == 0) sm.bcast32[2] = -1;
+    __syncthreads();
+    for (int k = 0; k < BPT; ++k)
+      if (sm.hist[tid * BPT + k] != 0ull) atomicMax(&sm.bcast32[2], tid * BPT + k);
+    __syncthreads();
+    fbin = sm.bcast32[2];
+    if (fbin < 0) return ~0ull;
+    unsigned long long pre = 0;
+    for (int k = 0; k < fbin; ++k) pre += sm.hist[k];
+    below_f = below_c + double(pre) * sc;
+    __syncthreads();
+  }
+  if (tid == 0) trace_hs(a, h, step, 10, now_ns());
+
+  // gather the members of the fine cut bin
+  auto member = [&](uint32_t k, unsigned long long* w) {
+    float t;
+    return anchored_bin(r, k, w, &t) == cb && anchored_fine(t) == fbin;
+  };
+  if (tid == 0) sm.bcast32[1] = 0;
+  __syncthreads();
+  for (int i = tid; i < n32; i += kDecThreads) {
+    const uint32_t k = E.key(i);
+    unsigned long long w;
+    if (member(k, &w)) {
+      const int sl = atomicAdd(&sm.bcast32[1], 1);
+      if (sl < 32) {
+        sm.cut_key[sl] = entry_key64(a, Entry{k, E.code(i)});
+        sm.cut_w[sl] = w;
+      }
+    }
+  }
+  __syncthreads();
+  const int cnt = sm.bcast32[1];
+  if (tid == 0) {
+    trace_hs(a, h, step, 12, now_ns());
+    trace_hs(a, h, step, 13, (unsigned long long)cnt);
+  }
+  if (cnt <= 32) {
+    if (tid < 32) {
+      unsigned long long k = tid < cnt ? sm.cut_key[tid] : ~0ull;
+      unsigned long long w = tid < cnt ? sm.cut_w[tid] : 0ull;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, stride);
+          const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+          const bool up = ((tid & size) == 0);
+          const bool lower = ((tid & stride) == 0);
+          const bool swap = (up == lower) ? (ok < k) : (ok > k);
+          if (swap) {
+            k = ok;
+            w = ow;
+          }
+        }
+      }
+      unsigned long long c = w;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, c, off);
+        if (tid >= off) c += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, tid < cnt && below_f + double(c) * sc >= T);
+      const int first = hit ? __ffs(hit) - 1 : max(cnt - 1, 0);
+      const unsigned long long cut = __shfl_sync(0xffffffffu, k, first);
+      if (tid == 0) sm.bcast64[1] = cnt > 0 ? cut : ~0ull;
+    }
+    __syncthreads();
+    return sm.bcast64[1];
+  }
+  // Many members share the fine cut bin (exact ties or near-ties): radix
+  // select on the 64-bit order key, 8 bits per pass, over those members.
+  unsigned long long prefix = 0, acc = 0;  // acc: exact mass of the members before the prefix's range
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = tid; i < 256; i += kDecThreads) sm.hist[i] = 0ull;
+    __syncthreads();
+    for (int i = tid; i < n32; i += kDecThreads) {
+      const uint32_t k = E.key(i);
+      unsigned long long w;
+      if (!member(k, &w)) continue;
+      const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
+      if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
+      atomicAdd(&sm.hist[(k64 >> shift) & 255], w);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      unsigned long long loc8 = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) loc8 += sm.hist[tid * 8 + k];
+      unsigned long long c = loc8;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, c, off);
+        if (tid >= off) c += y;
+      }
+      unsigned long long bef = acc + c - loc8;
+      int digit = -1, last = -1;
+      unsigned long long dbef = 0, lbef = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const unsigned long long hb = sm.hist[tid * 8 + k];
+        if (digit < 0 && below_f + double(bef + hb) * sc >= T) {
+          digit = tid * 8 + k;
+          dbef = bef;
+        }
+        if (hb) {
+          last = tid * 8 + k;
+          lbef = bef;
+        }
+        bef += hb;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, digit >= 0);
+      const unsigned any = __ballot_sync(0xffffffffu, last >= 0);
+      int dg;
+      unsigned long long db;
+      if (hit) {
+        const int src = __ffs(hit) - 1;
+        dg = __shfl_sync(0xffffffffu, digit, src);
+        db = __shfl_sync(0xffffffffu, dbef, src);
+      } else {  // rounding: fall back to the last non-empty digit
+        const int src = any ? 31 - __clz(any) : 31;
+        dg = __shfl_sync(0xffffffffu, last, src);
+        db = __shfl_sync(0xffffffffu, lbef, src);
+        if (!any) { dg = 255; db = acc; }
+      }
+      if (tid == 0) {
+        sm.bcast64[2] = prefix | (uint64_t(dg) << shift);
+        sm.bcast64[3] = db;
+      }
+    }
+    __syncthreads();
+    prefix = sm.bcast64[2];
+    acc = sm.bcast64[3];
+    __syncthreads();
+  }
+  return prefix;
+}
+
 // Grid barrier over all CTAs of the cooperative launch: a 64-bit arrival
 // counter that only grows; barrier k of a launch completes when it reaches
 // base + k * gridDim.x (the host tracks the base).  Returns true for every
@@ -625,19 +937,19 @@ __device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm, unsi
   return sm.fail != 0;
 }
 
-// Inclusive prefix of per-head counts held in sm.pref[1..nh] (pref[0] = 0); returns the total.
+// Inclusive prefix of per-head counts held in sm.pref()[1..nh] (pref[0] = 0); returns the total.
 __device__ __forceinline__ long long build_prefix(DecSmem& sm, int nh) {
   long long carry = 0;
   for (int base = 0; base < nh; base += kDecThreads) {
     const int i = base + threadIdx.x;
-    const unsigned long long v = i < nh ? (unsigned long long)sm.pref[1 + i] : 0ull;
+    const unsigned long long v = i < nh ? (unsigned long long)sm.pref()[1 + i] : 0ull;
     unsigned long long tot;
     const unsigned long long ex = block_scan_u64(v, sm.red64, &tot);
-    if (i < nh) sm.pref[1 + i] = carry + (long long)(ex + v);
+    if (i < nh) sm.pref()[1 + i] = carry + (long long)(ex + v);
     carry += (long long)tot;
     __syncthreads();
   }
-  if (threadIdx.x == 0) sm.pref[0] = 0;
+  if (threadIdx.x == 0) sm.pref()[0] = 0;
   __syncthreads();
   return carry;
 }
@@ -647,7 +959,7 @@ __device__ __forceinline__ int owner_of(const DecSmem& sm, int nh, long long i) 
   int lo = 0, hi = nh - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (sm.pref[mid] <= i) lo = mid; else hi = mid - 1;
+    if (sm.pref()[mid] <= i) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -676,30 +988,131 @@ __device__ __forceinline__ void cp_async_wait(int pending) {
   }
 }
 
+// ---------------------------------------------------------------- bulk copies
+// A node record is fetched with one bulk copy (cp.async.bulk, no multicast)
+// issued by one lane; completion is counted in bytes on a per-slot mbarrier.
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return unsigned(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Orders this thread's earlier shared-memory reads before later bulk-copy writes.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---------------------------------------------------------------- tensor-core estimate (bf16)
+// The q operand of the estimate, as B fragments of m16n8k16 (column 0 = q, the
+// other columns zero).  The k order of each k-step is a permutation of the
+// dimensions chosen so that a lane's A words are whole 16-byte chunks of a
+// record row: lane (g = lane/4, t = lane%4) reads chunks t*CPL .. t*CPL+CPL-1
+// of its rows; chunk c (8 dims) feeds k-steps 2c' and 2c'+1 (c' = c - t*CPL),
+// dims 0-3 the first and 4-7 the second, as (k 2t, 2t+1) and (k 2t+8, 2t+9).
+// The same permutation applied to q leaves the dot product unchanged.
+template <int D>
+__device__ __forceinline__ void q_fragments(const __nv_bfloat16* q, uint32_t (&qf)[D / 16][2], int lane) {
+  constexpr int CPL = D / 32;
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (g == 0) v = *reinterpret_cast<const uint4*>(q + (t * CPL + c) * 8);
+    qf[2 * c][0] = v.x;
+    qf[2 * c][1] = v.y;
+    qf[2 * c + 1][0] = v.z;
+    qf[2 * c + 1][1] = v.w;
+  }
+}
+
+// e = max_j (b_j + q.mu_j / sqrt d) of a bf16 record in shared memory: the
+// R x D slope rows times q on the tensor cores (fp32 accumulation), 16 rows
+// per m-tile; every lane returns the estimate.
+template <int D>
+__device__ __forceinline__ float score_record_mma(const unsigned char* rec, int R, float inv_sqrt_d,
+                                                  const uint32_t (&qf)[D / 16][2], int lane) {
+  constexpr int CPL = D / 32;
+  const int g = lane >> 2, t = lane & 3;
+  const float* bias = reinterpret_cast<const float*>(rec + size_t(R) * D * 2);
+  float best = -INFINITY;
+  for (int m0 = 0; m0 < R; m0 += 16) {
+    const int r0 = min(m0 + g, R - 1), r1 = min(m0 + g + 8, R - 1);  // rows past R: any valid row, masked below
+    const unsigned char* p0 = rec + size_t(r0) * D * 2 + t * CPL * 16;
+    const unsigned char* p1 = rec + size_t(r1) * D * 2 + t * CPL * 16;
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const uint4 x0 = *reinterpret_cast<const uint4*>(p0 + c * 16);
+      const uint4 x1 = *reinterpret_cast<const uint4*>(p1 + c * 16);
+      const uint32_t a0[4] = {x0.x, x1.x, x0.y, x1.y};
+      const uint32_t a1[4] = {x0.z, x1.z, x0.w, x1.w};
+      mma_bf16_16816(c0, a0, qf[2 * c]);
+      mma_bf16_16816(c1, a1, qf[2 * c + 1]);
+    }
+    if (t == 0) {
+      const int j0 = m0 + g, j1 = m0 + g + 8;
+      if (j0 < R) best = fmaxf(best, fmaf(c0[0] + c1[0], inv_sqrt_d, bias[j0]));
+      if (j1 < R) best = fmaxf(best, fmaf(c0[2] + c1[2], inv_sqrt_d, bias[j1]));
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+  return best;
+}
+
 // Estimate of a node whose record sits in shared memory (whole warp; the
-// lane's q slice covers elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR).
+// lane's q slice covers elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR).  Up
+// to kG reference rows per lane are in flight at once: their partial dot
+// products are formed independently, then reduced over the CPR lanes of each
+// row together, so that the shuffles of different rows overlap.  The
+// arithmetic (FMA order inside a lane, the butterfly over lanes) is the same
+// for every row count.
 template <typename T, int D>
 __device__ __forceinline__ float score_record_smem(const unsigned char* rec, int R, float inv_sqrt_d,
                                                    const float* qs, int lane) {
   constexpr int EPC = 16 / sizeof(T);
   constexpr int CPR = D * sizeof(T) / 16;
   constexpr int RPI = 32 / CPR;
+  constexpr int kG = 8;
   const float* bias = reinterpret_cast<const float*>(rec + size_t(R) * D * sizeof(T));
   const int sub = lane / CPR, cl = lane % CPR;
   float best = -INFINITY;
-  for (int j0 = 0; j0 < R; j0 += RPI) {
-    const int j = j0 + sub;
-    float part = 0.f;
-    if (j < R) {
-      const uint4 v = *reinterpret_cast<const uint4*>(rec + (size_t(j) * CPR + cl) * 16);
-      float x[EPC];
-      unpack16<T>(v, x);
+  for (int j0 = 0; j0 < R; j0 += RPI * kG) {
+    float part[kG];
 #pragma unroll
-      for (int i = 0; i < EPC; ++i) part = fmaf(x[i], qs[i], part);
+    for (int g = 0; g < kG; ++g) {
+      const int j = j0 + g * RPI + sub;
+      part[g] = 0.f;
+      if (j < R) {
+        const uint4 v = *reinterpret_cast<const uint4*>(rec + (size_t(j) * CPR + cl) * 16);
+        float x[EPC];
+        unpack16<T>(v, x);
+#pragma unroll
+        for (int i = 0; i < EPC; ++i) part[g] = fmaf(x[i], qs[i], part[g]);
+      }
     }
 #pragma unroll
-    for (int off = CPR / 2; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (j < R) best = fmaxf(best, fmaf(part, inv_sqrt_d, bias[j]));
+    for (int off = CPR / 2; off > 0; off >>= 1) {
+#pragma unroll
+      for (int g = 0; g < kG; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
+    }
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int j = j0 + g * RPI + sub;
+      if (j < R) best = fmaxf(best, fmaf(part[g], inv_sqrt_d, bias[j]));
+    }
   }
 #pragma unroll
   for (int off = 16; off >= CPR; off >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
@@ -707,7 +1120,7 @@ __device__ __forceinline__ float score_record_smem(const unsigned char* rec, int
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int EPC = 16 / sizeof(T);
   constexpr int CPR = D * sizeof(T) / 16;
   constexpr int KPW = 32 / CPR;  // keys per warp pass in the attention loop
@@ -717,244 +1130,354 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   const int nh = a.nheads;
   const int b = a.t.block;
   const int R = a.t.refs;
-  const long long gwarp = (long long)blockIdx.x * kDecWarps + wid;
-  const long long nwarps = (long long)gridDim.x * kDecWarps;
   unsigned long long bar_target = a.bar_base;
   auto ws = [&](int h) { return a.ws + uint64_t(h) * a.ws_per_bh; };
-  auto sel = [&](int h) { return reinterpret_cast<Entry*>(ws(h)); };
-  auto cand = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + a.cap_sel * sizeof(Entry)); };
-  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + a.cap_sel * (sizeof(Entry) + 4)); };
-  auto hstate = [&](int h) {
-    return reinterpret_cast<HeadState*>(ws(h) + a.cap_sel * (sizeof(Entry) + 4) + a.cap_list * 4);
+  // per-head workspace: step keys [2][cap4], step codes [2][cap4] (parity buffers: step s in s & 1),
+  // anchored histograms [2][kBins], kept entries of the last select [cap4], kept leaves [cap_list];
+  // leaf bitmaps live in the flow state
+  const int64_t cap4 = (a.cap_sel + 3) & ~int64_t(3);
+  auto keysP = [&](int h, int par) { return reinterpret_cast<uint32_t*>(ws(h) + par * cap4 * 4); };
+  auto codesP = [&](int h, int par) { return reinterpret_cast<uint32_t*>(ws(h) + (2 + par) * cap4 * 4); };
+  auto histP = [&](int h, int par) {
+    return reinterpret_cast<unsigned long long*>(ws(h) + 4 * cap4 * 4 + par * kBins * 8);
+  };
+  auto keptl = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 4 * cap4 * 4 + 2 * kBins * 8); };
+  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 5 * cap4 * 4 + 2 * kBins * 8); };
+  const int64_t bm_words = decode_bitmap_words(a.cap_sel);
+  auto hstate = [&](int h) { return reinterpret_cast<HeadState*>(a.flow) + h; };
+  auto bitmap = [&](int h) {
+    return reinterpret_cast<uint32_t*>(a.flow + size_t(nh) * sizeof(HeadState)) + h * bm_words;
   };
   auto q_slice = [&](int h, float* qs) {
     const T* q = static_cast<const T*>(a.Q) + size_t(h) * D + (lane % CPR) * EPC;
     unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
   };
   const int rec_bytes = int(a.t.rec_bytes);
-  const int rec_chunks = rec_bytes / 16;
-  const int nslot = max(1, min(kMaxSlots, (kUnionBytes / kDecWarps) / rec_bytes));
+  // scoring ring: nslot record slots per warp below the prefix area; warps past
+  // score_warps (only when a record is larger than a warp's share) do not score
+  const int nslot = max(1, min(kMaxSlots, (kPrefOff / kDecWarps) / rec_bytes));
+  const int score_warps = min(kDecWarps, kPrefOff / (nslot * rec_bytes));
   unsigned char* ring = sm.u + size_t(wid) * nslot * rec_bytes;
 
+  const bool routed = a.n_steps > 0 && a.n_roots > 0;
   stamp(a, 0);
-  for (int step = 0; step < a.n_steps; ++step) {
-    // ---------------- score (all CTAs)
-    for (int i = tid; i < nh; i += kDecThreads) {
-      long long c = a.n_roots;
-      if (step > 0) c = min64(max64(__ldcg(&hstate(i)->n_cand), 0), a.cap_sel);
-      sm.pref[1 + i] = c;
+  if (routed) {
+    // Step loop, in lock step over all heads: a scoring phase (all warps) makes
+    // step s's entries, a grid barrier, a select phase (one CTA per head) keeps
+    // a prefix of them, a grid barrier.  Step s's entries are the roots (s = 0,
+    // root i at position i) or the children of step s-1's kept non-leaves, at
+    // positions reserved per warp batch with one atomic add per head (their
+    // order varies from run to run; nothing downstream depends on it).  The
+    // phase after the last select only records the kept leaves.
+    constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
+    if (lane == 0) {
+      for (int k = 0; k < nslot; ++k) mbar_init(&sm.mbar[wid][k], 1);
+      mbar_init_fence();
     }
-    __syncthreads();
-    const long long total = build_prefix(sm, nh);
-    {
-      const long long i0 = gwarp * total / nwarps, i1 = (gwarp + 1) * total / nwarps;
-      const long long cnt = i1 - i0;
-      // codes of the next 32 items, one per lane
-      uint32_t code_reg = 0;
-      int head_reg = 0;
-      auto fetch_codes = [&](long long k0) {
-        const long long it = i0 + k0 + lane;
-        code_reg = 0;
-        head_reg = 0;
-        if (k0 + lane < cnt) {
-          const int h = owner_of(sm, nh, it);
-          const long long pos = it - sm.pref[h];
-          uint32_t code = step == 0 ? root_code(a, pos) : __ldcg(cand(h) + pos);
-          if (!valid_code(a, code)) {
-            raise_status(a.t.status, ZHA_ERR_CAPACITY);
-            code = 0;  // marks an item to skip
+    __syncwarp();
+    unsigned long long n_issued = 0, n_done = 0;  // records through this warp's ring so far (slot k % nslot)
+    float qs[EPC];
+    uint32_t qf[D / 16][2];
+    int qhead = -1;
+    const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
+    const long long nwarps = (long long)gridDim.x * score_warps;
+    for (int s = 0; s <= a.n_steps; ++s) {
+      const int par = s & 1;
+      // ---------------- scoring phase: units = roots (s = 0) or the kept entries of step s-1
+      for (int i = tid; i < nh; i += kDecThreads)
+        sm.pref()[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hstate(i)->kept), 0), a.cap_sel);
+      __syncthreads();
+      const long long total = build_prefix(sm, nh);
+      stamp(a, 2 + 2 * s);
+      const long long u0 = gwarp < 0 ? 0 : total * gwarp / nwarps;
+      const long long u1 = gwarp < 0 ? 0 : total * (gwarp + 1) / nwarps;
+      int cur_h = -1;           // lane 0: head of the pending min-key update
+      uint32_t cur_kmin = 0xffffffffu;
+      int cur_ovf = 0;
+      int ah = -1;              // head whose anchor is loaded
+      float anchor = 0.f;
+      for (long long ub = u0; ub < u1; ub += 32) {
+        // one unit per lane: its head, its first output position, its code
+        const long long u = ub + lane;
+        int uh = 0;
+        long long upos = 0;
+        uint32_t ucode = 0;
+        bool has = false;  // the unit makes records (a root, or a kept non-leaf)
+        if (u < u1) {
+          uh = owner_of(sm, nh, u);
+          const long long k = u - sm.pref()[uh];
+          if (s == 0) {
+            ucode = root_code(a, k);
+            upos = k;
+            has = valid_code(a, ucode);
+          } else {
+            const uint32_t idx = __ldcg(keptl(uh) + k);
+            const uint32_t code = idx < uint32_t(a.cap_sel) ? __ldcg(codesP(uh, par ^ 1) + idx) : 0u;
+            if (valid_code(a, code)) {
+              if (code_level(code) == 1) {
+                atomicOr(bitmap(uh) + (code_index(code) >> 5), 1u << (code_index(code) & 31u));
+              } else {
+                ucode = code;
+                has = true;
+              }
+            }
           }
-          code_reg = code;
-          head_reg = h;
         }
-      };
-      long long issued = 0, done = 0;
-      int qhead = -1;
-      float qs[EPC];
-      if (cnt > 0) fetch_codes(0);
-      while (done < cnt) {
-        // keep up to nslot records in flight
-        while (issued < cnt && issued - done < nslot && (issued >> 5) == (done >> 5)) {
-          const uint32_t code = __shfl_sync(0xffffffffu, code_reg, int(issued & 31));
-          const int h = __shfl_sync(0xffffffffu, head_reg, int(issued & 31));
-          unsigned char* slot = ring + size_t(issued % nslot) * rec_bytes;
-          if (code != 0) {
-            const int kvh = (h % a.t.hq) / a.t.group;
-            const unsigned char* src =
-                reinterpret_cast<const unsigned char*>(a.t.rec(code_level(code), kvh, code_index(code)));
-            for (int c = lane; c < rec_chunks; c += 32) cp_async16(slot + c * 16, src + c * 16);
+        if (s >= 1) {  // positions: one reservation per head segment of the batch
+          unsigned todo = __ballot_sync(0xffffffffu, has);
+          while (todo) {
+            const int l0 = __ffs(todo) - 1;
+            const int h0 = __shfl_sync(0xffffffffu, uh, l0);
+            const unsigned seg = __ballot_sync(0xffffffffu, has && uh == h0);
+            long long bs = 0;
+            if (lane == l0) {
+              const long long need = (long long)__popc(seg) * b;
+              bs = (long long)atomicAdd(reinterpret_cast<unsigned long long*>(&hstate(h0)->n[par]),
+                                        (unsigned long long)need);
+              if (bs + need > a.cap_sel) {
+                raise_status(a.t.status, ZHA_ERR_CAPACITY);
+                bs = -1;
+              }
+            }
+            bs = __shfl_sync(0xffffffffu, bs, l0);
+            if (has && uh == h0) {
+              upos = bs + (long long)__popc(seg & ((1u << lane) - 1u)) * b;
+              if (bs < 0) has = false;
+            }
+            todo &= ~seg;
           }
-          cp_async_commit();
-          ++issued;
         }
-        const uint32_t code = __shfl_sync(0xffffffffu, code_reg, int(done & 31));
-        const int h = __shfl_sync(0xffffffffu, head_reg, int(done & 31));
-        if (code != 0 && h != qhead) {  // load the head's query while the record is in flight
-          q_slice(h, qs);
-          qhead = h;
+        const unsigned mhas = __ballot_sync(0xffffffffu, has);
+        if (!mhas) continue;
+        const int per = s == 0 ? 1 : b;  // records per unit
+        const int items = __popc(mhas) * per;
+        // item k: record (k % per) of the (k / per)-th unit with records, in lane order
+        struct Cursor {
+          unsigned rem;
+          int child;
+        };
+        struct Item {
+          int h;
+          long long pos;
+          uint32_t code;
+        };
+        auto next_item = [&](Cursor& cur) -> Item {  // the whole warp calls it, in item order
+          const int pl = __ffs(cur.rem) - 1;
+          Item it;
+          it.h = __shfl_sync(0xffffffffu, uh, pl);
+          it.pos = __shfl_sync(0xffffffffu, upos, pl) + cur.child;
+          const uint32_t pc = __shfl_sync(0xffffffffu, ucode, pl);
+          it.code = s == 0 ? pc : node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(cur.child));
+          if (++cur.child == per) {
+            cur.child = 0;
+            cur.rem &= cur.rem - 1u;
+          }
+          return it;
+        };
+        Cursor cur_i{mhas, 0};
+        Item slot_item[kMaxSlots];
+        int issued = 0, done = 0;
+        while (done < items) {
+          while (issued < items && issued - done < nslot) {
+            const Item it = next_item(cur_i);
+            const int sl = int(n_issued % unsigned(nslot));
+            unsigned char* slot = ring + size_t(sl) * rec_bytes;
+            if (lane == 0) {
+              fence_proxy_async();  // the slot's last reads (generic proxy) before the copy writes it
+              const int kvh = (it.h % a.t.hq) / a.t.group;
+              bulk_load(slot, a.t.rec(code_level(it.code), kvh, code_index(it.code)), unsigned(rec_bytes),
+                        &sm.mbar[wid][sl]);
+            }
+#pragma unroll
+            for (int k = 0; k < kMaxSlots; ++k)
+              if (k == issued - done) slot_item[k] = it;
+            ++issued;
+            ++n_issued;
+          }
+          const int sl = int(n_done % unsigned(nslot));
+          const unsigned parity = unsigned((n_done / unsigned(nslot)) & 1ull);
+          {
+            long long it = 0;
+            while (!mbar_try_wait(&sm.mbar[wid][sl], parity)) {
+              if (++it > a.spin_limit) {  // a copy that never lands: report, then give it one more bound
+                if (lane == 0) raise_status(a.t.status, ZHA_ERR_TIMEOUT);
+                if (it > 2 * a.spin_limit) break;
+              }
+            }
+          }
+          __syncwarp();
+          const Item it = slot_item[0];
+#pragma unroll
+          for (int k = 0; k + 1 < kMaxSlots; ++k) slot_item[k] = slot_item[k + 1];
+          if (it.h != qhead) {
+            if constexpr (kMma) q_fragments<D>(static_cast<const __nv_bfloat16*>(a.Q) + size_t(it.h) * D, qf, lane);
+            else q_slice(it.h, qs);
+            qhead = it.h;
+          }
+          const unsigned char* rec = ring + size_t(sl) * rec_bytes;
+          float e;
+          if constexpr (kMma) e = score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
+          else e = score_record_smem<T, D>(rec, R, a.t.inv_sqrt_d, qs, lane);
+          if (lane == 0) {
+            const uint32_t key = desc_key(e);
+            keysP(it.h, par)[it.pos] = key;
+            codesP(it.h, par)[it.pos] = it.code;
+            if (it.h != cur_h) {  // flush the previous head's min key and overflow flag
+              if (cur_h >= 0) {
+                atomicMax(&hstate(cur_h)->kinv[par], ~cur_kmin);
+                if (cur_ovf) atomicOr(&hstate(cur_h)->ovf[par], 1);
+              }
+              cur_h = it.h;
+              cur_kmin = 0xffffffffu;
+              cur_ovf = 0;
+            }
+            cur_kmin = min(cur_kmin, key);
+            if (s >= 1) {
+              if (it.h != ah) {
+                anchor = __ldcg(&hstate(it.h)->anchor);
+                ah = it.h;
+              }
+              unsigned long long w;
+              float t;
+              const int bin = anchored_bin(anchor, key, &w, &t);
+              if (bin < 0) cur_ovf = 1;
+              else atomicAdd(histP(it.h, par) + bin, w);
+            }
+          }
+          __syncwarp();
+          ++done;
+          ++n_done;
         }
-        cp_async_wait(int(issued - done - 1));
-        __syncwarp();
-        if (code != 0) {
-          const float e = score_record_smem<T, D>(ring + size_t(done % nslot) * rec_bytes, R, a.t.inv_sqrt_d, qs,
-                                                  lane);
-          if (lane == 0) sel(h)[i0 + done - sm.pref[h]] = Entry{desc_key(e), code};
-        }
-        __syncwarp();
-        ++done;
-        if ((done & 31) == 0 && done < cnt) fetch_codes(done);
       }
-    }
-    stamp(a, 1 + 4 * step);
-    if (grid_sync(a, sm, bar_target)) return;
-    stamp(a, 2 + 4 * step);
+      if (lane == 0 && cur_h >= 0) {
+        atomicMax(&hstate(cur_h)->kinv[par], ~cur_kmin);
+        if (cur_ovf) atomicOr(&hstate(cur_h)->ovf[par], 1);
+      }
+      if (grid_sync(a, sm, bar_target)) return;
+      stamp(a, 3 + 2 * s);
+      if (s == a.n_steps) break;  // the last phase only recorded kept leaves
 
-    // ---------------- select (one CTA per head)
-    for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-      const long long n = sm.pref[h + 1] - sm.pref[h];
-      HeadState* hs = hstate(h);
-      long long n_leaf0 = 0, scored0 = 0;
-      int leaf0 = 0, steps0 = 0;
-      if (step > 0) {
-        n_leaf0 = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
-        scored0 = __ldcg(&hs->scored);
-        leaf0 = __ldcg(&hs->leaf0);
-        steps0 = __ldcg(&hs->steps);
-      }
-      if (n == 0) {
-        if (tid == 0) {
-          hs->n_cand = 0;
-          hs->n_leaf = n_leaf0;
-          hs->scored = scored0;
-          hs->leaf0 = leaf0;
-          hs->steps = steps0;
+      // ---------------- select phase: one CTA per head
+      for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+        HeadState* hs = hstate(h);
+        const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
+        if (n == 0) {
+          __syncthreads();
+          if (tid == 0) hs->kept = 0;
+          continue;
         }
-        continue;
-      }
-      const Entry* S = sel(h);
-      const int mode = n <= kCache8 ? 1 : (n <= kCache4 ? 2 : 0);
-      __syncthreads();
-      uint32_t kmin = 0xffffffffu;
-      if (mode == 1) {
-        Entry* ce = reinterpret_cast<Entry*>(sm.u);
-        for (long long i = tid; i < n; i += kDecThreads) {
-          const uint2 v = __ldcg(reinterpret_cast<const uint2*>(S + i));
-          ce[i] = Entry{v.x, v.y};
-          kmin = min(kmin, v.x);
+        const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
+        const float anchor_h = __ldcg(&hs->anchor);
+        const int ovf = __ldcg(&hs->ovf[par]);
+        const long long scored0 = __ldcg(&hs->scored);
+        const uint32_t* gk = keysP(h, par);
+        const uint32_t* gc = codesP(h, par);
+        if (a.scored) {  // codes of the scored nodes
+          int32_t* out = a.scored + size_t(h) * a.scored_cap;
+          for (long long i = tid; i < n; i += kDecThreads)
+            if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
         }
-      } else if (mode == 2) {
+        const float m = desc_key_value(kmin);
+        // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
+        const int ncache = n <= kDecThreads ? 0 : int(min64(n, kCacheKeys));
         uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
-        for (long long i = tid; i < n; i += kDecThreads) {
-          const uint32_t k = __ldcg(reinterpret_cast<const unsigned int*>(S + i));
-          ck[i] = k;
-          kmin = min(kmin, k);
+        for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
+        cp_async_commit();
+        cp_async_wait(0);
+        __syncthreads();
+        const StepView E{ck, ncache, gk, gc};
+        unsigned long long cut = ~0ull;
+        if (!a.p_all) {
+          if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
+          else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
+            cut = select_cut_anchored(a, E, n, anchor_h, histP(h, par), sm, h, s);
+          else cut = select_cut(a, E, n, kmin, sm, h, s);
         }
-      } else {
-        for (long long i = tid; i < n; i += kDecThreads)
-          kmin = min(kmin, __ldcg(reinterpret_cast<const unsigned int*>(S + i)));
-      }
-      kmin = block_min_u32(kmin, sm.red32);  // includes the barrier that publishes the cache
-      int my_leaf0 = 0;
-      uint32_t tot_leaf = 0, tot_par = 0;
-      auto select_and_rank = [&](const auto& E) {
-      if (a.scored) {
-        int32_t* out = a.scored + size_t(h) * a.scored_cap;
-        for (long long i = tid; i < n; i += kDecThreads)
-          if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
-      }
-      stamp(a, 32 + 3 * step);
-      const unsigned long long cut = select_cut(a, E, n, kmin, sm, step);
-      stamp(a, 33 + 3 * step);
-      const uint32_t cut32 = uint32_t(cut >> 32);
-      // ranks of the kept entries in canonical order: each warp owns a contiguous
-      // segment, walked 32 entries at a time (coalesced reads and writes)
-      const int64_t wseg = (n + kDecWarps - 1) / kDecWarps;
-      const int64_t wlo = min64(n, wid * wseg), whi = min64(n, wlo + wseg);
-      auto kept_entry = [&](long long i, uint32_t& code) {
-        const uint32_t k = E.key(i);
-        if (k > cut32) return false;
-        code = E.code(i);
-        return k < cut32 || entry_key64(a, Entry{k, code}) <= cut;
-      };
-      uint32_t wleaf = 0, wpar = 0;
-      for (int64_t base = wlo; base < whi; base += 128) {
-        bool kp[4];
-        uint32_t code[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t i = base + 32 * u + lane;
-          code[u] = 0;
-          kp[u] = i < whi && kept_entry(i, code[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          wleaf += __popc(__ballot_sync(0xffffffffu, kp[u] && code_level(code[u]) == 1));
-          wpar += __popc(__ballot_sync(0xffffffffu, kp[u] && code_level(code[u]) != 1));
-        }
-      }
-      if (lane == 0) {
-        sm.red32[wid] = wleaf;
-        sm.red32[kDecWarps + wid] = wpar;
-      }
-      __syncthreads();
-      stamp(a, 68 + 8 * step);
-      uint32_t leaf_off = 0, par_off = 0;
-      for (int w = 0; w < kDecWarps; ++w) {
-        const uint32_t l = sm.red32[w], q = sm.red32[kDecWarps + w];
-        if (w < wid) { leaf_off += l; par_off += q; }
-        tot_leaf += l;
-        tot_par += q;
-      }
-      const unsigned below_me = (1u << lane) - 1u;
-      for (int64_t base = wlo; base < whi; base += 32) {
-        const int64_t i = base + lane;
-        uint32_t code = 0;
-        const bool kp = i < whi && kept_entry(i, code);
-        const bool isleaf = kp && code_level(code) == 1;
-        const bool ispar = kp && code_level(code) != 1;
-        const unsigned ml = __ballot_sync(0xffffffffu, isleaf);
-        const unsigned mp = __ballot_sync(0xffffffffu, ispar);
-        if (isleaf) {
-          const long long g = n_leaf0 + leaf_off + __popc(ml & below_me);
-          if (code_index(code) == 0) my_leaf0 = 1;
-          if (g < a.cap_list) leaves(h)[g] = code_index(code);
-          else raise_status(a.t.status, ZHA_ERR_CAPACITY);
-          if (a.kept && g < a.kept_stride) a.kept[size_t(h) * a.kept_stride + g] = int32_t(code_index(code));
-        }
-        if (ispar) {
-          const long long pr = par_off + __popc(mp & below_me);
-          const uint32_t cl = code_level(code) - 1, ci = code_index(code) * uint32_t(b);
-          if ((pr + 1) * b <= a.cap_sel) {
-            for (int c = 0; c < b; ++c) cand(h)[pr * b + c] = node_code(cl, ci + uint32_t(c));
+        // the kept entries (order key <= cut), listed in entry
+        // order: each warp owns a contiguous segment; the code is read only for a
+        // key equal to the cut's
+        long long n_kept = 0;
+        {
+          const uint32_t cut32 = uint32_t(cut >> 32);
+          const int n32 = int(n);
+          const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
+          const int wlo = min(n32, wid * wseg), whi = min(n32, wlo + wseg);
+          auto kept_at = [&](int i) {
+            const uint32_t k = E.key(i);
+            return k < cut32 || (k == cut32 && entry_key64(a, Entry{k, E.code(i)}) <= cut);
+          };
+          uint32_t wk = 0;
+          for (int base = wlo; base < whi; base += 32) {
+            const int i = base + lane;
+            wk += __popc(__ballot_sync(0xffffffffu, i < whi && kept_at(i)));
+          }
+          if (lane == 0) sm.red32[wid] = wk;
+          __syncthreads();
+          uint32_t off = 0;
+          for (int w = 0; w < kDecWarps; ++w) {
+            if (w < wid) off += sm.red32[w];
+            n_kept += sm.red32[w];
+          }
+          uint32_t* kl = keptl(h);
+          for (int base = wlo; base < whi; base += 32) {
+            const int i = base + lane;
+            const bool kp = i < whi && kept_at(i);
+            const unsigned mk = __ballot_sync(0xffffffffu, kp);
+            if (kp) kl[off + __popc(mk & ((1u << lane) - 1u))] = uint32_t(i);
+            off += __popc(mk);
           }
         }
-        leaf_off += __popc(ml);
-        par_off += __popc(mp);
-      }
-      };
-      if (mode == 1) select_and_rank(ViewSmemEntries{reinterpret_cast<const Entry*>(sm.u)});
-      else if (mode == 2) select_and_rank(ViewSmemKeys{reinterpret_cast<const uint32_t*>(sm.u), S});
-      else select_and_rank(ViewGlobal{S});
-      my_leaf0 = __syncthreads_or(my_leaf0);
-      stamp(a, 69 + 8 * step);
-      if (tid == 0) {
-        long long nc = (long long)tot_par * b;
-        if (nc > a.cap_sel) {
-          raise_status(a.t.status, ZHA_ERR_CAPACITY);
-          nc = 0;
+        // state for the next step: its histogram cleared, its anchor = this step's max
+        unsigned long long* nhist = histP(h, par ^ 1);
+        for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
+        __syncthreads();
+        if (tid == 0) {
+          hs->kept = n_kept;
+          hs->n[par ^ 1] = 0;
+          hs->anchor = m;
+          hs->kinv[par ^ 1] = 0u;
+          hs->ovf[par ^ 1] = 0;
+          hs->scored = scored0 + n;
+          hs->steps = hs->steps + 1;
         }
-        hs->n_cand = nc;
-        hs->n_leaf = min64(n_leaf0 + tot_leaf, a.cap_list);
-        hs->scored = scored0 + n;
-        hs->leaf0 = leaf0 | my_leaf0;
-        hs->steps = steps0 + 1;
+      }
+      if (grid_sync(a, sm, bar_target)) return;
+    }
+    // ---------------- finalize: the kept leaves of each head, in block order, from its bitmap
+    for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+      uint32_t* bm = bitmap(h);
+      const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
+      long long carry = 0;
+      if (tid == 0) sm.bcast32[3] = 0;
+      for (long long w0 = 0; w0 < nw; w0 += kDecThreads) {
+        const long long wi = w0 + tid;
+        uint32_t bits = wi < nw ? __ldcg(bm + wi) : 0u;
+        if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
+        if (wi == 0 && (bits & 1u)) sm.bcast32[3] = 1;
+        uint32_t tot;
+        const uint32_t ex = block_scan_u32(uint32_t(__popc(bits)), sm.red32, &tot);
+        long long pos = carry + ex;
+        while (bits) {
+          const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
+          bits &= bits - 1u;
+          if (pos < a.cap_list) leaves(h)[pos] = idx;
+          if (a.kept && pos < a.kept_stride) a.kept[size_t(h) * a.kept_stride + pos] = int32_t(idx);
+          ++pos;
+        }
+        carry += tot;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        if (carry > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+        hstate(h)->n_leaf = min64(carry, a.cap_list);
+        hstate(h)->leaf0 = sm.bcast32[3];
       }
       __syncthreads();
     }
-    stamp(a, 3 + 4 * step);
     if (grid_sync(a, sm, bar_target)) return;
-    stamp(a, 4 + 4 * step);
   }
+  __syncthreads();
+  stamp(a, 1);
 
   // ---------------- attend (all CTAs)
   const long long n1 = a.nl[1];
@@ -962,7 +1485,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   auto head_keys = [&](int h, long long& nl, bool& sink) {
     nl = 0;
     int l0 = 0;
-    if (a.n_steps > 0) {
+    if (routed) {
       nl = min64(max64(__ldcg(&hstate(h)->n_leaf), 0), a.cap_list);
       l0 = __ldcg(&hstate(h)->leaf0);
     }
@@ -972,7 +1495,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   for (int i = tid; i < nh; i += kDecThreads) {
     long long nl;
     bool sink;
-    sm.pref[1 + i] = head_keys(i, nl, sink);
+    sm.pref()[1 + i] = head_keys(i, nl, sink);
   }
   __syncthreads();
   const long long total_keys = build_prefix(sm, nh);
@@ -982,7 +1505,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   for (int i = tid; i < nh; i += kDecThreads) {
     long long nl;
     bool sink;
-    sm.pref[1 + i] = (head_keys(i, nl, sink) + chunk - 1) / chunk;
+    sm.pref()[1 + i] = (head_keys(i, nl, sink) + chunk - 1) / chunk;
   }
   __syncthreads();
   const long long total_items = build_prefix(sm, nh);
@@ -996,7 +1519,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     constexpr int kU = 8;
     for (long long it = c0 + wid; it < c1; it += kDecWarps) {
       const int h = owner_of(sm, nh, it);
-      const long long ci = it - sm.pref[h];
+      const long long ci = it - sm.pref()[h];
       const int kvh = (h % a.t.hq) / a.t.group;
       long long nl;
       bool sink;
@@ -1101,8 +1624,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   // the global slot of the segment's first chunk
   for (long long seg = c0 + wid; seg < c1; seg += kDecWarps) {
     const int h = owner_of(sm, nh, seg);
-    if (seg != c0 && seg != sm.pref[h]) continue;  // not the first chunk of a segment
-    const long long send = min64(c1, sm.pref[h + 1]);
+    if (seg != c0 && seg != sm.pref()[h]) continue;  // not the first chunk of a segment
+    const long long send = min64(c1, sm.pref()[h + 1]);
     float M = -INFINITY;
     for (long long j = seg; j < send; ++j) M = fmaxf(M, part[j - c0][0]);
     float L = 0.f;
@@ -1133,7 +1656,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
   // ---------------- combine (one CTA per head)
   for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-    const long long p0 = sm.pref[h], p1 = sm.pref[h + 1];
+    const long long p0 = sm.pref()[h], p1 = sm.pref()[h + 1];
     // partial slots: one per CTA whose chunk range meets [p0, p1), at max(p0, range start)
     float M = -INFINITY;
     auto range_start = [&](long long c) { return (c * total_items) / (long long)gridDim.x; };
@@ -1179,11 +1702,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     if (tid == 0) {
       long long nl = 0, scored = 0;
       int l0 = 0, steps = 0;
-      if (a.n_steps > 0) {
-        nl = __ldcg(&hstate(h)->n_leaf);
-        l0 = __ldcg(&hstate(h)->leaf0);
-        scored = __ldcg(&hstate(h)->scored);
-        steps = __ldcg(&hstate(h)->steps);
+      if (routed) {
+        HeadState* hs = hstate(h);
+        nl = __ldcg(&hs->n_leaf);
+        l0 = __ldcg(&hs->leaf0);
+        scored = __ldcg(&hs->scored);
+        steps = __ldcg(&hs->steps);
+        // leave the head's state zeroed for the next launch
+        long long* z = reinterpret_cast<long long*>(hs);
+        for (int k = 0; k < int(sizeof(HeadState) / 8); ++k) z[k] = 0;
       }
       if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
       if (a.stats) {
@@ -1242,7 +1769,18 @@ int decode_grid(int dtype, int d) {
 }
 
 size_t decode_smem_bytes() { return sizeof(DecSmem); }
-size_t decode_head_state_bytes() { return sizeof(HeadState); }
+// Head states and leaf bitmaps, one region cleared together.
+size_t decode_flow_bytes(int nheads, int64_t cap_sel) {
+  return size_t(nheads) * (sizeof(HeadState) + size_t(decode_bitmap_words(cap_sel)) * 4);
+}
+// Grid barriers one decode launch takes.
+int decode_barriers(int n_steps, int n_roots) { return n_steps > 0 && n_roots > 0 ? 2 * n_steps + 3 : 1; }
+// Per-head routing workspace: step keys and codes in two parity buffers, two
+// anchored histograms, the kept entries of the last select, the kept leaves.
+uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list) {
+  const uint64_t cap4 = (uint64_t(cap_sel) + 3) & ~uint64_t(3);
+  return cap4 * 20 + 2 * kBins * 8 + uint64_t(cap_list) * 4;
+}
 int decode_max_heads() { return kMaxHeads; }
 int decode_items_per_cta() { return kItemsPerCta; }
 int decode_max_grid() { return kMaxDecodeGrid; }
