@@ -146,17 +146,21 @@ ZHA_API int64_t zha_tree_size(const zha_tree* tree);
  *   O        - [B][Hq][d] fp32, device; softmax attention over each head's
  *              attended set (kept blocks, token 0, tail tokens).
  *   kept     - optional [B][Hq][cap_leaves] int32 (cap_leaves = capacity / block):
- *              the kept level-1 block indices of each head, in no particular
- *              order; kept_cnt [B][Hq] int32 receives their number.  Both NULL
- *              or both non-NULL.
+ *              the kept level-1 block indices of each head, ascending;
+ *              kept_cnt [B][Hq] int32 receives their number.  Both NULL or
+ *              both non-NULL.
  *   stats    - optional [B][Hq][ZHA_STAT_COUNT] int64 counters.
  *   scored   - optional [B][Hq][scored_cap] int32: the codes (level << 27 | index)
- *              of every node the head scored, step by step; ZHA_STAT_NODES_SCORED
+ *              of every node the head scored, step by step (in no particular
+ *              order within a step); ZHA_STAT_NODES_SCORED
  *              gives how many (entries past scored_cap are dropped).  Used to
  *              count the bytes a decode must read; leave NULL on the hot path.
  * Requires 1 <= B <= max_batch and at least one cached token.  The call
- * launches one cooperative kernel (every SM takes part); calls on one tree
- * share its scratch and must be issued in order on one stream.
+ * launches a fixed sequence of kernels on `stream` (per routing step a scoring
+ * and a select kernel, then finalize, attention and combine kernels) and
+ * returns without synchronizing; calls on one tree share its scratch and must
+ * be issued in order on one stream.  A wait of a scoring warp on a record copy
+ * is bounded: when it runs out the status word reports ZHA_ERR_TIMEOUT.
  */
 ZHA_API int zha_decode(const zha_tree* tree, const void* Q, float* O, int32_t B, int32_t* kept,
                int32_t* kept_cnt, int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream);

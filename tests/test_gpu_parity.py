@@ -267,15 +267,15 @@ def test_errors():
     case.tree.status()
 
 
-def test_barrier_timeout_is_reported_and_recoverable(monkeypatch):
-    """A grid-barrier wait that runs out returns ZHA_ERR_TIMEOUT through the status word; the context stays usable.
+def test_wait_timeout_is_reported_and_recoverable(monkeypatch):
+    """A bounded wait that runs out returns ZHA_ERR_TIMEOUT through the status word; the context stays usable.
 
-    ZHA_SPIN_LIMIT=1 (read when a tree is created) makes every waiting CTA give up at once; the kernel
-    then returns without touching memory beyond its bounds-checked workspace.
+    ZHA_SPIN_LIMIT=0 (read when a tree is created) makes every wait of the scoring warps on a record copy give
+    up at its first check; the warp then waits, with its own bound, for the copies it has in flight and stops.
     """
     K, V, refs, Q = random_tree_case(21, n_tokens=3000, d=128, n_q_heads=8, n_kv_heads=1, n_refs=4, batch=2,
                                      dtype="bf16")
-    monkeypatch.setenv("ZHA_SPIN_LIMIT", "1")
+    monkeypatch.setenv("ZHA_SPIN_LIMIT", "0")
     bad = Case(K, V, refs, block=4, levels=3, p=0.9, n=3000, group=8)
     monkeypatch.delenv("ZHA_SPIN_LIMIT")
     bad.tree.decode(Q.cuda())

@@ -17,14 +17,10 @@ cudaError_t launch_tree_update(const TreeDev& t, int dtype, int64_t n_old, int64
 cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
                                cudaStream_t st);
 size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R);
-size_t decode_smem_bytes();
 size_t decode_flow_bytes(int nheads, int64_t cap_sel);
 uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list);
-int decode_barriers(int n_steps, int n_roots);
 int decode_max_heads();
-int decode_items_per_cta();
-int decode_max_grid();
-int decode_grid(int dtype, int d);
+uint64_t decode_part_items(int nheads);
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
 size_t dense_static_floats();
 cudaError_t dense_static_scratch(float** out);
@@ -65,14 +61,14 @@ struct Layout {
   uint64_t rec_off[kMaxLevels + 1], f_off[kMaxLevels + 1], up_off[kMaxLevels + 1];
   uint64_t rec_bytes, up_bytes, node_bytes;
   // scratch
-  uint64_t status_off, bar_off, part_off, part_items, flow_off, flow_bytes, ws_off, ws_per_bh, stage_off, scratch_bytes;
+  uint64_t status_off, part_off, part_items, flow_off, flow_bytes, ws_off, ws_per_bh, stage_off, scratch_bytes;
   int64_t cap_sel, cap_list;
   uint64_t stage_k, stage_v, stage_q, stage_o;
 };
 
 uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
-constexpr long long kDefaultSpinLimit = 1ll << 24;  // ~1 s of 40 ns sleeps  // CTAs of the decode launch (one per SM) the scratch is sized for
+constexpr long long kDefaultSpinLimit = 1ll << 22;  // bound of the decode's waits on record copies (try_wait rounds)
 
 int elem_size(int dtype) { return dtype == ZHA_BF16 ? 2 : 4; }
 
@@ -138,13 +134,12 @@ int make_layout(const zha_config* c, Layout* L) {
   // scratch: status word and grid barrier, attend partials, per (sequence,
   // query head) routing workspace, host-step staging
   L->status_off = 0;
-  L->bar_off = 64;
   const int64_t n1cap = L->cap_nodes[1] > 0 ? L->cap_nodes[1] : 1;
   L->cap_sel = n1cap;
   L->cap_list = n1cap + 64;
   const uint64_t nheads = uint64_t(c->max_batch) * c->n_q_heads;
   L->part_off = 256;
-  L->part_items = uint64_t(decode_max_grid()) * decode_items_per_cta() + nheads + 64;
+  L->part_items = decode_part_items(int(nheads));
   L->flow_off = align256(L->part_off + L->part_items * (c->d + 2) * 4);
   // head states and leaf bitmaps, cleared together
   L->flow_bytes = decode_flow_bytes(int(nheads), L->cap_sel);
@@ -173,8 +168,7 @@ struct zha_tree {
   char* scratch;
   int64_t n;
   int device;
-  long long spin_limit;  // grid-barrier spin bound of the decode kernel
-  unsigned long long bar_count;  // arrivals the decode kernels have made on the grid barrier so far
+  long long spin_limit;  // bound of the decode's waits on record copies
   bool flow_dirty;               // the routing flow state must be zeroed before the next decode
 };
 
@@ -225,11 +219,10 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
   t->scratch = static_cast<char*>(scratch);
   t->n = 0;
   t->spin_limit = kDefaultSpinLimit;
-  t->bar_count = 0;
   t->flow_dirty = true;
-  if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: force the barrier timeout path
+  if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: 0 makes every wait give up at once
     const long long x = std::atoll(v);
-    if (x > 0) t->spin_limit = x;
+    if (x >= 0 && (x > 0 || v[0] == '0')) t->spin_limit = x;
   }
   cudaGetDevice(&t->device);
   TreeDev& d = t->dev;
@@ -276,7 +269,6 @@ int zha_tree_build(zha_tree* t, int64_t n, void* stream) {
   e = launch_tree_update(t->dev, t->cfg.dtype, 0, n, st);
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_build");
   t->n = n;
-  t->bar_count = 0;
   t->flow_dirty = true;
   return ZHA_OK;
 }
@@ -319,8 +311,6 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->ws = t->scratch + t->L.ws_off;
   a->ws_per_bh = t->L.ws_per_bh;
   a->flow = reinterpret_cast<unsigned char*>(t->scratch + t->L.flow_off);
-  a->bar = reinterpret_cast<unsigned long long*>(t->scratch + t->L.bar_off);
-  a->bar_base = t->bar_count;
   a->attn_part = reinterpret_cast<float*>(t->scratch + t->L.part_off);
   a->spin_limit = t->spin_limit;
 #ifdef ZHA_PHASE_TIMING
@@ -357,15 +347,11 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
   if (scored && scored_cap < 1) return fail(ZHA_ERR_INVALID, "scored needs scored_cap >= 1");
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)
     return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
-  const int grid = decode_grid(t->cfg.dtype, t->cfg.d);
-  if (grid < 1) return fail(ZHA_ERR_CUDA, "the decode kernel does not fit on this device");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   zha_tree* tm = const_cast<zha_tree*>(t);
   if (tm->flow_dirty) {  // first decode of this tree, or the first after an error status
     cudaError_t e = cudaMemsetAsync(t->scratch + t->L.flow_off, 0, t->L.flow_bytes, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(t->scratch + t->L.bar_off, 0, 8, st);
-    if (e != cudaSuccess) return fail_cuda(e, "zha_decode: clearing the flow state");
-    tm->bar_count = 0;
+    if (e != cudaSuccess) return fail_cuda(e, "zha_decode: clearing the routing state");
     tm->flow_dirty = false;
   }
   DecodeArgs a;
@@ -376,8 +362,6 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
     tm->flow_dirty = true;
     return fail_cuda(e, "zha_decode");
   }
-  // every CTA arrives once on each grid barrier of the launch
-  tm->bar_count += uint64_t(decode_barriers(a.n_steps, a.n_roots)) * uint64_t(grid);
   return ZHA_OK;
 }
 

@@ -19,10 +19,8 @@ struct DecodeArgs {
   int64_t cap_sel;              // entries per step buffer (and kept parents)
   int64_t cap_list;             // kept leaves per head
   unsigned char* flow;          // per-head routing states, then leaf bitmaps (zero between launches)
-  unsigned long long* bar;      // grid barrier arrival counter (only grows)
-  unsigned long long bar_base;  // its value when this launch starts
   float* attn_part;             // attend partials, (2 + d) floats each
-  long long spin_limit;         // grid-barrier spin bound
+  long long spin_limit;         // bound of the waits on record copies
   int32_t* kept;
   int32_t* kept_cnt;
   int64_t* stats;

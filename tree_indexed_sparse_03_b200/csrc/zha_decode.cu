@@ -49,19 +49,23 @@ struct Entry {
   uint32_t code;  // node_code(level, index)
 };
 
-constexpr int kDecThreads = 512;                   // threads per CTA (one CTA per SM)
+constexpr int kDecThreads = 512;                   // threads of a scoring, select or finalize CTA
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kUnionBytes = 208 * 1024;            // select key cache / score rings / attend partials + prefix
-constexpr int kCacheKeys = kUnionBytes / 4;        // step keys a select caches in shared memory
+constexpr int kUnionBytes = 208 * 1024;            // select: step keys cached in shared memory
+constexpr int kCacheKeys = kUnionBytes / 4;
+constexpr int kRingBytes = 200 * 1024;             // scoring: record ring of the CTA's warps
 constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
 constexpr int kMaxHeads = 1024;                    // sequences x query heads per call
-constexpr int kItemsPerCta = 256;                  // attend chunks a CTA owns at most (plus one per head)
-constexpr int kMaxDecodeGrid = 512;                // CTAs per decode launch the scratch is laid out for
-constexpr int kPrefOff = kUnionBytes - (kMaxHeads + 1) * 8;  // per-head prefix (attend), inside the union
-constexpr int kPartSlots = kPrefOff / ((2 + 128) * 4);          // attend partials a CTA can hold
 constexpr int kMaxSlots = 8;                       // score ring slots per warp
-static_assert(kPartSlots >= kItemsPerCta + 16, "attend partial area too small");
+constexpr long long kDrainLimit = 1ll << 22;       // bound of the wait for copies in flight after a timeout
+constexpr int kAttThreads = 256;                   // threads of an attention CTA
+constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kAttItems = 32;                      // attend chunks a CTA owns at most
+constexpr int kMaxAttGrid = 1024;                  // attention CTAs the scratch is laid out for
+constexpr int kCombThreads = 1024;                 // threads of a combine CTA (one partial per thread)
+static_assert(kMaxAttGrid <= kCombThreads, "the combine takes one partial per thread");
+static_assert(kCombThreads % 128 == 0, "the combine splits its threads over the output elements");
 
 struct HeadState {  // per (sequence, query head)
   long long n[2];          // entries of the step built in each parity buffer (step 0: unused)
@@ -127,10 +131,23 @@ struct __align__(16) DecSmem {
   int bcast32[8];
   int fail;
   int job_h, job_s;           // select CTA: the request being served (-2: exit)
-  unsigned long long mbar[kDecWarps][kMaxSlots];  // scoring warps: one mbarrier per ring slot
-  // per-head prefix of attend work items (lives in the union after routing)
-  __device__ __forceinline__ long long* pref() { return reinterpret_cast<long long*>(u + kPrefOff); }
-  __device__ __forceinline__ const long long* pref() const { return reinterpret_cast<const long long*>(u + kPrefOff); }
+};
+
+// Division of 32-bit values by a fixed divisor d >= 2 with a multiply-high and
+// one correction step (m = floor(2^32 / d) underestimates x / d by less than 1).
+struct DivU32 {
+  uint32_t d, m;
+  __device__ explicit DivU32(uint32_t div) : d(div), m(uint32_t((1ull << 32) / div)) {}
+  __device__ __forceinline__ uint32_t div(uint32_t x, uint32_t* rem) const {
+    uint32_t q = __umulhi(x, m);
+    uint32_t r = x - q * d;
+    if (r >= d) {
+      ++q;
+      r -= d;
+    }
+    *rem = r;
+    return q;
+  }
 };
 
 // The step's entries of one head: keys [0, nc) cached in shared memory, the
@@ -229,6 +246,7 @@ __device__ __forceinline__ float score_node(const TreeDev& t, int head, uint32_t
 
 // Block-wide exclusive scan of one value per thread; returns the exclusive
 // prefix and writes the block total to *total (all threads).
+template <int NW = kDecWarps>
 __device__ __forceinline__ uint32_t block_scan_u32(uint32_t v, uint32_t* red, uint32_t* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint32_t x = v;
@@ -240,7 +258,7 @@ __device__ __forceinline__ uint32_t block_scan_u32(uint32_t v, uint32_t* red, ui
   if (lane == 31) red[wid] = x;
   __syncthreads();
   uint32_t base = 0, tot = 0;
-  for (int w = 0; w < kDecWarps; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const uint32_t s = red[w];
     if (w < wid) base += s;
     tot += s;
@@ -250,6 +268,7 @@ __device__ __forceinline__ uint32_t block_scan_u32(uint32_t v, uint32_t* red, ui
   return base + x - v;
 }
 
+template <int NW = kDecWarps>
 __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* red,
                                                              unsigned long long* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -262,7 +281,7 @@ __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long 
   if (lane == 31) red[wid] = x;
   __syncthreads();
   unsigned long long base = 0, tot = 0;
-  for (int w = 0; w < kDecWarps; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const unsigned long long s = red[w];
     if (w < wid) base += s;
     tot += s;
@@ -909,57 +928,31 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
   return prefix;
 }
 
-// Grid barrier over all CTAs of the cooperative launch: a 64-bit arrival
-// counter that only grows; barrier k of a launch completes when it reaches
-// base + k * gridDim.x (the host tracks the base).  Returns true for every
-// thread of the CTA if the wait gave up.
-__device__ __forceinline__ bool grid_sync(const DecodeArgs& a, DecSmem& sm, unsigned long long& target) {
-  target += gridDim.x;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    sm.fail = 0;
-    __threadfence();
-    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(a.bar) : "memory");
-    long long it = 0;
-    while (true) {
-      unsigned long long v;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.bar) : "memory");
-      if (v >= target) break;
-      if (++it > a.spin_limit) {
-        sm.fail = 1;
-        raise_status(a.t.status, ZHA_ERR_TIMEOUT);
-        break;
-      }
-      __nanosleep(20);
-    }
-  }
-  __syncthreads();
-  return sm.fail != 0;
-}
-
-// Inclusive prefix of per-head counts held in sm.pref()[1..nh] (pref[0] = 0); returns the total.
-__device__ __forceinline__ long long build_prefix(DecSmem& sm, int nh) {
+// Inclusive prefix of per-head counts held in pref[1..nh] (pref[0] = 0), NT
+// threads; returns the total.
+template <int NT>
+__device__ __forceinline__ long long build_prefix(long long* pref, unsigned long long* red64, int nh) {
   long long carry = 0;
-  for (int base = 0; base < nh; base += kDecThreads) {
+  for (int base = 0; base < nh; base += NT) {
     const int i = base + threadIdx.x;
-    const unsigned long long v = i < nh ? (unsigned long long)sm.pref()[1 + i] : 0ull;
+    const unsigned long long v = i < nh ? (unsigned long long)pref[1 + i] : 0ull;
     unsigned long long tot;
-    const unsigned long long ex = block_scan_u64(v, sm.red64, &tot);
-    if (i < nh) sm.pref()[1 + i] = carry + (long long)(ex + v);
+    const unsigned long long ex = block_scan_u64<NT / 32>(v, red64, &tot);
+    if (i < nh) pref[1 + i] = carry + (long long)(ex + v);
     carry += (long long)tot;
     __syncthreads();
   }
-  if (threadIdx.x == 0) sm.pref()[0] = 0;
+  if (threadIdx.x == 0) pref[0] = 0;
   __syncthreads();
   return carry;
 }
 
 // Head owning work item i: the largest h with pref[h] <= i.
-__device__ __forceinline__ int owner_of(const DecSmem& sm, int nh, long long i) {
+__device__ __forceinline__ int owner_of(const long long* pref, int nh, long long i) {
   int lo = 0, hi = nh - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (sm.pref()[mid] <= i) lo = mid; else hi = mid - 1;
+    if (pref[mid] <= i) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -1119,422 +1112,682 @@ __device__ __forceinline__ float score_record_smem(const unsigned char* rec, int
   return best;
 }
 
+// ---------------------------------------------------------------- per-call context
+// The scratch regions of one decode call and the views of them every phase uses.
 template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+struct Ctx {
+  const DecodeArgs& a;
+  int nh;
+  int64_t cap4, bm_words;
+  __device__ explicit Ctx(const DecodeArgs& args)
+      : a(args), nh(args.nheads), cap4((args.cap_sel + 3) & ~int64_t(3)), bm_words(decode_bitmap_words(args.cap_sel)) {}
+  // per-head workspace: step keys [2][cap4], step codes [2][cap4] (parity buffers: step s in s & 1),
+  // anchored histograms [2][kBins], kept entries of the last select [cap4], kept leaves [cap_list]
+  __device__ char* ws(int h) const { return a.ws + uint64_t(h) * a.ws_per_bh; }
+  __device__ uint32_t* keysP(int h, int par) const { return reinterpret_cast<uint32_t*>(ws(h) + par * cap4 * 4); }
+  __device__ uint32_t* codesP(int h, int par) const {
+    return reinterpret_cast<uint32_t*>(ws(h) + (2 + par) * cap4 * 4);
+  }
+  __device__ unsigned long long* histP(int h, int par) const {
+    return reinterpret_cast<unsigned long long*>(ws(h) + 4 * cap4 * 4 + par * kBins * 8);
+  }
+  __device__ uint32_t* keptl(int h) const { return reinterpret_cast<uint32_t*>(ws(h) + 4 * cap4 * 4 + 2 * kBins * 8); }
+  __device__ uint32_t* leaves(int h) const {
+    return reinterpret_cast<uint32_t*>(ws(h) + 5 * cap4 * 4 + 2 * kBins * 8);
+  }
+  // head states, then one leaf bitmap per head (one region, zero between calls)
+  __device__ HeadState* hstate(int h) const { return reinterpret_cast<HeadState*>(a.flow) + h; }
+  __device__ uint32_t* bitmap(int h) const {
+    return reinterpret_cast<uint32_t*>(a.flow + size_t(nh) * sizeof(HeadState)) + h * bm_words;
+  }
+  // the lane's q slice for the FMA estimates: elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR
+  __device__ void q_slice(int h, float* qs) const {
+    constexpr int EPC = 16 / sizeof(T);
+    constexpr int CPR = D * sizeof(T) / 16;
+    const T* q = static_cast<const T*>(a.Q) + size_t(h) * D + ((threadIdx.x & 31) % CPR) * EPC;
+    unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
+  }
+};
+
+// ---------------------------------------------------------------- scoring phase
+// Step s's entries: the roots (s = 0, root i at position i) or the children of
+// step s-1's kept non-leaves, at positions reserved per warp batch with one
+// atomic add per head (their order varies from run to run; nothing
+// downstream depends on it); kept leaves of step s-1 go to the head's bitmap.
+// Units (roots, or kept entries) of all heads are cut into contiguous ranges,
+// one per warp.  Each record is fetched with one bulk copy into the warp's
+// ring; the estimate is added to the step's anchored histogram (s >= 1).
+struct __align__(16) ScoreSmem {
+  unsigned char ring[kRingBytes];
+  long long pref[kMaxHeads + 1];
+  unsigned long long red64[kDecWarps];
+  unsigned long long mbar[kDecWarps][kMaxSlots];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_constant__ DecodeArgs a, int s) {
   constexpr int EPC = 16 / sizeof(T);
-  constexpr int CPR = D * sizeof(T) / 16;
-  constexpr int KPW = 32 / CPR;  // keys per warp pass in the attention loop
+  constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ScoreSmem& sp = *reinterpret_cast<ScoreSmem*>(smem_raw);
+  const Ctx<T, D> c(a);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nh = a.nheads, b = a.t.block, R = a.t.refs;
+  const int par = s & 1;
+  const int rec_bytes = int(a.t.rec_bytes);
+  // nslot record slots per warp; warps past score_warps (only when a record is
+  // larger than a warp's share of the ring) do not score
+  const int nslot = max(1, min(kMaxSlots, (kRingBytes / kDecWarps) / rec_bytes));
+  const int score_warps = min(kDecWarps, kRingBytes / (nslot * rec_bytes));
+  unsigned char* ring = sp.ring + size_t(wid) * nslot * rec_bytes;
+  if (lane == 0) {
+    for (int k = 0; k < nslot; ++k) mbar_init(&sp.mbar[wid][k], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  // ring cursors: slot of the next copy / the next record to consume, and the
+  // mbarrier phase parity of the latter (flips each time it wraps)
+  int slot_i = 0, slot_d = 0, in_flight = 0;
+  unsigned phase_d = 0;
+  float qs[EPC];
+  uint32_t qf[D / 16][2];
+  int qhead = -1;
+  const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
+  const long long nwarps = (long long)gridDim.x * score_warps;
+  // ---------------- scoring phase: units = roots (s = 0) or the kept entries of step s-1
+  for (int i = tid; i < nh; i += kDecThreads)
+    sp.pref[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&c.hstate(i)->kept), 0), a.cap_sel);
+  __syncthreads();
+  const long long total = build_prefix<kDecThreads>(sp.pref, sp.red64, nh);
+  const long long u0 = gwarp < 0 ? 0 : total * gwarp / nwarps;
+  const long long u1 = gwarp < 0 ? 0 : total * (gwarp + 1) / nwarps;
+  int cur_h = -1;           // lane 0: head of the pending min-key update
+  uint32_t cur_kmin = 0xffffffffu;
+  int cur_ovf = 0;
+  int ah = -1;              // head whose anchor is loaded
+  float anchor = 0.f;
+  for (long long ub = u0; ub < u1; ub += 32) {
+    // one unit per lane: its head, its first output position, its code
+    const long long u = ub + lane;
+    int uh = 0;
+    long long upos = 0;
+    uint32_t ucode = 0;
+    bool has = false;  // the unit makes records (a root, or a kept non-leaf)
+    if (u < u1) {
+      uh = owner_of(sp.pref, nh, u);
+      const long long k = u - sp.pref[uh];
+      if (s == 0) {
+        ucode = root_code(a, k);
+        upos = k;
+        has = valid_code(a, ucode);
+      } else {
+        const uint32_t idx = __ldcg(c.keptl(uh) + k);
+        const uint32_t code = idx < uint32_t(a.cap_sel) ? __ldcg(c.codesP(uh, par ^ 1) + idx) : 0u;
+        if (valid_code(a, code)) {
+          if (code_level(code) == 1) {
+            atomicOr(c.bitmap(uh) + (code_index(code) >> 5), 1u << (code_index(code) & 31u));
+          } else {
+            ucode = code;
+            has = true;
+          }
+        }
+      }
+    }
+    if (s >= 1) {  // positions: one reservation per head segment of the batch
+      unsigned todo = __ballot_sync(0xffffffffu, has);
+      while (todo) {
+        const int l0 = __ffs(todo) - 1;
+        const int h0 = __shfl_sync(0xffffffffu, uh, l0);
+        const unsigned seg = __ballot_sync(0xffffffffu, has && uh == h0);
+        long long bs = 0;
+        if (lane == l0) {
+          const long long need = (long long)__popc(seg) * b;
+          bs = (long long)atomicAdd(reinterpret_cast<unsigned long long*>(&c.hstate(h0)->n[par]),
+                                    (unsigned long long)need);
+          if (bs + need > a.cap_sel) {
+            raise_status(a.t.status, ZHA_ERR_CAPACITY);
+            bs = -1;
+          }
+        }
+        bs = __shfl_sync(0xffffffffu, bs, l0);
+        if (has && uh == h0) {
+          upos = bs + (long long)__popc(seg & ((1u << lane) - 1u)) * b;
+          if (bs < 0) has = false;
+        }
+        todo &= ~seg;
+      }
+    }
+    const unsigned mhas = __ballot_sync(0xffffffffu, has);
+    if (!mhas) continue;
+    const int per = s == 0 ? 1 : b;  // records per unit
+    const int items = __popc(mhas) * per;
+    // item k: record (k % per) of the (k / per)-th unit with records, in lane order
+    struct Cursor {
+      unsigned rem;
+      int child;
+    };
+    struct Item {
+      int h;
+      long long pos;
+      uint32_t code;
+    };
+    auto next_item = [&](Cursor& cur) -> Item {  // the whole warp calls it, in item order
+      const int pl = __ffs(cur.rem) - 1;
+      Item it;
+      it.h = __shfl_sync(0xffffffffu, uh, pl);
+      it.pos = __shfl_sync(0xffffffffu, upos, pl) + cur.child;
+      const uint32_t pc = __shfl_sync(0xffffffffu, ucode, pl);
+      it.code = s == 0 ? pc : node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(cur.child));
+      if (++cur.child == per) {
+        cur.child = 0;
+        cur.rem &= cur.rem - 1u;
+      }
+      return it;
+    };
+    Cursor cur_i{mhas, 0};
+    Item slot_item[kMaxSlots];
+    int issued = 0, done = 0;
+    while (done < items) {
+      while (issued < items && issued - done < nslot) {
+        const Item it = next_item(cur_i);
+        const int sl = slot_i;
+        slot_i = slot_i + 1 == nslot ? 0 : slot_i + 1;
+        unsigned char* slot = ring + size_t(sl) * rec_bytes;
+        if (lane == 0) {
+          fence_proxy_async();  // the slot's last reads (generic proxy) before the copy writes it
+          const int kvh = (it.h % a.t.hq) / a.t.group;
+          bulk_load(slot, a.t.rec(code_level(it.code), kvh, code_index(it.code)), unsigned(rec_bytes),
+                    &sp.mbar[wid][sl]);
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxSlots; ++k)
+          if (k == issued - done) slot_item[k] = it;
+        ++issued;
+        ++in_flight;
+      }
+      const int sl = slot_d;
+      const unsigned parity = phase_d;
+      {
+        // bounded wait; on running out: report, wait (again bounded) for the
+        // copies in flight, and stop this warp
+        long long it = 0;
+        bool out = false;
+        while (true) {
+          if (it >= a.spin_limit) {
+            out = true;
+            break;
+          }
+          if (mbar_try_wait(&sp.mbar[wid][sl], parity)) break;
+          ++it;
+        }
+        if (__any_sync(0xffffffffu, out)) {
+          if (lane == 0) raise_status(a.t.status, ZHA_ERR_TIMEOUT);
+          int ks = slot_d;
+          unsigned kp = phase_d;
+          for (int k = 0; k < in_flight; ++k) {
+            for (long long d = 0; d < kDrainLimit && !mbar_try_wait(&sp.mbar[wid][ks], kp); ++d) {
+            }
+            if (++ks == nslot) {
+              ks = 0;
+              kp ^= 1u;
+            }
+          }
+          return;
+        }
+      }
+      __syncwarp();
+      const Item it = slot_item[0];
+#pragma unroll
+      for (int k = 0; k + 1 < kMaxSlots; ++k) slot_item[k] = slot_item[k + 1];
+      if (it.h != qhead) {
+        if constexpr (kMma) q_fragments<D>(static_cast<const __nv_bfloat16*>(a.Q) + size_t(it.h) * D, qf, lane);
+        else c.q_slice(it.h, qs);
+        qhead = it.h;
+      }
+      const unsigned char* rec = ring + size_t(sl) * rec_bytes;
+      float e;
+      if constexpr (kMma) e = score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
+      else e = score_record_smem<T, D>(rec, R, a.t.inv_sqrt_d, qs, lane);
+      if (lane == 0) {
+        const uint32_t key = desc_key(e);
+        c.keysP(it.h, par)[it.pos] = key;
+        c.codesP(it.h, par)[it.pos] = it.code;
+        if (it.h != cur_h) {  // flush the previous head's min key and overflow flag
+          if (cur_h >= 0) {
+            atomicMax(&c.hstate(cur_h)->kinv[par], ~cur_kmin);
+            if (cur_ovf) atomicOr(&c.hstate(cur_h)->ovf[par], 1);
+          }
+          cur_h = it.h;
+          cur_kmin = 0xffffffffu;
+          cur_ovf = 0;
+        }
+        cur_kmin = min(cur_kmin, key);
+        if (s >= 1) {
+          if (it.h != ah) {
+            anchor = __ldcg(&c.hstate(it.h)->anchor);
+            ah = it.h;
+          }
+          unsigned long long w;
+          float t;
+          const int bin = anchored_bin(anchor, key, &w, &t);
+          if (bin < 0) cur_ovf = 1;
+          else atomicAdd(c.histP(it.h, par) + bin, w);
+        }
+      }
+      __syncwarp();
+      ++done;
+      --in_flight;
+      if (++slot_d == nslot) {
+        slot_d = 0;
+        phase_d ^= 1u;
+      }
+    }
+  }
+  if (lane == 0 && cur_h >= 0) {
+    atomicMax(&c.hstate(cur_h)->kinv[par], ~cur_kmin);
+    if (cur_ovf) atomicOr(&c.hstate(cur_h)->ovf[par], 1);
+  }
+}
+
+// ---------------------------------------------------------------- select phase
+// One CTA per head: the cut of step s (small path, anchored histogram or the
+// in-CTA histograms), the kept entries listed in entry order, and the state
+// of step s+1 (histogram cleared, anchor = step s's max).
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_constant__ DecodeArgs a, int s) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  const Ctx<T, D> c(a);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nh = a.nheads, b = a.t.block;
+  const int par = s & 1;
+  // ---------------- select phase: one CTA per head
+  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+    HeadState* hs = c.hstate(h);
+    const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
+    if (n == 0) {
+      __syncthreads();
+      if (tid == 0) hs->kept = 0;
+      continue;
+    }
+    const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
+    const float anchor_h = __ldcg(&hs->anchor);
+    const int ovf = __ldcg(&hs->ovf[par]);
+    const long long scored0 = __ldcg(&hs->scored);
+    const uint32_t* gk = c.keysP(h, par);
+    const uint32_t* gc = c.codesP(h, par);
+    if (a.scored) {  // codes of the scored nodes
+      int32_t* out = a.scored + size_t(h) * a.scored_cap;
+      for (long long i = tid; i < n; i += kDecThreads)
+        if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
+    }
+    const float m = desc_key_value(kmin);
+    // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
+    const int ncache = n <= kDecThreads ? 0 : int(min64(n, kCacheKeys));
+    uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
+    for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
+    cp_async_commit();
+    cp_async_wait(0);
+    __syncthreads();
+    const StepView E{ck, ncache, gk, gc};
+    unsigned long long cut = ~0ull;
+    if (!a.p_all) {
+      if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
+      else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
+        cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
+      else cut = select_cut(a, E, n, kmin, sm, h, s);
+    }
+    // the kept entries (order key <= cut), listed in entry
+    // order: each warp owns a contiguous segment; the code is read only for a
+    // key equal to the cut's
+    long long n_kept = 0;
+    {
+      const uint32_t cut32 = uint32_t(cut >> 32);
+      const int n32 = int(n);
+      const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
+      const int wlo = min(n32, wid * wseg), whi = min(n32, wlo + wseg);
+      auto kept_at = [&](int i) {
+        const uint32_t k = E.key(i);
+        return k < cut32 || (k == cut32 && entry_key64(a, Entry{k, E.code(i)}) <= cut);
+      };
+      uint32_t wk = 0;
+      for (int base = wlo; base < whi; base += 32) {
+        const int i = base + lane;
+        wk += __popc(__ballot_sync(0xffffffffu, i < whi && kept_at(i)));
+      }
+      if (lane == 0) sm.red32[wid] = wk;
+      __syncthreads();
+      uint32_t off = 0;
+      for (int w = 0; w < kDecWarps; ++w) {
+        if (w < wid) off += sm.red32[w];
+        n_kept += sm.red32[w];
+      }
+      uint32_t* kl = c.keptl(h);
+      for (int base = wlo; base < whi; base += 32) {
+        const int i = base + lane;
+        const bool kp = i < whi && kept_at(i);
+        const unsigned mk = __ballot_sync(0xffffffffu, kp);
+        if (kp) kl[off + __popc(mk & ((1u << lane) - 1u))] = uint32_t(i);
+        off += __popc(mk);
+      }
+    }
+    // state for the next step: its histogram cleared, its anchor = this step's max
+    unsigned long long* nhist = c.histP(h, par ^ 1);
+    for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
+    __syncthreads();
+    if (tid == 0) {
+      hs->kept = n_kept;
+      hs->n[par ^ 1] = 0;
+      hs->anchor = m;
+      hs->kinv[par ^ 1] = 0u;
+      hs->ovf[par ^ 1] = 0;
+      hs->scored = scored0 + n;
+      hs->steps = hs->steps + 1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- finalize
+// One CTA per head: the kept leaves in block order from the head's bitmap
+// (each warp owns a contiguous run of words: counts, one scan over warps, then
+// writes), which it leaves zeroed.
+struct FinSmem {
+  uint32_t red32[kDecWarps];
+};
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads) finalize_kernel(const __grid_constant__ DecodeArgs a) {
+  __shared__ FinSmem sm;
+  const Ctx<T, D> c(a);
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int nh = a.nheads;
-  const int b = a.t.block;
-  const int R = a.t.refs;
-  unsigned long long bar_target = a.bar_base;
-  auto ws = [&](int h) { return a.ws + uint64_t(h) * a.ws_per_bh; };
-  // per-head workspace: step keys [2][cap4], step codes [2][cap4] (parity buffers: step s in s & 1),
-  // anchored histograms [2][kBins], kept entries of the last select [cap4], kept leaves [cap_list];
-  // leaf bitmaps live in the flow state
-  const int64_t cap4 = (a.cap_sel + 3) & ~int64_t(3);
-  auto keysP = [&](int h, int par) { return reinterpret_cast<uint32_t*>(ws(h) + par * cap4 * 4); };
-  auto codesP = [&](int h, int par) { return reinterpret_cast<uint32_t*>(ws(h) + (2 + par) * cap4 * 4); };
-  auto histP = [&](int h, int par) {
-    return reinterpret_cast<unsigned long long*>(ws(h) + 4 * cap4 * 4 + par * kBins * 8);
-  };
-  auto keptl = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 4 * cap4 * 4 + 2 * kBins * 8); };
-  auto leaves = [&](int h) { return reinterpret_cast<uint32_t*>(ws(h) + 5 * cap4 * 4 + 2 * kBins * 8); };
-  const int64_t bm_words = decode_bitmap_words(a.cap_sel);
-  auto hstate = [&](int h) { return reinterpret_cast<HeadState*>(a.flow) + h; };
-  auto bitmap = [&](int h) {
-    return reinterpret_cast<uint32_t*>(a.flow + size_t(nh) * sizeof(HeadState)) + h * bm_words;
-  };
-  auto q_slice = [&](int h, float* qs) {
-    const T* q = static_cast<const T*>(a.Q) + size_t(h) * D + (lane % CPR) * EPC;
-    unpack16<T>(*reinterpret_cast<const uint4*>(q), qs);
-  };
-  const int rec_bytes = int(a.t.rec_bytes);
-  // scoring ring: nslot record slots per warp below the prefix area; warps past
-  // score_warps (only when a record is larger than a warp's share) do not score
-  const int nslot = max(1, min(kMaxSlots, (kPrefOff / kDecWarps) / rec_bytes));
-  const int score_warps = min(kDecWarps, kPrefOff / (nslot * rec_bytes));
-  unsigned char* ring = sm.u + size_t(wid) * nslot * rec_bytes;
-
-  const bool routed = a.n_steps > 0 && a.n_roots > 0;
-  stamp(a, 0);
-  if (routed) {
-    // Step loop, in lock step over all heads: a scoring phase (all warps) makes
-    // step s's entries, a grid barrier, a select phase (one CTA per head) keeps
-    // a prefix of them, a grid barrier.  Step s's entries are the roots (s = 0,
-    // root i at position i) or the children of step s-1's kept non-leaves, at
-    // positions reserved per warp batch with one atomic add per head (their
-    // order varies from run to run; nothing downstream depends on it).  The
-    // phase after the last select only records the kept leaves.
-    constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
-    if (lane == 0) {
-      for (int k = 0; k < nslot; ++k) mbar_init(&sm.mbar[wid][k], 1);
-      mbar_init_fence();
-    }
-    __syncwarp();
-    unsigned long long n_issued = 0, n_done = 0;  // records through this warp's ring so far (slot k % nslot)
-    float qs[EPC];
-    uint32_t qf[D / 16][2];
-    int qhead = -1;
-    const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
-    const long long nwarps = (long long)gridDim.x * score_warps;
-    for (int s = 0; s <= a.n_steps; ++s) {
-      const int par = s & 1;
-      // ---------------- scoring phase: units = roots (s = 0) or the kept entries of step s-1
-      for (int i = tid; i < nh; i += kDecThreads)
-        sm.pref()[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hstate(i)->kept), 0), a.cap_sel);
-      __syncthreads();
-      const long long total = build_prefix(sm, nh);
-      stamp(a, 2 + 2 * s);
-      const long long u0 = gwarp < 0 ? 0 : total * gwarp / nwarps;
-      const long long u1 = gwarp < 0 ? 0 : total * (gwarp + 1) / nwarps;
-      int cur_h = -1;           // lane 0: head of the pending min-key update
-      uint32_t cur_kmin = 0xffffffffu;
-      int cur_ovf = 0;
-      int ah = -1;              // head whose anchor is loaded
-      float anchor = 0.f;
-      for (long long ub = u0; ub < u1; ub += 32) {
-        // one unit per lane: its head, its first output position, its code
-        const long long u = ub + lane;
-        int uh = 0;
-        long long upos = 0;
-        uint32_t ucode = 0;
-        bool has = false;  // the unit makes records (a root, or a kept non-leaf)
-        if (u < u1) {
-          uh = owner_of(sm, nh, u);
-          const long long k = u - sm.pref()[uh];
-          if (s == 0) {
-            ucode = root_code(a, k);
-            upos = k;
-            has = valid_code(a, ucode);
-          } else {
-            const uint32_t idx = __ldcg(keptl(uh) + k);
-            const uint32_t code = idx < uint32_t(a.cap_sel) ? __ldcg(codesP(uh, par ^ 1) + idx) : 0u;
-            if (valid_code(a, code)) {
-              if (code_level(code) == 1) {
-                atomicOr(bitmap(uh) + (code_index(code) >> 5), 1u << (code_index(code) & 31u));
-              } else {
-                ucode = code;
-                has = true;
-              }
-            }
-          }
-        }
-        if (s >= 1) {  // positions: one reservation per head segment of the batch
-          unsigned todo = __ballot_sync(0xffffffffu, has);
-          while (todo) {
-            const int l0 = __ffs(todo) - 1;
-            const int h0 = __shfl_sync(0xffffffffu, uh, l0);
-            const unsigned seg = __ballot_sync(0xffffffffu, has && uh == h0);
-            long long bs = 0;
-            if (lane == l0) {
-              const long long need = (long long)__popc(seg) * b;
-              bs = (long long)atomicAdd(reinterpret_cast<unsigned long long*>(&hstate(h0)->n[par]),
-                                        (unsigned long long)need);
-              if (bs + need > a.cap_sel) {
-                raise_status(a.t.status, ZHA_ERR_CAPACITY);
-                bs = -1;
-              }
-            }
-            bs = __shfl_sync(0xffffffffu, bs, l0);
-            if (has && uh == h0) {
-              upos = bs + (long long)__popc(seg & ((1u << lane) - 1u)) * b;
-              if (bs < 0) has = false;
-            }
-            todo &= ~seg;
-          }
-        }
-        const unsigned mhas = __ballot_sync(0xffffffffu, has);
-        if (!mhas) continue;
-        const int per = s == 0 ? 1 : b;  // records per unit
-        const int items = __popc(mhas) * per;
-        // item k: record (k % per) of the (k / per)-th unit with records, in lane order
-        struct Cursor {
-          unsigned rem;
-          int child;
-        };
-        struct Item {
-          int h;
-          long long pos;
-          uint32_t code;
-        };
-        auto next_item = [&](Cursor& cur) -> Item {  // the whole warp calls it, in item order
-          const int pl = __ffs(cur.rem) - 1;
-          Item it;
-          it.h = __shfl_sync(0xffffffffu, uh, pl);
-          it.pos = __shfl_sync(0xffffffffu, upos, pl) + cur.child;
-          const uint32_t pc = __shfl_sync(0xffffffffu, ucode, pl);
-          it.code = s == 0 ? pc : node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(cur.child));
-          if (++cur.child == per) {
-            cur.child = 0;
-            cur.rem &= cur.rem - 1u;
-          }
-          return it;
-        };
-        Cursor cur_i{mhas, 0};
-        Item slot_item[kMaxSlots];
-        int issued = 0, done = 0;
-        while (done < items) {
-          while (issued < items && issued - done < nslot) {
-            const Item it = next_item(cur_i);
-            const int sl = int(n_issued % unsigned(nslot));
-            unsigned char* slot = ring + size_t(sl) * rec_bytes;
-            if (lane == 0) {
-              fence_proxy_async();  // the slot's last reads (generic proxy) before the copy writes it
-              const int kvh = (it.h % a.t.hq) / a.t.group;
-              bulk_load(slot, a.t.rec(code_level(it.code), kvh, code_index(it.code)), unsigned(rec_bytes),
-                        &sm.mbar[wid][sl]);
-            }
+  const int64_t bm_words = c.bm_words;
+  // ---------------- finalize: the kept leaves of each head, in block order, from its bitmap
+  // (each warp owns a contiguous run of words: counts, one block scan over warps, then writes)
+  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
+    uint32_t* bm = c.bitmap(h);
+    const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
+    const long long wseg = (nw + kDecWarps - 1) / kDecWarps;
+    const long long w_lo = min64(nw, wid * wseg), w_hi = min64(nw, w_lo + wseg);
+    uint32_t cnt = 0;
+    for (long long wi = w_lo + lane; wi < w_hi; wi += 32) cnt += __popc(__ldcg(bm + wi));
 #pragma unroll
-            for (int k = 0; k < kMaxSlots; ++k)
-              if (k == issued - done) slot_item[k] = it;
-            ++issued;
-            ++n_issued;
-          }
-          const int sl = int(n_done % unsigned(nslot));
-          const unsigned parity = unsigned((n_done / unsigned(nslot)) & 1ull);
-          {
-            long long it = 0;
-            while (!mbar_try_wait(&sm.mbar[wid][sl], parity)) {
-              if (++it > a.spin_limit) {  // a copy that never lands: report, then give it one more bound
-                if (lane == 0) raise_status(a.t.status, ZHA_ERR_TIMEOUT);
-                if (it > 2 * a.spin_limit) break;
-              }
-            }
-          }
-          __syncwarp();
-          const Item it = slot_item[0];
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if (lane == 0) sm.red32[wid] = cnt;
+    __syncthreads();
+    long long pos = 0, total = 0;
+    for (int w = 0; w < kDecWarps; ++w) {
+      if (w < wid) pos += sm.red32[w];
+      total += sm.red32[w];
+    }
+    const int leaf0 = nw > 0 ? int(__ldcg(bm) & 1u) : 0;
+    __syncthreads();
+    for (long long wb = w_lo; wb < w_hi; wb += 32) {
+      const long long wi = wb + lane;
+      uint32_t bits = wi < w_hi ? __ldcg(bm + wi) : 0u;
+      uint32_t pc = __popc(bits), ex = pc;
 #pragma unroll
-          for (int k = 0; k + 1 < kMaxSlots; ++k) slot_item[k] = slot_item[k + 1];
-          if (it.h != qhead) {
-            if constexpr (kMma) q_fragments<D>(static_cast<const __nv_bfloat16*>(a.Q) + size_t(it.h) * D, qf, lane);
-            else q_slice(it.h, qs);
-            qhead = it.h;
-          }
-          const unsigned char* rec = ring + size_t(sl) * rec_bytes;
-          float e;
-          if constexpr (kMma) e = score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
-          else e = score_record_smem<T, D>(rec, R, a.t.inv_sqrt_d, qs, lane);
-          if (lane == 0) {
-            const uint32_t key = desc_key(e);
-            keysP(it.h, par)[it.pos] = key;
-            codesP(it.h, par)[it.pos] = it.code;
-            if (it.h != cur_h) {  // flush the previous head's min key and overflow flag
-              if (cur_h >= 0) {
-                atomicMax(&hstate(cur_h)->kinv[par], ~cur_kmin);
-                if (cur_ovf) atomicOr(&hstate(cur_h)->ovf[par], 1);
-              }
-              cur_h = it.h;
-              cur_kmin = 0xffffffffu;
-              cur_ovf = 0;
-            }
-            cur_kmin = min(cur_kmin, key);
-            if (s >= 1) {
-              if (it.h != ah) {
-                anchor = __ldcg(&hstate(it.h)->anchor);
-                ah = it.h;
-              }
-              unsigned long long w;
-              float t;
-              const int bin = anchored_bin(anchor, key, &w, &t);
-              if (bin < 0) cur_ovf = 1;
-              else atomicAdd(histP(it.h, par) + bin, w);
-            }
-          }
-          __syncwarp();
-          ++done;
-          ++n_done;
-        }
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, ex, off);
+        if (lane >= off) ex += y;
       }
-      if (lane == 0 && cur_h >= 0) {
-        atomicMax(&hstate(cur_h)->kinv[par], ~cur_kmin);
-        if (cur_ovf) atomicOr(&hstate(cur_h)->ovf[par], 1);
+      const uint32_t wtot = __shfl_sync(0xffffffffu, ex, 31);
+      long long p = pos + ex - pc;
+      if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
+      while (bits) {
+        const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
+        bits &= bits - 1u;
+        if (p < a.cap_list) c.leaves(h)[p] = idx;
+        if (a.kept && p < a.kept_stride) a.kept[size_t(h) * a.kept_stride + p] = int32_t(idx);
+        ++p;
       }
-      if (grid_sync(a, sm, bar_target)) return;
-      stamp(a, 3 + 2 * s);
-      if (s == a.n_steps) break;  // the last phase only recorded kept leaves
-
-      // ---------------- select phase: one CTA per head
-      for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-        HeadState* hs = hstate(h);
-        const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
-        if (n == 0) {
-          __syncthreads();
-          if (tid == 0) hs->kept = 0;
-          continue;
-        }
-        const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
-        const float anchor_h = __ldcg(&hs->anchor);
-        const int ovf = __ldcg(&hs->ovf[par]);
-        const long long scored0 = __ldcg(&hs->scored);
-        const uint32_t* gk = keysP(h, par);
-        const uint32_t* gc = codesP(h, par);
-        if (a.scored) {  // codes of the scored nodes
-          int32_t* out = a.scored + size_t(h) * a.scored_cap;
-          for (long long i = tid; i < n; i += kDecThreads)
-            if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
-        }
-        const float m = desc_key_value(kmin);
-        // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
-        const int ncache = n <= kDecThreads ? 0 : int(min64(n, kCacheKeys));
-        uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
-        for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
-        cp_async_commit();
-        cp_async_wait(0);
-        __syncthreads();
-        const StepView E{ck, ncache, gk, gc};
-        unsigned long long cut = ~0ull;
-        if (!a.p_all) {
-          if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
-          else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
-            cut = select_cut_anchored(a, E, n, anchor_h, histP(h, par), sm, h, s);
-          else cut = select_cut(a, E, n, kmin, sm, h, s);
-        }
-        // the kept entries (order key <= cut), listed in entry
-        // order: each warp owns a contiguous segment; the code is read only for a
-        // key equal to the cut's
-        long long n_kept = 0;
-        {
-          const uint32_t cut32 = uint32_t(cut >> 32);
-          const int n32 = int(n);
-          const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
-          const int wlo = min(n32, wid * wseg), whi = min(n32, wlo + wseg);
-          auto kept_at = [&](int i) {
-            const uint32_t k = E.key(i);
-            return k < cut32 || (k == cut32 && entry_key64(a, Entry{k, E.code(i)}) <= cut);
-          };
-          uint32_t wk = 0;
-          for (int base = wlo; base < whi; base += 32) {
-            const int i = base + lane;
-            wk += __popc(__ballot_sync(0xffffffffu, i < whi && kept_at(i)));
-          }
-          if (lane == 0) sm.red32[wid] = wk;
-          __syncthreads();
-          uint32_t off = 0;
-          for (int w = 0; w < kDecWarps; ++w) {
-            if (w < wid) off += sm.red32[w];
-            n_kept += sm.red32[w];
-          }
-          uint32_t* kl = keptl(h);
-          for (int base = wlo; base < whi; base += 32) {
-            const int i = base + lane;
-            const bool kp = i < whi && kept_at(i);
-            const unsigned mk = __ballot_sync(0xffffffffu, kp);
-            if (kp) kl[off + __popc(mk & ((1u << lane) - 1u))] = uint32_t(i);
-            off += __popc(mk);
-          }
-        }
-        // state for the next step: its histogram cleared, its anchor = this step's max
-        unsigned long long* nhist = histP(h, par ^ 1);
-        for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
-        __syncthreads();
-        if (tid == 0) {
-          hs->kept = n_kept;
-          hs->n[par ^ 1] = 0;
-          hs->anchor = m;
-          hs->kinv[par ^ 1] = 0u;
-          hs->ovf[par ^ 1] = 0;
-          hs->scored = scored0 + n;
-          hs->steps = hs->steps + 1;
-        }
-      }
-      if (grid_sync(a, sm, bar_target)) return;
+      pos += wtot;
     }
-    // ---------------- finalize: the kept leaves of each head, in block order, from its bitmap
-    for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-      uint32_t* bm = bitmap(h);
-      const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
-      long long carry = 0;
-      if (tid == 0) sm.bcast32[3] = 0;
-      for (long long w0 = 0; w0 < nw; w0 += kDecThreads) {
-        const long long wi = w0 + tid;
-        uint32_t bits = wi < nw ? __ldcg(bm + wi) : 0u;
-        if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
-        if (wi == 0 && (bits & 1u)) sm.bcast32[3] = 1;
-        uint32_t tot;
-        const uint32_t ex = block_scan_u32(uint32_t(__popc(bits)), sm.red32, &tot);
-        long long pos = carry + ex;
-        while (bits) {
-          const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
-          bits &= bits - 1u;
-          if (pos < a.cap_list) leaves(h)[pos] = idx;
-          if (a.kept && pos < a.kept_stride) a.kept[size_t(h) * a.kept_stride + pos] = int32_t(idx);
-          ++pos;
-        }
-        carry += tot;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        if (carry > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
-        hstate(h)->n_leaf = min64(carry, a.cap_list);
-        hstate(h)->leaf0 = sm.bcast32[3];
-      }
-      __syncthreads();
+    if (tid == 0) {
+      if (total > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+      c.hstate(h)->n_leaf = min64(total, a.cap_list);
+      c.hstate(h)->leaf0 = leaf0;
     }
-    if (grid_sync(a, sm, bar_target)) return;
+    __syncthreads();
   }
-  __syncthreads();
-  stamp(a, 1);
+}
 
-  // ---------------- attend (all CTAs)
+// ---------------------------------------------------------------- attention
+// Attended keys of head h: its kept blocks, the sink (token 0) unless block 0
+// is kept, the tail after the last complete block.
+template <typename T, int D>
+__device__ __forceinline__ long long att_head_keys(const Ctx<T, D>& c, int h, long long* nl, bool* sink) {
+  const DecodeArgs& a = c.a;
   const long long n1 = a.nl[1];
-  const long long tail = a.n_tokens - n1 * b;
-  auto head_keys = [&](int h, long long& nl, bool& sink) {
-    nl = 0;
-    int l0 = 0;
-    if (routed) {
-      nl = min64(max64(__ldcg(&hstate(h)->n_leaf), 0), a.cap_list);
-      l0 = __ldcg(&hstate(h)->leaf0);
-    }
-    sink = (n1 > 0) && !l0;
-    return nl * b + (sink ? 1 : 0) + tail;
-  };
-  for (int i = tid; i < nh; i += kDecThreads) {
+  const long long tail = a.n_tokens - n1 * a.t.block;
+  *nl = 0;
+  int l0 = 0;
+  if (a.n_steps > 0 && a.n_roots > 0) {
+    *nl = min64(max64(__ldcg(&c.hstate(h)->n_leaf), 0), a.cap_list);
+    l0 = __ldcg(&c.hstate(h)->leaf0);
+  }
+  *sink = (n1 > 0) && !l0;
+  return *nl * a.t.block + (*sink ? 1 : 0) + tail;
+}
+
+// The chunk partition of all heads' attended keys over `grid` CTAs (the same
+// in the attention and combine kernels): chunk size (>= 32 keys, so that a CTA
+// owns at most about kAttItems chunks), and per-head chunk prefix in pref[0..nh].
+template <typename T, int D, int NT>
+__device__ __forceinline__ void att_partition(const Ctx<T, D>& c, long long* pref, unsigned long long* red64,
+                                              int grid, long long* chunk_out, long long* total_out) {
+  const int nh = c.nh;
+  for (int i = threadIdx.x; i < nh; i += NT) {
     long long nl;
     bool sink;
-    sm.pref()[1 + i] = head_keys(i, nl, sink);
+    pref[1 + i] = att_head_keys<T, D>(c, i, &nl, &sink);
   }
   __syncthreads();
-  const long long total_keys = build_prefix(sm, nh);
-  // chunk size: at least 32 keys, large enough that a CTA owns <= kItemsPerCta chunks (+1 per head)
-  long long chunk = (total_keys + (long long)gridDim.x * kItemsPerCta - 1) / ((long long)gridDim.x * kItemsPerCta);
+  const long long total_keys = build_prefix<NT>(pref, red64, nh);
+  long long chunk = (total_keys + (long long)grid * kAttItems - 1) / ((long long)grid * kAttItems);
   chunk = max64(32, chunk);
-  for (int i = tid; i < nh; i += kDecThreads) {
+  for (int i = threadIdx.x; i < nh; i += NT) {
     long long nl;
     bool sink;
-    sm.pref()[1 + i] = (head_keys(i, nl, sink) + chunk - 1) / chunk;
+    pref[1 + i] = (att_head_keys<T, D>(c, i, &nl, &sink) + chunk - 1) / chunk;
   }
   __syncthreads();
-  const long long total_items = build_prefix(sm, nh);
-  stamp(a, 60);
+  *total_out = build_prefix<NT>(pref, red64, nh);
+  *chunk_out = chunk;
+}
+
+// Every head's attended keys (kept blocks, sink, tail) are cut into chunks of
+// >= 32 keys; CTAs own contiguous ranges of chunks, each warp runs a chunk at a
+// time (batches of keys: scores first, then one rescale of the running sums),
+// and each CTA merges its chunks per head into one partial.
+constexpr int kAttSlots = kAttItems + 16;  // partial slots of a CTA (per-head rounding adds up to one per head)
+struct __align__(16) AttSmem {
+  float part[kAttSlots][2 + 128];
+  long long pref[kMaxHeads + 1];
+  unsigned long long red64[kAttWarps];
+};
+
+// CTAs per SM the attention kernel is compiled for: two for the tensor-core
+// (bf16) path, whose tiles need up to 128 registers, three for the fp32 path.
+template <typename T>
+constexpr int att_ctas_per_sm() { return std::is_same<T, __nv_bfloat16>::value ? 2 : 3; }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int EPC = 16 / sizeof(T);
+  constexpr int CPR = D * sizeof(T) / 16;
+  constexpr int KPW = 32 / CPR;  // keys per warp pass
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  AttSmem& sm = *reinterpret_cast<AttSmem*>(smem_raw);
+  const Ctx<T, D> c(a);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nh = a.nheads, b = a.t.block;
+  const long long n1 = a.nl[1];
+  const DivU32 divb{uint32_t(b)};  // key index -> (block, token within it); keys per head < 2^31
+  long long chunk, total_items;
+  att_partition<T, D, kAttThreads>(c, sm.pref, sm.red64, int(gridDim.x), &chunk, &total_items);
   const long long c0 = (long long)blockIdx.x * total_items / gridDim.x;
-  const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kPartSlots);
+  const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kAttSlots);
   if (tid == 0 && (long long)(blockIdx.x + 1) * total_items / gridDim.x > c1) raise_status(a.t.status, ZHA_ERR_CAPACITY);
-  float (*part)[2 + 128] = reinterpret_cast<float (*)[2 + 128]>(sm.u);
+  float (*part)[2 + 128] = sm.part;
   {
     const int sub = lane / CPR, cl = lane % CPR;
-    constexpr int kU = 8;
-    for (long long it = c0 + wid; it < c1; it += kDecWarps) {
-      const int h = owner_of(sm, nh, it);
-      const long long ci = it - sm.pref()[h];
+    constexpr int kU = 4;
+    for (long long it = c0 + wid; it < c1; it += kAttWarps) {
+      const int h = owner_of(sm.pref, nh, it);
+      const long long ci = it - sm.pref[h];
       const int kvh = (h % a.t.hq) / a.t.group;
       long long nl;
       bool sink;
-      const long long kh = head_keys(h, nl, sink);
+      const long long kh = att_head_keys<T, D>(c, h, &nl, &sink);
       const long long leaf_keys = nl * b;
       const long long k0 = ci * chunk, k1 = min64(kh, k0 + chunk);
       float qs[EPC];
-      q_slice(h, qs);
+      c.q_slice(h, qs);
       const T* Kh = static_cast<const T*>(a.t.K) + size_t(kvh) * a.t.capacity * D;
       const T* Vh = static_cast<const T*>(a.t.V) + size_t(kvh) * a.t.capacity * D;
-      const uint32_t* lv = leaves(h);
+      const uint32_t* lv = c.leaves(h);
       // leaf indices of the chunk's first 32 blocks, one per lane
-      const long long lf0 = k0 / b;
+      uint32_t r0;
+      const long long lf0 = divb.div(uint32_t(k0), &r0);
       uint32_t leaf_reg = 0;
       if (lf0 + lane < nl) leaf_reg = __ldcg(lv + lf0 + lane);
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // tensor-core path: 16-key tiles, S = K q^T and O^T += V^T P with
+        // mma.sync m16n8k16 as in the dense kernel, q in column 0 of the B
+        // operand (the other columns are zero and ignored); the fp32 sums l
+        // use the unrounded weights, O^T the weights split into hi + lo bf16
+        // parts (relative rounding about 2^-16 instead of 2^-8)
+        constexpr int NV = D / 32, MT = D / 16, VW = D / 64;
+        const int g = lane >> 2, t4 = lane & 3;
+        const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(Kh);
+        const __nv_bfloat16* Vb = reinterpret_cast<const __nv_bfloat16*>(Vh);
+        uint4 qv[NV];
+        {
+          const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.Q) + size_t(h) * D;
+#pragma unroll
+          for (int v = 0; v < NV; ++v)
+            qv[v] = g == 0 ? *reinterpret_cast<const uint4*>(q + 8 * t4 + 32 * v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // token of attended key idx (the whole warp calls it; idx < k1)
+        auto tok_of = [&](long long idx) -> long long {
+          uint32_t rb;
+          const long long li = divb.div(uint32_t(idx), &rb);
+          const uint32_t lr = __shfl_sync(0xffffffffu, leaf_reg, int((li - lf0) & 31));
+          long long tok;
+          if (idx < leaf_keys) tok = int64_t((li - lf0 < 32) ? lr : __ldcg(lv + li)) * b + rb;
+          else if (sink && idx == leaf_keys) tok = 0;
+          else tok = n1 * b + (idx - leaf_keys - (sink ? 1 : 0));
+          if (tok < 0 || tok >= a.n_tokens) {  // a corrupted leaf index: read token 0, report
+            raise_status(a.t.status, ZHA_ERR_CAPACITY);
+            tok = 0;
+          }
+          return tok;
+        };
+        float om[MT][4];
+#pragma unroll
+        for (int i = 0; i < MT; ++i) om[i][0] = om[i][1] = om[i][2] = om[i][3] = 0.f;
+        float mr[2] = {-INFINITY, -INFINITY}, lr2[2] = {0.f, 0.f};
+        for (long long t0 = k0; t0 < k1; t0 += 16) {
+          const long long last = k1 - 1;
+          const long long tk0 = tok_of(min64(t0 + g, last)), tk1 = tok_of(min64(t0 + g + 8, last));
+          uint4 kr0[NV], kr1[NV];
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            kr0[v] = ldg_stream(Kb + size_t(tk0) * D + 8 * t4 + 32 * v);
+            kr1[v] = ldg_stream(Kb + size_t(tk1) * D + 8 * t4 + 32 * v);
+          }
+          long long tv[4];
+          tv[0] = tok_of(min64(t0 + 2 * t4, last));
+          tv[1] = tok_of(min64(t0 + 2 * t4 + 1, last));
+          tv[2] = tok_of(min64(t0 + 2 * t4 + 8, last));
+          tv[3] = tok_of(min64(t0 + 2 * t4 + 9, last));
+          uint4 vr[4][VW];
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int w = 0; w < VW; ++w) vr[rr][w] = ldg_stream(Vb + size_t(tv[rr]) * D + (D / 8) * g + 8 * w);
+          float sv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j) {
+            const int v = j >> 1, hf = j & 1;
+            const uint32_t af[4] = {word_of(kr0[v], 2 * hf), word_of(kr1[v], 2 * hf), word_of(kr0[v], 2 * hf + 1),
+                                    word_of(kr1[v], 2 * hf + 1)};
+            const uint32_t bf[2] = {word_of(qv[v], 2 * hf), word_of(qv[v], 2 * hf + 1)};
+            mma_bf16_16816(sv, af, bf);
+          }
+          const bool v0 = t0 + g < k1, v1 = t0 + g + 8 < k1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sv[i] *= a.t.inv_sqrt_d;
+          if (!v0) sv[0] = sv[1] = -INFINITY;
+          if (!v1) sv[2] = sv[3] = -INFINITY;
+          float pp[4];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {  // key t0 (row 0) is always valid: mx is finite
+            float mx = fmaxf(sv[hh], sv[2 + hh]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mn = fmaxf(mr[hh], mx);
+            const float sc = expf(mr[hh] - mn);
+            pp[hh] = expf(sv[hh] - mn);
+            pp[2 + hh] = expf(sv[2 + hh] - mn);
+            lr2[hh] = fmaf(lr2[hh], sc, pp[hh] + pp[2 + hh]);
+            mr[hh] = mn;
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+              om[i][hh] *= sc;
+              om[i][2 + hh] *= sc;
+            }
+          }
+          // P as hi + lo bf16 parts (two products), so that its rounding stays near fp32
+          float plo[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) plo[i] = pp[i] - __bfloat162float(__float2bfloat16_rn(pp[i]));
+          const uint32_t pb[2] = {movmatrix_trans(pack_bf16(pp[0], pp[1])), movmatrix_trans(pack_bf16(pp[2], pp[3]))};
+          const uint32_t pl[2] = {movmatrix_trans(pack_bf16(plo[0], plo[1])),
+                                  movmatrix_trans(pack_bf16(plo[2], plo[3]))};
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            uint32_t af[4];
+            if (D == 128) {
+              const int w = i >> 1;
+              const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+              af[0] = __byte_perm(word_of(vr[0][0], w), word_of(vr[1][0], w), sel);
+              af[1] = __byte_perm(word_of(vr[0][VW - 1], w), word_of(vr[1][VW - 1], w), sel);
+              af[2] = __byte_perm(word_of(vr[2][0], w), word_of(vr[3][0], w), sel);
+              af[3] = __byte_perm(word_of(vr[2][VW - 1], w), word_of(vr[3][VW - 1], w), sel);
+            } else {
+              const int w0 = i >> 1, w1 = (4 + i) >> 1;
+              const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+              af[0] = __byte_perm(word_of(vr[0][0], w0), word_of(vr[1][0], w0), sel);
+              af[1] = __byte_perm(word_of(vr[0][0], w1), word_of(vr[1][0], w1), sel);
+              af[2] = __byte_perm(word_of(vr[2][0], w0), word_of(vr[3][0], w0), sel);
+              af[3] = __byte_perm(word_of(vr[2][0], w1), word_of(vr[3][0], w1), sel);
+            }
+            mma_bf16_16816(om[i], af, pb);
+            mma_bf16_16816(om[i], af, pl);
+          }
+        }
+        // column 0: l over the 8 lanes that share t4; m is already common to them
+        lr2[0] += __shfl_xor_sync(0xffffffffu, lr2[0], 4);
+        lr2[0] += __shfl_xor_sync(0xffffffffu, lr2[0], 8);
+        lr2[0] += __shfl_xor_sync(0xffffffffu, lr2[0], 16);
+        float* P = part[it - c0];
+        if (lane == 0) {
+          P[0] = mr[0];
+          P[1] = lr2[0];
+        }
+        if (t4 == 0) {
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            const int dA = (D == 128) ? 16 * g + i : 8 * g + i;
+            const int dB = (D == 128) ? 16 * g + 8 + i : 8 * g + 4 + i;
+            P[2 + dA] = om[i][0];
+            P[2 + dB] = om[i][2];
+          }
+        }
+        continue;
+      }
       float m_run = -INFINITY, l_run = 0.f, o[EPC];
 #pragma unroll
       for (int i = 0; i < EPC; ++i) o[i] = 0.f;
@@ -1546,12 +1799,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           const long long idx = wb + (long long)u * KPW + sub;
           ok[u] = idx < k1;
           long long tok = 0;
-          const long long li = idx / b;
+          uint32_t rb;
+          const long long li = divb.div(uint32_t(idx), &rb);
           // every lane takes part in the shuffle; only leaf keys use the value
           const uint32_t lr = __shfl_sync(0xffffffffu, leaf_reg, int((li - lf0) & 31));
           if (idx < leaf_keys) {
             const uint32_t leaf = (li - lf0 < 32) ? lr : __ldcg(lv + li);
-            tok = int64_t(leaf) * b + idx % b;
+            tok = int64_t(leaf) * b + rb;
           } else if (sink && idx == leaf_keys) {
             tok = 0;
           } else {
@@ -1566,29 +1820,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             vv[u] = ldg_stream(Vh + size_t(tok) * D + cl * EPC);
           }
         }
+        // the batch's scores, independently; then one rescale of the running sums
+        float sc8[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
           float kx[EPC];
-          float s = 0.f;
+          float sv = 0.f;
           if (ok[u]) {
             unpack16<T>(kv[u], kx);
 #pragma unroll
-            for (int i = 0; i < EPC; ++i) s = fmaf(kx[i], qs[i], s);
+            for (int i = 0; i < EPC; ++i) sv = fmaf(kx[i], qs[i], sv);
           }
+          sc8[u] = sv;
+        }
 #pragma unroll
-          for (int off = CPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-          if (ok[u]) {
-            s *= a.t.inv_sqrt_d;
-            const float mn = fmaxf(m_run, s);
-            const float sc = expf(m_run - mn);
-            const float pk = expf(s - mn);
-            l_run = l_run * sc + pk;
+        for (int off = CPR / 2; off > 0; off >>= 1) {
+#pragma unroll
+          for (int u = 0; u < kU; ++u) sc8[u] += __shfl_xor_sync(0xffffffffu, sc8[u], off);
+        }
+        float mb = m_run;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          sc8[u] = ok[u] ? sc8[u] * a.t.inv_sqrt_d : -INFINITY;
+          mb = fmaxf(mb, sc8[u]);
+        }
+        if (mb != -INFINITY) {
+          const float r = expf(m_run - mb);
+          l_run *= r;
+#pragma unroll
+          for (int i = 0; i < EPC; ++i) o[i] *= r;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            if (!ok[u]) continue;
+            const float pk = expf(sc8[u] - mb);
+            l_run += pk;
             float vx[EPC];
             unpack16<T>(vv[u], vx);
 #pragma unroll
-            for (int i = 0; i < EPC; ++i) o[i] = fmaf(pk, vx[i], o[i] * sc);
-            m_run = mn;
+            for (int i = 0; i < EPC; ++i) o[i] = fmaf(pk, vx[i], o[i]);
           }
+          m_run = mb;
         }
       }
       // merge the KPW lane groups of the warp (lanes l, l+CPR, ... hold the same d-range)
@@ -1619,13 +1890,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
   }
   __syncthreads();
-  stamp(a, 26);
   // merge this CTA's chunks per head segment; one partial per segment, stored at
   // the global slot of the segment's first chunk
-  for (long long seg = c0 + wid; seg < c1; seg += kDecWarps) {
-    const int h = owner_of(sm, nh, seg);
-    if (seg != c0 && seg != sm.pref()[h]) continue;  // not the first chunk of a segment
-    const long long send = min64(c1, sm.pref()[h + 1]);
+  for (long long seg = c0 + wid; seg < c1; seg += kAttWarps) {
+    const int h = owner_of(sm.pref, nh, seg);
+    if (seg != c0 && seg != sm.pref[h]) continue;  // not the first chunk of a segment
+    const long long send = min64(c1, sm.pref[h + 1]);
     float M = -INFINITY;
     for (long long j = seg; j < send; ++j) M = fmaxf(M, part[j - c0][0]);
     float L = 0.f;
@@ -1650,65 +1920,94 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     for (int q = 0; q < (D + 31) / 32; ++q)
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
   }
-  stamp(a, 27);
-  if (grid_sync(a, sm, bar_target)) return;
-  stamp(a, 28);
+}
 
-  // ---------------- combine (one CTA per head)
+// ---------------------------------------------------------------- combine
+// One CTA per head: the partials of the head (one per attention CTA that met
+// it) rescaled to their common max and summed -> O; the head's statistics and
+// kept count; the head's state zeroed for the next call.
+template <typename T, int D>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_constant__ DecodeArgs a, int att_grid) {
+  __shared__ long long pref[kMaxHeads + 1];
+  __shared__ unsigned long long red64[kCombThreads / 32];
+  __shared__ uint32_t red32[kCombThreads / 32];
+  __shared__ float pm[kCombThreads];
+  __shared__ long long ps[kCombThreads];
+  __shared__ float redf[kCombThreads];
+  const Ctx<T, D> c(a);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nh = a.nheads, b = a.t.block;
+  constexpr int NW = kCombThreads / 32;
+  long long chunk, total_items;
+  att_partition<T, D, kCombThreads>(c, pref, red64, att_grid, &chunk, &total_items);
+  const long long n1 = a.nl[1];
+  const long long tail = a.n_tokens - n1 * b;
   for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-    const long long p0 = sm.pref()[h], p1 = sm.pref()[h + 1];
-    // partial slots: one per CTA whose chunk range meets [p0, p1), at max(p0, range start)
-    float M = -INFINITY;
-    auto range_start = [&](long long c) { return (c * total_items) / (long long)gridDim.x; };
-    long long cfirst = (p0 * gridDim.x) / max64(total_items, 1);
+    const long long p0 = pref[h], p1 = pref[h + 1];
+    // partial slots: one per attention CTA whose chunk range meets [p0, p1), at
+    // max(p0, range start); thread t takes the t-th of them
+    auto range_start = [&](long long cc) { return (cc * total_items) / (long long)att_grid; };
+    long long cfirst = (p0 * att_grid) / max64(total_items, 1);
     while (cfirst > 0 && range_start(cfirst) > p0) --cfirst;
-    while (cfirst + 1 < gridDim.x && range_start(cfirst + 1) <= p0) ++cfirst;
-    for (long long c = cfirst + tid; c < gridDim.x; c += kDecThreads) {
-      const long long cs = max64(p0, range_start(c));
-      if (cs >= p1) break;
-      if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
-      M = fmaxf(M, __ldcg(a.attn_part + size_t(cs) * (2 + D)));
+    while (cfirst + 1 < att_grid && range_start(cfirst + 1) <= p0) ++cfirst;
+    float mt = -INFINITY, lt = 0.f;
+    long long myslot = -1;
+    {
+      const long long cc = cfirst + tid;
+      if (cc < att_grid) {
+        const long long cs = max64(p0, range_start(cc));
+        if (cs < p1 && cs < min64(p1, range_start(cc + 1))) {
+          myslot = cs;
+          const float* G = a.attn_part + size_t(cs) * (2 + D);
+          mt = __ldcg(G);
+          lt = __ldcg(G + 1);
+        }
+      }
     }
+    float M = mt;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) sm.red32[wid] = __float_as_uint(M);
+    if (lane == 0) red32[wid] = __float_as_uint(M);
     __syncthreads();
     M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, __uint_as_float(sm.red32[w]));
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, __uint_as_float(red32[w]));
+    const float sct = (myslot < 0 || mt == -INFINITY) ? 0.f : expf(mt - M);
+    pm[tid] = sct;
+    ps[tid] = myslot;
+    float Lw = sct * lt;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Lw += __shfl_xor_sync(0xffffffffu, Lw, off);
     __syncthreads();
-    float L = 0.f, acc = 0.f;
-    const int e = tid % D, prt = tid / D;  // NP threads per output element
-    constexpr int NP = kDecThreads / D;
-    float Lp = 0.f;
-    for (long long c = cfirst + prt; c < gridDim.x; c += NP) {
-      const long long cs = max64(p0, range_start(c));
-      if (cs >= p1) break;
-      if (cs >= min64(p1, range_start(c + 1))) continue;  // empty range
-      const float* G = a.attn_part + size_t(cs) * (2 + D);
-      const float mg = __ldcg(G), lg = __ldcg(G + 1), og = __ldcg(G + 2 + e);  // independent loads
-      const float sc = mg == -INFINITY ? 0.f : expf(mg - M);
-      Lp = fmaf(sc, lg, Lp);
-      acc = fmaf(sc, og, acc);
+    if (lane == 0) red32[wid] = __float_as_uint(Lw);
+    __syncthreads();
+    float L = 0.f;
+    for (int w = 0; w < NW; ++w) L += __uint_as_float(red32[w]);
+    // outputs: NP threads per element, each over every NP-th partial (independent loads)
+    constexpr int NP = kCombThreads / D;
+    const int e = tid % D, prt = tid / D;
+    const int npart = int(min64(att_grid - cfirst, kCombThreads));
+    float acc = 0.f;
+    for (int t = prt; t < npart; t += NP) {
+      const long long cs = ps[t];
+      if (cs < 0) continue;
+      acc = fmaf(pm[t], __ldcg(a.attn_part + size_t(cs) * (2 + D) + 2 + e), acc);
     }
-    float* red = reinterpret_cast<float*>(sm.hist);  // [NP][D] + [NP]
-    red[prt * D + e] = acc;
-    if (e == 0) red[NP * D + prt] = Lp;
+    redf[prt * D + e] = acc;
     __syncthreads();
     if (prt == 0) {
-      for (int q = 1; q < NP; ++q) acc += red[q * D + e];
-      for (int q = 0; q < NP; ++q) L += red[NP * D + q];
+      for (int q = 1; q < NP; ++q) acc += redf[q * D + e];
       a.O[size_t(h) * D + e] = acc / L;
     }
     if (tid == 0) {
       long long nl = 0, scored = 0;
       int l0 = 0, steps = 0;
-      if (routed) {
-        HeadState* hs = hstate(h);
+      if (a.n_steps > 0 && a.n_roots > 0) {
+        HeadState* hs = c.hstate(h);
         nl = __ldcg(&hs->n_leaf);
         l0 = __ldcg(&hs->leaf0);
         scored = __ldcg(&hs->scored);
         steps = __ldcg(&hs->steps);
-        // leave the head's state zeroed for the next launch
+        // leave the head's state zeroed for the next call
         long long* z = reinterpret_cast<long long*>(hs);
         for (int k = 0; k < int(sizeof(HeadState) / 8); ++k) z[k] = 0;
       }
@@ -1723,38 +2022,53 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     __syncthreads();
   }
-  stamp(a, 29);
 }
 
 // ------------------------------------------------------------------ host launcher
-template <typename T, int D>
-static int grid_size_t() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
-  auto kern = decode_kernel<T, D>;
-  const size_t smem = sizeof(DecSmem);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
-  int per_sm = 0, dev = 0, sms = 0;
+static int device_sms() {
+  int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  cached = min(per_sm * sms, kMaxDecodeGrid);
-  return cached;
+  return sms;
 }
 
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
-  auto kern = decode_kernel<T, D>;
-  const int grid = grid_size_t<T, D>();
-  if (grid < 1) return cudaErrorLaunchOutOfResources;
-  DecodeArgs args = a;
-  void* params[] = {&args};
-  count_launches(1);
-  return cudaLaunchCooperativeKernel((const void*)kern, dim3(unsigned(grid)), dim3(kDecThreads), params,
-                                     sizeof(DecSmem), st);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(score_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(sizeof(ScoreSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(select_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(sizeof(DecSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attend_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(sizeof(AttSmem)));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int sms = device_sms();
+  const unsigned nh = unsigned(a.nheads);
+  const bool routed = a.n_steps > 0 && a.n_roots > 0;
+  int launches = 0;
+  if (routed) {
+    for (int s = 0; s <= a.n_steps; ++s) {
+      score_kernel<T, D><<<unsigned(sms), kDecThreads, sizeof(ScoreSmem), st>>>(a, s);
+      ++launches;
+      if (s < a.n_steps) {
+        select_kernel<T, D><<<nh, kDecThreads, sizeof(DecSmem), st>>>(a, s);
+        ++launches;
+      }
+    }
+    finalize_kernel<T, D><<<nh, kDecThreads, 0, st>>>(a);
+    ++launches;
+  }
+  const int att_grid = min(kMaxAttGrid, att_ctas_per_sm<T>() * sms);  // one wave
+  attend_kernel<T, D><<<unsigned(att_grid), kAttThreads, sizeof(AttSmem), st>>>(a);
+  combine_kernel<T, D><<<nh, kCombThreads, 0, st>>>(a, att_grid);
+  launches += 2;
+  count_launches(launches);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
@@ -1763,18 +2077,10 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
   return a.t.d == 128 ? launch_decode_t<float, 128>(a, st) : launch_decode_t<float, 64>(a, st);
 }
 
-int decode_grid(int dtype, int d) {
-  if (dtype == ZHA_BF16) return d == 128 ? grid_size_t<__nv_bfloat16, 128>() : grid_size_t<__nv_bfloat16, 64>();
-  return d == 128 ? grid_size_t<float, 128>() : grid_size_t<float, 64>();
-}
-
-size_t decode_smem_bytes() { return sizeof(DecSmem); }
 // Head states and leaf bitmaps, one region cleared together.
 size_t decode_flow_bytes(int nheads, int64_t cap_sel) {
   return size_t(nheads) * (sizeof(HeadState) + size_t(decode_bitmap_words(cap_sel)) * 4);
 }
-// Grid barriers one decode launch takes.
-int decode_barriers(int n_steps, int n_roots) { return n_steps > 0 && n_roots > 0 ? 2 * n_steps + 3 : 1; }
 // Per-head routing workspace: step keys and codes in two parity buffers, two
 // anchored histograms, the kept entries of the last select, the kept leaves.
 uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list) {
@@ -1782,7 +2088,7 @@ uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list) {
   return cap4 * 20 + 2 * kBins * 8 + uint64_t(cap_list) * 4;
 }
 int decode_max_heads() { return kMaxHeads; }
-int decode_items_per_cta() { return kItemsPerCta; }
-int decode_max_grid() { return kMaxDecodeGrid; }
+// attention partial slots of one call: at most kAttItems per CTA, one more per head
+uint64_t decode_part_items(int nheads) { return uint64_t(kMaxAttGrid) * (kAttItems + 16) + uint64_t(nheads) + 64; }
 
 }  // namespace zha

@@ -28,21 +28,6 @@ constexpr int kDenseThreads = 128;
 constexpr int kDenseWarps = kDenseThreads / 32;
 constexpr int kDenseTile = 16;
 
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
-  return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
-}
-
 // Combine the split partials of one query head: one CTA per (head, sequence).
 // o = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s with M = max_s m_s.
 template <int D>
