@@ -32,12 +32,6 @@ using namespace zha;
 
 static std::atomic<uint64_t> g_launches{0};
 
-#ifdef ZHA_PHASE_TIMING
-// Profiling builds only: a device buffer [grid][32] of %globaltimer stamps that
-// the decode kernel fills at its phase boundaries.
-static unsigned long long* g_phase_ns = nullptr;
-extern "C" ZHA_API void zha_debug_phase_buffer(void* p) { g_phase_ns = static_cast<unsigned long long*>(p); }
-#endif
 void zha::count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
 
 namespace {
@@ -313,9 +307,6 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->flow = reinterpret_cast<unsigned char*>(t->scratch + t->L.flow_off);
   a->attn_part = reinterpret_cast<float*>(t->scratch + t->L.part_off);
   a->spin_limit = t->spin_limit;
-#ifdef ZHA_PHASE_TIMING
-  a->phase_ns = g_phase_ns;
-#endif
   a->cap_sel = t->L.cap_sel;
   a->cap_list = t->L.cap_list;
   a->kept = kept;

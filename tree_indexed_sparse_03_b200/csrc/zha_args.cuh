@@ -30,7 +30,6 @@ struct DecodeArgs {
   uint32_t p_mant;              // p = p_mant * 2^-p_shift  (p < 1)
   int p_shift;
   int p_all;                    // p >= 1: keep every candidate
-  unsigned long long* phase_ns; // optional per-CTA phase timestamps (profiling builds), else NULL
 };
 
 struct DenseArgs {

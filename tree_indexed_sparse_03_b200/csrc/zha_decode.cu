@@ -62,8 +62,8 @@ constexpr long long kDrainLimit = 1ll << 22;       // bound of the wait for copi
 constexpr int kAttThreads = 256;                   // threads of an attention CTA
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttItems = 32;                      // attend chunks a CTA owns at most
-constexpr int kMaxAttGrid = 1024;                  // attention CTAs the scratch is laid out for
-constexpr int kCombThreads = 1024;                 // threads of a combine CTA (one partial per thread)
+constexpr int kMaxAttGrid = 512;                   // attention CTAs the scratch is laid out for
+constexpr int kCombThreads = 512;                  // threads of a combine CTA (one partial per thread)
 static_assert(kMaxAttGrid <= kCombThreads, "the combine takes one partial per thread");
 static_assert(kCombThreads % 128 == 0, "the combine splits its threads over the output elements");
 
@@ -321,25 +321,6 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
 }
 
-// Phase timestamp (profiling builds pass a buffer of 128 slots per CTA).
-__device__ __forceinline__ void stamp(const DecodeArgs& a, int slot) {
-  if (a.phase_ns != nullptr && threadIdx.x == 0 && slot < 128) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    a.phase_ns[blockIdx.x * 128 + slot] = t;
-  }
-}
-
-// Per (head, step) event times for profiling builds (heads < 64, steps < 8).
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void trace_hs(const DecodeArgs& a, int h, int step, int field, unsigned long long v) {
-  if (a.phase_ns != nullptr && h < 64 && step < 8) a.phase_ns[40960 + (h * 8 + step) * 32 + field] = v;
-}
-
 // Add mass w to shared-memory histogram bin `bin` for every lane of
 // the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
 // a bin (siblings sit next to each other in a step's candidate list), so the
@@ -395,42 +376,62 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 }
 
 
-// The cut for at most kDecThreads entries: thread i takes entry i, counts the
-// entries ordered before it (its rank), the masses are placed in rank order
-// and scanned, and the cut is the first entry whose running mass reaches T.
+// The cut for at most kDecThreads entries: thread i takes entry i; the (order
+// key, mass) pairs are sorted by a bitonic network in shared memory (strides
+// below 32 within a warp by shuffles), the masses scanned in sorted order, and
+// the cut is the first entry whose running mass reaches T.
 template <class View>
 __device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
-                                               DecSmem& sm) {
-  const int tid = threadIdx.x;
-  unsigned long long* k64s = sm.hist;                        // [n] order keys
-  unsigned long long* wr = sm.hist + kDecThreads;            // [n] masses in rank order
-  unsigned long long myk = ~0ull, myw = 0;
+                                                            DecSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  unsigned long long* ks = sm.hist;                // [np] order keys
+  unsigned long long* ws = sm.hist + kDecThreads;  // [np] masses
+  int np = 32;
+  while (np < n) np <<= 1;  // <= kDecThreads
+  unsigned long long k = ~0ull, w = 0;
   if (tid < n) {
-    const uint32_t k = E.key(tid);
-    myk = entry_key64(a, Entry{k, E.code(tid)});
-    myw = entry_mass(m, k);
-    k64s[tid] = myk;
+    const uint32_t key = E.key(tid);
+    k = entry_key64(a, Entry{key, E.code(tid)});
+    w = entry_mass(m, key);
   }
-  __syncthreads();
-  int rank = 0;
-  if (tid < n) {
-    for (int j = 0; j < n; ++j) rank += k64s[j] < myk;
-    wr[rank] = myw;
+  if (tid < np) {
+    for (int size = 2; size <= np; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const bool up = (tid & size) == 0;
+        unsigned long long ok, ow;
+        if (stride >= 32) {  // partner in another warp: through shared memory
+          ks[tid] = k;
+          ws[tid] = w;
+          asm volatile("bar.sync 1, %0;" ::"r"(np) : "memory");
+          ok = ks[tid ^ stride];
+          ow = ws[tid ^ stride];
+          asm volatile("bar.sync 1, %0;" ::"r"(np) : "memory");
+        } else {
+          ok = __shfl_xor_sync(0xffffffffu, k, stride);
+          ow = __shfl_xor_sync(0xffffffffu, w, stride);
+        }
+        const bool lower = (tid & stride) == 0;
+        const bool take = (up == lower) ? (ok < k) : (ok > k);
+        if (take) {
+          k = ok;
+          w = ow;
+        }
+      }
+    }
   }
-  __syncthreads();
-  const unsigned long long w_sorted = tid < n ? wr[tid] : 0ull;
+  (void)lane;
   unsigned long long Z;
-  const unsigned long long before = block_scan_u64(w_sorted, sm.red64, &Z);
+  const unsigned long long before = block_scan_u64(tid < np ? w : 0ull, sm.red64, &Z);
   const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);
-  // sorted position of the cut: the first with before + w >= T
-  if (tid == 0) sm.bcast32[2] = int(n) - 1;
+  // sorted position of the cut: the first with before + w >= T (else the last entry)
+  if (tid == 0) sm.bcast64[1] = ~0ull;
   __syncthreads();
-  if (tid < n && before < T && before + w_sorted >= T) sm.bcast32[2] = tid;
+  if (tid < n && before < T && before + w >= T) sm.bcast64[1] = k;
   __syncthreads();
-  const int cut_pos = sm.bcast32[2];
-  if (tid < n && rank == cut_pos) sm.bcast64[1] = myk;
-  __syncthreads();
-  const unsigned long long cut = sm.bcast64[1];
+  unsigned long long cut = sm.bcast64[1];
+  if (cut == ~0ull) {  // T out of reach by rounding: keep everything
+    cut = ~0ull;
+  }
   __syncthreads();
   return cut;
 }
@@ -495,7 +496,6 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
     block_scan_u64(local, sm.red64, &Z);
   }
   const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);  // keep while mass before < T
-  if (tid == 0) trace_hs(a, h, step, 8, now_ns());
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
@@ -503,7 +503,6 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   // keys of coarse bin cb form the contiguous range [klo, khi)
   const unsigned long long klo = first_key_at_least(kmin, cb, cbin);
   const unsigned long long khi = cb + 1 < kBins ? first_key_at_least(uint32_t(klo), cb + 1, cbin) : 0x100000000ull;
-  if (tid == 0) trace_hs(a, h, step, 9, now_ns());
 
   // fine histogram inside the cut coarse bin: the fine cut bin's key range
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
@@ -528,7 +527,6 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
     for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, bin[u], w[u]);
   }
   __syncthreads();
-  if (tid == 0) trace_hs(a, h, step, 10, now_ns());
   unsigned long long below2;
   const int fb = find_cut_bin(sm, below, T, &below2);
   if (fb < 0) return ~0ull;
@@ -540,7 +538,6 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   unsigned long long fhi = fb + 1 < kBins ? first_key_at_least(uint32_t(flo), fb + 1, fbin) : khi;
   if (fhi > khi) fhi = khi;
   auto in_cut = [&](uint32_t k) { return k >= flo && k < fhi; };
-  if (tid == 0) trace_hs(a, h, step, 11, now_ns());
 
   // gather the entries around the cut
   if (tid == 0) sm.bcast32[1] = 0;
@@ -557,10 +554,6 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   }
   __syncthreads();
   const int cnt = sm.bcast32[1];
-  if (tid == 0) {
-    trace_hs(a, h, step, 12, now_ns());
-    trace_hs(a, h, step, 13, (unsigned long long)cnt);
-  }
   if (cnt <= 32) {
     if (tid < 32) {
       unsigned long long k = tid < cnt ? sm.cut_key[tid] : ~0ull;
@@ -722,16 +715,61 @@ __device__ __forceinline__ int find_cut_bin_f64(DecSmem& sm, const double* m, do
   return bin;
 }
 
+// Bin of a key for anchor r (the anchored_bin bin alone, no mass), and the
+// bin's sub-bin, as monotone non-decreasing functions of the key: -1 for an
+// estimate above the anchor span.
+__device__ __forceinline__ int anchored_bin_of(float r, uint32_t key) {
+  const float x = __fadd_rn(__fsub_rn(r, desc_key_value(key)), kAnchorSpan);
+  if (!(x >= 0.f)) return -1;
+  return min(int(__fmul_rn(x, kBinScale)), kBins - 1);
+}
+// (coarse bin, sub-bin) ordered as one number: coarse * kBins + fine
+__device__ __forceinline__ long long anchored_code_of(float r, uint32_t key) {
+  const float x = __fadd_rn(__fsub_rn(r, desc_key_value(key)), kAnchorSpan);
+  if (!(x >= 0.f)) return -1;
+  const int b = min(int(__fmul_rn(x, kBinScale)), kBins - 1);
+  const float t = __fsub_rn(x, __fmul_rn(float(b), 1.f / kBinScale));
+  return (long long)b * kBins + anchored_fine(t);
+}
+
+// Smallest key in [lo, 2^32) whose f(key) >= target, for f monotone
+// non-decreasing over the keys; 2^32 if none.  One warp, 32-ary search: each
+// round the lanes probe 32 keys spread over the remaining interval (7 rounds
+// for 2^32 keys).  Every lane returns the answer.
+template <typename F>
+__device__ __forceinline__ unsigned long long warp_first_key(unsigned long long lo, long long target, F f) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long L = lo, H = 0x100000000ull;  // answer in [L, H]
+  while (L < H) {
+    const unsigned long long span = H - L;
+    const unsigned long long p = L + (span * unsigned(lane)) / 32u;
+    const bool ge = f(uint32_t(p)) >= target;
+    const unsigned m = __ballot_sync(0xffffffffu, ge);
+    if (m == 0u) {
+      L = __shfl_sync(0xffffffffu, p, 31) + 1;  // all probes below: past the last one
+    } else {
+      const int j = __ffs(m) - 1;
+      const unsigned long long pj = __shfl_sync(0xffffffffu, p, j);
+      if (j == 0) return pj;  // the first probe is L itself
+      L = __shfl_sync(0xffffffffu, p, j - 1) + 1;
+      H = pj;
+    }
+  }
+  return L;
+}
+
 // The cut of a step from its anchored histogram (global, kBins sums): the
-// coarse cut bin from the histogram alone, then one pass over the keys for
-// the fine histogram of that bin's members, one more to gather the members of
-// the fine cut bin, which are ordered by (e desc, start asc).  Every thread
-// returns the same value.
+// coarse cut bin from the histogram alone; the exact key ranges of that bin
+// and of its sub-bins from warp searches; one pass over the keys for the
+// sub-bin histogram of the bin's members, one more to gather the members of
+// the cut sub-bin, which are ordered by (e desc, start asc).  Passes read four
+// keys per lane and do real work only for members.  Every thread returns the
+// same value.
 template <class View>
 __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs& a, const View& E, int64_t n,
-                                                                  float r, const unsigned long long* ghist,
-                                                                  DecSmem& sm, int h, int step) {
-  const int tid = threadIdx.x, lane = tid & 31;
+                                                               float r, const unsigned long long* ghist,
+                                                               DecSmem& sm, int h, int step) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   constexpr int BPT = kBins / kDecThreads;
   double* red = reinterpret_cast<double*>(sm.red64);
   const double p = ldexp(double(a.p_mant), -a.p_shift);
@@ -749,31 +787,42 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
   const int cb = find_cut_bin_f64(sm, mb, before, T, &below_c);
   if (cb < 0) return ~0ull;  // rounding kept T out of reach: keep everything
   const double sc = anchored_scale(cb);
-  if (tid == 0) trace_hs(a, h, step, 8, now_ns());
-
-  // fine histogram of the cut bin's members (exact integer masses)
+  // key range [klo, khi) of the coarse bin
+  if (wid < 2) {
+    const unsigned long long k =
+        warp_first_key(0ull, cb + wid, [&](uint32_t key) { return (long long)anchored_bin_of(r, key); });
+    if (lane == 0) sm.bcast64[wid] = k;
+  }
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
+  const unsigned long long klo = sm.bcast64[0], khi = sm.bcast64[1];
+  __syncthreads();
   const int n32 = int(n);
-  const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
-  const int wlo = min(n32, (tid >> 5) * wseg), whi = min(n32, wlo + wseg);
-  constexpr int U = 4;
-  for (int base = wlo; base < whi; base += 32 * U) {
-    int fb[U];
-    unsigned long long w[U];
+  // sub-bin histogram of the members (exact integer masses), four keys per lane
+  auto keys4 = [&](int i0, uint32_t* k) {  // keys i0 .. i0+3 (past n: 0xffffffff, never a member)
+    if (i0 + 4 <= E.nc) {
+      const uint4 v = *reinterpret_cast<const uint4*>(E.ck + i0);
+      k[0] = v.x;
+      k[1] = v.y;
+      k[2] = v.z;
+      k[3] = v.w;
+    } else {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + 32 * u + lane;
-      fb[u] = -1;
-      w[u] = 0;
-      if (i < whi) {
+      for (int u = 0; u < 4; ++u) k[u] = i0 + u < n32 ? E.key(i0 + u) : 0xffffffffu;
+    }
+  };
+  for (int i0 = 4 * tid; i0 < n32; i0 += 4 * kDecThreads) {
+    uint32_t k[4];
+    keys4(i0, k);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (k[u] >= klo && k[u] < khi) {
+        unsigned long long w;
         float t;
-        if (anchored_bin(r, E.key(i), &w[u], &t) == cb) fb[u] = anchored_fine(t);
-        else w[u] = 0;
+        anchored_bin(r, k[u], &w, &t);
+        atomicAdd(&sm.hist[anchored_fine(t)], w);
       }
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) hist_add_warp(sm.hist, fb[u], w[u]);
   }
   __syncthreads();
   double fm[BPT];
@@ -800,32 +849,36 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     below_f = below_c + double(pre) * sc;
     __syncthreads();
   }
-  if (tid == 0) trace_hs(a, h, step, 10, now_ns());
-
-  // gather the members of the fine cut bin
-  auto member = [&](uint32_t k, unsigned long long* w) {
-    float t;
-    return anchored_bin(r, k, w, &t) == cb && anchored_fine(t) == fbin;
-  };
+  // key range [flo, fhi) of the cut sub-bin
+  if (wid < 2) {
+    const long long target = (long long)cb * kBins + fbin + wid;
+    const unsigned long long k = warp_first_key(klo, target, [&](uint32_t key) { return anchored_code_of(r, key); });
+    if (lane == 0) sm.bcast64[2 + wid] = min(k, khi);
+  }
   if (tid == 0) sm.bcast32[1] = 0;
   __syncthreads();
-  for (int i = tid; i < n32; i += kDecThreads) {
-    const uint32_t k = E.key(i);
-    unsigned long long w;
-    if (member(k, &w)) {
-      const int sl = atomicAdd(&sm.bcast32[1], 1);
-      if (sl < 32) {
-        sm.cut_key[sl] = entry_key64(a, Entry{k, E.code(i)});
-        sm.cut_w[sl] = w;
+  const unsigned long long flo = sm.bcast64[2], fhi = sm.bcast64[3];
+  __syncthreads();
+  // gather the members of the cut sub-bin
+  for (int i0 = 4 * tid; i0 < n32; i0 += 4 * kDecThreads) {
+    uint32_t k[4];
+    keys4(i0, k);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (k[u] >= flo && k[u] < fhi) {
+        unsigned long long w;
+        float t;
+        anchored_bin(r, k[u], &w, &t);
+        const int sl = atomicAdd(&sm.bcast32[1], 1);
+        if (sl < 32) {
+          sm.cut_key[sl] = entry_key64(a, Entry{k[u], E.code(i0 + u)});
+          sm.cut_w[sl] = w;
+        }
       }
     }
   }
   __syncthreads();
   const int cnt = sm.bcast32[1];
-  if (tid == 0) {
-    trace_hs(a, h, step, 12, now_ns());
-    trace_hs(a, h, step, 13, (unsigned long long)cnt);
-  }
   if (cnt <= 32) {
     if (tid < 32) {
       unsigned long long k = tid < cnt ? sm.cut_key[tid] : ~0ull;
@@ -859,7 +912,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     __syncthreads();
     return sm.bcast64[1];
   }
-  // Many members share the fine cut bin (exact ties or near-ties): radix
+  // Many members share the cut sub-bin (exact ties or near-ties): radix
   // select on the 64-bit order key, 8 bits per pass, over those members.
   unsigned long long prefix = 0, acc = 0;  // acc: exact mass of the members before the prefix's range
   for (int pass = 0; pass < 8; ++pass) {
@@ -868,8 +921,10 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     __syncthreads();
     for (int i = tid; i < n32; i += kDecThreads) {
       const uint32_t k = E.key(i);
+      if (!(k >= flo && k < fhi)) continue;
       unsigned long long w;
-      if (!member(k, &w)) continue;
+      float t;
+      anchored_bin(r, k, &w, &t);
       const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
       atomicAdd(&sm.hist[(k64 >> shift) & 255], w);
@@ -913,7 +968,10 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
         const int src = any ? 31 - __clz(any) : 31;
         dg = __shfl_sync(0xffffffffu, last, src);
         db = __shfl_sync(0xffffffffu, lbef, src);
-        if (!any) { dg = 255; db = acc; }
+        if (!any) {
+          dg = 255;
+          db = acc;
+        }
       }
       if (tid == 0) {
         sm.bcast64[2] = prefix | (uint64_t(dg) << shift);
@@ -1112,6 +1170,16 @@ __device__ __forceinline__ float score_record_smem(const unsigned char* rec, int
   return best;
 }
 
+// ---------------------------------------------------------------- launch overlap
+// Every decode kernel is launched with programmatic stream serialization: it
+// may start while the kernel before it finishes, lets the next one start too,
+// and waits for the one before to complete (memory visible) before it reads
+// anything that kernel wrote.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- per-call context
 // The scratch regions of one decode call and the views of them every phase uses.
 template <typename T, int D>
@@ -1149,6 +1217,205 @@ struct Ctx {
   }
 };
 
+// ---------------------------------------------------------------- select
+// One head, whole CTA: the cut of step s (small path, anchored histogram or
+// the in-CTA histograms), the kept entries listed in entry order, and the
+// state of step s+1 (histogram cleared, anchor = step s's max).
+template <typename T, int D>
+__device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c, DecSmem& sm, int h, int s) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int par = s & 1;
+  {
+    HeadState* hs = c.hstate(h);
+    const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
+    if (n == 0) {
+      if (tid == 0) hs->kept = 0;
+      return;
+    }
+    const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
+    const float anchor_h = __ldcg(&hs->anchor);
+    const int ovf = __ldcg(&hs->ovf[par]);
+    const long long scored0 = __ldcg(&hs->scored);
+    const uint32_t* gk = c.keysP(h, par);
+    const uint32_t* gc = c.codesP(h, par);
+    if (a.scored) {  // codes of the scored nodes
+      int32_t* out = a.scored + size_t(h) * a.scored_cap;
+      for (long long i = tid; i < n; i += kDecThreads)
+        if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
+    }
+    const float m = desc_key_value(kmin);
+    // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
+    const int ncache = int(min64(n, kCacheKeys));
+    uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
+    for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
+    cp_async_commit();
+    cp_async_wait(0);
+    __syncthreads();
+    const StepView E{ck, ncache, gk, gc};
+    unsigned long long cut = ~0ull;
+    if (!a.p_all) {
+      if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
+      else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
+        cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
+      else cut = select_cut(a, E, n, kmin, sm, h, s);
+    }
+    // the kept entries (order key <= cut), listed in entry order: each warp
+    // owns a contiguous run of 128-entry groups, four entries per lane; the
+    // code is read only for a key equal to the cut's
+    long long n_kept = 0;
+    {
+      const uint32_t cut32 = uint32_t(cut >> 32);
+      const int n32 = int(n);
+      const int groups = (n32 + 127) / 128;
+      const int gseg = (groups + kDecWarps - 1) / kDecWarps;
+      const int wlo = min(n32, wid * gseg * 128), whi = min(n32, wlo + gseg * 128);
+      auto kept4 = [&](int i0) -> unsigned {  // bit u: entry i0 + u is kept (i0 + u < whi)
+        uint32_t k[4];
+        if (i0 + 4 <= E.nc && i0 + 4 <= whi) {
+          const uint4 v = *reinterpret_cast<const uint4*>(E.ck + i0);
+          k[0] = v.x;
+          k[1] = v.y;
+          k[2] = v.z;
+          k[3] = v.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) k[u] = i0 + u < whi ? E.key(i0 + u) : 0xffffffffu;
+        }
+        unsigned bits = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool kp = i0 + u < whi &&
+                          (k[u] < cut32 || (k[u] == cut32 && entry_key64(a, Entry{k[u], E.code(i0 + u)}) <= cut));
+          bits |= kp ? (1u << u) : 0u;
+        }
+        return bits;
+      };
+      uint32_t wk = 0;
+      for (int base = wlo; base < whi; base += 128) wk += __popc(kept4(base + 4 * lane));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) wk += __shfl_xor_sync(0xffffffffu, wk, off);
+      if (lane == 0) sm.red32[wid] = wk;
+      __syncthreads();
+      uint32_t off = 0;
+      for (int w = 0; w < kDecWarps; ++w) {
+        if (w < wid) off += sm.red32[w];
+        n_kept += sm.red32[w];
+      }
+      uint32_t* kl = c.keptl(h);
+      for (int base = wlo; base < whi; base += 128) {
+        const int i0 = base + 4 * lane;
+        unsigned bits = kept4(i0);
+        const uint32_t pc = __popc(bits);
+        uint32_t ex = pc;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, ex, o2);
+          if (lane >= o2) ex += y;
+        }
+        uint32_t pos = off + ex - pc;
+        while (bits) {
+          const int u = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          kl[pos++] = uint32_t(i0 + u);
+        }
+        off += __shfl_sync(0xffffffffu, ex, 31);
+      }
+    }
+    // state for the next step: its histogram cleared, its anchor = this step's max
+    unsigned long long* nhist = c.histP(h, par ^ 1);
+    for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
+    __syncthreads();
+    if (tid == 0) {
+      hs->kept = n_kept;
+      hs->n[par ^ 1] = 0;
+      hs->anchor = m;
+      hs->kinv[par ^ 1] = 0u;
+      hs->ovf[par ^ 1] = 0;
+      hs->scored = scored0 + n;
+      hs->steps = hs->steps + 1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- finalize
+// One head, whole CTA: the kept leaves in block order from the head's bitmap
+// (each warp owns a contiguous run of words: counts, one scan over warps, then
+// writes), which it leaves zeroed.
+template <typename T, int D>
+__device__ __noinline__ void finalize_head(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int64_t bm_words = c.bm_words;
+  {
+    uint32_t* bm = c.bitmap(h);
+    const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
+    const long long wseg = (nw + kDecWarps - 1) / kDecWarps;
+    const long long w_lo = min64(nw, wid * wseg), w_hi = min64(nw, w_lo + wseg);
+    uint32_t cnt = 0;
+    for (long long wi = w_lo + lane; wi < w_hi; wi += 32) cnt += __popc(__ldcg(bm + wi));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if (lane == 0) red32[wid] = cnt;
+    __syncthreads();
+    long long pos = 0, total = 0;
+    for (int w = 0; w < kDecWarps; ++w) {
+      if (w < wid) pos += red32[w];
+      total += red32[w];
+    }
+    const int leaf0 = nw > 0 ? int(__ldcg(bm) & 1u) : 0;
+    __syncthreads();
+    for (long long wb = w_lo; wb < w_hi; wb += 32) {
+      const long long wi = wb + lane;
+      uint32_t bits = wi < w_hi ? __ldcg(bm + wi) : 0u;
+      uint32_t pc = __popc(bits), ex = pc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, ex, off);
+        if (lane >= off) ex += y;
+      }
+      const uint32_t wtot = __shfl_sync(0xffffffffu, ex, 31);
+      long long p = pos + ex - pc;
+      if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
+      while (bits) {
+        const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
+        bits &= bits - 1u;
+        if (p < a.cap_list) c.leaves(h)[p] = idx;
+        if (a.kept && p < a.kept_stride) a.kept[size_t(h) * a.kept_stride + p] = int32_t(idx);
+        ++p;
+      }
+      pos += wtot;
+    }
+    if (tid == 0) {
+      if (total > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
+      c.hstate(h)->n_leaf = min64(total, a.cap_list);
+      c.hstate(h)->leaf0 = leaf0;
+    }
+    __syncthreads();
+  }
+}
+
+// One CTA per head.
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_constant__ DecodeArgs a, int s) {
+  pdl_wait_and_release();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  const Ctx<T, D> c(a);
+  for (int h = blockIdx.x; h < a.nheads; h += gridDim.x) {
+    select_head<T, D>(a, c, sm, h, s);
+    __syncthreads();
+  }
+}
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads) finalize_kernel(const __grid_constant__ DecodeArgs a) {
+  pdl_wait_and_release();
+  __shared__ uint32_t red32[kDecWarps];
+  const Ctx<T, D> c(a);
+  for (int h = blockIdx.x; h < a.nheads; h += gridDim.x) {
+    finalize_head<T, D>(a, c, red32, h);
+    __syncthreads();
+  }
+}
+
 // ---------------------------------------------------------------- scoring phase
 // Step s's entries: the roots (s = 0, root i at position i) or the children of
 // step s-1's kept non-leaves, at positions reserved per warp batch with one
@@ -1157,6 +1424,7 @@ struct Ctx {
 // Units (roots, or kept entries) of all heads are cut into contiguous ranges,
 // one per warp.  Each record is fetched with one bulk copy into the warp's
 // ring; the estimate is added to the step's anchored histogram (s >= 1).
+
 struct __align__(16) ScoreSmem {
   unsigned char ring[kRingBytes];
   long long pref[kMaxHeads + 1];
@@ -1166,6 +1434,7 @@ struct __align__(16) ScoreSmem {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_constant__ DecodeArgs a, int s) {
+  pdl_wait_and_release();
   constexpr int EPC = 16 / sizeof(T);
   constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -1192,6 +1461,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   float qs[EPC];
   uint32_t qf[D / 16][2];
   int qhead = -1;
+  bool failed = false;  // a copy never landed: this warp stops scoring
   const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
   const long long nwarps = (long long)gridDim.x * score_warps;
   // ---------------- scoring phase: units = roots (s = 0) or the kept entries of step s-1
@@ -1332,7 +1602,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
               kp ^= 1u;
             }
           }
-          return;
+          failed = true;
+          break;
         }
       }
       __syncwarp();
@@ -1382,172 +1653,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
         phase_d ^= 1u;
       }
     }
+    if (failed) break;
   }
   if (lane == 0 && cur_h >= 0) {
     atomicMax(&c.hstate(cur_h)->kinv[par], ~cur_kmin);
     if (cur_ovf) atomicOr(&c.hstate(cur_h)->ovf[par], 1);
-  }
-}
-
-// ---------------------------------------------------------------- select phase
-// One CTA per head: the cut of step s (small path, anchored histogram or the
-// in-CTA histograms), the kept entries listed in entry order, and the state
-// of step s+1 (histogram cleared, anchor = step s's max).
-template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_constant__ DecodeArgs a, int s) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
-  const Ctx<T, D> c(a);
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int nh = a.nheads, b = a.t.block;
-  const int par = s & 1;
-  // ---------------- select phase: one CTA per head
-  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-    HeadState* hs = c.hstate(h);
-    const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
-    if (n == 0) {
-      __syncthreads();
-      if (tid == 0) hs->kept = 0;
-      continue;
-    }
-    const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
-    const float anchor_h = __ldcg(&hs->anchor);
-    const int ovf = __ldcg(&hs->ovf[par]);
-    const long long scored0 = __ldcg(&hs->scored);
-    const uint32_t* gk = c.keysP(h, par);
-    const uint32_t* gc = c.codesP(h, par);
-    if (a.scored) {  // codes of the scored nodes
-      int32_t* out = a.scored + size_t(h) * a.scored_cap;
-      for (long long i = tid; i < n; i += kDecThreads)
-        if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
-    }
-    const float m = desc_key_value(kmin);
-    // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
-    const int ncache = n <= kDecThreads ? 0 : int(min64(n, kCacheKeys));
-    uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
-    for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
-    cp_async_commit();
-    cp_async_wait(0);
-    __syncthreads();
-    const StepView E{ck, ncache, gk, gc};
-    unsigned long long cut = ~0ull;
-    if (!a.p_all) {
-      if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
-      else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
-        cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
-      else cut = select_cut(a, E, n, kmin, sm, h, s);
-    }
-    // the kept entries (order key <= cut), listed in entry
-    // order: each warp owns a contiguous segment; the code is read only for a
-    // key equal to the cut's
-    long long n_kept = 0;
-    {
-      const uint32_t cut32 = uint32_t(cut >> 32);
-      const int n32 = int(n);
-      const int wseg = (n32 + kDecWarps - 1) / kDecWarps;
-      const int wlo = min(n32, wid * wseg), whi = min(n32, wlo + wseg);
-      auto kept_at = [&](int i) {
-        const uint32_t k = E.key(i);
-        return k < cut32 || (k == cut32 && entry_key64(a, Entry{k, E.code(i)}) <= cut);
-      };
-      uint32_t wk = 0;
-      for (int base = wlo; base < whi; base += 32) {
-        const int i = base + lane;
-        wk += __popc(__ballot_sync(0xffffffffu, i < whi && kept_at(i)));
-      }
-      if (lane == 0) sm.red32[wid] = wk;
-      __syncthreads();
-      uint32_t off = 0;
-      for (int w = 0; w < kDecWarps; ++w) {
-        if (w < wid) off += sm.red32[w];
-        n_kept += sm.red32[w];
-      }
-      uint32_t* kl = c.keptl(h);
-      for (int base = wlo; base < whi; base += 32) {
-        const int i = base + lane;
-        const bool kp = i < whi && kept_at(i);
-        const unsigned mk = __ballot_sync(0xffffffffu, kp);
-        if (kp) kl[off + __popc(mk & ((1u << lane) - 1u))] = uint32_t(i);
-        off += __popc(mk);
-      }
-    }
-    // state for the next step: its histogram cleared, its anchor = this step's max
-    unsigned long long* nhist = c.histP(h, par ^ 1);
-    for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
-    __syncthreads();
-    if (tid == 0) {
-      hs->kept = n_kept;
-      hs->n[par ^ 1] = 0;
-      hs->anchor = m;
-      hs->kinv[par ^ 1] = 0u;
-      hs->ovf[par ^ 1] = 0;
-      hs->scored = scored0 + n;
-      hs->steps = hs->steps + 1;
-    }
-  }
-}
-
-// ---------------------------------------------------------------- finalize
-// One CTA per head: the kept leaves in block order from the head's bitmap
-// (each warp owns a contiguous run of words: counts, one scan over warps, then
-// writes), which it leaves zeroed.
-struct FinSmem {
-  uint32_t red32[kDecWarps];
-};
-template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads) finalize_kernel(const __grid_constant__ DecodeArgs a) {
-  __shared__ FinSmem sm;
-  const Ctx<T, D> c(a);
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int nh = a.nheads;
-  const int64_t bm_words = c.bm_words;
-  // ---------------- finalize: the kept leaves of each head, in block order, from its bitmap
-  // (each warp owns a contiguous run of words: counts, one block scan over warps, then writes)
-  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-    uint32_t* bm = c.bitmap(h);
-    const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
-    const long long wseg = (nw + kDecWarps - 1) / kDecWarps;
-    const long long w_lo = min64(nw, wid * wseg), w_hi = min64(nw, w_lo + wseg);
-    uint32_t cnt = 0;
-    for (long long wi = w_lo + lane; wi < w_hi; wi += 32) cnt += __popc(__ldcg(bm + wi));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (lane == 0) sm.red32[wid] = cnt;
-    __syncthreads();
-    long long pos = 0, total = 0;
-    for (int w = 0; w < kDecWarps; ++w) {
-      if (w < wid) pos += sm.red32[w];
-      total += sm.red32[w];
-    }
-    const int leaf0 = nw > 0 ? int(__ldcg(bm) & 1u) : 0;
-    __syncthreads();
-    for (long long wb = w_lo; wb < w_hi; wb += 32) {
-      const long long wi = wb + lane;
-      uint32_t bits = wi < w_hi ? __ldcg(bm + wi) : 0u;
-      uint32_t pc = __popc(bits), ex = pc;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, ex, off);
-        if (lane >= off) ex += y;
-      }
-      const uint32_t wtot = __shfl_sync(0xffffffffu, ex, 31);
-      long long p = pos + ex - pc;
-      if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
-      while (bits) {
-        const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
-        bits &= bits - 1u;
-        if (p < a.cap_list) c.leaves(h)[p] = idx;
-        if (a.kept && p < a.kept_stride) a.kept[size_t(h) * a.kept_stride + p] = int32_t(idx);
-        ++p;
-      }
-      pos += wtot;
-    }
-    if (tid == 0) {
-      if (total > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
-      c.hstate(h)->n_leaf = min64(total, a.cap_list);
-      c.hstate(h)->leaf0 = leaf0;
-    }
-    __syncthreads();
   }
 }
 
@@ -1613,6 +1723,7 @@ constexpr int att_ctas_per_sm() { return std::is_same<T, __nv_bfloat16>::value ?
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kernel(const __grid_constant__ DecodeArgs a) {
+  pdl_wait_and_release();
   constexpr int EPC = 16 / sizeof(T);
   constexpr int CPR = D * sizeof(T) / 16;
   constexpr int KPW = 32 / CPR;  // keys per warp pass
@@ -1928,6 +2039,7 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
 // kept count; the head's state zeroed for the next call.
 template <typename T, int D>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_constant__ DecodeArgs a, int att_grid) {
+  pdl_wait_and_release();
   __shared__ long long pref[kMaxHeads + 1];
   __shared__ unsigned long long red64[kCombThreads / 32];
   __shared__ uint32_t red32[kCombThreads / 32];
@@ -1986,11 +2098,19 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_cons
     constexpr int NP = kCombThreads / D;
     const int e = tid % D, prt = tid / D;
     const int npart = int(min64(att_grid - cfirst, kCombThreads));
+    // 8 independent loads in flight per thread (partials past npart or empty add 0)
     float acc = 0.f;
-    for (int t = prt; t < npart; t += NP) {
-      const long long cs = ps[t];
-      if (cs < 0) continue;
-      acc = fmaf(pm[t], __ldcg(a.attn_part + size_t(cs) * (2 + D) + 2 + e), acc);
+    for (int t0 = prt; t0 < npart; t0 += 8 * NP) {
+      float x[8], w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u * NP;
+        const long long cs = t < npart ? ps[t] : -1;
+        w[u] = cs >= 0 ? pm[t] : 0.f;
+        x[u] = cs >= 0 ? __ldcg(a.attn_part + size_t(cs) * (2 + D) + 2 + e) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc = fmaf(w[u], x[u], acc);
     }
     redf[prt * D + e] = acc;
     __syncthreads();
@@ -2032,6 +2152,23 @@ static int device_sms() {
   return sms;
 }
 
+// Launch with programmatic stream serialization (see pdl_wait_and_release).
+template <typename... Args>
+static void launch_pdl(void (*kern)(Args...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   static bool configured = false;
@@ -2053,19 +2190,19 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   int launches = 0;
   if (routed) {
     for (int s = 0; s <= a.n_steps; ++s) {
-      score_kernel<T, D><<<unsigned(sms), kDecThreads, sizeof(ScoreSmem), st>>>(a, s);
+      launch_pdl(score_kernel<T, D>, unsigned(sms), kDecThreads, sizeof(ScoreSmem), st, a, s);
       ++launches;
       if (s < a.n_steps) {
-        select_kernel<T, D><<<nh, kDecThreads, sizeof(DecSmem), st>>>(a, s);
+        launch_pdl(select_kernel<T, D>, nh, kDecThreads, sizeof(DecSmem), st, a, s);
         ++launches;
       }
     }
-    finalize_kernel<T, D><<<nh, kDecThreads, 0, st>>>(a);
+    launch_pdl(finalize_kernel<T, D>, nh, kDecThreads, 0, st, a);
     ++launches;
   }
   const int att_grid = min(kMaxAttGrid, att_ctas_per_sm<T>() * sms);  // one wave
-  attend_kernel<T, D><<<unsigned(att_grid), kAttThreads, sizeof(AttSmem), st>>>(a);
-  combine_kernel<T, D><<<nh, kCombThreads, 0, st>>>(a, att_grid);
+  launch_pdl(attend_kernel<T, D>, unsigned(att_grid), kAttThreads, sizeof(AttSmem), st, a);
+  launch_pdl(combine_kernel<T, D>, nh, kCombThreads, 0, st, a, att_grid);
   launches += 2;
   count_launches(launches);
   return cudaGetLastError();
