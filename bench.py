@@ -8,11 +8,12 @@ the step's queries (zha_decode).  The default workload is the deep tree at
 queries, p=0.95, batch 1), synthetic and seeded.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zha|reference] [--workload NAME]
+  python bench.py --profile [--workload NAME] [--n N] [--warmup W] [--steps K]   (untimed decodes, for ncu)
 
 One JSON line on stdout (rank 0).  Timing: CUDA events on the launching
-stream around every step (and around the decode kernel alone), the L2 flushed
+stream around every step (and around the decode call alone), the L2 flushed
 before every step (a 2x L2-sized write outside the timed events), warm-up
-steps untimed, max over ranks.  Algorithmic bytes of the decode kernel are
+steps untimed, max over ranks.  Algorithmic bytes of the decode call are
 counted from the nodes each query head scored and the keys it attended,
 taking the union over each GQA group (the bytes the method has to move), on
 an untimed repeat of every timed decode.  With --gpus N > 1 every rank runs
@@ -54,6 +55,8 @@ def parse_args():
     ap.add_argument("--dense-steps", type=int, default=30)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="build the workload's tree, run --warmup + --steps decodes untimed, exit (for ncu)")
     return ap.parse_args()
 
 
@@ -65,8 +68,11 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        # NCCL between the GPU replicas; gloo lets the host-only reference arm run under torchrun on CPU
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -82,7 +88,8 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -148,6 +155,40 @@ def measured_peaks():
             return json.load(fh), "measured"
     except (OSError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------------ measured traffic
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic_deep256k.txt")
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources of the library (a traffic figure is valid only for the kernels it measured)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tree_indexed_sparse_03_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload_name: str):
+    """DRAM bytes (read + write) of one decode call from the committed ncu summary, if it measured these
+    kernels on this workload; else None."""
+    try:
+        vals = {}
+        with open(TRAFFIC_FILE) as fh:
+            for line in fh:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("workload") != workload_name or vals.get("source_hash") != kernel_source_hash():
+            return None
+        return int(float(vals["dram_bytes_per_decode"]))
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 # ------------------------------------------------------------------ workload
@@ -234,6 +275,29 @@ def run_reference(args, world, rank):
         "e2e": {"value": round(us, 3), "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ profiling mode
+def run_profile(args):
+    """Build the workload's tree and run decodes without timing, so a profiler can capture the kernels."""
+    import tree_indexed_sparse_03_b200 as z
+    from synth.workloads import generate
+
+    w = load_workload(args)
+    dev = torch.device("cuda", 0)
+    inp = generate(w)
+    n = w.n_tokens
+    cfg = z.make_config(d=w.d, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, block=w.block, levels=w.levels,
+                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=n, max_batch=w.batch)
+    tree = z.ZhaTree(cfg, inp.K.to(dev), inp.V.to(dev), inp.refs.to(dev))
+    tree.build(n)
+    Qs = inp.Q.to(dev)
+    for i in range(args.warmup + args.steps):
+        tree.decode(Qs[i % w.n_query_sets])
+    torch.cuda.synchronize(dev)
+    tree.status()
+    log(f"[bench] profile mode: {args.warmup + args.steps} decodes of {w.name} (N={n}), "
+        f"{args.warmup} first, {args.steps} after")
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -403,10 +467,13 @@ def run_zha(args, world, rank, local):
         "keys_frac": round(statistics.mean(keys_ph) / n_final, 6),
         "route_bytes": int(statistics.mean(route_b)),
         "attend_bytes": int(statistics.mean(attend_b)),
-        "roofline": {"bound": "hbm", "kernel": "zha decode (route + attend, one launch)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "zha_decode call: per routing step a scoring and a select kernel, then finalize, "
+                               "attention and combine kernels",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "frac_of_8tbs": round(achieved / 8000.0, 4), "traffic": None},
+                     "frac_of_8tbs": round(achieved / 8000.0, 4), "traffic": measured_traffic(w.name),
+                     "algorithmic_bytes": int(alg_bytes)},
         "clocks": clk.summary(),
         "e2e": ({"value": round(statistics.mean(e2e_ms) * 1000, 3), "unit": "us", "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h} if e2e_ms else None),
@@ -427,6 +494,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.profile:
+            run_profile(args)
         else:
             run_zha(args, world, rank, local)
     finally:

@@ -77,13 +77,19 @@ class Workload:
 
 
 def workload(name: str, n_tokens: Optional[int] = None) -> Workload:
-    """The named workloads (tiny fp32, deep and wide 256K trees, the light sweep, build+batch)."""
+    """The named workloads (tiny fp32, deep and wide 256K trees, the deep tree at any size, the light
+    sweep, build+batch)."""
     if name == "tiny4k_fp32":
         return Workload(name, d=64, n_q_heads=1, n_kv_heads=1, n_tokens=4096, block=4, levels=3,
                         n_refs=4, p=0.9, batch=8, dtype="f32", gen="needles", seed=0)
     if name == "deep256k_bf16":
         return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=262144, block=4,
                         levels=6, n_refs=16, p=0.95, batch=1, dtype="bf16", gen="topics", seed=1)
+    if name == "deep_bf16":  # the deep tree's shape at another context length (profiling cases)
+        n = n_tokens if n_tokens is not None else 262144
+        return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=n, block=4,
+                        levels=levels_for_top(n, 4, max_top=64), n_refs=16, p=0.95, batch=1, dtype="bf16",
+                        gen="topics", seed=1)
     if name == "wide256k_bf16":
         return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=262144, block=256,
                         levels=1, n_refs=16, p=0.95, batch=1, dtype="bf16", gen="topics", seed=1)
