@@ -1,0 +1,108 @@
+"""Parity at full size: the 256K deep tree (GQA 32/4, d=128, bf16, block 4, 6 levels, 16 refs, p=0.95,
+batch 1) in the configuration the benchmark times.
+
+The oracle cannot rebuild the whole tree quickly, so the build is checked on sampled nodes (the first,
+the last and seeded random ones at every level of every KV head), each computed by the oracle straight
+from the raw keys it covers.  Routing and attention are cheap for the oracle even at this size, so
+every query head of several query sets is checked, before and after single-token appends.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.zha_oracle as zo
+from parity_helpers import assert_close_out, compare_planes, compare_route, f64, oracle_attend_on_sets, p32
+from synth.workloads import generate, workload
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import tree_indexed_sparse_03_b200 as z
+
+N_APPEND = 5
+
+
+@pytest.fixture(scope="module")
+def deep256k():
+    w = workload("deep256k_bf16")
+    n = w.n_tokens
+    inp = generate(w, n_total=n + N_APPEND)
+    cap = n + N_APPEND
+    cfg = z.make_config(d=w.d, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, block=w.block, levels=w.levels,
+                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=cap, max_batch=w.batch)
+    K = torch.zeros(w.n_kv_heads, cap, w.d, dtype=inp.K.dtype, device="cuda")
+    V = torch.zeros_like(K)
+    K[:, :n] = inp.K[:, :n].cuda()
+    V[:, :n] = inp.V[:, :n].cuda()
+    tree = z.ZhaTree(cfg, K, V, inp.refs.cuda().contiguous())
+    tree.build(n)
+    torch.cuda.synchronize()
+    tree.status()
+    return w, inp, tree
+
+
+def _sample_nodes(count: int, k: int, rng) -> np.ndarray:
+    if count <= k:
+        return np.arange(count)
+    idx = {0, count - 1} | set(int(i) for i in rng.choice(count, k - 2, replace=False))
+    return np.array(sorted(idx))
+
+
+def test_build_sampled_nodes(deep256k):
+    w, inp, tree = deep256k
+    rng = np.random.default_rng(7)
+    n = tree.size
+    for level in range(1, w.levels + 1):
+        mu, bias, f = tree.level_planes(level)
+        count = n // w.block ** level
+        for kvh in range(w.n_kv_heads):
+            Kh = f64(inp.K[kvh, :n])
+            refs = f64(inp.refs[kvh])
+            idx = _sample_nodes(count, 24, rng)
+            direct = [zo.node_planes_direct(Kh, refs, (level, int(i)), w.block) for i in idx]
+            orc = zo.Planes(np.concatenate([p.f for p in direct]), np.concatenate([p.mu for p in direct]),
+                            np.concatenate([p.bias for p in direct]))
+            it = torch.as_tensor(idx, dtype=torch.long)
+            compare_planes(f64(mu[kvh].cpu()[it]), f64(bias[kvh].cpu()[it]), f64(f[kvh].cpu()[it]), orc, w.dtype,
+                           refs, label=f"kv{kvh} level {level}")
+
+
+def _check_decode(w, inp, tree, Q):
+    O_bench = tree.decode(Q)  # the benchmark's call: no exports
+    O, (kept, cnt), stats = tree.decode(Q, want_kept=True, want_stats=True)
+    torch.cuda.synchronize()
+    tree.status()
+    # the exports do not change the computation
+    assert torch.equal(O_bench, O)
+    n = tree.size
+    group = w.n_q_heads // w.n_kv_heads
+    rep = compare_route(tree, Q, kept, cnt, p32(w.p), n, w.block, w.levels, group)
+    assert not rep.failures, "\n".join(rep.failures[:5])
+    assert rep.flagged <= 0.2 * rep.heads + 1, (rep.flagged, rep.heads)
+    ref = oracle_attend_on_sets(inp.K, inp.V, Q, kept, cnt, n, w.block, group)
+    atol = 2e-5 * float(inp.V[:, :n].abs().max()) + 1e-6
+    assert_close_out(O.cpu().numpy(), ref, atol, f"attend at N={n}")
+    assert torch.equal(stats.cpu()[..., 1], cnt.cpu().long())
+    return rep
+
+
+def test_route_attend_full_size(deep256k):
+    w, inp, tree = deep256k
+    Qs = inp.Q.cuda()
+    for s in (0, 5, 11):
+        rep = _check_decode(w, inp, tree, Qs[s])
+        print(f"query set {s}: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+
+
+def test_append_then_decode_full_size(deep256k):
+    w, inp, tree = deep256k
+    n0 = tree.size
+    Qs = inp.Q.cuda()
+    for i in range(N_APPEND):
+        t = n0 + i
+        # one token per append, as in a decode step: [Hkv, 1, d]
+        tree.append(inp.K[:, t:t + 1].cuda(), inp.V[:, t:t + 1].cuda())
+    torch.cuda.synchronize()
+    tree.status()
+    assert tree.size == n0 + N_APPEND
+    _check_decode(w, inp, tree, Qs[3])
