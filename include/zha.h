@@ -157,7 +157,7 @@ ZHA_API int64_t zha_tree_size(const zha_tree* tree);
  *              count the bytes a decode must read; leave NULL on the hot path.
  * Requires 1 <= B <= max_batch and at least one cached token.  The call
  * launches a fixed sequence of kernels on `stream` (per routing step a scoring
- * and a select kernel, then finalize, attention and combine kernels) and
+ * and a select kernel, then one attention kernel) and
  * returns without synchronizing; calls on one tree share its scratch and must
  * be issued in order on one stream.  A wait of a scoring warp on a record copy
  * is bounded: when it runs out the status word reports ZHA_ERR_TIMEOUT.

@@ -14,30 +14,35 @@
 // mass >= p; ties in e go to the lower start token; tokens after the last
 // complete block (the tail) are always attended.
 //
-// GPU design.  One persistent cooperative launch per decode call; all query
-// heads of all sequences are routed together so that the whole GPU shares
-// the work of the heads whose routing is diffuse.  Phases are separated by a
-// software grid barrier (a monotonic arrival counter; bounded spin: on
-// timeout the kernel raises ZHA_ERR_TIMEOUT and returns):
-//   score   (all CTAs) the step's candidates of every head form one list that
-//           is cut into contiguous per-warp ranges; each warp streams the node
-//           records of its range through a ring of shared-memory slots with
-//           cp.async (several records in flight per warp), computes the
-//           estimates in fp32 and writes (descending key of e, node code) at
-//           the candidate's position in its head's step buffer;
-//   select  (one CTA per head) masses w = exp(e - max e) as 2^-40 fixed-point
-//           integers (exact, order-independent sums); a 1024-bin histogram of
-//           the masses over (max e - e) in 1/32-logit bins, then 1024 sub-bins
-//           of the cut bin, isolate the few entries around the cut, which are
-//           ordered by (e desc, start asc); kept = every entry at or before the
-//           cut.  The children of the kept non-leaf nodes, in rank order, are
-//           written as the next step's candidates; kept leaves are appended to
-//           the head's attend list;
-//   attend  (all CTAs) every head's attended keys (kept blocks, sink, tail)
-//           are cut into chunks; CTAs own contiguous ranges of chunks, warps
-//           run an online softmax per chunk, and each CTA merges its chunks per
-//           head into one partial;
-//   combine (one CTA per head) the partials of each head -> O.
+// GPU design.  A decode call is a fixed sequence of kernels on the caller's
+// stream, each launched with programmatic stream serialization (it may start
+// while the one before drains and waits for it before reading its output);
+// all query heads of all sequences are routed together so that the whole GPU
+// shares the work of the heads whose routing is diffuse.  Per routing step s:
+//   score   (one CTA per SM) the step's units of every head (the roots, or the
+//           kept non-leaves of step s-1) form one list cut into contiguous
+//           per-warp ranges; each warp fetches the node records (the roots,
+//           or the b children of each unit) with bulk copies into a ring of
+//           shared-memory slots, computes the estimates (tensor cores for
+//           bf16) and writes (descending key of e, node code) at the entry's
+//           position in its head's step buffer, adding the entry's
+//           fixed-point mass to the step's histogram anchored at the largest
+//           estimate of step s-1;
+//   select  (one CTA per head) the cut: masses as 2^-40 fixed-point integers
+//           (exact, order-independent sums); the cut bin from the anchored
+//           histogram (or histograms built in the CTA), then its sub-bins,
+//           isolate the few entries around the cut, which are ordered by
+//           (e desc, start asc); kept = every entry at or before the cut.
+//           Kept non-leaves become the next step's units, kept leaves are
+//           appended to the head's attend list.
+// Then
+//   attend  (two CTAs per SM) every head's attended keys (kept blocks, sink,
+//           tail) are cut into chunks; CTAs own contiguous ranges of chunks,
+//           warps run an online softmax per chunk (tensor cores for bf16), each
+//           CTA merges its chunks per head into one partial, and the warp that
+//           writes a head's last partial combines the head's partials -> O.
+// The only waits inside a kernel are a scoring warp's waits for its own bulk
+// copies; they are bounded (on running out the kernel raises ZHA_ERR_TIMEOUT).
 #include <type_traits>
 
 #include "zha_args.cuh"
@@ -49,10 +54,11 @@ struct Entry {
   uint32_t code;  // node_code(level, index)
 };
 
-constexpr int kDecThreads = 512;                   // threads of a scoring, select or finalize CTA
+constexpr int kDecThreads = 512;                   // threads of a scoring or select CTA
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kUnionBytes = 208 * 1024;            // select: step keys cached in shared memory
-constexpr int kCacheKeys = kUnionBytes / 4;
+constexpr int kUnionBytes = 208 * 1024;            // select: step keys and codes cached in shared memory
+constexpr int kCacheEnt = kUnionBytes / 8;          // entries (key + code) the cache holds
+constexpr int kSpecEnt = 512;                       // entries a select fetches before it knows the step's size
 constexpr int kRingBytes = 200 * 1024;             // scoring: record ring of the CTA's warps
 constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
@@ -63,27 +69,27 @@ constexpr int kAttThreads = 256;                   // threads of an attention CT
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttItems = 32;                      // attend chunks a CTA owns at most
 constexpr int kMaxAttGrid = 512;                   // attention CTAs the scratch is laid out for
-constexpr int kCombThreads = 512;                  // threads of a combine CTA (one partial per thread)
-static_assert(kMaxAttGrid <= kCombThreads, "the combine takes one partial per thread");
-static_assert(kCombThreads % 128 == 0, "the combine splits its threads over the output elements");
 
 struct HeadState {  // per (sequence, query head)
   long long n[2];          // entries of the step built in each parity buffer (step 0: unused)
-  long long kept;          // entries kept by the last select (units of the next scoring phase)
+  long long units;         // kept non-leaves of the last select (units of the next scoring phase)
   long long scored;        // nodes scored so far
-  long long n_leaf;        // kept level-1 blocks (set when routing ends)
+  long long n_leaf;        // kept level-1 blocks listed so far
   unsigned int kinv[2];    // ~(smallest key) of the step built in each parity buffer
   int ovf[2];              // an estimate of that step lies above its anchor span
   float anchor;            // histogram anchor of the step being built (max e of the step before)
   int steps;               // selects done
   int leaf0;               // leaf block 0 kept (token 0 already attended)
-  int pad_i;
+  int ticket;              // attention partials of the head written so far
   long long pad[23];
 };
 static_assert(sizeof(HeadState) == 256, "HeadState layout");
 
-// Per-head routing state and leaf bitmaps live in one scratch region that
-// every decode leaves zeroed for the next (the combine phase clears it).
+// Per-head routing state and leaf bitmaps live in one scratch region.  The
+// first select of a decode starts the head's counters from zero, the last
+// one leaves both parities' step extremes cleared, the combining warp resets
+// the ticket and the export clears the bitmap, so a decode leaves the region
+// ready for the next one (after an error status the host zeroes it).
 
 // 32-bit words of a head's leaf bitmap (one bit per level-1 block), a multiple of 4.
 __host__ __device__ __forceinline__ int64_t decode_bitmap_words(int64_t cap_sel) {
@@ -130,7 +136,6 @@ struct __align__(16) DecSmem {
   unsigned long long bcast64[4];
   int bcast32[8];
   int fail;
-  int job_h, job_s;           // select CTA: the request being served (-2: exit)
 };
 
 // Division of 32-bit values by a fixed divisor d >= 2 with a multiply-high and
@@ -154,11 +159,12 @@ struct DivU32 {
 // rest (and every code) read from the global step buffers.
 struct StepView {
   const uint32_t* ck;  // cached keys
-  int nc;
+  const uint32_t* cc;  // cached codes
+  int nc;              // entries cached
   const uint32_t* gk;  // global keys
   const uint32_t* gc;  // global codes
   __device__ __forceinline__ uint32_t key(int64_t i) const { return i < nc ? ck[i] : __ldcg(gk + i); }
-  __device__ __forceinline__ uint32_t code(int64_t i) const { return __ldcg(gc + i); }
+  __device__ __forceinline__ uint32_t code(int64_t i) const { return i < nc ? cc[i] : __ldcg(gc + i); }
 };
 
 __device__ __forceinline__ uint32_t root_code(const DecodeArgs& a, int64_t i) {
@@ -1190,7 +1196,7 @@ struct Ctx {
   __device__ explicit Ctx(const DecodeArgs& args)
       : a(args), nh(args.nheads), cap4((args.cap_sel + 3) & ~int64_t(3)), bm_words(decode_bitmap_words(args.cap_sel)) {}
   // per-head workspace: step keys [2][cap4], step codes [2][cap4] (parity buffers: step s in s & 1),
-  // anchored histograms [2][kBins], kept entries of the last select [cap4], kept leaves [cap_list]
+  // anchored histograms [2][kBins], units of the next scoring phase [cap4], kept leaves [cap_list]
   __device__ char* ws(int h) const { return a.ws + uint64_t(h) * a.ws_per_bh; }
   __device__ uint32_t* keysP(int h, int par) const { return reinterpret_cast<uint32_t*>(ws(h) + par * cap4 * 4); }
   __device__ uint32_t* codesP(int h, int par) const {
@@ -1199,7 +1205,7 @@ struct Ctx {
   __device__ unsigned long long* histP(int h, int par) const {
     return reinterpret_cast<unsigned long long*>(ws(h) + 4 * cap4 * 4 + par * kBins * 8);
   }
-  __device__ uint32_t* keptl(int h) const { return reinterpret_cast<uint32_t*>(ws(h) + 4 * cap4 * 4 + 2 * kBins * 8); }
+  __device__ uint32_t* units(int h) const { return reinterpret_cast<uint32_t*>(ws(h) + 4 * cap4 * 4 + 2 * kBins * 8); }
   __device__ uint32_t* leaves(int h) const {
     return reinterpret_cast<uint32_t*>(ws(h) + 5 * cap4 * 4 + 2 * kBins * 8);
   }
@@ -1219,177 +1225,198 @@ struct Ctx {
 
 // ---------------------------------------------------------------- select
 // One head, whole CTA: the cut of step s (small path, anchored histogram or
-// the in-CTA histograms), the kept entries listed in entry order, and the
-// state of step s+1 (histogram cleared, anchor = step s's max).
+// the in-CTA histograms), then the kept entries in entry order, split by
+// level: kept non-leaves become the units of step s+1 (unit u's b children
+// are scored into positions u*b .. u*b+b-1 of step s+1), kept level-1 blocks
+// are appended to the head's leaf list.  The head's state and the step's
+// first kSpecEnt keys and codes are fetched together; a larger step's other
+// keys and codes follow once its size is known.
+template <typename T, int D>
+__device__ __noinline__ void export_kept(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h);
+
 template <typename T, int D>
 __device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c, DecSmem& sm, int h, int s) {
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int tid = threadIdx.x;
   const int par = s & 1;
-  {
-    HeadState* hs = c.hstate(h);
-    const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
-    if (n == 0) {
-      if (tid == 0) hs->kept = 0;
-      return;
-    }
-    const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
-    const float anchor_h = __ldcg(&hs->anchor);
-    const int ovf = __ldcg(&hs->ovf[par]);
-    const long long scored0 = __ldcg(&hs->scored);
-    const uint32_t* gk = c.keysP(h, par);
-    const uint32_t* gc = c.codesP(h, par);
-    if (a.scored) {  // codes of the scored nodes
-      int32_t* out = a.scored + size_t(h) * a.scored_cap;
-      for (long long i = tid; i < n; i += kDecThreads)
-        if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(__ldcg(gc + i));
-    }
-    const float m = desc_key_value(kmin);
-    // the step's keys, cached in shared memory as far as they fit (16-byte async copies)
-    const int ncache = int(min64(n, kCacheKeys));
-    uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
-    for (int v = tid; v < (ncache + 3) / 4; v += kDecThreads) cp_async16(ck + 4 * v, gk + 4 * v);
-    cp_async_commit();
-    cp_async_wait(0);
-    __syncthreads();
-    const StepView E{ck, ncache, gk, gc};
-    unsigned long long cut = ~0ull;
-    if (!a.p_all) {
-      if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
-      else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
-        cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
-      else cut = select_cut(a, E, n, kmin, sm, h, s);
-    }
-    // the kept entries (order key <= cut), listed in entry order: each warp
-    // owns a contiguous run of 128-entry groups, four entries per lane; the
-    // code is read only for a key equal to the cut's
-    long long n_kept = 0;
-    {
-      const uint32_t cut32 = uint32_t(cut >> 32);
-      const int n32 = int(n);
-      const int groups = (n32 + 127) / 128;
-      const int gseg = (groups + kDecWarps - 1) / kDecWarps;
-      const int wlo = min(n32, wid * gseg * 128), whi = min(n32, wlo + gseg * 128);
-      auto kept4 = [&](int i0) -> unsigned {  // bit u: entry i0 + u is kept (i0 + u < whi)
-        uint32_t k[4];
-        if (i0 + 4 <= E.nc && i0 + 4 <= whi) {
-          const uint4 v = *reinterpret_cast<const uint4*>(E.ck + i0);
-          k[0] = v.x;
-          k[1] = v.y;
-          k[2] = v.z;
-          k[3] = v.w;
-        } else {
+  const bool last = s + 1 == a.n_steps;
+  const int b = a.t.block;
+  HeadState* hs = c.hstate(h);
+  const uint32_t* gk = c.keysP(h, par);
+  const uint32_t* gc = c.codesP(h, par);
+  uint32_t* ck = reinterpret_cast<uint32_t*>(sm.u);
+  uint32_t* cc = ck + kCacheEnt;
+  const int spec = int(min64(kSpecEnt, c.cap4));
+  for (int v = tid; v < spec / 4; v += kDecThreads) {
+    cp_async16(ck + 4 * v, gk + 4 * v);
+    cp_async16(cc + 4 * v, gc + 4 * v);
+  }
+  cp_async_commit();
+  // step 0 starts the head's counters afresh
+  const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
+  const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
+  const float anchor_h = __ldcg(&hs->anchor);
+  const int ovf = __ldcg(&hs->ovf[par]);
+  const long long scored0 = s == 0 ? 0 : __ldcg(&hs->scored);
+  const long long leaves0 = s == 0 ? 0 : min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
+  const int leaf0_in = s == 0 ? 0 : __ldcg(&hs->leaf0);
+  const int steps0 = s == 0 ? 0 : __ldcg(&hs->steps);
+  const int ncache = int(min64(n, kCacheEnt));
+  for (int v = spec / 4 + tid; v < (ncache + 3) / 4; v += kDecThreads) {
+    cp_async16(ck + 4 * v, gk + 4 * v);
+    cp_async16(cc + 4 * v, gc + 4 * v);
+  }
+  cp_async_commit();
+  cp_async_wait(0);
+  __syncthreads();
+  const StepView E{ck, cc, ncache, gk, gc};
+  if (a.scored) {  // codes of the scored nodes
+    int32_t* out = a.scored + size_t(h) * a.scored_cap;
+    for (long long i = tid; i < n; i += kDecThreads)
+      if (scored0 + i < a.scored_cap) out[scored0 + i] = int32_t(E.code(i));
+  }
+  const float m = desc_key_value(kmin);
+  unsigned long long cut = ~0ull;
+  if (!a.p_all && n > 0) {
+    if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
+    else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
+      cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
+    else cut = select_cut(a, E, n, kmin, sm, h, s);
+  }
+  // the kept entries (order key <= cut) in entry order, four per thread and
+  // round; one block scan per round gives both lists' positions (units in the
+  // high half of the packed count, leaves in the low half)
+  const uint32_t cut32 = uint32_t(cut >> 32);
+  const int n32 = int(n);
+  uint32_t* un = c.units(h);
+  uint32_t* lv = c.leaves(h);
+  uint32_t* bm = c.bitmap(h);
+  long long nu = 0, nlf = 0;
+  int leaf0 = 0;
+  for (int base = 0; base < n32; base += 4 * kDecThreads) {
+    const int i0 = base + 4 * tid;
+    uint32_t k[4], cd[4];
+    if (i0 + 4 <= ncache) {
+      const uint4 kv = *reinterpret_cast<const uint4*>(ck + i0);
+      const uint4 cv = *reinterpret_cast<const uint4*>(cc + i0);
+      k[0] = kv.x; k[1] = kv.y; k[2] = kv.z; k[3] = kv.w;
+      cd[0] = cv.x; cd[1] = cv.y; cd[2] = cv.z; cd[3] = cv.w;
+    } else {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) k[u] = i0 + u < whi ? E.key(i0 + u) : 0xffffffffu;
-        }
-        unsigned bits = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool kp = i0 + u < whi &&
-                          (k[u] < cut32 || (k[u] == cut32 && entry_key64(a, Entry{k[u], E.code(i0 + u)}) <= cut));
-          bits |= kp ? (1u << u) : 0u;
-        }
-        return bits;
-      };
-      uint32_t wk = 0;
-      for (int base = wlo; base < whi; base += 128) wk += __popc(kept4(base + 4 * lane));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) wk += __shfl_xor_sync(0xffffffffu, wk, off);
-      if (lane == 0) sm.red32[wid] = wk;
-      __syncthreads();
-      uint32_t off = 0;
-      for (int w = 0; w < kDecWarps; ++w) {
-        if (w < wid) off += sm.red32[w];
-        n_kept += sm.red32[w];
-      }
-      uint32_t* kl = c.keptl(h);
-      for (int base = wlo; base < whi; base += 128) {
-        const int i0 = base + 4 * lane;
-        unsigned bits = kept4(i0);
-        const uint32_t pc = __popc(bits);
-        uint32_t ex = pc;
-#pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, ex, o2);
-          if (lane >= o2) ex += y;
-        }
-        uint32_t pos = off + ex - pc;
-        while (bits) {
-          const int u = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          kl[pos++] = uint32_t(i0 + u);
-        }
-        off += __shfl_sync(0xffffffffu, ex, 31);
+      for (int u = 0; u < 4; ++u) {
+        k[u] = i0 + u < n32 ? E.key(i0 + u) : 0xffffffffu;
+        cd[u] = i0 + u < n32 ? E.code(i0 + u) : 0u;
       }
     }
-    // state for the next step: its histogram cleared, its anchor = this step's max
+    unsigned kb = 0, lb = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool kp = i0 + u < n32 &&
+                      (k[u] < cut32 || (k[u] == cut32 && entry_key64(a, Entry{k[u], cd[u]}) <= cut));
+      if (kp && valid_code(a, cd[u])) {  // (codes come from the scoring kernel; the check guards the writes)
+        kb |= 1u << u;
+        if (code_level(cd[u]) == 1) lb |= 1u << u;
+      }
+    }
+    unsigned long long tot;
+    const unsigned long long ex =
+        block_scan_u64((unsigned long long)__popc(kb & ~lb) << 32 | (unsigned long long)__popc(lb), sm.red64, &tot);
+    long long pu = nu + (long long)(ex >> 32);
+    long long pl = leaves0 + nlf + (long long)(ex & 0xffffffffull);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!((kb >> u) & 1u)) continue;
+      if ((lb >> u) & 1u) {
+        const uint32_t li = code_index(cd[u]);
+        if (pl < a.cap_list) lv[pl] = li;
+        ++pl;
+        leaf0 |= li == 0u ? 1 : 0;
+        if (a.kept) atomicOr(bm + (li >> 5), 1u << (li & 31u));
+      } else {
+        un[pu++] = cd[u];
+      }
+    }
+    nu += (long long)(tot >> 32);
+    nlf += (long long)(tot & 0xffffffffull);
+  }
+  const int any_leaf0 = __syncthreads_or(leaf0);
+  // state for the next step: its histogram cleared, its anchor = this step's max
+  if (!last) {
     unsigned long long* nhist = c.histP(h, par ^ 1);
     for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
-    __syncthreads();
-    if (tid == 0) {
-      hs->kept = n_kept;
-      hs->n[par ^ 1] = 0;
-      hs->anchor = m;
-      hs->kinv[par ^ 1] = 0u;
-      hs->ovf[par ^ 1] = 0;
-      hs->scored = scored0 + n;
-      hs->steps = hs->steps + 1;
+  }
+  if (tid == 0) {
+    long long U = nu, NL = leaves0 + nlf;
+    if (U * b > a.cap_sel) {
+      raise_status(a.t.status, ZHA_ERR_CAPACITY);
+      U = a.cap_sel / b;
     }
+    if (NL > a.cap_list) {
+      raise_status(a.t.status, ZHA_ERR_CAPACITY);
+      NL = a.cap_list;
+    }
+    hs->units = U;
+    hs->n[par ^ 1] = U * b;
+    hs->n_leaf = NL;
+    hs->leaf0 = leaf0_in | any_leaf0;
+    hs->anchor = m;
+    hs->kinv[par ^ 1] = 0u;
+    hs->ovf[par ^ 1] = 0;
+    hs->scored = scored0 + n;
+    hs->steps = steps0 + (n > 0 ? 1 : 0);
+    if (last) {  // the next decode's first step finds its extremes cleared
+      hs->kinv[par] = 0u;
+      hs->ovf[par] = 0;
+    }
+  }
+  if (last && a.kept) {
+    __threadfence();
+    __syncthreads();
+    export_kept(a, c, sm.red32, h);
   }
 }
 
-// ---------------------------------------------------------------- finalize
-// One head, whole CTA: the kept leaves in block order from the head's bitmap
-// (each warp owns a contiguous run of words: counts, one scan over warps, then
-// writes), which it leaves zeroed.
+// ---------------------------------------------------------------- kept export
+// The head's kept leaves in ascending block order from its bitmap (every
+// select of a call with the export sets the bits of the leaves it keeps),
+// which it leaves zeroed.  Each warp owns a contiguous run of words: counts,
+// one scan over warps, then writes.
 template <typename T, int D>
-__device__ __noinline__ void finalize_head(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h) {
+__device__ __noinline__ void export_kept(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int64_t bm_words = c.bm_words;
-  {
-    uint32_t* bm = c.bitmap(h);
-    const long long nw = min64((a.nl[1] + 31) / 32, bm_words);
-    const long long wseg = (nw + kDecWarps - 1) / kDecWarps;
-    const long long w_lo = min64(nw, wid * wseg), w_hi = min64(nw, w_lo + wseg);
-    uint32_t cnt = 0;
-    for (long long wi = w_lo + lane; wi < w_hi; wi += 32) cnt += __popc(__ldcg(bm + wi));
+  uint32_t* bm = c.bitmap(h);
+  const long long nw = min64((a.nl[1] + 31) / 32, c.bm_words);
+  const long long wseg = (nw + kDecWarps - 1) / kDecWarps;
+  const long long w_lo = min64(nw, wid * wseg), w_hi = min64(nw, w_lo + wseg);
+  uint32_t cnt = 0;
+  for (long long wi = w_lo + lane; wi < w_hi; wi += 32) cnt += __popc(__ldcg(bm + wi));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (lane == 0) red32[wid] = cnt;
-    __syncthreads();
-    long long pos = 0, total = 0;
-    for (int w = 0; w < kDecWarps; ++w) {
-      if (w < wid) pos += red32[w];
-      total += red32[w];
-    }
-    const int leaf0 = nw > 0 ? int(__ldcg(bm) & 1u) : 0;
-    __syncthreads();
-    for (long long wb = w_lo; wb < w_hi; wb += 32) {
-      const long long wi = wb + lane;
-      uint32_t bits = wi < w_hi ? __ldcg(bm + wi) : 0u;
-      uint32_t pc = __popc(bits), ex = pc;
+  for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+  if (lane == 0) red32[wid] = cnt;
+  __syncthreads();
+  long long pos = 0;
+  for (int w = 0; w < wid; ++w) pos += red32[w];
+  __syncthreads();
+  int32_t* out = a.kept + size_t(h) * a.kept_stride;
+  for (long long wb = w_lo; wb < w_hi; wb += 32) {
+    const long long wi = wb + lane;
+    uint32_t bits = wi < w_hi ? __ldcg(bm + wi) : 0u;
+    const uint32_t pc = __popc(bits);
+    uint32_t ex = pc;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, ex, off);
-        if (lane >= off) ex += y;
-      }
-      const uint32_t wtot = __shfl_sync(0xffffffffu, ex, 31);
-      long long p = pos + ex - pc;
-      if (bits) bm[wi] = 0u;  // leave the bitmap zeroed for the next decode
-      while (bits) {
-        const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
-        bits &= bits - 1u;
-        if (p < a.cap_list) c.leaves(h)[p] = idx;
-        if (a.kept && p < a.kept_stride) a.kept[size_t(h) * a.kept_stride + p] = int32_t(idx);
-        ++p;
-      }
-      pos += wtot;
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ex, off);
+      if (lane >= off) ex += y;
     }
-    if (tid == 0) {
-      if (total > a.cap_list) raise_status(a.t.status, ZHA_ERR_CAPACITY);
-      c.hstate(h)->n_leaf = min64(total, a.cap_list);
-      c.hstate(h)->leaf0 = leaf0;
+    const uint32_t wtot = __shfl_sync(0xffffffffu, ex, 31);
+    long long p = pos + ex - pc;
+    if (bits) bm[wi] = 0u;
+    while (bits) {
+      const uint32_t idx = uint32_t(wi) * 32u + uint32_t(__ffs(bits) - 1);
+      bits &= bits - 1u;
+      if (p < a.kept_stride) out[p] = int32_t(idx);
+      ++p;
     }
-    __syncthreads();
+    pos += wtot;
   }
 }
 
@@ -1405,29 +1432,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_con
     __syncthreads();
   }
 }
-template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads) finalize_kernel(const __grid_constant__ DecodeArgs a) {
-  pdl_wait_and_release();
-  __shared__ uint32_t red32[kDecWarps];
-  const Ctx<T, D> c(a);
-  for (int h = blockIdx.x; h < a.nheads; h += gridDim.x) {
-    finalize_head<T, D>(a, c, red32, h);
-    __syncthreads();
-  }
-}
 
 // ---------------------------------------------------------------- scoring phase
 // Step s's entries: the roots (s = 0, root i at position i) or the children of
-// step s-1's kept non-leaves, at positions reserved per warp batch with one
-// atomic add per head (their order varies from run to run; nothing
-// downstream depends on it); kept leaves of step s-1 go to the head's bitmap.
-// Units (roots, or kept entries) of all heads are cut into contiguous ranges,
-// one per warp.  Each record is fetched with one bulk copy into the warp's
-// ring; the estimate is added to the step's anchored histogram (s >= 1).
+// step s-1's kept non-leaves (unit u of the head: positions u*b .. u*b+b-1).
+// Units of all heads are cut into contiguous ranges, one per warp.  Each
+// record is fetched with one bulk copy into the warp's ring; the estimate is
+// added to the step's anchored histogram (s >= 1).
 
 struct __align__(16) ScoreSmem {
   unsigned char ring[kRingBytes];
   long long pref[kMaxHeads + 1];
+  float anchor[kMaxHeads];
   unsigned long long red64[kDecWarps];
   unsigned long long mbar[kDecWarps][kMaxSlots];
 };
@@ -1464,9 +1480,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   bool failed = false;  // a copy never landed: this warp stops scoring
   const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
   const long long nwarps = (long long)gridDim.x * score_warps;
-  // ---------------- scoring phase: units = roots (s = 0) or the kept entries of step s-1
-  for (int i = tid; i < nh; i += kDecThreads)
-    sp.pref[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&c.hstate(i)->kept), 0), a.cap_sel);
+  // ---------------- units = roots (s = 0) or the kept non-leaves of step s-1
+  for (int i = tid; i < nh; i += kDecThreads) {
+    sp.pref[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&c.hstate(i)->units), 0), a.cap_sel);
+    sp.anchor[i] = s == 0 ? 0.f : __ldcg(&c.hstate(i)->anchor);
+  }
   __syncthreads();
   const long long total = build_prefix<kDecThreads>(sp.pref, sp.red64, nh);
   const long long u0 = gwarp < 0 ? 0 : total * gwarp / nwarps;
@@ -1474,8 +1492,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   int cur_h = -1;           // lane 0: head of the pending min-key update
   uint32_t cur_kmin = 0xffffffffu;
   int cur_ovf = 0;
-  int ah = -1;              // head whose anchor is loaded
-  float anchor = 0.f;
   for (long long ub = u0; ub < u1; ub += 32) {
     // one unit per lane: its head, its first output position, its code
     const long long u = ub + lane;
@@ -1491,40 +1507,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
         upos = k;
         has = valid_code(a, ucode);
       } else {
-        const uint32_t idx = __ldcg(c.keptl(uh) + k);
-        const uint32_t code = idx < uint32_t(a.cap_sel) ? __ldcg(c.codesP(uh, par ^ 1) + idx) : 0u;
-        if (valid_code(a, code)) {
-          if (code_level(code) == 1) {
-            atomicOr(c.bitmap(uh) + (code_index(code) >> 5), 1u << (code_index(code) & 31u));
-          } else {
-            ucode = code;
-            has = true;
-          }
+        const uint32_t code = __ldcg(c.units(uh) + k);
+        if (valid_code(a, code) && code_level(code) >= 2) {
+          ucode = code;
+          upos = k * b;
+          has = true;
         }
-      }
-    }
-    if (s >= 1) {  // positions: one reservation per head segment of the batch
-      unsigned todo = __ballot_sync(0xffffffffu, has);
-      while (todo) {
-        const int l0 = __ffs(todo) - 1;
-        const int h0 = __shfl_sync(0xffffffffu, uh, l0);
-        const unsigned seg = __ballot_sync(0xffffffffu, has && uh == h0);
-        long long bs = 0;
-        if (lane == l0) {
-          const long long need = (long long)__popc(seg) * b;
-          bs = (long long)atomicAdd(reinterpret_cast<unsigned long long*>(&c.hstate(h0)->n[par]),
-                                    (unsigned long long)need);
-          if (bs + need > a.cap_sel) {
-            raise_status(a.t.status, ZHA_ERR_CAPACITY);
-            bs = -1;
-          }
-        }
-        bs = __shfl_sync(0xffffffffu, bs, l0);
-        if (has && uh == h0) {
-          upos = bs + (long long)__popc(seg & ((1u << lane) - 1u)) * b;
-          if (bs < 0) has = false;
-        }
-        todo &= ~seg;
       }
     }
     const unsigned mhas = __ballot_sync(0xffffffffu, has);
@@ -1634,13 +1622,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
         }
         cur_kmin = min(cur_kmin, key);
         if (s >= 1) {
-          if (it.h != ah) {
-            anchor = __ldcg(&c.hstate(it.h)->anchor);
-            ah = it.h;
-          }
           unsigned long long w;
           float t;
-          const int bin = anchored_bin(anchor, key, &w, &t);
+          const int bin = anchored_bin(sp.anchor[it.h], key, &w, &t);
           if (bin < 0) cur_ovf = 1;
           else atomicAdd(c.histP(it.h, par) + bin, w);
         }
@@ -1679,8 +1663,7 @@ __device__ __forceinline__ long long att_head_keys(const Ctx<T, D>& c, int h, lo
   return *nl * a.t.block + (*sink ? 1 : 0) + tail;
 }
 
-// The chunk partition of all heads' attended keys over `grid` CTAs (the same
-// in the attention and combine kernels): chunk size (>= 32 keys, so that a CTA
+// The chunk partition of all heads' attended keys over `grid` CTAs: chunk size (>= 32 keys, so that a CTA
 // owns at most about kAttItems chunks), and per-head chunk prefix in pref[0..nh].
 template <typename T, int D, int NT>
 __device__ __forceinline__ void att_partition(const Ctx<T, D>& c, long long* pref, unsigned long long* red64,
@@ -1715,6 +1698,91 @@ struct __align__(16) AttSmem {
   long long pref[kMaxHeads + 1];
   unsigned long long red64[kAttWarps];
 };
+
+// ---------------------------------------------------------------- combine
+// The partials of head h (one per attention CTA whose chunk range meets the
+// head's chunks [P0, P1), at slot max(P0, range start)) rescaled to their
+// common max and summed -> O, by one warp of the CTA that wrote the head's
+// last partial; then the head's statistics and kept count, and its ticket
+// reset.  The sums run over the partials in CTA order (deterministic).
+template <typename T, int D>
+__device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& c, int h, long long P0, long long P1,
+                                          long long total_items, int grid) {
+  const int lane = threadIdx.x & 31;
+  constexpr int NQ = (D + 31) / 32;
+  auto range_start = [&](long long cc) { return (cc * total_items) / (long long)grid; };
+  long long cfirst = (P0 * grid) / max64(total_items, 1);
+  while (cfirst > 0 && range_start(cfirst) > P0) --cfirst;
+  while (cfirst + 1 < grid && range_start(cfirst + 1) <= P0) ++cfirst;
+  // slot of CTA cfirst + i, or -1 if that CTA has no chunk of the head
+  auto slot_of = [&](long long cc) -> long long {
+    if (cc >= grid) return -1;
+    const long long cs = max64(P0, range_start(cc));
+    return (cs < P1 && cs < range_start(cc + 1)) ? cs : -1;
+  };
+  float M = -INFINITY;
+  for (long long cc = cfirst + lane; cc < grid && range_start(cc) < P1; cc += 32) {
+    const long long sl = slot_of(cc);
+    if (sl >= 0) M = fmaxf(M, __ldcg(a.attn_part + size_t(sl) * (2 + D)));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f, acc[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+  for (long long cb = cfirst; cb < grid && range_start(cb) < P1; cb += 32) {
+    const long long sl = slot_of(cb + lane);
+    float sc = 0.f;
+    if (sl >= 0) {
+      const float mj = __ldcg(a.attn_part + size_t(sl) * (2 + D));
+      sc = mj == -INFINITY ? 0.f : expf(mj - M);
+      L = fmaf(sc, __ldcg(a.attn_part + size_t(sl) * (2 + D) + 1), L);
+    }
+    for (int t0 = 0; t0 < 32; t0 += 8) {  // 8 partials' loads in flight per lane
+      float x[8][NQ], w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const long long st = __shfl_sync(0xffffffffu, sl, t0 + u);
+        w[u] = __shfl_sync(0xffffffffu, sc, t0 + u);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          x[u][q] = (st >= 0 && q * 32 + lane < D) ? __ldcg(a.attn_part + size_t(st) * (2 + D) + 2 + q * 32 + lane)
+                                                  : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+    if (q * 32 + lane < D) a.O[size_t(h) * D + q * 32 + lane] = acc[q] / L;
+  if (lane == 0) {
+    const long long n1 = a.nl[1], b = a.t.block;
+    const long long tail = a.n_tokens - n1 * b;
+    long long nl = 0, scored = 0;
+    int l0 = 0, steps = 0;
+    HeadState* hs = c.hstate(h);
+    if (a.n_steps > 0 && a.n_roots > 0) {
+      nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
+      l0 = __ldcg(&hs->leaf0);
+      scored = __ldcg(&hs->scored);
+      steps = __ldcg(&hs->steps);
+    }
+    hs->ticket = 0;
+    if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
+    if (a.stats) {
+      int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
+      st[ZHA_STAT_NODES_SCORED] = scored;
+      st[ZHA_STAT_LEAVES_KEPT] = nl;
+      st[ZHA_STAT_KEYS] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
+      st[ZHA_STAT_STEPS] = steps;
+    }
+  }
+}
 
 // CTAs per SM the attention kernel is compiled for: two for the tensor-core
 // (bf16) path, whose tiles need up to 128 registers, three for the fp32 path.
@@ -2030,117 +2098,19 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
 #pragma unroll
     for (int q = 0; q < (D + 31) / 32; ++q)
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
-  }
-}
-
-// ---------------------------------------------------------------- combine
-// One CTA per head: the partials of the head (one per attention CTA that met
-// it) rescaled to their common max and summed -> O; the head's statistics and
-// kept count; the head's state zeroed for the next call.
-template <typename T, int D>
-__global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_constant__ DecodeArgs a, int att_grid) {
-  pdl_wait_and_release();
-  __shared__ long long pref[kMaxHeads + 1];
-  __shared__ unsigned long long red64[kCombThreads / 32];
-  __shared__ uint32_t red32[kCombThreads / 32];
-  __shared__ float pm[kCombThreads];
-  __shared__ long long ps[kCombThreads];
-  __shared__ float redf[kCombThreads];
-  const Ctx<T, D> c(a);
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int nh = a.nheads, b = a.t.block;
-  constexpr int NW = kCombThreads / 32;
-  long long chunk, total_items;
-  att_partition<T, D, kCombThreads>(c, pref, red64, att_grid, &chunk, &total_items);
-  const long long n1 = a.nl[1];
-  const long long tail = a.n_tokens - n1 * b;
-  for (int h = blockIdx.x; h < nh; h += gridDim.x) {
-    const long long p0 = pref[h], p1 = pref[h + 1];
-    // partial slots: one per attention CTA whose chunk range meets [p0, p1), at
-    // max(p0, range start); thread t takes the t-th of them
-    auto range_start = [&](long long cc) { return (cc * total_items) / (long long)att_grid; };
-    long long cfirst = (p0 * att_grid) / max64(total_items, 1);
-    while (cfirst > 0 && range_start(cfirst) > p0) --cfirst;
-    while (cfirst + 1 < att_grid && range_start(cfirst + 1) <= p0) ++cfirst;
-    float mt = -INFINITY, lt = 0.f;
-    long long myslot = -1;
-    {
-      const long long cc = cfirst + tid;
-      if (cc < att_grid) {
-        const long long cs = max64(p0, range_start(cc));
-        if (cs < p1 && cs < min64(p1, range_start(cc + 1))) {
-          myslot = cs;
-          const float* G = a.attn_part + size_t(cs) * (2 + D);
-          mt = __ldcg(G);
-          lt = __ldcg(G + 1);
-        }
-      }
+    // the head's chunks done so far; the warp that completes them combines
+    __threadfence();
+    __syncwarp();
+    int done = 0;
+    if (lane == 0) {
+      const int mine = int(send - seg);
+      const int prev = atomicAdd(&c.hstate(h)->ticket, mine);
+      done = prev + mine == int(sm.pref[h + 1] - sm.pref[h]) ? 1 : 0;
     }
-    float M = mt;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) red32[wid] = __float_as_uint(M);
-    __syncthreads();
-    M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, __uint_as_float(red32[w]));
-    const float sct = (myslot < 0 || mt == -INFINITY) ? 0.f : expf(mt - M);
-    pm[tid] = sct;
-    ps[tid] = myslot;
-    float Lw = sct * lt;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Lw += __shfl_xor_sync(0xffffffffu, Lw, off);
-    __syncthreads();
-    if (lane == 0) red32[wid] = __float_as_uint(Lw);
-    __syncthreads();
-    float L = 0.f;
-    for (int w = 0; w < NW; ++w) L += __uint_as_float(red32[w]);
-    // outputs: NP threads per element, each over every NP-th partial (independent loads)
-    constexpr int NP = kCombThreads / D;
-    const int e = tid % D, prt = tid / D;
-    const int npart = int(min64(att_grid - cfirst, kCombThreads));
-    // 8 independent loads in flight per thread (partials past npart or empty add 0)
-    float acc = 0.f;
-    for (int t0 = prt; t0 < npart; t0 += 8 * NP) {
-      float x[8], w[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = t0 + u * NP;
-        const long long cs = t < npart ? ps[t] : -1;
-        w[u] = cs >= 0 ? pm[t] : 0.f;
-        x[u] = cs >= 0 ? __ldcg(a.attn_part + size_t(cs) * (2 + D) + 2 + e) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc = fmaf(w[u], x[u], acc);
+    if (__shfl_sync(0xffffffffu, done, 0)) {
+      __threadfence();
+      combine_head<T, D>(a, c, h, sm.pref[h], sm.pref[h + 1], total_items, int(gridDim.x));
     }
-    redf[prt * D + e] = acc;
-    __syncthreads();
-    if (prt == 0) {
-      for (int q = 1; q < NP; ++q) acc += redf[q * D + e];
-      a.O[size_t(h) * D + e] = acc / L;
-    }
-    if (tid == 0) {
-      long long nl = 0, scored = 0;
-      int l0 = 0, steps = 0;
-      if (a.n_steps > 0 && a.n_roots > 0) {
-        HeadState* hs = c.hstate(h);
-        nl = __ldcg(&hs->n_leaf);
-        l0 = __ldcg(&hs->leaf0);
-        scored = __ldcg(&hs->scored);
-        steps = __ldcg(&hs->steps);
-        // leave the head's state zeroed for the next call
-        long long* z = reinterpret_cast<long long*>(hs);
-        for (int k = 0; k < int(sizeof(HeadState) / 8); ++k) z[k] = 0;
-      }
-      if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
-      if (a.stats) {
-        int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
-        st[ZHA_STAT_NODES_SCORED] = scored;
-        st[ZHA_STAT_LEAVES_KEPT] = nl;
-        st[ZHA_STAT_KEYS] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
-        st[ZHA_STAT_STEPS] = steps;
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -2189,21 +2159,15 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   const bool routed = a.n_steps > 0 && a.n_roots > 0;
   int launches = 0;
   if (routed) {
-    for (int s = 0; s <= a.n_steps; ++s) {
+    for (int s = 0; s < a.n_steps; ++s) {
       launch_pdl(score_kernel<T, D>, unsigned(sms), kDecThreads, sizeof(ScoreSmem), st, a, s);
-      ++launches;
-      if (s < a.n_steps) {
-        launch_pdl(select_kernel<T, D>, nh, kDecThreads, sizeof(DecSmem), st, a, s);
-        ++launches;
-      }
+      launch_pdl(select_kernel<T, D>, nh, kDecThreads, sizeof(DecSmem), st, a, s);
+      launches += 2;
     }
-    launch_pdl(finalize_kernel<T, D>, nh, kDecThreads, 0, st, a);
-    ++launches;
   }
   const int att_grid = min(kMaxAttGrid, att_ctas_per_sm<T>() * sms);  // one wave
   launch_pdl(attend_kernel<T, D>, unsigned(att_grid), kAttThreads, sizeof(AttSmem), st, a);
-  launch_pdl(combine_kernel<T, D>, nh, kCombThreads, 0, st, a, att_grid);
-  launches += 2;
+  launches += 1;
   count_launches(launches);
   return cudaGetLastError();
 }
@@ -2219,7 +2183,7 @@ size_t decode_flow_bytes(int nheads, int64_t cap_sel) {
   return size_t(nheads) * (sizeof(HeadState) + size_t(decode_bitmap_words(cap_sel)) * 4);
 }
 // Per-head routing workspace: step keys and codes in two parity buffers, two
-// anchored histograms, the kept entries of the last select, the kept leaves.
+// anchored histograms, the units of the next scoring phase, the kept leaves.
 uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list) {
   const uint64_t cap4 = (uint64_t(cap_sel) + 3) & ~uint64_t(3);
   return cap4 * 20 + 2 * kBins * 8 + uint64_t(cap_list) * 4;
