@@ -136,10 +136,15 @@ def _unit(x: torch.Tensor) -> torch.Tensor:
 def generate(w: Workload, device: str = "cpu", n_total: Optional[int] = None) -> Inputs:
     """Draw the workload's tensors.
 
-    ``n_total`` defaults to ``n_tokens + append``: the appended tokens continue
-    the same segment/topic process and are simply the tail of K and V.
+    The workload's own tokens (``n_tokens + append``) do not depend on
+    ``n_total``: asking for fewer returns a prefix, asking for more draws the
+    extra tokens from a second seeded stream (same distribution; under
+    "topics" they continue the last segment's topic), so a benchmark's step
+    count never changes the context it runs on.
     """
-    n = w.n_tokens + w.append if n_total is None else n_total
+    n_base = w.n_tokens + w.append
+    n_want = n_base if n_total is None else n_total
+    n = n_base
     g = torch.Generator(device=device)
     g.manual_seed(w.seed)
     f32 = torch.float32
@@ -205,6 +210,23 @@ def generate(w: Workload, device: str = "cpu", n_total: Optional[int] = None) ->
     else:
         raise KeyError(w.gen)
 
+    if n_want < n:
+        K, V = K[:, :n_want], V[:, :n_want]
+    elif n_want > n:
+        g2 = torch.Generator(device=device)
+        g2.manual_seed(w.seed * 1000003 + 7919)
+        m = n_want - n
+        Kx = torch.randn(Hkv, m, d, generator=g2, device=device, dtype=f32)
+        Vx = torch.randn(Hkv, m, d, generator=g2, device=device, dtype=f32)
+        if w.gen == "needles":
+            Kx *= 0.5
+        else:
+            last = int(tok_topic[-1])
+            for h in range(Hkv):
+                Kx[h] += w.topic_amp * T[h, last]
+                Vx[h] += w.topic_amp * T[h, last]
+        K, V = torch.cat([K, Kx], 1), torch.cat([V, Vx], 1)
+    meta["n_total"] = n_want
     dt = DTYPES[w.dtype]
     return Inputs(K=K.to(dt).contiguous(), V=V.to(dt).contiguous(), refs=refs.to(dt).contiguous(),
                   Q=Q.to(dt).contiguous(), needle_pos=pos, meta=meta)
