@@ -80,8 +80,9 @@ struct HeadState {  // per (sequence, query head)
   float anchor;            // histogram anchor of the step being built (max e of the step before)
   int steps;               // selects done
   int leaf0;               // leaf block 0 kept (token 0 already attended)
-  int ticket;              // attention partials of the head written so far
-  long long pad[23];
+  int ticket;              // attention chunks of the head merged in group results so far
+  int gticket[32];         // per group of attention CTAs: chunks of the head written so far
+  long long pad[7];
 };
 static_assert(sizeof(HeadState) == 256, "HeadState layout");
 
@@ -1700,63 +1701,124 @@ struct __align__(16) AttSmem {
 };
 
 // ---------------------------------------------------------------- combine
-// The partials of head h (one per attention CTA whose chunk range meets the
-// head's chunks [P0, P1), at slot max(P0, range start)) rescaled to their
-// common max and summed -> O, by one warp of the CTA that wrote the head's
-// last partial; then the head's statistics and kept count, and its ticket
-// reset.  The sums run over the partials in CTA order (deterministic).
-template <typename T, int D>
-__device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& c, int h, long long P0, long long P1,
-                                          long long total_items, int grid) {
+// Partials (m, l, o[D]) are merged by rescaling to their common max:
+// M = max m_j, L = sum e^(m_j - M) l_j, o = sum e^(m_j - M) o_j, in slot order
+// (deterministic).  One warp; lane owns elements q*32 + lane.  cnt <= 32
+// partials, slot_of(j) their slots (-1: none).
+template <int D, class SlotFn>
+__device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotFn slot_of, float& M, float& L,
+                                               float (&acc)[(D + 31) / 32]) {
   const int lane = threadIdx.x & 31;
   constexpr int NQ = (D + 31) / 32;
-  auto range_start = [&](long long cc) { return (cc * total_items) / (long long)grid; };
-  long long cfirst = (P0 * grid) / max64(total_items, 1);
-  while (cfirst > 0 && range_start(cfirst) > P0) --cfirst;
-  while (cfirst + 1 < grid && range_start(cfirst + 1) <= P0) ++cfirst;
-  // slot of CTA cfirst + i, or -1 if that CTA has no chunk of the head
-  auto slot_of = [&](long long cc) -> long long {
-    if (cc >= grid) return -1;
-    const long long cs = max64(P0, range_start(cc));
-    return (cs < P1 && cs < range_start(cc + 1)) ? cs : -1;
-  };
-  float M = -INFINITY;
-  for (long long cc = cfirst + lane; cc < grid && range_start(cc) < P1; cc += 32) {
-    const long long sl = slot_of(cc);
-    if (sl >= 0) M = fmaxf(M, __ldcg(a.attn_part + size_t(sl) * (2 + D)));
-  }
+  const long long sl = lane < cnt ? slot_of(lane) : -1;
+  const float mj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D)) : -INFINITY;
+  const float lj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D) + 1) : 0.f;
+  M = mj;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float L = 0.f, acc[NQ];
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
-  for (long long cb = cfirst; cb < grid && range_start(cb) < P1; cb += 32) {
-    const long long sl = slot_of(cb + lane);
-    float sc = 0.f;
-    if (sl >= 0) {
-      const float mj = __ldcg(a.attn_part + size_t(sl) * (2 + D));
-      sc = mj == -INFINITY ? 0.f : expf(mj - M);
-      L = fmaf(sc, __ldcg(a.attn_part + size_t(sl) * (2 + D) + 1), L);
-    }
-    for (int t0 = 0; t0 < 32; t0 += 8) {  // 8 partials' loads in flight per lane
-      float x[8][NQ], w[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const long long st = __shfl_sync(0xffffffffu, sl, t0 + u);
-        w[u] = __shfl_sync(0xffffffffu, sc, t0 + u);
-#pragma unroll
-        for (int q = 0; q < NQ; ++q)
-          x[u][q] = (st >= 0 && q * 32 + lane < D) ? __ldcg(a.attn_part + size_t(st) * (2 + D) + 2 + q * 32 + lane)
-                                                  : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
-    }
-  }
+  const float sc = (sl >= 0 && mj != -INFINITY) ? expf(mj - M) : 0.f;
+  L = sc * lj;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+  for (int t0 = 0; t0 < cnt; t0 += 8) {  // 8 partials' loads in flight per lane
+    float x[8][NQ], w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long st = __shfl_sync(0xffffffffu, sl, (t0 + u) & 31);
+      w[u] = __shfl_sync(0xffffffffu, sc, (t0 + u) & 31);
+      const bool ok = t0 + u < cnt && st >= 0;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        x[u][q] = (ok && q * 32 + lane < D) ? __ldcg(part + size_t(st) * (2 + D) + 2 + q * 32 + lane) : 0.f;
+      if (!ok) w[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
+  }
+}
+
+// Combine of head h, whose chunks [P0, P1) were spread over attention CTAs in
+// contiguous chunk ranges (CTA cc starts at range_start(cc)).  CTAs form
+// groups of kCombGroup; the warp that writes the last partial of the head in
+// a group merges that group's partials (at most kCombGroup) into the slot of
+// the group's first chunk of the head; the warp that completes the last group
+// merges the group results (at most 32) -> O, the head's statistics and kept
+// count, and resets the head's tickets.  Called by the warp that wrote CTA
+// blockIdx.x's partial of the head, `mine` chunks at slot `seg`.
+constexpr int kCombGroup = 16;
+static_assert(kMaxAttGrid / kCombGroup <= 32, "group results merge in one pass of 32 lanes");
+template <typename T, int D>
+__device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& c, int h, long long P0, long long P1,
+                                          long long seg, long long mine, long long total_items, int grid) {
+  const int lane = threadIdx.x & 31;
+  constexpr int NQ = (D + 31) / 32;
+  HeadState* hs = c.hstate(h);
+  auto range_start = [&](long long cc) { return cc >= grid ? total_items : (cc * total_items) / (long long)grid; };
+  const int g = int(blockIdx.x) / kCombGroup;
+  const long long g0 = max64(P0, range_start((long long)g * kCombGroup));
+  const long long g1 = min64(P1, range_start((long long)(g + 1) * kCombGroup));
+  // level 1: this group's chunks of the head
+  int done = 0;
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) {
+    const int prev = atomicAdd(&hs->gticket[g], int(mine));
+    done = prev + int(mine) == int(g1 - g0) ? 1 : 0;
+  }
+  if (!__shfl_sync(0xffffffffu, done, 0)) return;
+  __threadfence();
+  const bool one_group = g0 == P0 && g1 == P1;
+  float M, L, acc[NQ];
+  {
+    // partials of the group's CTAs: slot max(P0, start) for each CTA whose range meets [g0, g1)
+    const long long cbase = (long long)g * kCombGroup;
+    auto slot_of = [&](int j) -> long long {
+      const long long cc = cbase + j;
+      if (cc >= grid) return -1;
+      const long long cs = max64(g0, range_start(cc));
+      return (cs < g1 && cs < range_start(cc + 1)) ? cs : -1;
+    };
+    merge_partials<D>(a.attn_part, kCombGroup, slot_of, M, L, acc);
+  }
+  if (!one_group) {
+    float* G = a.attn_part + size_t(g0) * (2 + D);  // the group result replaces its first partial
+    if (lane == 0) {
+      G[0] = M;
+      G[1] = L;
+      hs->gticket[g] = 0;
+    }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
+    // level 2: the head's chunks over all groups
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      const int prev = atomicAdd(&hs->ticket, int(g1 - g0));
+      last = prev + int(g1 - g0) == int(P1 - P0) ? 1 : 0;
+    }
+    if (!__shfl_sync(0xffffffffu, last, 0)) return;
+    __threadfence();
+    // groups meeting [P0, P1): the first is the group of the CTA holding chunk P0
+    long long cfirst = (P0 * grid) / max64(total_items, 1);
+    while (cfirst > 0 && range_start(cfirst) > P0) --cfirst;
+    while (cfirst + 1 < grid && range_start(cfirst + 1) <= P0) ++cfirst;
+    const int gfirst = int(cfirst / kCombGroup);
+    const int ngroups = (grid + kCombGroup - 1) / kCombGroup;
+    auto gslot_of = [&](int j) -> long long {
+      const int gg = gfirst + j;
+      if (gg >= ngroups) return -1;
+      const long long s0 = max64(P0, range_start((long long)gg * kCombGroup));
+      const long long s1 = min64(P1, range_start((long long)(gg + 1) * kCombGroup));
+      return s0 < s1 ? s0 : -1;
+    };
+    merge_partials<D>(a.attn_part, min(32, ngroups - gfirst), gslot_of, M, L, acc);
+  }
 #pragma unroll
   for (int q = 0; q < NQ; ++q)
     if (q * 32 + lane < D) a.O[size_t(h) * D + q * 32 + lane] = acc[q] / L;
@@ -1765,7 +1827,6 @@ __device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& 
     const long long tail = a.n_tokens - n1 * b;
     long long nl = 0, scored = 0;
     int l0 = 0, steps = 0;
-    HeadState* hs = c.hstate(h);
     if (a.n_steps > 0 && a.n_roots > 0) {
       nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
       l0 = __ldcg(&hs->leaf0);
@@ -1773,6 +1834,7 @@ __device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& 
       steps = __ldcg(&hs->steps);
     }
     hs->ticket = 0;
+    hs->gticket[g] = 0;
     if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
     if (a.stats) {
       int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
@@ -2098,19 +2160,7 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
 #pragma unroll
     for (int q = 0; q < (D + 31) / 32; ++q)
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
-    // the head's chunks done so far; the warp that completes them combines
-    __threadfence();
-    __syncwarp();
-    int done = 0;
-    if (lane == 0) {
-      const int mine = int(send - seg);
-      const int prev = atomicAdd(&c.hstate(h)->ticket, mine);
-      done = prev + mine == int(sm.pref[h + 1] - sm.pref[h]) ? 1 : 0;
-    }
-    if (__shfl_sync(0xffffffffu, done, 0)) {
-      __threadfence();
-      combine_head<T, D>(a, c, h, sm.pref[h], sm.pref[h + 1], total_items, int(gridDim.x));
-    }
+    combine_head<T, D>(a, c, h, sm.pref[h], sm.pref[h + 1], seg, send - seg, total_items, int(gridDim.x));
   }
 }
 
