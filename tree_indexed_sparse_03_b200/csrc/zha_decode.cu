@@ -19,11 +19,10 @@
 // while the one before drains and waits for it before reading its output);
 // all query heads of all sequences are routed together so that the whole GPU
 // shares the work of the heads whose routing is diffuse.  Per routing step s:
-//   score   (one CTA per SM) the step's units of every head (the roots, or the
-//           kept non-leaves of step s-1) form one list cut into contiguous
-//           per-warp ranges; each warp fetches the node records (the roots,
-//           or the b children of each unit) with bulk copies into a ring of
-//           shared-memory slots, computes the estimates (tensor cores for
+//   score   (one CTA per SM) the step's records of every head (the roots, or
+//           the b children of each kept non-leaf of step s-1) form one list
+//           cut into contiguous per-warp ranges; each warp fetches its node
+//           records with bulk copies into a ring of shared-memory slots, computes the estimates (tensor cores for
 //           bf16) and writes (descending key of e, node code) at the entry's
 //           position in its head's step buffer, adding the entry's
 //           fixed-point mass to the step's histogram anchored at the largest
@@ -1437,7 +1436,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_con
 // ---------------------------------------------------------------- scoring phase
 // Step s's entries: the roots (s = 0, root i at position i) or the children of
 // step s-1's kept non-leaves (unit u of the head: positions u*b .. u*b+b-1).
-// Units of all heads are cut into contiguous ranges, one per warp.  Each
+// The records of all heads are cut into contiguous ranges, one per warp.  Each
 // record is fetched with one bulk copy into the warp's ring; the estimate is
 // added to the step's anchored histogram (s >= 1).
 
@@ -1481,9 +1480,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   bool failed = false;  // a copy never landed: this warp stops scoring
   const long long gwarp = wid < score_warps ? (long long)blockIdx.x * score_warps + wid : -1;
   const long long nwarps = (long long)gridDim.x * score_warps;
-  // ---------------- units = roots (s = 0) or the kept non-leaves of step s-1
+  // ---------------- records = the roots (s = 0) or the b children of each kept
+  // non-leaf of step s-1; the records of all heads are cut into contiguous
+  // per-warp ranges (a small step gives most warps one record or none)
   for (int i = tid; i < nh; i += kDecThreads) {
-    sp.pref[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&c.hstate(i)->units), 0), a.cap_sel);
+    sp.pref[1 + i] = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&c.hstate(i)->units), 0), a.cap_sel) * b;
     sp.anchor[i] = s == 0 ? 0.f : __ldcg(&c.hstate(i)->anchor);
   }
   __syncthreads();
@@ -1494,33 +1495,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   uint32_t cur_kmin = 0xffffffffu;
   int cur_ovf = 0;
   for (long long ub = u0; ub < u1; ub += 32) {
-    // one unit per lane: its head, its first output position, its code
+    // one record per lane: its head, its position in the head's step buffer
+    // (child c of unit u at u*b + c), its node code
     const long long u = ub + lane;
     int uh = 0;
     long long upos = 0;
     uint32_t ucode = 0;
-    bool has = false;  // the unit makes records (a root, or a kept non-leaf)
+    bool has = false;
     if (u < u1) {
       uh = owner_of(sp.pref, nh, u);
       const long long k = u - sp.pref[uh];
+      upos = k;
       if (s == 0) {
         ucode = root_code(a, k);
-        upos = k;
         has = valid_code(a, ucode);
       } else {
-        const uint32_t code = __ldcg(c.units(uh) + k);
-        if (valid_code(a, code) && code_level(code) >= 2) {
-          ucode = code;
-          upos = k * b;
+        const long long unit = k / b;
+        const uint32_t pc = __ldcg(c.units(uh) + unit);
+        if (valid_code(a, pc) && code_level(pc) >= 2) {
+          ucode = node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(k - unit * b));
           has = true;
         }
       }
     }
     const unsigned mhas = __ballot_sync(0xffffffffu, has);
     if (!mhas) continue;
-    const int per = s == 0 ? 1 : b;  // records per unit
-    const int items = __popc(mhas) * per;
-    // item k: record (k % per) of the (k / per)-th unit with records, in lane order
+    constexpr int per = 1;  // records per lane
+    const int items = __popc(mhas);
+    // item k: the record of the k-th lane with one
     struct Cursor {
       unsigned rem;
       int child;
@@ -1534,9 +1536,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
       const int pl = __ffs(cur.rem) - 1;
       Item it;
       it.h = __shfl_sync(0xffffffffu, uh, pl);
-      it.pos = __shfl_sync(0xffffffffu, upos, pl) + cur.child;
-      const uint32_t pc = __shfl_sync(0xffffffffu, ucode, pl);
-      it.code = s == 0 ? pc : node_code(code_level(pc) - 1, code_index(pc) * uint32_t(b) + uint32_t(cur.child));
+      it.pos = __shfl_sync(0xffffffffu, upos, pl);
+      it.code = __shfl_sync(0xffffffffu, ucode, pl);
       if (++cur.child == per) {
         cur.child = 0;
         cur.rem &= cur.rem - 1u;
