@@ -468,8 +468,8 @@ def run_zha(args, world, rank, local):
         "route_bytes": int(statistics.mean(route_b)),
         "attend_bytes": int(statistics.mean(attend_b)),
         "roofline": {"bound": "hbm",
-                     "kernel": "zha_decode call: per routing step a scoring and a select kernel, then finalize, "
-                               "attention and combine kernels",
+                     "kernel": "zha_decode call: per routing step a scoring and a select kernel, then one "
+                               "attention kernel",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_8tbs": round(achieved / 8000.0, 4), "traffic": measured_traffic(w.name),
