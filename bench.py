@@ -9,6 +9,7 @@ queries, p=0.95, batch 1), synthetic and seeded.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zha|reference] [--workload NAME]
   python bench.py --profile [--workload NAME] [--n N] [--warmup W] [--steps K]   (untimed decodes, for ncu)
+  python bench.py --sweep [N,N,...] [--steps K] [--warmup W]   (light sweep 32K..4M: ZHA vs dense, crossover)
 
 One JSON line on stdout (rank 0).  Timing: CUDA events on the launching
 stream around every step (and around the decode call alone), the L2 flushed
@@ -57,6 +58,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="build the workload's tree, run --warmup + --steps decodes untimed, exit (for ncu)")
+    ap.add_argument("--sweep", nargs="?", const="32768,65536,131072,262144,524288,1048576,2097152,4194304",
+                    default=None, help="run the light sweep workload at these context lengths (one process each) "
+                                       "and print one line per N plus the measured dense/ZHA crossover")
     return ap.parse_args()
 
 
@@ -307,7 +311,8 @@ def run_zha(args, world, rank, local):
 
     w = load_workload(args)
     dev = torch.device("cuda", local if world > 1 else 0)
-    n0 = w.n_tokens
+    n_build = w.n_tokens
+    n0 = n_build + w.append  # context after the workload's own block append (if any)
     total_steps = args.warmup + args.steps + args.e2e_steps + 2
     t_gen = time.perf_counter()
     inp = generate(w, n_total=n0 + total_steps)
@@ -318,8 +323,8 @@ def run_zha(args, world, rank, local):
     dt = inp.K.dtype
     K = torch.zeros(w.n_kv_heads, cap, w.d, dtype=dt, device=dev)
     V = torch.zeros_like(K)
-    K[:, :n0] = inp.K[:, :n0].to(dev)
-    V[:, :n0] = inp.V[:, :n0].to(dev)
+    K[:, :n_build] = inp.K[:, :n_build].to(dev)
+    V[:, :n_build] = inp.V[:, :n_build].to(dev)
     # per-step new tokens, each [Hkv, 1, d] contiguous
     Kn = inp.K[:, n0:].permute(1, 0, 2).contiguous().unsqueeze(2).to(dev)
     Vn = inp.V[:, n0:].permute(1, 0, 2).contiguous().unsqueeze(2).to(dev)
@@ -331,11 +336,22 @@ def run_zha(args, world, rank, local):
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    tree.build(n0)
+    tree.build(n_build)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     tree.status()
     build_ms = e0.elapsed_time(e1)
+    append_block = None
+    if w.append > 0:  # the workload's block append, timed once (new rows and newly complete nodes)
+        Ka = inp.K[:, n_build:n0].contiguous().to(dev)
+        Va = inp.V[:, n_build:n0].contiguous().to(dev)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        tree.append(Ka, Va)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tree.status()
+        append_block = {"tokens": w.append, "us": round(e0.elapsed_time(e1) * 1000, 3)}
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
@@ -451,7 +467,7 @@ def run_zha(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": w.name, "n_tokens": n0, "block": w.block, "levels": w.levels, "n_refs": w.n_refs,
                    "p": w.p, "batch": w.batch, "gqa": f"{w.n_q_heads}/{w.n_kv_heads}", "d": w.d,
-                   "step": "append 1 token + route + attend", "l2": "flushed before every step",
+                   "built": n_build, "step": "append 1 token + route + attend", "l2": "flushed before every step",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "queries": f"{w.n_query_sets} seeded query sets, rotated"},
         "median_us": round(statistics.median(step_ms) * 1000, 3),
@@ -463,6 +479,7 @@ def run_zha(args, world, rank, local):
         "speedup_vs_dense": round(statistics.mean(dense_ms) / step_ms_mean, 3) if dense_ms else None,
         "dense_gbs": round(dense_bytes / (statistics.mean(dense_ms) * 1e-3) / 1e9, 1) if dense_ms else None,
         "build_ms": round(build_ms, 3),
+        "append_block": append_block,
         "keys_per_head": round(statistics.mean(keys_ph), 1),
         "keys_frac": round(statistics.mean(keys_ph) / n_final, 6),
         "route_bytes": int(statistics.mean(route_b)),
@@ -488,8 +505,42 @@ def run_zha(args, world, rank, local):
     del tree
 
 
+def run_sweep(args):
+    """The light sweep: one bench process per context length, then the dense/ZHA crossover."""
+    lines = []
+    for n in [int(x) for x in args.sweep.split(",") if x]:
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", "sweep_bf16", "--n", str(n),
+               "--steps", str(args.steps), "--warmup", str(args.warmup), "--e2e-steps", "0",
+               "--dense-steps", str(max(args.dense_steps, 5)), "--no-cpu-baseline"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            log(r.stderr[-2000:])
+            raise SystemExit(f"sweep point N={n} failed")
+        line = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+        lines.append(line)
+        print(json.dumps({"sweep_point": n, "decode_us": line["decode_us"], "dense_us": line["dense_us"],
+                          "speedup_vs_dense": round(line["dense_us"] / line["decode_us"], 3),
+                          "keys_per_head": line["keys_per_head"], "roofline_frac": line["roofline"]["frac"],
+                          "levels": line["config"]["levels"], "clocks": line["clocks"]}), flush=True)
+    # crossover: the first N from which the routed decode call is faster than the dense decode,
+    # interpolated linearly in log N between the two bracketing points
+    cross = None
+    for a, b in zip(lines, lines[1:]):
+        da, db = a["dense_us"] - a["decode_us"], b["dense_us"] - b["decode_us"]
+        if da < 0 <= db:
+            na, nb = math.log(a["config"]["n_tokens"]), math.log(b["config"]["n_tokens"])
+            cross = int(round(math.exp(na + (nb - na) * (-da) / (db - da))))
+    if lines and cross is None and lines[0]["dense_us"] >= lines[0]["decode_us"]:
+        cross = f"<= {lines[0]['config']['n_tokens']}"
+    print(json.dumps({"sweep": "light sweep bf16 (GQA 32/4, d=128, b=8, R=1, p=0.75, batch 1)",
+                      "crossover_n": cross, "unit": "us per decode call"}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
