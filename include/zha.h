@@ -212,6 +212,25 @@ ZHA_API int zha_dense_decode(const zha_config* cfg, const void* K, const void* V
 ZHA_API int zha_dense_decode_noalloc(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n,
                              const void* Q, float* O, int32_t B, void* stream);
 
+/*
+ * zha_tree_set_step_p: top-p thresholds per routing step, for routing whose
+ * threshold changes with the depth in the tree and with the context length
+ * ("Zyphra Hierarchical Attention", closing section on matching the degree of
+ * compression to the predictive information in the data: a fixed top-p at
+ * every level is not enough, the threshold has to evolve with tree depth and
+ * context length; the "ZHA 階層注意力研究" review, section on thresholds that
+ * follow depth and content).  The pages give no schedule, so the caller
+ * chooses one.
+ *   p - host array of n thresholds, p[s] for routing step s (s = 0 scores the
+ *       roots, step s the children of step s-1's kept nodes); steps past n-1
+ *       use p[n-1].  Each value in (0, 1]; 1 keeps every candidate of the step.
+ *   n - 0 .. 20; n = 0 returns to the configuration's single p.
+ * Applies to the decode calls issued after it; copied (the array may be
+ * freed).  ZHA_ERR_INVALID for a NULL tree, n out of range, a NULL p with
+ * n > 0, or a value outside (0, 1].
+ */
+ZHA_API int zha_tree_set_step_p(zha_tree* tree, const float* p, int32_t n);
+
 /* Synchronise `stream` and return the tree's device status word (ZHA_OK or a
  * ZHA_ERR_* code raised inside a kernel); clears it. */
 ZHA_API int zha_tree_status(zha_tree* tree, void* stream);

@@ -190,6 +190,7 @@ class RouteStep:
     order: np.ndarray         # candidate indices in (ehat desc, start asc) order
     cum: np.ndarray           # cumulative softmax mass along ``order``
     k: int                    # number kept (a prefix of ``order``)
+    p: float = 1.0            # the step's threshold
 
 
 @dataclass
@@ -218,7 +219,22 @@ def top_p_count(ehat: np.ndarray, order: np.ndarray, p: float) -> Tuple[int, np.
     return k, cum
 
 
-def route(planes: PlanesFn, q: np.ndarray, p: float, n_tokens: int, block: int,
+def step_threshold(p, s: int) -> float:
+    """Threshold of routing step s (s = 0 scores the roots).
+
+    ``p`` is one value for every step, or a sequence with one value per step
+    (later steps take the last one): the blog's closing section ("matching the
+    degree of compression to the predictive information") and the review's
+    section on thresholds that follow depth and content say a fixed top-p at
+    every level is not enough and the threshold should change with tree depth
+    and context length; they give no schedule, so the schedule is an input.
+    """
+    if np.ndim(p) == 0:
+        return float(p)
+    return float(p[min(s, len(p) - 1)])
+
+
+def route(planes: PlanesFn, q: np.ndarray, p, n_tokens: int, block: int,
           levels: int) -> RouteTrace:
     """Top-down top-p routing of one query head ([blog] "Routing in the tree").
 
@@ -226,11 +242,13 @@ def route(planes: PlanesFn, q: np.ndarray, p: float, n_tokens: int, block: int,
     requested nodes - the oracle's own tree or planes read back from the GPU.
     Start: the forest roots.  Each step softmaxes the candidate estimates,
     keeps the smallest prefix (ehat descending, lower start token first on
-    ties) reaching mass p; kept level-1 nodes are final, kept higher nodes
-    contribute their ``block`` children to the next candidate set.
+    ties) reaching mass p (``step_threshold(p, s)`` at step s); kept level-1
+    nodes are final, kept higher nodes contribute their ``block`` children to
+    the next candidate set.
     """
     trace = RouteTrace()
     cand = forest_roots(n_tokens, block, levels)
+    s = 0
     while cand:
         ehat = np.empty(len(cand))
         lv = np.array([c[0] for c in cand])
@@ -241,8 +259,10 @@ def route(planes: PlanesFn, q: np.ndarray, p: float, n_tokens: int, block: int,
             ehat[sel] = estimate(mu, bias, q)
         start = ix * np.array([block ** int(v) for v in lv])
         order = np.lexsort((start, -ehat))        # primary: ehat desc; secondary: start asc
-        k, cum = top_p_count(ehat, order, p)
-        trace.steps.append(RouteStep(cand, ehat, order, cum, k))
+        ps = step_threshold(p, s)
+        k, cum = top_p_count(ehat, order, ps)
+        trace.steps.append(RouteStep(cand, ehat, order, cum, k, ps))
+        s += 1
         nxt: List[Node] = []
         for j in order[:k]:
             node = cand[j]
@@ -287,7 +307,7 @@ def dense(K: np.ndarray, V: np.ndarray, q: np.ndarray, n_tokens: int) -> np.ndar
     return attend(K, V, q, np.arange(n_tokens))
 
 
-def decode_head(K: np.ndarray, V: np.ndarray, planes: PlanesFn, q: np.ndarray, p: float,
+def decode_head(K: np.ndarray, V: np.ndarray, planes: PlanesFn, q: np.ndarray, p,
                 n_tokens: int, block: int, levels: int) -> Tuple[np.ndarray, RouteTrace]:
     """Route + attend for one query head of one sequence."""
     trace = route(planes, q, p, n_tokens, block, levels)

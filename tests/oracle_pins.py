@@ -232,6 +232,34 @@ def pin_minimal_prefix(zo):
             assert sorted(step.order[: step.k].tolist()) == sorted(want)
 
 
+def pin_step_thresholds(zo):
+    """Per-step thresholds: a constant schedule equals the single p; every step keeps a minimum-cardinality
+    set reaching its own threshold (brute force); a threshold of 1 at a step keeps all of that step."""
+    rng = _rng(21)
+    d = 8
+    for trial in range(10):
+        b = int(rng.integers(2, 5))
+        L = int(rng.integers(2, 4))
+        n = int(rng.integers(b ** 2, min(b ** (L + 1) * 2, 60)))
+        K = rng.normal(size=(n, d)) * 2
+        refs = rng.normal(size=(2, d))
+        tree = zo.build_tree(K, refs, n, b, L)
+        pf = zo.tree_planes_fn(tree)
+        q = rng.normal(size=d) * 2
+        p = float(rng.choice([0.4, 0.8, 0.95]))
+        assert zo.route(pf, q, [p] * L, n, b, L).leaves == zo.route(pf, q, p, n, b, L).leaves
+        sched = [float(x) for x in rng.choice([0.3, 0.6, 0.9, 1.0], size=int(rng.integers(1, L + 1)))]
+        trace = zo.route(pf, q, sched, n, b, L)
+        for s, step in enumerate(trace.steps):
+            ps = sched[min(s, len(sched) - 1)]
+            assert step.p == ps
+            if ps >= 1:
+                assert step.k == len(step.cand)
+            if len(step.cand) <= 14:
+                start = np.array([zo.node_span(c, b)[0] for c in step.cand])
+                assert step.k == _brute_top_p(step.ehat, start, ps), (trial, s, step.k)
+
+
 def pin_cut_reaches_p_exactly(zo):
     """Four equal estimates at p = 0.5: mass 0.25 + 0.25 reaches p, so exactly two are kept."""
     e = np.zeros(4)

@@ -30,9 +30,11 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def p32(p: float) -> float:
-    """The threshold as the library sees it (a C float)."""
-    return float(np.float32(p))
+def p32(p):
+    """The threshold (or per-step thresholds) as the library sees it (C floats)."""
+    if np.ndim(p) == 0:
+        return float(np.float32(p))
+    return [float(np.float32(x)) for x in p]
 
 
 # --------------------------------------------------------------------------- build
@@ -79,12 +81,13 @@ def ehat_error_bound(mu: np.ndarray, bias: np.ndarray, q: np.ndarray) -> np.ndar
     return (d + 8) * U32 * mag.max(axis=1) + 1e-7
 
 
-def trace_flags(trace: zo.RouteTrace, planes, q: np.ndarray, p: float, block: int) -> List[str]:
+def trace_flags(trace: zo.RouteTrace, planes, q: np.ndarray, p, block: int) -> List[str]:
     """Boundary / near-tie cases along the oracle's path (the places where fp32 and fp64 may differ)."""
     flags = []
-    if p >= 1:
-        return flags
     for s, st in enumerate(trace.steps):
+        p = st.p
+        if p >= 1:
+            continue
         n = len(st.cand)
         lv = np.array([c[0] for c in st.cand])
         ix = np.array([c[1] for c in st.cand])
@@ -119,7 +122,7 @@ def gpu_planes_fn(tree, kv_head: int, levels: int):
     return fn
 
 
-def compare_route(tree, Q: torch.Tensor, kept: torch.Tensor, cnt: torch.Tensor, p: float, n_tokens: int,
+def compare_route(tree, Q: torch.Tensor, kept: torch.Tensor, cnt: torch.Tensor, p, n_tokens: int,
                   block: int, levels: int, group: int, heads=None) -> RouteReport:
     """Oracle routing on the GPU planes vs the GPU kept sets, for every (sequence, head)."""
     rep = RouteReport()

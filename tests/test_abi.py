@@ -114,6 +114,7 @@ def test_null_arguments_fail_before_any_device_work(built):
     assert L.zha_decode(None, None, None, 1, None, None, None, None, 0, None) == zb.ZHA_ERR_INVALID
     assert L.zha_launch_count() == 0
     assert L.zha_tree_status(None, None) == zb.ZHA_ERR_INVALID
+    assert L.zha_tree_set_step_p(None, None, 0) == zb.ZHA_ERR_INVALID
     assert L.zha_tree_size(None) == -1
     assert L.zha_dense_decode(ctypes.byref(c), None, None, 1, 1, None, None, 1, None, None) == zb.ZHA_ERR_INVALID
     L.zha_tree_destroy(None)

@@ -242,6 +242,30 @@ def test_many_candidates_in_cut_bin():
     check_decode(case, Q)
 
 
+def test_step_thresholds():
+    """Per-step top-p thresholds (zha_tree_set_step_p) against the oracle's route with the same schedule."""
+    w = small_topics(20011, d=128, n_q_heads=8, n_kv_heads=1, block=4, levels=4, n_refs=8, p=0.95, batch=2)
+    inp = generate(w)
+    case = Case(inp.K, inp.V, inp.refs, block=4, levels=4, p=0.95, n=20011, group=8)
+    Q = inp.Q[1]
+    O_cfg = case.decode(Q)[0]
+    for sched in ([0.99, 0.9, 0.8, 0.7], [1.0, 0.5], [0.6]):
+        case.tree.set_step_p(sched)
+        case.p = sched
+        rep, *_ = check_decode(case, Q)
+        print(f"schedule {sched}: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+    # a constant schedule is the configuration's p; an empty one restores it
+    case.tree.set_step_p([0.95])
+    assert torch.equal(case.decode(Q)[0], O_cfg)
+    case.tree.set_step_p(None)
+    case.p = 0.95
+    assert torch.equal(case.decode(Q)[0], O_cfg)
+    with pytest.raises(z.ZhaError):
+        case.tree.set_step_p([0.5, 1.5])
+    with pytest.raises(z.ZhaError):
+        case.tree.set_step_p([0.0])
+
+
 def test_append_then_decode():
     w = small_topics(6000, d=128, n_q_heads=8, n_kv_heads=1, block=4, levels=3, n_refs=4, p=0.9, batch=1)
     inp = generate(w, n_total=6000)

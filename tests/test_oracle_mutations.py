@@ -127,9 +127,14 @@ def _attend_no_scale(K, V, q, tokens):
     return (w / w.sum()) @ V[tokens]
 
 
+def _step_threshold_first(p, s):
+    return float(p) if np.ndim(p) == 0 else float(p[0])
+
+
 def _route_ties_high(planes, q, p, n_tokens, block, levels):
     trace = zo.RouteTrace()
     cand = zo.forest_roots(n_tokens, block, levels)
+    s = 0
     while cand:
         lv = np.array([c[0] for c in cand])
         ix = np.array([c[1] for c in cand])
@@ -140,8 +145,10 @@ def _route_ties_high(planes, q, p, n_tokens, block, levels):
             ehat[sel] = zo.estimate(mu, bias, q)
         start = ix * np.array([block ** int(v) for v in lv])
         order = np.lexsort((-start, -ehat))            # higher start first on ties
-        k, cum = zo.top_p_count(ehat, order, p)
-        trace.steps.append(zo.RouteStep(cand, ehat, order, cum, k))
+        ps = zo.step_threshold(p, s)
+        k, cum = zo.top_p_count(ehat, order, ps)
+        trace.steps.append(zo.RouteStep(cand, ehat, order, cum, k, ps))
+        s += 1
         nxt = []
         for j in order[:k]:
             node = cand[j]
@@ -173,6 +180,7 @@ MUTATIONS = {
     "tail forgotten": ("attended_tokens", _attended_no_tail),
     "attention without 1/sqrt(d)": ("attend", _attend_no_scale),
     "ties to the higher start": ("route", _route_ties_high),
+    "step thresholds ignored after the first": ("step_threshold", _step_threshold_first),
 }
 
 

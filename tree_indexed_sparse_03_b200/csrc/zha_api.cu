@@ -164,6 +164,8 @@ struct zha_tree {
   int device;
   long long spin_limit;  // bound of the decode's waits on record copies
   bool flow_dirty;               // the routing flow state must be zeroed before the next decode
+  float step_p[kMaxLevels];      // per-step thresholds (n_step_p of them; 0: the configuration's p)
+  int n_step_p;
 };
 
 extern "C" {
@@ -214,6 +216,7 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
   t->n = 0;
   t->spin_limit = kDefaultSpinLimit;
   t->flow_dirty = true;
+  t->n_step_p = 0;
   if (const char* v = std::getenv("ZHA_SPIN_LIMIT")) {  // test hook: 0 makes every wait give up at once
     const long long x = std::atoll(v);
     if (x >= 0 && (x > 0 || v[0] == '0')) t->spin_limit = x;
@@ -315,14 +318,16 @@ static int fill_decode_args(const zha_tree* t, const void* Q, float* O, int32_t*
   a->scored = scored;
   a->scored_cap = scored ? scored_cap : 0;
   a->kept_stride = t->L.cap_nodes[1];
-  const float p = t->cfg.p;
-  if (p >= 1.f) {
-    a->p_all = 1;
-  } else {
-    int ex = 0;
-    const float fr = std::frexp(p, &ex);           // p = fr * 2^ex, fr in [0.5, 1)
-    a->p_mant = uint32_t(std::ldexp(fr, 24));      // exact: fr has 24 significant bits
-    a->p_shift = 24 - ex;
+  for (int s = 0; s < kMaxLevels; ++s) {
+    const float p = t->n_step_p > 0 ? t->step_p[s < t->n_step_p ? s : t->n_step_p - 1] : t->cfg.p;
+    if (p >= 1.f) {
+      a->p_all[s] = 1;
+    } else {
+      int ex = 0;
+      const float fr = std::frexp(p, &ex);           // p = fr * 2^ex, fr in [0.5, 1)
+      a->p_mant[s] = uint32_t(std::ldexp(fr, 24));   // exact: fr has 24 significant bits
+      a->p_shift[s] = 24 - ex;
+    }
   }
   return ZHA_OK;
 }
@@ -464,6 +469,17 @@ int zha_dense_decode_noalloc(const zha_config* cfg, const void* K, const void* V
   a.inv_sqrt_d = 1.0f / std::sqrt(float(cfg->d));
   e = launch_dense(a, cfg->dtype, cfg->d, B, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "zha_dense_decode_noalloc");
+  return ZHA_OK;
+}
+
+int zha_tree_set_step_p(zha_tree* t, const float* p, int32_t n) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (n < 0 || n > kMaxLevels) return fail(ZHA_ERR_INVALID, "n must be in 0..20");
+  if (n > 0 && !p) return fail(ZHA_ERR_INVALID, "p is NULL");
+  for (int i = 0; i < n; ++i)
+    if (!(p[i] > 0.f) || !(p[i] <= 1.f)) return fail(ZHA_ERR_INVALID, "every threshold must be in (0, 1]");
+  for (int i = 0; i < n; ++i) t->step_p[i] = p[i];
+  t->n_step_p = n;
   return ZHA_OK;
 }
 

@@ -27,9 +27,11 @@ struct DecodeArgs {
   int32_t* scored;
   int64_t scored_cap;
   int64_t kept_stride;
-  uint32_t p_mant;              // p = p_mant * 2^-p_shift  (p < 1)
-  int p_shift;
-  int p_all;                    // p >= 1: keep every candidate
+  // top-p threshold of routing step s (s = 0: the roots): p = p_mant[s] * 2^-p_shift[s] (p < 1);
+  // p_all[s]: p >= 1, keep every candidate of the step
+  uint32_t p_mant[kMaxLevels];
+  int p_shift[kMaxLevels];
+  int p_all[kMaxLevels];
 };
 
 struct DenseArgs {

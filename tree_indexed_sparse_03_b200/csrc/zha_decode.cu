@@ -388,7 +388,7 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 // the cut is the first entry whose running mass reaches T.
 template <class View>
 __device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
-                                                            DecSmem& sm) {
+                                                            DecSmem& sm, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
   unsigned long long* ks = sm.hist;                // [np] order keys
   unsigned long long* ws = sm.hist + kDecThreads;  // [np] masses
@@ -428,7 +428,7 @@ __device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a,
   (void)lane;
   unsigned long long Z;
   const unsigned long long before = block_scan_u64(tid < np ? w : 0ull, sm.red64, &Z);
-  const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);
+  const unsigned long long T = ceil_p_times(Z, a.p_mant[step], a.p_shift[step]);
   // sorted position of the cut: the first with before + w >= T (else the last entry)
   if (tid == 0) sm.bcast64[1] = ~0ull;
   __syncthreads();
@@ -464,9 +464,9 @@ template <class View>
 __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const View& E, int64_t n, uint32_t kmin,
                                          DecSmem& sm, int h, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
-  if (a.p_all) return ~0ull;
+  if (a.p_all[step]) return ~0ull;
   const float m = desc_key_value(kmin);
-  if (n <= kDecThreads) return select_cut_small(a, E, n, m, sm);
+  if (n <= kDecThreads) return select_cut_small(a, E, n, m, sm, step);
 
   // coarse histogram of the masses (and counts); total mass Z and the target T = ceil(p Z)
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
@@ -501,7 +501,7 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
     for (int k = 0; k < BPT; ++k) local += sm.hist[tid * BPT + k];
     block_scan_u64(local, sm.red64, &Z);
   }
-  const unsigned long long T = ceil_p_times(Z, a.p_mant, a.p_shift);  // keep while mass before < T
+  const unsigned long long T = ceil_p_times(Z, a.p_mant[step], a.p_shift[step]);  // keep while mass before < T
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
@@ -778,7 +778,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   constexpr int BPT = kBins / kDecThreads;
   double* red = reinterpret_cast<double*>(sm.red64);
-  const double p = ldexp(double(a.p_mant), -a.p_shift);
+  const double p = ldexp(double(a.p_mant[step]), -a.p_shift[step]);
   double mb[BPT], loc = 0.0;
 #pragma unroll
   for (int k = 0; k < BPT; ++k) {
@@ -1276,8 +1276,8 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c
   }
   const float m = desc_key_value(kmin);
   unsigned long long cut = ~0ull;
-  if (!a.p_all && n > 0) {
-    if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm);
+  if (!a.p_all[s] && n > 0) {
+    if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm, s);
     else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
       cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
     else cut = select_cut(a, E, n, kmin, sm, h, s);

@@ -44,6 +44,7 @@ _SIGS = {
     "zha_dense_decode_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64,
                                             _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p]),
     "zha_tree_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
+    "zha_tree_set_step_p": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int32]),
     "zha_tree_destroy": (None, [_c.c_void_p]),
     "zha_last_error": (_c.c_char_p, []),
     "zha_launch_count": (_c.c_uint64, []),
@@ -198,6 +199,13 @@ class ZhaTree:
         B = q_host.shape[0]
         _check(lib().zha_decode_step_host(self._h, _ptr(k_host), _ptr(v_host), q_host.data_ptr(), o_host.data_ptr(),
                                           B, _stream(stream)))
+
+    def set_step_p(self, p) -> None:
+        """Top-p threshold per routing step (p[s] for step s, the last value for later steps); [] or None
+        returns to the configuration's p."""
+        vals = [] if p is None else [float(x) for x in p]
+        arr = (_c.c_float * max(len(vals), 1))(*vals)
+        _check(lib().zha_tree_set_step_p(self._h, _c.cast(arr, _c.c_void_p) if vals else None, len(vals)))
 
     def status(self, stream=None) -> None:
         _check(lib().zha_tree_status(self._h, _stream(stream)))
