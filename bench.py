@@ -205,7 +205,8 @@ def load_workload(args):
 def union_bytes(w, scored: np.ndarray, nscored: np.ndarray, kept: np.ndarray, kcnt: np.ndarray, n_tokens: int):
     """Algorithmic bytes of one decode call: union over each GQA group of the planes scored and keys attended."""
     es = 2 if w.dtype == "bf16" else 4
-    plane = w.n_refs * (w.d * es + 4)            # mu and intercepts; f is not read by routing
+    # mu and intercepts of a node (f is not read by routing); FP4 router planes: codes, scales, intercepts
+    plane = w.n_refs * (w.d // 2 + w.d // 16 + 4) if w.planes == "fp4" else w.n_refs * (w.d * es + 4)
     kv = 2 * w.d * es
     n1 = n_tokens // w.block
     tail = n_tokens - n1 * w.block
@@ -292,7 +293,8 @@ def run_profile(args):
     inp = generate(w)
     n = w.n_tokens
     cfg = z.make_config(d=w.d, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, block=w.block, levels=w.levels,
-                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=n, max_batch=w.batch)
+                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=n, max_batch=w.batch,
+                        planes=w.planes)
     tree = z.ZhaTree(cfg, inp.K.to(dev), inp.V.to(dev), inp.refs.to(dev))
     tree.build(n)
     Qs = inp.Q.to(dev)
@@ -319,7 +321,8 @@ def run_zha(args, world, rank, local):
     log(f"[bench] generated {w.name} in {time.perf_counter() - t_gen:.1f}s")
     cap = n0 + total_steps
     cfg = z.make_config(d=w.d, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, block=w.block, levels=w.levels,
-                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=cap, max_batch=w.batch)
+                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=cap, max_batch=w.batch,
+                        planes=w.planes)
     dt = inp.K.dtype
     K = torch.zeros(w.n_kv_heads, cap, w.d, dtype=dt, device=dev)
     V = torch.zeros_like(K)
@@ -467,7 +470,7 @@ def run_zha(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": w.name, "n_tokens": n0, "block": w.block, "levels": w.levels, "n_refs": w.n_refs,
                    "p": w.p, "batch": w.batch, "gqa": f"{w.n_q_heads}/{w.n_kv_heads}", "d": w.d,
-                   "built": n_build, "step": "append 1 token + route + attend", "l2": "flushed before every step",
+                   "router_planes": w.planes, "built": n_build, "step": "append 1 token + route + attend", "l2": "flushed before every step",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "queries": f"{w.n_query_sets} seeded query sets, rotated"},
         "median_us": round(statistics.median(step_ms) * 1000, 3),

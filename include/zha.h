@@ -63,6 +63,22 @@ enum {
 
 enum { ZHA_F32 = 0, ZHA_BF16 = 1 };
 
+/* Router planes: the slopes the routing steps read.  ZHA_PLANES_KEY reads the
+ * stored nodes (mu in the element type).  ZHA_PLANES_FP4 keeps, beside them,
+ * a copy of every node's slopes in 4-bit e2m1 with one e4m3 scale per 16
+ * dimensions (an FP4 router; the pages report that one was tried, without
+ * details), which the routing steps read instead: a record is
+ * R*(d/2 + d/16 + 4) bytes (1216 at R = 16, d = 128) instead of
+ * R*(d*es + 4).  Quantisation of a group of 16 stored slopes v (converted
+ * exactly to fp32): amax = max |v|; scale = e4m3(amax / 6) (the division in
+ * fp32, then round to nearest, ties to even, at most 448; 0 when amax is 0);
+ * code of v = e2m1(v / scale) (fp32 division, nearest value of
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6} with the sign, ties to the even mantissa,
+ * at most 6; 0 when the scale is 0).  The slope the router uses is
+ * code * scale (exact in fp16).  Intercepts stay fp32 and unchanged.
+ * bf16 configurations only (ZHA_ERR_UNSUPPORTED otherwise). */
+enum { ZHA_PLANES_KEY = 0, ZHA_PLANES_FP4 = 1 };
+
 /* Geometry and limits of one layer's tree.  Passed by pointer, read only. */
 typedef struct {
   int32_t d;           /* head dimension: 64 or 128 */
@@ -75,6 +91,7 @@ typedef struct {
   int32_t dtype;       /* ZHA_F32 or ZHA_BF16 */
   int64_t capacity;    /* maximum number of cached tokens per KV head */
   int32_t max_batch;   /* maximum decode batch B per zha_decode call */
+  int32_t planes;      /* ZHA_PLANES_KEY (0) or ZHA_PLANES_FP4 */
 } zha_config;
 
 typedef struct zha_tree zha_tree; /* opaque host handle */
@@ -110,6 +127,16 @@ ZHA_API int zha_tree_bytes(const zha_config* cfg, size_t* node_bytes, size_t* sc
  */
 ZHA_API int zha_tree_layout(const zha_config* cfg, int32_t level, size_t* rec_offset, size_t* f_offset,
                     int64_t* cap_nodes, size_t* rec_bytes);
+
+/*
+ * zha_tree_layout_fp4: where the FP4 router records of level `level` live
+ * inside node_buf (configurations with planes = ZHA_PLANES_FP4; else
+ * ZHA_ERR_INVALID).  Records [Hkv][cap_nodes] of rec_bytes each: codes
+ * [R][d/2] bytes (dimension 2i in the low nibble, 2i+1 in the high one; e2m1
+ * bits s|e1 e0|m), then scales [R][d/16] e4m3 bytes, then bias[R] fp32, zero
+ * padded to a multiple of 16 bytes.  Host only.
+ */
+ZHA_API int zha_tree_layout_fp4(const zha_config* cfg, int32_t level, size_t* rec_offset, size_t* rec_bytes);
 
 /*
  * zha_tree_create: bind caller-owned buffers into a tree handle (host only).

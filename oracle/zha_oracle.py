@@ -180,6 +180,87 @@ def log_mass(K: np.ndarray, node: Node, q: np.ndarray, block: int) -> float:
     return float(m + np.log(np.exp(z - m).sum()))
 
 
+# --------------------------------------------------------------------------- FP4 router planes
+# [blog] "How does this give subquadratic scaling?" / the review pages mention that an FP4 router was
+# also tried, without details.  Reading: the router reads each slope row as 4-bit e2m1 codes with one
+# e4m3 scale per 16 dimensions (the OCP microscaling element and scale formats), quantised from the
+# stored slopes by round-to-nearest; the intercepts stay fp32.  The decisions (scale, codes) are taken in
+# fp32 arithmetic, as the stored slopes are fp32-representable; the values are then exact.
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e4m3_nearest(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Nearest e4m3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448) of
+    each x >= 0, ties to the even mantissa, at most 448: (values, encodings)."""
+    x = np.asarray(x, dtype=np.float64)
+    vals = np.zeros_like(x)
+    bits = np.zeros(x.shape, dtype=np.uint8)
+    for i in np.ndindex(x.shape):
+        v = float(x[i])
+        if not v > 0:
+            continue
+        if v >= 448.0:
+            vals[i], bits[i] = 448.0, 0x7E
+            continue
+        E = math.frexp(v)[1] - 1                  # v in [2^E, 2^(E+1))
+        if E < -6:                                # subnormals: multiples of 2^-9
+            m = float(np.rint(v * 2.0 ** 9))
+            vals[i], bits[i] = m * 2.0 ** -9, int(m)
+            continue
+        m = float(np.rint(v * 2.0 ** (3 - E)))   # in [8, 16]
+        if m == 16.0:
+            m, E = 8.0, E + 1
+        val = m * 2.0 ** (E - 3)
+        if val > 448.0:
+            vals[i], bits[i] = 448.0, 0x7E
+        else:
+            vals[i], bits[i] = val, ((E + 7) << 3) | (int(m) - 8)
+    return vals, bits
+
+
+def e4m3_decode(bits: np.ndarray) -> np.ndarray:
+    """Values of e4m3 encodings (finite ones)."""
+    b = np.asarray(bits).astype(np.int64)
+    e, m = (b >> 3) & 15, (b & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    return np.where((b & 128) != 0, -mag, mag)
+
+
+def e2m1_code(y: np.ndarray) -> np.ndarray:
+    """e2m1 code (bit 3 the sign, bits 0-2 the index into E2M1_VALUES) of the nearest representable value
+    of each y, ties to the even mantissa, magnitude at most 6; magnitude 0 is coded +0."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    # index i has mantissa bit i & 1 (i >= 1): a tie between i and i+1 goes to the even one
+    idx = np.zeros(a.shape, dtype=np.uint8)
+    for i in range(1, 8):
+        lo, hi = E2M1_VALUES[i - 1], E2M1_VALUES[i]
+        mid = (lo + hi) / 2
+        up = (a > mid) | ((a == mid) & (i % 2 == 0))   # above the midpoint, or at it with i even
+        idx = np.where(up, np.uint8(i), idx)
+    return np.where(idx == 0, 0, idx | np.where(y < 0, 8, 0)).astype(np.uint8)
+
+
+def quantize_fp4(mu: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Codes [..., d] and scale encodings [..., d/16] of slope rows mu [..., d] (fp32-representable)."""
+    m32 = np.asarray(mu, dtype=np.float32)
+    g = m32.reshape(*m32.shape[:-1], m32.shape[-1] // 16, 16)
+    amax = np.abs(g).max(axis=-1)
+    sval, sbits = e4m3_nearest((amax / np.float32(6)).astype(np.float32))   # fp32 division
+    s32 = sval.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = (g / s32[..., None]).astype(np.float32)                            # fp32 division
+    codes = np.where(s32[..., None] > 0, e2m1_code(y), 0).astype(np.uint8)
+    return codes.reshape(m32.shape), sbits
+
+
+def dequantize_fp4(codes: np.ndarray, sbits: np.ndarray) -> np.ndarray:
+    """Slopes code * scale (exact) from codes [..., d] and scale encodings [..., d/16]."""
+    c = np.asarray(codes).astype(np.int64)
+    v = E2M1_VALUES[c & 7] * np.where((c & 8) != 0, -1.0, 1.0)
+    return v * np.repeat(e4m3_decode(sbits), 16, axis=-1)
+
+
 # --------------------------------------------------------------------------- routing
 @dataclass
 class RouteStep:

@@ -57,6 +57,7 @@ class Workload:
     seed: int
     n_query_sets: int = 16
     append: int = 0        # tokens appended after the initial build
+    planes: str = "key"    # router planes: "key" (the stored slopes) or "fp4"
     # topic / needle constants (logit gains are in units of q.k/sqrt(d))
     n_topics: int = 64
     n_segments: int = 256
@@ -85,6 +86,9 @@ def workload(name: str, n_tokens: Optional[int] = None) -> Workload:
     if name == "deep256k_bf16":
         return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=262144, block=4,
                         levels=6, n_refs=16, p=0.95, batch=1, dtype="bf16", gen="topics", seed=1)
+    if name == "deep256k_fp4":  # the deep 256K tree, routed on FP4 router planes
+        return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=262144, block=4,
+                        levels=6, n_refs=16, p=0.95, batch=1, dtype="bf16", gen="topics", seed=1, planes="fp4")
     if name == "deep_bf16":  # the deep tree's shape at another context length (profiling cases)
         n = n_tokens if n_tokens is not None else 262144
         return Workload(name, d=128, n_q_heads=32, n_kv_heads=4, n_tokens=n, block=4,

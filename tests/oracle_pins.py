@@ -260,6 +260,60 @@ def pin_step_thresholds(zo):
                 assert step.k == _brute_top_p(step.ehat, start, ps), (trial, s, step.k)
 
 
+def pin_e4m3_grid(zo):
+    """Every finite non-negative e4m3 encoding decodes to its value and rounds back to itself; the values
+    rise strictly from 0 through 2^-9 (smallest subnormal) and 2^-6 (smallest normal) to 448."""
+    bits = np.arange(0, 127, dtype=np.uint8)          # 0x7F would be NaN
+    vals = zo.e4m3_decode(bits)
+    assert vals[0] == 0 and vals[1] == 2.0 ** -9 and vals[8] == 2.0 ** -6 and vals[-1] == 448.0
+    assert np.all(np.diff(vals) > 0)
+    v2, b2 = zo.e4m3_nearest(vals)
+    assert np.array_equal(v2, vals) and np.array_equal(b2, bits)
+    # midpoints go to the neighbour with the even mantissa, points off them to the nearer neighbour
+    mids = (vals[1:] + vals[:-1]) / 2
+    got, _ = zo.e4m3_nearest(mids)
+    even = np.where(bits[:-1] % 2 == 0, vals[:-1], vals[1:])
+    assert np.array_equal(got, even)
+    below, _ = zo.e4m3_nearest(mids * (1 - 1e-9))
+    above, _ = zo.e4m3_nearest(mids * (1 + 1e-9))
+    assert np.array_equal(below, vals[:-1]) and np.array_equal(above, vals[1:])
+    assert zo.e4m3_nearest(np.array([1e6]))[0][0] == 448.0
+
+
+def pin_e2m1_codes(zo):
+    """The eight e2m1 magnitudes code to themselves with either sign; midpoints go to the even mantissa
+    (0, 1, 2, 4 are even); beyond 6 saturates."""
+    vals = zo.E2M1_VALUES
+    assert np.array_equal(zo.E2M1_VALUES[zo.e2m1_code(vals) & 7], vals)
+    assert np.array_equal(zo.E2M1_VALUES[zo.e2m1_code(-vals) & 7], vals)
+    assert np.all((zo.e2m1_code(-vals[1:]) & 8) == 8) and zo.e2m1_code(np.array([-0.1]))[0] == 0
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    assert np.array_equal(zo.E2M1_VALUES[zo.e2m1_code(ties)], [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0])
+    assert zo.E2M1_VALUES[zo.e2m1_code(np.array([7.0, 100.0])) & 7].tolist() == [6.0, 6.0]
+
+
+def pin_fp4_quantize(zo):
+    """A group whose largest magnitude is 6 * (an e4m3 value) gets exactly that scale and codes it as +-6;
+    every slope is within one scale step (the widest e2m1 gap is 4 to 6) of its value, within a quarter
+    step where |v| / scale <= 2; an all-zero group has scale 0 and zero codes."""
+    rng = _rng(31)
+    mu = rng.normal(size=(6, 64)).astype(np.float32)
+    mu[0, :16] = 0.0
+    mu[1, 16:32] = np.float32(0.75) * rng.uniform(-1, 1, 16).astype(np.float32)
+    mu[1, 16] = np.float32(6 * 0.125)                   # amax = 6 * 0.125, 0.125 is an e4m3 value
+    codes, sb = zo.quantize_fp4(mu)
+    dq = zo.dequantize_fp4(codes, sb)
+    sc = np.repeat(zo.e4m3_decode(sb), 16, axis=-1)
+    assert np.all(np.abs(dq - mu) <= sc + 1e-12)
+    small = np.abs(mu) <= 2 * sc
+    assert np.all(np.abs(dq - mu)[small] <= 0.25 * sc[small] + 1e-12)
+    assert sb[0, 0] == 0 and np.all(codes[0, :16] == 0)
+    assert zo.e4m3_decode(sb[1, 1]) == 0.125 and dq[1, 16] == 0.75
+    # symmetric: negating the slopes negates the values
+    c2, s2 = zo.quantize_fp4(-mu)
+    assert np.array_equal(zo.dequantize_fp4(c2, s2), -dq)
+
+
 def pin_cut_reaches_p_exactly(zo):
     """Four equal estimates at p = 0.5: mass 0.25 + 0.25 reaches p, so exactly two are kept."""
     e = np.zeros(4)

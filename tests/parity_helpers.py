@@ -108,12 +108,13 @@ def trace_flags(trace: zo.RouteTrace, planes, q: np.ndarray, p, block: int) -> L
 
 
 def gpu_planes_fn(tree, kv_head: int, levels: int):
-    """planes(level, idx) over the GPU-stored planes (bf16/fp32 upcast to fp64), read lazily."""
+    """planes(level, idx) over the planes the GPU router reads (the stored bf16/fp32 slopes, or the FP4
+    router copies' exact values), upcast to fp64, read lazily."""
     cache: Dict[int, Tuple[torch.Tensor, torch.Tensor]] = {}
 
     def fn(level, idx):
         if level not in cache:
-            mu, bias, _ = tree.level_planes(level)
+            mu, bias = tree.router_planes(level)
             cache[level] = (mu[kv_head].cpu(), bias[kv_head].cpu())
         mu, bias = cache[level]
         idx_t = torch.as_tensor(np.asarray(idx), dtype=torch.long)

@@ -96,6 +96,32 @@ def test_sizes_and_layout(built):
     assert lay.rec_bytes == 3 * 64 * 4 + 16
 
 
+def test_fp4_router_layout(built):
+    """FP4 router records: R*(d/2 + d/16) bytes of codes and scales, then R floats padded to 16 bytes,
+    after the key planes; bf16 only; a key-plane configuration has none."""
+    c = cfg(planes="fp4")
+    nb_fp4, _ = z.tree_bytes(c)
+    nb_key, _ = z.tree_bytes(cfg())
+    total = 0
+    for level in range(1, 7):
+        off, rb = z.zha.tree_layout_fp4(c, level)
+        assert rb == 16 * (64 + 8) + 64 == 1216
+        assert off % 256 == 0 and off >= nb_key
+        total += 4 * (262144 // 4 ** level) * rb
+    assert nb_fp4 >= nb_key + total
+    with pytest.raises(z.ZhaError) as e:
+        z.zha.tree_layout_fp4(cfg(), 1)
+    assert e.value.code == zb.ZHA_ERR_INVALID
+    with pytest.raises(z.ZhaError) as e:
+        z.tree_bytes(cfg(planes="fp4", dtype="f32"))
+    assert e.value.code == zb.ZHA_ERR_UNSUPPORTED
+    bad = cfg()
+    bad.planes = 7
+    with pytest.raises(z.ZhaError) as e:
+        z.tree_bytes(bad)
+    assert e.value.code == zb.ZHA_ERR_INVALID
+
+
 def test_dense_scratch_bytes(built):
     c = cfg()
     assert z.dense_scratch_bytes(c, 1, 262144) > 0

@@ -25,14 +25,15 @@ if torch.cuda.is_available():
 class Case:
     """A tree over the first n tokens of (K, V), with room to append the rest."""
 
-    def __init__(self, K, V, refs, *, block, levels, p, n, group, max_batch=16, capacity=None):
+    def __init__(self, K, V, refs, *, block, levels, p, n, group, max_batch=16, capacity=None, planes="key"):
         self.Kall, self.Vall, self.refs_cpu = K, V, refs
         Hkv, ntot, d = K.shape
         self.dtype = "bf16" if K.dtype == torch.bfloat16 else "f32"
         self.block, self.levels, self.p, self.group = block, levels, p, group
         cap = capacity or max(ntot, 1)
         self.cfg = z.make_config(d=d, n_q_heads=Hkv * group, n_kv_heads=Hkv, block=block, levels=levels,
-                                 n_refs=refs.shape[1], p=p, dtype=self.dtype, capacity=cap, max_batch=max_batch)
+                                 n_refs=refs.shape[1], p=p, dtype=self.dtype, capacity=cap, max_batch=max_batch,
+                                 planes=planes)
         self.Kc = torch.zeros(Hkv, cap, d, dtype=K.dtype, device="cuda")
         self.Vc = torch.zeros_like(self.Kc)
         self.Kc[:, :n] = K[:, :n].cuda()
@@ -264,6 +265,42 @@ def test_step_thresholds():
         case.tree.set_step_p([0.5, 1.5])
     with pytest.raises(z.ZhaError):
         case.tree.set_step_p([0.0])
+
+
+def check_fp4_records(case: Case):
+    """The FP4 router records are the oracle's quantisation of the stored slopes (bit-exact) and carry the
+    stored intercepts."""
+    for level in range(1, case.levels + 1):
+        n_l = case.n // case.block ** level
+        if n_l == 0:
+            continue
+        mu, bias, _ = case.tree.level_planes(level)
+        codes, sbits, b4 = case.tree.fp4_records(level)
+        for kvh in range(case.Kall.shape[0]):
+            oc, osb = zo.quantize_fp4(mu[kvh, :n_l].float().cpu().numpy())
+            assert np.array_equal(codes[kvh, :n_l].cpu().numpy(), oc), f"level {level} codes"
+            assert np.array_equal(sbits[kvh, :n_l].cpu().numpy(), osb), f"level {level} scales"
+            assert torch.equal(b4[kvh, :n_l].cpu(), bias[kvh, :n_l].cpu())
+
+
+@pytest.mark.parametrize("d,block,levels,R,G", [(128, 4, 4, 8, 8), (64, 8, 2, 16, 4), (128, 3, 5, 1, 2)])
+def test_fp4_router_planes(d, block, levels, R, G):
+    """Routing on FP4 router records: quantisation bit-exact against the oracle's, route and attention
+    against the oracle on the planes the router reads, including after appends."""
+    n = 20011
+    w = small_topics(n + 300, d=d, n_q_heads=G, n_kv_heads=1, block=block, levels=levels, n_refs=R, p=0.95,
+                     batch=2)
+    inp = generate(w)
+    case = Case(inp.K, inp.V, inp.refs, block=block, levels=levels, p=0.95, n=n, group=G, planes="fp4")
+    check_build(case)
+    check_fp4_records(case)
+    for s in range(2):
+        rep, *_ = check_decode(case, inp.Q[s])
+        print(f"fp4 d={d} b={block}: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+    for m in (1, 3, 296):
+        case.append(m)
+    check_fp4_records(case)
+    check_decode(case, inp.Q[2])
 
 
 def test_append_then_decode():

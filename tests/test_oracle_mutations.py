@@ -127,6 +127,28 @@ def _attend_no_scale(K, V, q, tokens):
     return (w / w.sum()) @ V[tokens]
 
 
+def _e2m1_ties_up(y):
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    idx = np.zeros(a.shape, dtype=np.uint8)
+    for i in range(1, 8):
+        mid = (zo.E2M1_VALUES[i - 1] + zo.E2M1_VALUES[i]) / 2
+        idx = np.where(a >= mid, np.uint8(i), idx)       # ties away from zero
+    return np.where(idx == 0, 0, idx | np.where(y < 0, 8, 0)).astype(np.uint8)
+
+
+def _quantize_scale_amax4(mu):
+    m32 = np.asarray(mu, dtype=np.float32)
+    g = m32.reshape(*m32.shape[:-1], m32.shape[-1] // 16, 16)
+    amax = np.abs(g).max(axis=-1)
+    sval, sbits = zo.e4m3_nearest((amax / np.float32(4)).astype(np.float32))
+    s32 = sval.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = (g / s32[..., None]).astype(np.float32)
+    codes = np.where(s32[..., None] > 0, zo.e2m1_code(y), 0).astype(np.uint8)
+    return codes.reshape(m32.shape), sbits
+
+
 def _step_threshold_first(p, s):
     return float(p) if np.ndim(p) == 0 else float(p[0])
 
@@ -181,6 +203,8 @@ MUTATIONS = {
     "attention without 1/sqrt(d)": ("attend", _attend_no_scale),
     "ties to the higher start": ("route", _route_ties_high),
     "step thresholds ignored after the first": ("step_threshold", _step_threshold_first),
+    "e2m1 ties away from zero": ("e2m1_code", _e2m1_ties_up),
+    "fp4 scale from amax / 4": ("quantize_fp4", _quantize_scale_amax4),
 }
 
 

@@ -53,6 +53,7 @@ struct Layout {
   int64_t cap_nodes[kMaxLevels + 1];
   int64_t pow_b[kMaxLevels + 1];
   uint64_t rec_off[kMaxLevels + 1], f_off[kMaxLevels + 1], up_off[kMaxLevels + 1];
+  uint64_t rec4_off[kMaxLevels + 1], rec4_bytes;  // FP4 router records (planes = ZHA_PLANES_FP4)
   uint64_t rec_bytes, up_bytes, node_bytes;
   // scratch
   uint64_t status_off, part_off, part_items, flow_off, flow_bytes, ws_off, ws_per_bh, stage_off, scratch_bytes;
@@ -79,6 +80,10 @@ int validate(const zha_config* c) {
   if (c->capacity < 1 || c->capacity >= (int64_t(1) << 31)) return fail(ZHA_ERR_INVALID, "capacity must be in [1, 2^31)");
   if (c->capacity / c->block >= (int64_t(1) << 27)) return fail(ZHA_ERR_UNSUPPORTED, "capacity / block must be < 2^27");
   if (c->max_batch < 1 || c->max_batch > 65535) return fail(ZHA_ERR_INVALID, "max_batch must be in [1, 65535]");
+  if (c->planes != ZHA_PLANES_KEY && c->planes != ZHA_PLANES_FP4)
+    return fail(ZHA_ERR_INVALID, "planes must be ZHA_PLANES_KEY or ZHA_PLANES_FP4");
+  if (c->planes == ZHA_PLANES_FP4 && c->dtype != ZHA_BF16)
+    return fail(ZHA_ERR_UNSUPPORTED, "FP4 router planes need a bf16 configuration");
   if (int64_t(c->max_batch) * c->n_q_heads > decode_max_heads())
     return fail(ZHA_ERR_UNSUPPORTED, "max_batch * n_q_heads must be <= 1024");
   // block^levels must fit comfortably in int64
@@ -123,6 +128,14 @@ int make_layout(const zha_config* c, Layout* L) {
   for (int l = L->S; l < c->levels; ++l) {
     L->up_off[l] = off;
     off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * L->up_bytes);
+  }
+  if (c->planes == ZHA_PLANES_FP4) {
+    L->rec4_bytes = uint64_t(c->n_refs) * (c->d / 2 + c->d / 16) + ((uint64_t(c->n_refs) * 4 + 15) & ~uint64_t(15));
+    L->rec4_bytes = (L->rec4_bytes + 15) & ~uint64_t(15);
+    for (int l = 1; l <= c->levels; ++l) {
+      L->rec4_off[l] = off;
+      off = align256(off + uint64_t(c->n_kv_heads) * L->cap_nodes[l] * L->rec4_bytes);
+    }
   }
   L->node_bytes = off > 0 ? off : 256;
   // scratch: status word and grid barrier, attend partials, per (sequence,
@@ -196,6 +209,17 @@ int zha_tree_layout(const zha_config* cfg, int32_t level, size_t* rec_offset, si
   return ZHA_OK;
 }
 
+int zha_tree_layout_fp4(const zha_config* cfg, int32_t level, size_t* rec_offset, size_t* rec_bytes) {
+  Layout L;
+  int rc = make_layout(cfg, &L);
+  if (rc) return rc;
+  if (cfg->planes != ZHA_PLANES_FP4) return fail(ZHA_ERR_INVALID, "the configuration has no FP4 router planes");
+  if (level < 1 || level > cfg->levels) return fail(ZHA_ERR_INVALID, "level out of range");
+  if (rec_offset) *rec_offset = L.rec4_off[level];
+  if (rec_bytes) *rec_bytes = L.rec4_bytes;
+  return ZHA_OK;
+}
+
 int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, void* node_buf, void* scratch,
                     zha_tree** out) {
   if (!out) return fail(ZHA_ERR_INVALID, "out is NULL");
@@ -239,8 +263,11 @@ int zha_tree_create(const zha_config* cfg, void* K, void* V, const void* refs, v
     d.rec_off[l] = L.rec_off[l];
     d.f_off[l] = L.f_off[l];
     d.up_off[l] = L.up_off[l];
+    d.rec4_off[l] = L.rec4_off[l];
   }
   d.rec_bytes = L.rec_bytes;
+  d.planes = cfg->planes;
+  d.rec4_bytes = L.rec4_bytes;
   d.up_bytes = L.up_bytes;
   d.nodes = static_cast<char*>(node_buf);
   d.K = K;

@@ -291,6 +291,47 @@ __global__ void __launch_bounds__(kBuildThreads) upper_kernel(TreeDev t, int lev
   }
 }
 
+// FP4 router records of the nodes [first, first + gridDim.x) of one level, from
+// the stored records: one thread per (reference row, group of 16 dimensions)
+// quantises the group (scale = e4m3(amax / 6), codes = e2m1(v / scale), both
+// rounded to nearest, ties to even) and writes its 8 code bytes and its scale
+// byte; the intercepts are copied and the padding zeroed.
+template <typename T, int D>
+__global__ void quant4_kernel(TreeDev t, int level, int64_t first) {
+  using E = Elem<T>;
+  const int h = blockIdx.y;
+  const int64_t gi = first + blockIdx.x;
+  const int R = t.refs;
+  constexpr int G = D / 16;
+  const T* src = reinterpret_cast<const T*>(t.rec(level, h, gi));
+  unsigned char* dst = reinterpret_cast<unsigned char*>(t.rec4(level, h, gi));
+  for (int i = threadIdx.x; i < R * G; i += blockDim.x) {
+    const int j = i / G, g = i % G;
+    float v[16];
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      v[k] = E::to_f(src[size_t(j) * D + g * 16 + k]);
+      amax = fmaxf(amax, fabsf(v[k]));
+    }
+    uint32_t sbits;
+    const float sc = e4m3_nearest(__fdiv_rn(amax, 6.f), &sbits);
+    uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t c = sc > 0.f ? e2m1_code(__fdiv_rn(v[k], sc)) : 0u;
+      if (k < 8) w0 |= c << (4 * k);
+      else w1 |= c << (4 * (k - 8));
+    }
+    *reinterpret_cast<uint2*>(dst + size_t(j) * (D / 2) + g * 8) = make_uint2(w0, w1);
+    dst[size_t(R) * (D / 2) + size_t(j) * G + g] = (unsigned char)sbits;
+  }
+  const float* bsrc = reinterpret_cast<const float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T));
+  float* bdst = reinterpret_cast<float*>(dst + size_t(R) * (D / 2 + G));
+  const int padded = int((t.rec4_bytes - size_t(R) * (D / 2 + G)) / 4);
+  for (int j = threadIdx.x; j < padded; j += blockDim.x) bdst[j] = j < R ? bsrc[j] : 0.f;
+}
+
 // Copy m new tokens ([Hkv][m][d] rows) into the cache at positions [n, n+m).
 template <typename T, int D>
 __global__ void append_copy_kernel(TreeDev t, const T* Knew, const T* Vnew, int64_t n, int64_t m) {
@@ -337,6 +378,17 @@ static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_ne
     upper_kernel<T, D><<<grid, kBuildThreads, sm, st>>>(t, level, a0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+  }
+  if (t.planes == ZHA_PLANES_FP4) {  // the router copies of the nodes this call completed
+    for (int level = 1; level <= t.levels; ++level) {
+      const int64_t a0 = n_old / t.pow_b[level], a1 = n_new / t.pow_b[level];
+      if (a1 <= a0) continue;
+      dim3 grid(unsigned(a1 - a0), unsigned(t.hkv));
+      count_launches(1);
+      quant4_kernel<T, D><<<grid, 128, 0, st>>>(t, level, a0);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaSuccess;
 }

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -61,6 +62,90 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, cons
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+__device__ __forceinline__ void mma_f16_16816(float* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// ---------------------------------------------------------------- FP4 router planes
+// Values of the e2m1 codes by magnitude index 0..7 (the code's low three bits; bit 3 is the sign).
+// A group of 16 slopes shares one e4m3 scale; the slope is code * scale (see zha.h, ZHA_PLANES_FP4).
+
+// Nearest e4m3 value of x >= 0, ties to the even mantissa, at most 448 (the largest finite e4m3);
+// *bits receives its encoding (sign 0, exponent bias 7, 3 mantissa bits).  Scaling by powers of two
+// and rintf (round half to even) are exact, so the result is the correctly rounded one.
+__device__ __forceinline__ float e4m3_nearest(float x, uint32_t* bits) {
+  if (!(x > 0.f)) {
+    *bits = 0u;
+    return 0.f;
+  }
+  if (x >= 448.f) {
+    *bits = 0x7Eu;
+    return 448.f;
+  }
+  int e2;
+  frexpf(x, &e2);
+  int E = e2 - 1;  // x in [2^E, 2^(E+1))
+  if (E < -6) {    // subnormal range: multiples of 2^-9
+    const float m = rintf(ldexpf(x, 9));
+    *bits = uint32_t(m);  // m == 8 is the smallest normal (exponent field 1, mantissa 0)
+    return ldexpf(m, -9);
+  }
+  float m = rintf(ldexpf(x, 3 - E));  // in [8, 16]
+  if (m == 16.f) {
+    m = 8.f;
+    ++E;
+  }
+  const float v = ldexpf(m, E - 3);
+  if (v > 448.f) {
+    *bits = 0x7Eu;
+    return 448.f;
+  }
+  *bits = (uint32_t(E + 7) << 3) | (uint32_t(m) - 8u);
+  return v;
+}
+
+// e2m1 code of y: nearest of {0, 0.5, 1, 1.5, 2, 3, 4, 6} with the sign of y, ties to the even
+// mantissa, at most 6; magnitude 0 is coded +0.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  uint32_t i;
+  if (a <= 0.25f) i = 0u;
+  else if (a < 0.75f) i = 1u;
+  else if (a <= 1.25f) i = 2u;
+  else if (a < 1.75f) i = 3u;
+  else if (a <= 2.5f) i = 4u;
+  else if (a < 3.5f) i = 5u;
+  else if (a <= 5.f) i = 6u;
+  else i = 7u;
+  return i == 0u ? 0u : (i | (y < 0.f ? 8u : 0u));
+}
+
+// Two e2m1 codes (low nibble first) -> f16x2 (low half first), exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte2) {
+  uint32_t r;
+  asm("{\n .reg .b8 lo8, hi8;\n mov.b16 {lo8, hi8}, %1;\n cvt.rn.f16x2.e2m1x2 %0, lo8;\n}"
+      : "=r"(r)
+      : "h"((unsigned short)(byte2 & 0xffu)));
+  return r;
+}
+
+// Two e4m3 values (low byte first) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((unsigned short)(two & 0xffffu)));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -109,6 +194,9 @@ struct TreeDev {
   uint64_t up_off[kMaxLevels + 1];     // fp32 full nodes, levels chunk_level .. levels-1
   uint64_t rec_bytes;                  // mu[R][d] (element type) + bias[R] fp32, padded to 16 B
   uint64_t up_bytes;                   // mu[R][d] fp32 + f[R] + g[R]
+  int planes;                          // ZHA_PLANES_KEY or ZHA_PLANES_FP4 (the routing steps read rec4)
+  uint64_t rec4_off[kMaxLevels + 1];   // FP4 router records: codes[R][d/2], scales[R][d/16], bias[R]
+  uint64_t rec4_bytes;
   char* nodes;
   void* K;
   void* V;
@@ -118,6 +206,9 @@ struct TreeDev {
 
   __device__ __forceinline__ char* rec(int level, int head, int64_t i) const {
     return nodes + rec_off[level] + (uint64_t(head) * cap_nodes[level] + i) * rec_bytes;
+  }
+  __device__ __forceinline__ char* rec4(int level, int head, int64_t i) const {
+    return nodes + rec4_off[level] + (uint64_t(head) * cap_nodes[level] + i) * rec4_bytes;
   }
   __device__ __forceinline__ float* fval(int level, int head, int64_t i) const {
     return reinterpret_cast<float*>(nodes + f_off[level]) +

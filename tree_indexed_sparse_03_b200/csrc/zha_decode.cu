@@ -1129,6 +1129,82 @@ __device__ __forceinline__ float score_record_mma(const unsigned char* rec, int 
   return best;
 }
 
+// The q operand for FP4 router records: the bf16 fragments of q_fragments
+// converted to f16 (exact for the normal f16 range).
+template <int D>
+__device__ __forceinline__ void q_fragments_f16(const __nv_bfloat16* q, uint32_t (&qf)[D / 16][2], int lane) {
+  q_fragments<D>(q, qf, lane);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float lo = __uint_as_float(qf[k][u] << 16), hi = __uint_as_float(qf[k][u] & 0xffff0000u);
+      const __half2 h = __floats2half2_rn(lo, hi);
+      qf[k][u] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
+// e = max_j (b_j + q.mu_j / sqrt d) of an FP4 router record in shared memory:
+// the lane's 4-bit codes of its two rows are turned into f16 (exact) and
+// multiplied by their groups' e4m3 scales (exact in f16), then fed to the
+// tensor cores in the same operand layout as score_record_mma (f16, fp32
+// accumulation); every lane returns the estimate.
+template <int D>
+__device__ __forceinline__ float score_record_fp4(const unsigned char* rec, int R, float inv_sqrt_d,
+                                                  const uint32_t (&qf)[D / 16][2], int lane) {
+  constexpr int CPL = D / 32;  // 8-dimension chunks per lane
+  const int g = lane >> 2, t = lane & 3;
+  const unsigned char* scales = rec + size_t(R) * (D / 2);
+  const float* bias = reinterpret_cast<const float*>(rec + size_t(R) * (D / 2 + D / 16));
+  float best = -INFINITY;
+  for (int m0 = 0; m0 < R; m0 += 16) {
+    const int r0 = min(m0 + g, R - 1), r1 = min(m0 + g + 8, R - 1);  // rows past R: masked below
+    uint32_t w0[CPL], w1[CPL];  // 4 code bytes (8 dimensions) per chunk
+    uint32_t s0, s1;            // the rows' scales of the lane's groups, as f16x2
+    if constexpr (D == 128) {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(rec + size_t(r0) * (D / 2) + t * 16);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(rec + size_t(r1) * (D / 2) + t * 16);
+      w0[0] = v0.x; w0[1] = v0.y; w0[2] = v0.z; w0[3] = v0.w;
+      w1[0] = v1.x; w1[1] = v1.y; w1[2] = v1.z; w1[3] = v1.w;
+      s0 = e4m3x2_to_f16x2(*reinterpret_cast<const unsigned short*>(scales + size_t(r0) * (D / 16) + 2 * t));
+      s1 = e4m3x2_to_f16x2(*reinterpret_cast<const unsigned short*>(scales + size_t(r1) * (D / 16) + 2 * t));
+    } else {
+      const uint2 v0 = *reinterpret_cast<const uint2*>(rec + size_t(r0) * (D / 2) + t * 8);
+      const uint2 v1 = *reinterpret_cast<const uint2*>(rec + size_t(r1) * (D / 2) + t * 8);
+      w0[0] = v0.x; w0[1] = v0.y;
+      w1[0] = v1.x; w1[1] = v1.y;
+      const uint32_t b0 = scales[size_t(r0) * (D / 16) + t], b1 = scales[size_t(r1) * (D / 16) + t];
+      s0 = e4m3x2_to_f16x2(b0 | (b0 << 8));
+      s1 = e4m3x2_to_f16x2(b1 | (b1 << 8));
+    }
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      // chunk c lies in group c/2 of the lane's (D = 128) or in its only group (D = 64)
+      const uint32_t sel = (D == 128 && c >= 2) ? 0x3232u : 0x1010u;
+      const uint32_t S0 = __byte_perm(s0, s0, sel), S1 = __byte_perm(s1, s1, sel);
+      uint32_t x0[4], x1[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        x0[q] = hmul2_u32(e2m1x2_to_f16x2(w0[c] >> (8 * q)), S0);
+        x1[q] = hmul2_u32(e2m1x2_to_f16x2(w1[c] >> (8 * q)), S1);
+      }
+      const uint32_t a0[4] = {x0[0], x1[0], x0[1], x1[1]};
+      const uint32_t a1[4] = {x0[2], x1[2], x0[3], x1[3]};
+      mma_f16_16816(c0, a0, qf[2 * c]);
+      mma_f16_16816(c1, a1, qf[2 * c + 1]);
+    }
+    if (t == 0) {
+      const int j0 = m0 + g, j1 = m0 + g + 8;
+      if (j0 < R) best = fmaxf(best, fmaf(c0[0] + c1[0], inv_sqrt_d, bias[j0]));
+      if (j1 < R) best = fmaxf(best, fmaf(c0[2] + c1[2], inv_sqrt_d, bias[j1]));
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+  return best;
+}
+
 // Estimate of a node whose record sits in shared memory (whole warp; the
 // lane's q slice covers elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR).  Up
 // to kG reference rows per lane are in flight at once: their partial dot
@@ -1459,7 +1535,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int nh = a.nheads, b = a.t.block, R = a.t.refs;
   const int par = s & 1;
-  const int rec_bytes = int(a.t.rec_bytes);
+  const bool fp4 = kMma && a.t.planes == ZHA_PLANES_FP4;  // the routing steps read the FP4 router records
+  const int rec_bytes = int(fp4 ? a.t.rec4_bytes : a.t.rec_bytes);
   // nslot record slots per warp; warps past score_warps (only when a record is
   // larger than a warp's share of the ring) do not score
   const int nslot = max(1, min(kMaxSlots, (kRingBytes / kDecWarps) / rec_bytes));
@@ -1556,8 +1633,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
         if (lane == 0) {
           fence_proxy_async();  // the slot's last reads (generic proxy) before the copy writes it
           const int kvh = (it.h % a.t.hq) / a.t.group;
-          bulk_load(slot, a.t.rec(code_level(it.code), kvh, code_index(it.code)), unsigned(rec_bytes),
-                    &sp.mbar[wid][sl]);
+          const int lv = code_level(it.code);
+          const int64_t ix = code_index(it.code);
+          bulk_load(slot, fp4 ? a.t.rec4(lv, kvh, ix) : a.t.rec(lv, kvh, ix), unsigned(rec_bytes), &sp.mbar[wid][sl]);
         }
 #pragma unroll
         for (int k = 0; k < kMaxSlots; ++k)
@@ -1601,13 +1679,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
 #pragma unroll
       for (int k = 0; k + 1 < kMaxSlots; ++k) slot_item[k] = slot_item[k + 1];
       if (it.h != qhead) {
-        if constexpr (kMma) q_fragments<D>(static_cast<const __nv_bfloat16*>(a.Q) + size_t(it.h) * D, qf, lane);
-        else c.q_slice(it.h, qs);
+        if constexpr (kMma) {
+          const __nv_bfloat16* qh = static_cast<const __nv_bfloat16*>(a.Q) + size_t(it.h) * D;
+          if (fp4) q_fragments_f16<D>(qh, qf, lane);
+          else q_fragments<D>(qh, qf, lane);
+        } else {
+          c.q_slice(it.h, qs);
+        }
         qhead = it.h;
       }
       const unsigned char* rec = ring + size_t(sl) * rec_bytes;
       float e;
-      if constexpr (kMma) e = score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
+      if constexpr (kMma) e = fp4 ? score_record_fp4<D>(rec, R, a.t.inv_sqrt_d, qf, lane)
+                                  : score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
       else e = score_record_smem<T, D>(rec, R, a.t.inv_sqrt_d, qs, lane);
       if (lane == 0) {
         const uint32_t key = desc_key(e);

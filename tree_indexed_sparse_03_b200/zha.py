@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libzha.so")
 
 ZHA_OK, ZHA_ERR_INVALID, ZHA_ERR_CAPACITY, ZHA_ERR_UNSUPPORTED, ZHA_ERR_CUDA, ZHA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 ZHA_F32, ZHA_BF16 = 0, 1
+ZHA_PLANES_KEY, ZHA_PLANES_FP4 = 0, 1
+PLANES_CODE = {"key": ZHA_PLANES_KEY, "fp4": ZHA_PLANES_FP4}
 STAT_NODES_SCORED, STAT_LEAVES_KEPT, STAT_KEYS, STAT_STEPS, STAT_COUNT = 0, 1, 2, 3, 4
 
 TORCH_DTYPE = {ZHA_F32: torch.float32, ZHA_BF16: torch.bfloat16}
@@ -30,6 +32,7 @@ _SIGS = {
     "zha_tree_bytes": (_c.c_int, [_c.c_void_p, _c.POINTER(_c.c_size_t), _c.POINTER(_c.c_size_t)]),
     "zha_tree_layout": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.POINTER(_c.c_size_t), _c.POINTER(_c.c_size_t),
                                    _c.POINTER(_c.c_int64), _c.POINTER(_c.c_size_t)]),
+    "zha_tree_layout_fp4": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.POINTER(_c.c_size_t), _c.POINTER(_c.c_size_t)]),
     "zha_tree_create": (_c.c_int, [_c.c_void_p] * 6 + [_c.POINTER(_c.c_void_p)]),
     "zha_tree_build": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_void_p]),
     "zha_tree_append": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p]),
@@ -83,12 +86,13 @@ class ZhaConfig(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("block", ctypes.c_int32), ("levels", ctypes.c_int32), ("n_refs", ctypes.c_int32),
                 ("p", ctypes.c_float), ("dtype", ctypes.c_int32), ("capacity", ctypes.c_int64),
-                ("max_batch", ctypes.c_int32)]
+                ("max_batch", ctypes.c_int32), ("planes", ctypes.c_int32)]
 
 
 def make_config(*, d: int, n_q_heads: int, n_kv_heads: int, block: int, levels: int, n_refs: int, p: float,
-                dtype, capacity: int, max_batch: int = 1) -> ZhaConfig:
-    return ZhaConfig(d, n_q_heads, n_kv_heads, block, levels, n_refs, p, DTYPE_CODE[dtype], capacity, max_batch)
+                dtype, capacity: int, max_batch: int = 1, planes: str = "key") -> ZhaConfig:
+    return ZhaConfig(d, n_q_heads, n_kv_heads, block, levels, n_refs, p, DTYPE_CODE[dtype], capacity, max_batch,
+                     PLANES_CODE[planes])
 
 
 def _stream(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
@@ -120,6 +124,31 @@ def tree_layout(cfg: ZhaConfig, level: int) -> LevelLayout:
     _check(lib().zha_tree_layout(ctypes.byref(cfg), level, ctypes.byref(ro), ctypes.byref(fo), ctypes.byref(cap),
                                  ctypes.byref(rb)))
     return LevelLayout(ro.value, fo.value, cap.value, rb.value)
+
+
+def tree_layout_fp4(cfg: ZhaConfig, level: int) -> Tuple[int, int]:
+    """(byte offset, bytes per record) of the FP4 router records of a level."""
+    ro, rb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().zha_tree_layout_fp4(ctypes.byref(cfg), level, ctypes.byref(ro), ctypes.byref(rb)))
+    return ro.value, rb.value
+
+
+E2M1_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def e2m1_value(codes: torch.Tensor) -> torch.Tensor:
+    """Values of 4-bit e2m1 codes (uint8 tensor of codes 0..15), fp32."""
+    tab = torch.tensor(E2M1_VALUES, dtype=torch.float32, device=codes.device)
+    v = tab[(codes & 7).long()]
+    return torch.where((codes & 8) != 0, -v, v)
+
+
+def e4m3_value(bits: torch.Tensor) -> torch.Tensor:
+    """Values of e4m3 bytes (finite encodings), fp32."""
+    b = bits.long()
+    e, m = (b >> 3) & 15, (b & 7).to(torch.float32)
+    mag = torch.where(e == 0, torch.ldexp(m, torch.full_like(e, -9)), torch.ldexp(1.0 + m / 8.0, e - 7))
+    return torch.where((b & 128) != 0, -mag, mag)
 
 
 class ZhaTree:
@@ -224,6 +253,31 @@ class ZhaTree:
         f = self.nodes[lay.f_offset: lay.f_offset + n * c.n_refs * 4].view(torch.float32).view(
             c.n_kv_heads, lay.cap_nodes, c.n_refs)
         return mu, bias, f
+
+    def fp4_records(self, level: int):
+        """FP4 router records of one level: (codes [Hkv, cap, R, d] uint8 (one code per dimension),
+        scales [Hkv, cap, R, d/16] uint8 e4m3, bias [Hkv, cap, R] fp32)."""
+        c = self.cfg
+        off, rb = tree_layout_fp4(c, level)
+        cap = tree_layout(c, level).cap_nodes
+        rec = self.nodes[off: off + c.n_kv_heads * cap * rb].view(c.n_kv_heads, cap, rb)
+        R, D = c.n_refs, c.d
+        packed = rec[..., : R * D // 2].reshape(c.n_kv_heads, cap, R, D // 2)
+        codes = torch.stack([packed & 15, packed >> 4], dim=-1).reshape(c.n_kv_heads, cap, R, D)
+        scales = rec[..., R * D // 2: R * (D // 2 + D // 16)].reshape(c.n_kv_heads, cap, R, D // 16)
+        b0 = R * (D // 2 + D // 16)
+        bias = rec[..., b0: b0 + 4 * R].contiguous().view(torch.float32)
+        return codes, scales, bias
+
+    def router_planes(self, level: int):
+        """The planes the routing steps read: (mu [Hkv, cap, R, d], bias [Hkv, cap, R] fp32); for FP4 router
+        planes mu = code * scale (exact)."""
+        if self.cfg.planes != ZHA_PLANES_FP4:
+            mu, bias, _ = self.level_planes(level)
+            return mu, bias
+        codes, scales, bias = self.fp4_records(level)
+        sc = e4m3_value(scales).repeat_interleave(16, dim=-1)
+        return e2m1_value(codes) * sc, bias
 
 
 def launch_count() -> int:
