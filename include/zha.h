@@ -66,8 +66,9 @@ enum { ZHA_F32 = 0, ZHA_BF16 = 1 };
 /* Router planes: the slopes the routing steps read.  ZHA_PLANES_KEY reads the
  * stored nodes (mu in the element type).  ZHA_PLANES_FP4 keeps, beside them,
  * a copy of every node's slopes in 4-bit e2m1 with one e4m3 scale per 16
- * dimensions (an FP4 router; the pages report that one was tried, without
- * details), which the routing steps read instead: a record is
+ * dimensions (an FP4 router: the tanhow.com summary "Zyphra发布ZHA稀疏注意力方法,
+ * 可改造冻结大模型", TL;DR, reports that one was tested, without details),
+ * which the routing steps read instead: a record is
  * R*(d/2 + d/16 + 4) bytes (1216 at R = 16, d = 128) instead of
  * R*(d*es + 4).  Quantisation of a group of 16 stored slopes v (converted
  * exactly to fp32): amax = max |v|; scale = e4m3(amax / 6) (the division in

@@ -181,8 +181,8 @@ def log_mass(K: np.ndarray, node: Node, q: np.ndarray, block: int) -> float:
 
 
 # --------------------------------------------------------------------------- FP4 router planes
-# [blog] "How does this give subquadratic scaling?" / the review pages mention that an FP4 router was
-# also tried, without details.  Reading: the router reads each slope row as 4-bit e2m1 codes with one
+# [summary] TL;DR: an FP4 router variant was also tested (no details given).  Reading: the router
+# reads each slope row as 4-bit e2m1 codes with one
 # e4m3 scale per 16 dimensions (the OCP microscaling element and scale formats), quantised from the
 # stored slopes by round-to-nearest; the intercepts stay fp32.  The decisions (scale, codes) are taken in
 # fp32 arithmetic, as the stored slopes are fp32-representable; the values are then exact.
