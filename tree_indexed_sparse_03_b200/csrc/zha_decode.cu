@@ -382,62 +382,49 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 }
 
 
-// The cut for at most kDecThreads entries: thread i takes entry i; the (order
-// key, mass) pairs are sorted by a bitonic network in shared memory (strides
-// below 32 within a warp by shuffles), the masses scanned in sorted order, and
-// the cut is the first entry whose running mass reaches T.
+// The cut for at most kDecThreads entries: thread i takes entry i; the order
+// keys are sorted by a bitonic network in shared memory (strides below 32
+// within a warp by shuffles), the masses scanned in sorted order, and the cut
+// is the first entry whose running mass reaches T.
 template <class View>
 __device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
                                                             DecSmem& sm, int step) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  unsigned long long* ks = sm.hist;                // [np] order keys
-  unsigned long long* ws = sm.hist + kDecThreads;  // [np] masses
+  const int tid = threadIdx.x;
+  unsigned long long* ks = sm.hist;  // [np] order keys
   int np = 32;
   while (np < n) np <<= 1;  // <= kDecThreads
-  unsigned long long k = ~0ull, w = 0;
-  if (tid < n) {
-    const uint32_t key = E.key(tid);
-    k = entry_key64(a, Entry{key, E.code(tid)});
-    w = entry_mass(m, key);
-  }
+  unsigned long long k = ~0ull;
+  if (tid < n) k = entry_key64(a, Entry{E.key(tid), E.code(tid)});
+  // the network moves the order keys alone: an entry's mass is a function of its estimate (the key's
+  // high half), recomputed after the sort
   if (tid < np) {
     for (int size = 2; size <= np; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
         const bool up = (tid & size) == 0;
-        unsigned long long ok, ow;
+        unsigned long long ok;
         if (stride >= 32) {  // partner in another warp: through shared memory
           ks[tid] = k;
-          ws[tid] = w;
           asm volatile("bar.sync 1, %0;" ::"r"(np) : "memory");
           ok = ks[tid ^ stride];
-          ow = ws[tid ^ stride];
           asm volatile("bar.sync 1, %0;" ::"r"(np) : "memory");
         } else {
           ok = __shfl_xor_sync(0xffffffffu, k, stride);
-          ow = __shfl_xor_sync(0xffffffffu, w, stride);
         }
         const bool lower = (tid & stride) == 0;
-        const bool take = (up == lower) ? (ok < k) : (ok > k);
-        if (take) {
-          k = ok;
-          w = ow;
-        }
+        if ((up == lower) ? (ok < k) : (ok > k)) k = ok;
       }
     }
   }
-  (void)lane;
+  const unsigned long long w = tid < n ? entry_mass(m, uint32_t(k >> 32)) : 0ull;  // sorted: valid first
   unsigned long long Z;
-  const unsigned long long before = block_scan_u64(tid < np ? w : 0ull, sm.red64, &Z);
+  const unsigned long long before = block_scan_u64(w, sm.red64, &Z);
   const unsigned long long T = ceil_p_times(Z, a.p_mant[step], a.p_shift[step]);
-  // sorted position of the cut: the first with before + w >= T (else the last entry)
+  // sorted position of the cut: the first with before + w >= T (none: keep everything)
   if (tid == 0) sm.bcast64[1] = ~0ull;
   __syncthreads();
   if (tid < n && before < T && before + w >= T) sm.bcast64[1] = k;
   __syncthreads();
-  unsigned long long cut = sm.bcast64[1];
-  if (cut == ~0ull) {  // T out of reach by rounding: keep everything
-    cut = ~0ull;
-  }
+  const unsigned long long cut = sm.bcast64[1];
   __syncthreads();
   return cut;
 }
