@@ -525,18 +525,24 @@ def run_sweep(args):
                           "speedup_vs_dense": round(line["dense_us"] / line["decode_us"], 3),
                           "keys_per_head": line["keys_per_head"], "roofline_frac": line["roofline"]["frac"],
                           "levels": line["config"]["levels"], "clocks": line["clocks"]}), flush=True)
-    # crossover: the first N from which the routed decode call is faster than the dense decode,
-    # interpolated linearly in log N between the two bracketing points
-    cross = None
-    for a, b in zip(lines, lines[1:]):
-        da, db = a["dense_us"] - a["decode_us"], b["dense_us"] - b["decode_us"]
-        if da < 0 <= db:
-            na, nb = math.log(a["config"]["n_tokens"]), math.log(b["config"]["n_tokens"])
-            cross = int(round(math.exp(na + (nb - na) * (-da) / (db - da))))
-    if lines and cross is None and lines[0]["dense_us"] >= lines[0]["decode_us"]:
-        cross = f"<= {lines[0]['config']['n_tokens']}"
+    cross = crossover([(ln["config"]["n_tokens"], ln["decode_us"], ln["dense_us"]) for ln in lines])
     print(json.dumps({"sweep": "light sweep bf16 (GQA 32/4, d=128, b=8, R=1, p=0.75, batch 1)",
                       "crossover_n": cross, "unit": "us per decode call"}), flush=True)
+
+
+def crossover(points):
+    """Context length from which the routed decode is faster than the dense one: points are
+    (N, routed us, dense us) in increasing N; the last sign change of dense - routed from negative to
+    non-negative, interpolated linearly in log N; "<= N0" if routed is never slower; None if never faster."""
+    cross = None
+    for (na, ra, da), (nb, rb, db) in zip(points, points[1:]):
+        ga, gb = da - ra, db - rb
+        if ga < 0 <= gb:
+            la, lb = math.log(na), math.log(nb)
+            cross = int(round(math.exp(la + (lb - la) * (-ga) / (gb - ga))))
+    if points and cross is None and all(d >= r for _, r, d in points):
+        cross = f"<= {points[0][0]}"
+    return cross
 
 
 def main():

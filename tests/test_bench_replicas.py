@@ -74,3 +74,17 @@ def test_reference_arm_under_torchrun():
 
 if __name__ == "__main__":
     pytest.main([__file__, "-q"])
+
+
+def test_sweep_crossover():
+    """The crossover is interpolated in log N between the bracketing sweep points."""
+    import math
+    sys.path.insert(0, ROOT)
+    import bench
+    pts = [(32768, 150.0, 34.0), (262144, 200.0, 105.0), (524288, 140.0, 190.0), (1048576, 220.0, 350.0)]
+    x = bench.crossover(pts)
+    g0, g1 = 105.0 - 200.0, 190.0 - 140.0
+    want = math.exp(math.log(262144) + (math.log(524288) - math.log(262144)) * (-g0) / (g1 - g0))
+    assert x == int(round(want)) and 262144 < x < 524288
+    assert bench.crossover([(1024, 1.0, 2.0), (2048, 1.0, 3.0)]) == "<= 1024"
+    assert bench.crossover([(1024, 3.0, 2.0), (2048, 4.0, 3.0)]) is None
