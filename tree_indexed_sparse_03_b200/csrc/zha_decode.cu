@@ -87,43 +87,13 @@ static_assert(sizeof(HeadState) == 256, "HeadState layout");
 
 // Per-head routing state and leaf bitmaps live in one scratch region.  The
 // first select of a decode starts the head's counters from zero, the last
-// one leaves both parities' step extremes cleared, the combining warp resets
-// the ticket and the export clears the bitmap, so a decode leaves the region
+// one leaves both parities' step extremes cleared, the combining warps reset
+// the tickets and the export clears the bitmap, so a decode leaves the region
 // ready for the next one (after an error status the host zeroes it).
 
 // 32-bit words of a head's leaf bitmap (one bit per level-1 block), a multiple of 4.
 __host__ __device__ __forceinline__ int64_t decode_bitmap_words(int64_t cap_sel) {
   return (((cap_sel + 31) / 32) + 3) & ~int64_t(3);
-}
-
-// Loads and stores of the routing flow state.  Stores that publish work are
-// releases at GPU scope and the loads that find it acquires, so that what the
-// publisher wrote before (entries, candidate codes, counters) is visible to
-// whoever takes the work.
-__device__ __forceinline__ int ld_volatile_i(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
-__device__ __forceinline__ long long ld_volatile_ll(const long long* p) {
-  return *reinterpret_cast<const volatile long long*>(p);
-}
-__device__ __forceinline__ int ld_acquire_i(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
-  return *reinterpret_cast<const volatile unsigned long long*>(p);
-}
-// After a relaxed load that found published work: orders the reads of that work after it.
-__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-__device__ __forceinline__ void st_release_i(int* p, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 struct __align__(16) DecSmem {
@@ -135,7 +105,6 @@ struct __align__(16) DecSmem {
   uint32_t red32[kDecWarps * 2];
   unsigned long long bcast64[4];
   int bcast32[8];
-  int fail;
 };
 
 // Division of 32-bit values by a fixed divisor d >= 2 with a multiply-high and
@@ -204,76 +173,8 @@ __device__ __forceinline__ unsigned long long ceil_p_times(uint64_t Z, uint32_t 
   return q + (rem_nz ? 1ull : 0ull);
 }
 
-// Estimate e(q) of one node, computed by a whole warp.  The lane's q slice
-// covers elements [cl*EPC, cl*EPC+EPC) with cl = lane % CPR.
-template <typename T, int D>
-__device__ __forceinline__ float score_node(const TreeDev& t, int head, uint32_t code, const float* qs,
-                                            int lane) {
-  constexpr int EPC = 16 / sizeof(T);
-  constexpr int CPR = D * sizeof(T) / 16;  // 16-byte chunks per ref row
-  constexpr int RPI = 32 / CPR;            // refs per warp pass
-  const int R = t.refs;
-  const char* rec = t.rec(code_level(code), head, code_index(code));
-  const float* bias = reinterpret_cast<const float*>(rec + size_t(R) * D * sizeof(T));
-  const int sub = lane / CPR, cl = lane % CPR;
-  float best = -INFINITY;
-  constexpr int kBatch = 8;
-  for (int j0 = 0; j0 < R; j0 += RPI * kBatch) {
-    uint4 v[kBatch];
-    float bj[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int j = j0 + u * RPI + sub;
-      if (j < R) {
-        v[u] = ldg_stream(rec + (size_t(j) * CPR + cl) * 16);
-        bj[u] = __ldg(bias + j);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int j = j0 + u * RPI + sub;
-      float part = 0.f;
-      if (j < R) {
-        float x[EPC];
-        unpack16<T>(v[u], x);
-#pragma unroll
-        for (int i = 0; i < EPC; ++i) part = fmaf(x[i], qs[i], part);
-      }
-#pragma unroll
-      for (int off = CPR / 2; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (j < R) best = fmaxf(best, fmaf(part, t.inv_sqrt_d, bj[u]));
-      if (j0 + (u + 1) * RPI >= R) break;
-    }
-  }
-#pragma unroll
-  for (int off = 16; off >= CPR; off >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
-  return best;
-}
-
 // Block-wide exclusive scan of one value per thread; returns the exclusive
 // prefix and writes the block total to *total (all threads).
-template <int NW = kDecWarps>
-__device__ __forceinline__ uint32_t block_scan_u32(uint32_t v, uint32_t* red, uint32_t* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  uint32_t x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) red[wid] = x;
-  __syncthreads();
-  uint32_t base = 0, tot = 0;
-  for (int w = 0; w < NW; ++w) {
-    const uint32_t s = red[w];
-    if (w < wid) base += s;
-    tot += s;
-  }
-  __syncthreads();
-  *total = tot;
-  return base + x - v;
-}
-
 template <int NW = kDecWarps>
 __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* red,
                                                              unsigned long long* total) {
@@ -297,17 +198,6 @@ __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long 
   return base + x - v;
 }
 
-__device__ __forceinline__ uint32_t block_min_u32(uint32_t v, uint32_t* red) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, off));
-  if (lane == 0) red[wid] = v;
-  __syncthreads();
-  uint32_t m = 0xffffffffu;
-  for (int w = 0; w < kDecWarps; ++w) m = min(m, red[w]);
-  __syncthreads();
-  return m;
-}
 
 // Distance of an entry below the maximum estimate, in fp32: x = m - e >= 0.
 // Bins over x are monotone in e (fp32 subtraction and power-of-two scaling
