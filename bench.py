@@ -258,6 +258,8 @@ def oracle_sample(w, inp, n_tokens, budget_s, q_sets):
     desc = (f"{len(per_head)} (query head, query set) decodes of KV head 0 at N={n_tokens}, oracle tree of that "
             f"head built beforehand (untimed); mean per head x {w.n_q_heads * w.batch} heads per step; "
             f"one-token append not included")
+    if w.planes != "key":
+        desc += "; the oracle routes on the unquantised slopes (its FP4 quantiser is not on this timed path)"
     return us, desc, threads
 
 

@@ -88,3 +88,30 @@ def test_sweep_crossover():
     assert x == int(round(want)) and 262144 < x < 524288
     assert bench.crossover([(1024, 1.0, 2.0), (2048, 1.0, 3.0)]) == "<= 1024"
     assert bench.crossover([(1024, 3.0, 2.0), (2048, 4.0, 3.0)]) is None
+
+
+def test_union_bytes_counts_each_group_once():
+    """Algorithmic bytes: planes scored and keys attended are counted once per (sequence, KV group)."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth.workloads import Workload
+    w = Workload("t", d=64, n_q_heads=4, n_kv_heads=2, n_tokens=1000, block=4, levels=2, n_refs=2, p=0.9,
+                 batch=1, dtype="bf16", gen="topics", seed=0)
+    # heads 0,1 share KV head 0; 2,3 share KV head 1
+    scored = np.array([[[5, 6, 7, 0], [6, 7, 8, 0], [1, 0, 0, 0], [2, 0, 0, 0]]], dtype=np.int32)
+    nscored = np.array([[3, 3, 1, 1]])
+    kept = np.array([[[0, 3, 0], [3, 4, 0], [9, 0, 0], [9, 0, 0]]], dtype=np.int32)
+    kcnt = np.array([[2, 2, 1, 1]])
+    route, attend, kph = bench.union_bytes(w, scored, nscored, kept, kcnt, 1002)
+    plane = 2 * (64 * 2 + 4)
+    assert route == (4 + 2) * plane                       # {5,6,7,8} and {1,2}
+    kv = 2 * 64 * 2
+    tail = 1002 - 250 * 4                                 # 2 tail tokens
+    # group 0: leaves {0,3,4} (block 0 kept: no extra sink); group 1: {9} + sink
+    assert attend == (3 * 4 + tail) * kv + (1 * 4 + tail + 1) * kv + 1 * 4 * 64 * (2 + 4)
+    assert kph == [2 * 4 + tail, 2 * 4 + tail + 1, 4 + tail + 1, 4 + tail + 1]
+    w4 = Workload("t4", d=64, n_q_heads=4, n_kv_heads=2, n_tokens=1000, block=4, levels=2, n_refs=2, p=0.9,
+                  batch=1, dtype="bf16", gen="topics", seed=0, planes="fp4")
+    route4, _, _ = bench.union_bytes(w4, scored, nscored, kept, kcnt, 1002)
+    assert route4 == (4 + 2) * 2 * (32 + 4 + 4)
