@@ -115,3 +115,19 @@ def test_union_bytes_counts_each_group_once():
                   batch=1, dtype="bf16", gen="topics", seed=0, planes="fp4")
     route4, _, _ = bench.union_bytes(w4, scored, nscored, kept, kcnt, 1002)
     assert route4 == (4 + 2) * 2 * (32 + 4 + 4)
+
+
+def test_traffic_figure_only_for_the_measured_kernels(tmp_path, monkeypatch):
+    """roofline.traffic is read from the ncu summary only while its workload and source hash match."""
+    sys.path.insert(0, ROOT)
+    import bench
+    f = tmp_path / "traffic.txt"
+    f.write_text(f"# comment: x\nworkload: deep256k_bf16\nsource_hash: {bench.kernel_source_hash()}\n"
+                 "dram_bytes_per_decode: 123456\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.measured_traffic("deep256k_bf16") == 123456
+    assert bench.measured_traffic("wide256k_bf16") is None
+    f.write_text("workload: deep256k_bf16\nsource_hash: 0000000000000000\ndram_bytes_per_decode: 123456\n")
+    assert bench.measured_traffic("deep256k_bf16") is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.txt"))
+    assert bench.measured_traffic("deep256k_bf16") is None
