@@ -161,8 +161,9 @@ class ZhaTree:
         for name, t in (("K", K), ("V", V)):
             if tuple(t.shape) != shape or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {shape}")
-        if tuple(refs.shape) != (cfg.n_kv_heads, cfg.n_refs, cfg.d) or refs.dtype != dt or not refs.is_contiguous():
-            raise ValueError("refs must be a contiguous tensor [Hkv, R, d] of the cache dtype")
+        if (tuple(refs.shape) != (cfg.n_kv_heads, cfg.n_refs, cfg.d) or refs.dtype != dt or not refs.is_cuda
+                or not refs.is_contiguous()):
+            raise ValueError("refs must be a contiguous CUDA tensor [Hkv, R, d] of the cache dtype")
         self.K, self.V, self.refs = K, V, refs
         nb, sb = tree_bytes(cfg)
         self.nodes = torch.zeros(nb, dtype=torch.uint8, device=K.device)
@@ -187,6 +188,13 @@ class ZhaTree:
 
     def append(self, K_new: torch.Tensor, V_new: torch.Tensor, stream=None) -> None:
         """Append tokens K_new, V_new [Hkv, m, d] (CUDA, cache dtype)."""
+        c = self.cfg
+        for name, t in (("K_new", K_new), ("V_new", V_new)):
+            if (t.dim() != 3 or t.shape[0] != c.n_kv_heads or t.shape[2] != c.d or t.dtype != TORCH_DTYPE[c.dtype]
+                    or not t.is_cuda):
+                raise ValueError(f"{name} must be a CUDA {TORCH_DTYPE[c.dtype]} tensor [{c.n_kv_heads}, m, {c.d}]")
+        if K_new.shape != V_new.shape:
+            raise ValueError("K_new and V_new must have the same shape")
         m = K_new.shape[1]
         K_new = K_new.contiguous()
         V_new = V_new.contiguous()
@@ -195,7 +203,13 @@ class ZhaTree:
     def decode(self, Q: torch.Tensor, *, want_kept: bool = False, want_stats: bool = False, out=None,
                scored_cap: int = 0, stream=None):
         """Decode queries Q [B, Hq, d].  Returns O [B, Hq, d] fp32 (and kept lists / stats when asked)."""
+        c = self.cfg
+        if Q.dim() != 3 or tuple(Q.shape[1:]) != (c.n_q_heads, c.d) or Q.dtype != TORCH_DTYPE[c.dtype] or not Q.is_cuda:
+            raise ValueError(f"Q must be a CUDA {TORCH_DTYPE[c.dtype]} tensor [B, {c.n_q_heads}, {c.d}]")
         B = Q.shape[0]
+        if out is not None and (tuple(out.shape) != (B, c.n_q_heads, c.d) or out.dtype != torch.float32
+                                or not out.is_cuda or not out.is_contiguous()):
+            raise ValueError(f"out must be a contiguous CUDA float32 tensor [{B}, {c.n_q_heads}, {c.d}]")
         Q = Q.contiguous()
         O = out if out is not None else torch.empty(B, self.cfg.n_q_heads, self.cfg.d, dtype=torch.float32,
                                                     device=Q.device)
