@@ -505,6 +505,14 @@ def run_zha(args, world, rank, local):
         us, desc, threads = oracle_sample(w, inp, n0, args.cpu_seconds, w.n_query_sets)
         res["cpu_baseline"] = {"value": round(us, 1), "unit": "us", "cores": threads, "kind": "oracle",
                                "sample": desc}
+        try:  # the same sample on one host thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                us1, desc1, _ = oracle_sample(w, inp, n0, min(args.cpu_seconds, 6.0), w.n_query_sets)
+            res["cpu_baseline_1t"] = {"value": round(us1, 1), "unit": "us", "cores": 1, "kind": "oracle",
+                                      "sample": desc1}
+        except ImportError:
+            pass
     if rank == 0:
         print(json.dumps(res), flush=True)
     del tree
