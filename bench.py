@@ -17,7 +17,7 @@ before every step (a 2x L2-sized write outside the timed events), warm-up
 steps untimed, max over ranks.  Algorithmic bytes of the decode call are
 counted from the nodes each query head scored and the keys it attended,
 taking the union over each GQA group (the bytes the method has to move), on
-an untimed repeat of every timed decode.  With --gpus N > 1 every rank runs
+untimed repeats of the timed decodes (one per query set).  With --gpus N > 1 every rank runs
 an independent replica (the path does not shard across GPUs here).
 """
 from __future__ import annotations
