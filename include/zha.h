@@ -29,8 +29,8 @@
  *   - Return value: ZHA_OK (0) or a negative ZHA_ERR_* code.  Nothing throws
  *     across the ABI; zha_last_error() gives a thread-local message for the
  *     last failing call on the calling thread.  Device-side faults that the
- *     kernels detect (a capacity bound that would be exceeded) set a status
- *     word that zha_tree_status() returns.
+ *     kernels detect (a capacity bound that would be exceeded, a bounded wait
+ *     that ran out) set a status word that zha_tree_status() returns.
  *   - Element types: ZHA_F32 stores K, V, Q, refs and the node slopes (mu) as
  *     fp32; ZHA_BF16 stores them as bf16 (round-to-nearest-even).  Node values
  *     f and intercepts b are always fp32, all arithmetic accumulates in fp32,
@@ -58,7 +58,7 @@ enum {
   ZHA_ERR_CAPACITY = -2,    /* more tokens / batch than the tree was created for */
   ZHA_ERR_UNSUPPORTED = -3, /* head dim not 64/128, block < 2, levels < 1, n_refs > 32 ... */
   ZHA_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
-  ZHA_ERR_TIMEOUT = -5      /* reserved: a bounded device-side wait gave up */
+  ZHA_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up (reported through the status word) */
 };
 
 enum { ZHA_F32 = 0, ZHA_BF16 = 1 };
