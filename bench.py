@@ -263,6 +263,47 @@ def oracle_sample(w, inp, n_tokens, budget_s, q_sets):
     return us, desc, threads
 
 
+def parity_sample(w, inp, tree, Qs, runs):
+    """Parity of the timed path on a bounded sample (KV head 0's query heads, the first timed query sets, on
+    the final tree), outside the timed region: the oracle's route on the GPU-stored planes (exact heads and
+    heads excused at a boundary of the cut), the oracle's attention on the GPU's kept blocks, and the whole
+    path against the oracle's own tree built in fp64 from the raw keys (kept-set Jaccard, output error)."""
+    import oracle.zha_oracle as zo
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity_helpers import compare_route, end_to_end, f64, oracle_attend_on_sets
+
+    t0 = time.perf_counter()
+    n = tree.size
+    p = float(np.float32(w.p))
+    heads = list(range(w.group))  # the query heads of KV head 0
+    otree = zo.build_tree(f64(inp.K[0, :n]), f64(inp.refs[0]), n, w.block, w.levels)
+    out = {"sample": f"query heads 0-{w.group - 1} (KV head 0), batch element 0, query sets "
+                     f"{[r[0] for r in runs]}, N={n}", "heads": 0, "exact": 0, "flagged": 0, "failed": 0}
+    jac, err, err_m, att = [], [], [], 0.0
+    for qi, O, kept, cnt in runs:
+        Q = Qs[qi].cpu()
+        rep = compare_route(tree, Q, kept, cnt, p, n, w.block, w.levels, w.group, heads=heads)
+        out["heads"] += rep.heads
+        out["exact"] += rep.exact
+        out["flagged"] += rep.flagged
+        out["failed"] += len(rep.failures)
+        ref = oracle_attend_on_sets(inp.K, inp.V, Q[:1], kept[:1], cnt[:1], n, w.block, w.group, heads=heads)
+        att = max(att, float(np.abs(O[0, heads].numpy() - ref[0, heads]).max()))
+        e2e = end_to_end(inp.K, inp.V, inp.refs, Q, O, kept, cnt, n, w.block, w.levels, p, w.group, 0, (0,),
+                         oracle_tree=otree)
+        jac += e2e.jaccard
+        err += e2e.err
+        err_m += e2e.err_matched
+    out["attend_max_abs_err"] = att
+    out["e2e_jaccard"] = round(float(np.mean(jac)), 5) if jac else None
+    out["e2e_jaccard_min"] = round(float(np.min(jac)), 5) if jac else None
+    out["e2e_matched_sets"] = len(err_m)
+    out["max_abs_err"] = float(np.max(err)) if err else None
+    out["max_abs_err_matched"] = float(np.max(err_m)) if err_m else None
+    out["seconds"] = round(time.perf_counter() - t0, 1)
+    return out
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -382,7 +423,6 @@ def run_zha(args, world, rank, local):
     tree.status()
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    scored_cap = 1 << 16
     route_b, attend_b, keys_ph = [], [], []
     launches0 = z.launch_count()
     barrier(world)
@@ -400,18 +440,27 @@ def run_zha(args, world, rank, local):
     dec_ms = [ev[1].elapsed_time(ev[2]) for ev in events]
     app_ms = [ev[0].elapsed_time(ev[1]) for ev in events]
 
-    # untimed repeat of each timed decode's query on the final tree for the byte counts
+    # untimed repeat of each timed decode's query on the final tree for the byte counts; the scored-node
+    # export is sized from the heads' own counters (a first decode with the counters alone)
     n_final = tree.size
+    parity_runs = []  # (query set, O, kept, cnt) of the first repeats, for the oracle's parity sample
     for i in range(min(args.steps, w.n_query_sets)):
-        q = Qs[(args.warmup + i) % w.n_query_sets]
-        _, (kept, cnt), stats, scored = tree.decode(q, want_kept=True, want_stats=True, scored_cap=scored_cap)
+        qi = (args.warmup + i) % w.n_query_sets
+        q = Qs[qi]
+        _, st0 = tree.decode(q, want_stats=True)
         torch.cuda.synchronize(dev)
+        scored_cap = max(1, int(st0[..., z.STAT_NODES_SCORED].max()))
+        O_i, (kept, cnt), stats, scored = tree.decode(q, want_kept=True, want_stats=True, scored_cap=scored_cap)
+        torch.cuda.synchronize(dev)
+        assert int(stats[..., z.STAT_NODES_SCORED].max()) <= scored_cap
         mk = max(1, int(cnt.max()))
         rb, ab, kph = union_bytes(w, scored.cpu().numpy(), stats[..., 0].cpu().numpy(), kept[..., :mk].cpu().numpy(),
                                   cnt.cpu().numpy(), n_final)
         route_b.append(rb)
         attend_b.append(ab)
         keys_ph.extend(kph)
+        if len(parity_runs) < 2:
+            parity_runs.append((qi, O_i.cpu(), kept.cpu(), cnt.cpu()))
     alg_bytes = statistics.mean(route_b) + statistics.mean(attend_b)
 
     # end to end through the C ABI with pinned host buffers (copies inside the timed region)
@@ -502,10 +551,14 @@ def run_zha(args, world, rank, local):
         "gpu_launches": launches,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle leg: the CPU baseline timing, then the parity sample (untimed, after the GPU timing)
         us, desc, threads = oracle_sample(w, inp, n0, args.cpu_seconds, w.n_query_sets)
-        res["cpu_baseline"] = {"value": round(us, 1), "unit": "us", "cores": threads, "kind": "oracle",
-                               "sample": desc}
-        try:  # the same sample on one host thread
+        res["cpu_baseline"] = {"value": round(us, 1), "unit": "us", "cores": 1, "kind": "oracle",
+                               "sample": desc + f"; effectively one thread: the oracle's route is a Python loop "
+                                               f"(numpy's BLAS pool has {threads} threads; the one-thread run "
+                                               f"below takes the same time)",
+                               "blas_threads": threads}
+        try:  # the same sample with the BLAS pool limited to one thread
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
                 us1, desc1, _ = oracle_sample(w, inp, n0, min(args.cpu_seconds, 6.0), w.n_query_sets)
@@ -513,6 +566,7 @@ def run_zha(args, world, rank, local):
                                       "sample": desc1}
         except ImportError:
             pass
+        res["parity"] = parity_sample(w, inp, tree, Qs, parity_runs)
     if rank == 0:
         print(json.dumps(res), flush=True)
     del tree

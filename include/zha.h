@@ -208,10 +208,13 @@ ZHA_API int zha_decode_step_host(zha_tree* tree, const void* k_host, const void*
  * queries over tokens [0, n) of K, V (the in-run comparator; no tree).
  *   K, V   - [Hkv][ld][d] element type (ld = row stride in tokens >= n).
  *   Q      - [B][Hq][d]; O - [B][Hq][d] fp32.
- *   scratch - zha_dense_scratch_bytes(cfg, B, n) bytes (0 for an invalid request),
- *            zero-filled before the first call; each call leaves its completion
- *            counters zero-filled again, so one scratch serves any later call with
- *            B' <= B and n' <= n.  B <= cfg->max_batch.
+ *   scratch - at least zha_dense_scratch_bytes(cfg, B, n) bytes (0 for an invalid
+ *            request): the split partials of every call with B' <= B sequences
+ *            and n' <= n tokens fit in it, so one scratch serves all such calls.
+ *            Its contents need no initialisation; each call writes the partials
+ *            it reads.  B <= cfg->max_batch.  A smaller scratch is not detected
+ *            (the call takes no size): the caller must size it with this
+ *            function.
  */
 ZHA_API size_t zha_dense_scratch_bytes(const zha_config* cfg, int32_t B, int64_t n);
 ZHA_API int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n,

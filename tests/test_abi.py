@@ -151,3 +151,30 @@ def test_binding_refuses_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(zb, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         zb.lib()
+
+
+def _dense_plan(B, hkv, n):
+    """The dense decode's split plan (zha_dense.cu, dense_plan): about four CTAs per SM of 148, splits of a
+    multiple of 64 keys."""
+    s = (148 * 4 + B * hkv - 1) // (B * hkv)
+    s = max(1, min(s, (n + 63) // 64))
+    per = max(64, ((n + s - 1) // s + 63) // 64 * 64)
+    return max(1, (n + per - 1) // per)
+
+
+@pytest.mark.parametrize("hkv,hq,d,B,n", [(1, 8, 128, 1, 37915), (4, 32, 128, 1, 262144), (2, 16, 64, 3, 5003),
+                                          (1, 1, 64, 1, 130)])
+def test_dense_scratch_covers_every_smaller_call(built, hkv, hq, d, B, n):
+    """One scratch of zha_dense_scratch_bytes(B, n) holds the split partials of every call with B' <= B and
+    n' <= n, although the split count itself is not monotone in n."""
+    c = cfg(d=d, n_q_heads=hq, n_kv_heads=hkv, levels=1, n_refs=1, capacity=max(n, 64), max_batch=B)
+    have = z.dense_scratch_bytes(c, B, n)
+    assert have > 0
+    worst = 0
+    for b in range(1, B + 1):
+        for m in list(range(1, min(n, 2048) + 1)) + list(range(max(1, n - 4096), n + 1)):
+            worst = max(worst, b * hq * _dense_plan(b, hkv, m) * (d + 2) * 4)
+    assert worst <= have, (worst, have)
+    # the advisor's case: the plan at n is smaller than at a shorter length
+    if (hkv, B, n) == (1, 1, 37915):
+        assert _dense_plan(1, 1, 37915) < _dense_plan(1, 1, 37851)

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle.zha_oracle as zo
-from parity_helpers import assert_close_out, compare_planes, compare_route, f64, oracle_attend_on_sets, p32
+from parity_helpers import (assert_close_out, compare_planes, compare_route, end_to_end, f64, oracle_attend_on_sets,
+                            p32)
 from synth.workloads import generate, workload
 
 pytestmark = pytest.mark.gpu
@@ -77,21 +78,55 @@ def _check_decode(w, inp, tree, Q):
     n = tree.size
     group = w.n_q_heads // w.n_kv_heads
     rep = compare_route(tree, Q, kept, cnt, p32(w.p), n, w.block, w.levels, group)
+    print(f"route at N={n}: {rep.summary()}")
     assert not rep.failures, "\n".join(rep.failures[:5])
-    assert rep.flagged <= 0.2 * rep.heads + 1, (rep.flagged, rep.heads)
+    # boundary cases are rare on this workload: at most one excused head per query set
+    assert rep.flagged <= 1, rep.summary()
     ref = oracle_attend_on_sets(inp.K, inp.V, Q, kept, cnt, n, w.block, group)
     atol = 2e-5 * float(inp.V[:, :n].abs().max()) + 1e-6
     assert_close_out(O.cpu().numpy(), ref, atol, f"attend at N={n}")
     assert torch.equal(stats.cpu()[..., 1], cnt.cpu().long())
-    return rep
+    return rep, O, kept, cnt
 
 
 def test_route_attend_full_size(deep256k):
     w, inp, tree = deep256k
     Qs = inp.Q.cuda()
     for s in (0, 5, 11):
-        rep = _check_decode(w, inp, tree, Qs[s])
+        rep, *_ = _check_decode(w, inp, tree, Qs[s])
         print(f"query set {s}: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+
+
+E2E_JACCARD_MEAN = 0.97   # bf16 rounding of the stored slopes moves a few cuts (fp64 simulation: 0.991 mean)
+E2E_JACCARD_MIN = 0.85    # (simulation: 0.915 worst head)
+E2E_ERR = 0.25            # output error when a cut moved: a different attended set, not an arithmetic error
+E2E_ERR_MATCHED = 2e-2    # the bf16 output tolerance, for heads whose sets match
+
+
+def check_end_to_end(rep, label):
+    s = rep.summary()
+    print(f"end to end {label}: {s}")
+    assert s["jaccard_mean"] >= E2E_JACCARD_MEAN, s
+    assert s["jaccard_min"] >= E2E_JACCARD_MIN, s
+    assert s["max_abs_err_matched"] <= E2E_ERR_MATCHED, s
+    assert s["max_abs_err"] <= E2E_ERR, s
+
+
+def test_end_to_end_against_oracle_tree(deep256k):
+    """The whole path against the oracle's own tree (fp64 planes from the raw keys) for the eight query heads
+    of KV head 0 and three query sets: kept-set Jaccard and output error."""
+    w, inp, tree = deep256k
+    n = tree.size
+    Kh = f64(inp.K[0, :n])
+    otree = zo.build_tree(Kh, f64(inp.refs[0]), n, w.block, w.levels)
+    for s in (0, 7, 15):
+        Q = inp.Q[s].cuda()
+        O, (kept, cnt) = tree.decode(Q, want_kept=True)
+        torch.cuda.synchronize()
+        tree.status()
+        rep = end_to_end(inp.K, inp.V, inp.refs, Q.cpu(), O, kept, cnt, n, w.block, w.levels, p32(w.p), w.group, 0,
+                         range(Q.shape[0]), oracle_tree=otree)
+        check_end_to_end(rep, f"query set {s}")
 
 
 def test_append_then_decode_full_size(deep256k):

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle.zha_oracle as zo
-from parity_helpers import assert_close_out, compare_planes, compare_route, f64, p32
+from parity_helpers import assert_close_out, compare_planes, compare_route, end_to_end, f64, p32
 from synth.workloads import generate, workload
 
 pytestmark = pytest.mark.gpu
@@ -70,8 +70,9 @@ def _check_decode(w, inp, tree, Q, attend_heads):
     n = tree.size
     group = w.n_q_heads // w.n_kv_heads
     rep = compare_route(tree, Q, kept, cnt, p32(w.p), n, w.block, w.levels, group)
+    print(f"route at N={n}: {rep.summary()}")
     assert not rep.failures, "\n".join(rep.failures[:5])
-    assert rep.flagged <= 0.2 * rep.heads + 1, (rep.flagged, rep.heads)
+    assert rep.flagged <= max(1, rep.heads // 64), rep.summary()
     kept, cnt = kept.cpu(), cnt.cpu()
     vmax = 0.0
     for bb, h in attend_heads:
@@ -83,7 +84,7 @@ def _check_decode(w, inp, tree, Q, attend_heads):
         ref = zo.attend(Ks, Vs, f64(Q[bb, h]), np.arange(len(toks)))
         assert_close_out(O[bb, h].cpu().numpy()[None], ref[None], 2e-5 * float(inp.V[kvh].abs().max()) + 1e-6,
                          f"attend seq {bb} head {h}")
-    return rep
+    return rep, O, kept, cnt
 
 
 def test_build_append_batched_decode_1m():
@@ -98,8 +99,16 @@ def test_build_append_batched_decode_1m():
     _check_nodes(w, inp, tree, kvh=1, per_level=12, seed=3)
     Q = inp.Q[0].cuda()
     heads = [(bb, h) for bb in (0, 7, 15) for h in (0, 9, 18, 31)]
-    rep = _check_decode(w, inp, tree, Q, heads)
+    rep, O, kept, cnt = _check_decode(w, inp, tree, Q, heads)
     print(f"1M batch 16: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")
+    # the whole path against the oracle's own tree of KV head 0 (fp64 planes from the raw keys, including the
+    # appended block), for three of the sixteen sequences
+    e2e = end_to_end(inp.K, inp.V, inp.refs, inp.Q[0], O, kept, cnt, n0, w.block, w.levels, p32(w.p), w.group, 0,
+                     (0, 7, 15))
+    s = e2e.summary()
+    print(f"end to end 1M: {s}")
+    assert s["jaccard_mean"] >= 0.97 and s["jaccard_min"] >= 0.85, s
+    assert s["max_abs_err_matched"] <= 2e-2 and s["max_abs_err"] <= 0.25, s
 
 
 @pytest.mark.skipif(not torch.cuda.is_available() or _host_memory_gb() < 48,
@@ -110,5 +119,5 @@ def test_light_sweep_4m():
     tree = _tree(w, inp, w.n_tokens, w.n_tokens)
     _check_nodes(w, inp, tree, kvh=0, per_level=8, seed=5)
     Q = inp.Q[0].cuda()
-    rep = _check_decode(w, inp, tree, Q, [(0, h) for h in (0, 3, 5, 8)])
+    rep, *_ = _check_decode(w, inp, tree, Q, [(0, h) for h in (0, 3, 5, 8)])
     print(f"4M sweep: {rep.exact}/{rep.heads} exact, {rep.flagged} flagged")

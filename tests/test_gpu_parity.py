@@ -73,6 +73,7 @@ def check_build(case: Case):
 def check_decode(case: Case, Q, allow_flagged_frac=0.2):
     O, kept, cnt, stats = case.decode(Q)
     rep = compare_route(case.tree, Q, kept, cnt, p32(case.p), case.n, case.block, case.levels, case.group)
+    print(f"route: {rep.summary()}")
     assert not rep.failures, "\n".join(rep.failures[:5])
     assert rep.flagged <= allow_flagged_frac * rep.heads + 1, (rep.flagged, rep.heads)
     ref = oracle_attend_on_sets(case.Kall, case.Vall, Q, kept, cnt, case.n, case.block, case.group)
@@ -101,9 +102,11 @@ def test_dense_decode(dtype, d, hq, hkv, n):
         G = hq // hkv
         ref = np.stack([[zo.dense(f64(K[h // G]), f64(V[h // G]), f64(Q[b, h]), n) for h in range(hq)]
                         for b in range(3)])
-        # bf16 P in the tensor-core path rounds each softmax weight to 8 bits
-        atol = (2e-2 if dtype == "bf16" else 2e-5) * max(1.0, float(V.abs().max()))
+        # bf16: the stated bound of 2e-2 absolute (the tensor-core path keeps the weights as hi + lo bf16
+        # parts, so its error is far below it); fp32: 2e-5 of the value scale, tighter than 1e-4 relative
+        atol = 2e-2 if dtype == "bf16" else 2e-5 * max(1.0, float(V.abs().max()))
         assert_close_out(O.cpu().numpy(), ref, atol, f"dense {dtype} d={d} n={n}")
+        print(f"dense {dtype} d={d} n={n}: max abs err {np.abs(O.cpu().numpy() - ref).max():.2e}")
 
 
 # ------------------------------------------------------------------ build

@@ -8,7 +8,6 @@ ordinary entry point (caller-provided scratch) on two calls in a row.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -33,17 +32,13 @@ def test_noalloc_matches_caller_scratch(dtype, d, hq, hkv, n, B):
                         capacity=n, max_batch=B)
     ref = z.DenseDecoder(cfg, B, n)(Kc, Vc, n, Qc)
     torch.cuda.synchronize()
-    # the tolerance of the dense-decode parity tests (bf16 softmax weights in the tensor-core path)
-    atol = (2e-2 if dtype == "bf16" else 2e-5) * max(1.0, float(V.abs().max()))
-    outs = []
+    # the same kernels with the same split plan run on both paths; only where the partials live differs,
+    # so the outputs must be identical bit for bit (the oracle comparison is test_dense_decode's)
     for _ in range(2):
         O = torch.full((B, hq, d), float("nan"), dtype=torch.float32, device="cuda")
         assert _call_noalloc(z, cfg, Kc, Vc, n, Qc, O) == 0, z.lib().zha_last_error()
         torch.cuda.synchronize()
-        assert torch.isfinite(O).all()
-        assert np.abs(O.cpu().numpy() - ref.cpu().numpy()).max() <= atol
-        outs.append(O.cpu())
-    assert torch.equal(outs[0], outs[1])
+        assert torch.equal(O, ref)
 
 
 def test_noalloc_rejects_requests_beyond_the_fixed_scratch():

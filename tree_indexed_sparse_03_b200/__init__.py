@@ -5,5 +5,6 @@ this package only marshals arguments to it.
 """
 from .zha import (  # noqa: F401
     DenseDecoder, LevelLayout, ZhaConfig, ZhaError, ZhaTree, dense_decode, dense_scratch_bytes, lib,
-    make_config, tree_bytes, tree_layout, launch_count, LIB_PATH, ZHA_BF16, ZHA_F32,
+    make_config, tree_bytes, tree_layout, launch_count, LIB_PATH, ZHA_BF16, ZHA_F32, STAT_NODES_SCORED,
+    STAT_LEAVES_KEPT, STAT_KEYS, STAT_STEPS,
 )

@@ -22,6 +22,7 @@ uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list);
 int decode_max_heads();
 uint64_t decode_part_items(int nheads);
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per);
+int dense_target_splits();
 size_t dense_static_floats();
 cudaError_t dense_static_scratch(float** out);
 }  // namespace zha
@@ -138,8 +139,8 @@ int make_layout(const zha_config* c, Layout* L) {
     }
   }
   L->node_bytes = off > 0 ? off : 256;
-  // scratch: status word and grid barrier, attend partials, per (sequence,
-  // query head) routing workspace, host-step staging
+  // scratch: status word, attend partials, per (sequence, query head)
+  // routing state and workspace, host-step staging
   L->status_off = 0;
   const int64_t n1cap = L->cap_nodes[1] > 0 ? L->cap_nodes[1] : 1;
   L->cap_sel = n1cap;
@@ -420,13 +421,21 @@ int zha_decode_step_host(zha_tree* t, const void* k_host, const void* v_host, co
   return ZHA_OK;
 }
 
+// Split partials of any dense decode with B' <= B sequences over n' <= n tokens.  dense_plan gives
+// splits' <= min(ceil(X / B'), ceil(n' / 64)) with X = ceil(dense_target / Hkv) (its split count is not
+// monotone in n, so the bound is taken over the plan's caps, not over one plan): B' * ceil(X / B') <=
+// X + B' - 1 <= X + B - 1, and B' * ceil(n' / 64) <= B * ceil(n / 64).
+static uint64_t dense_part_floats_bound(const zha_config* cfg, int32_t B, int64_t n) {
+  const uint64_t X = (uint64_t(dense_target_splits()) + cfg->n_kv_heads - 1) / cfg->n_kv_heads;
+  const uint64_t by_target = X + uint64_t(B) - 1;
+  const uint64_t by_len = uint64_t(B) * uint64_t((n + 63) / 64);
+  const uint64_t seq_splits = by_target < by_len ? by_target : by_len;  // bound on B' * splits'
+  return uint64_t(cfg->n_q_heads) * seq_splits * uint64_t(cfg->d + 2);
+}
+
 size_t zha_dense_scratch_bytes(const zha_config* cfg, int32_t B, int64_t n) {
   if (validate(cfg) || B < 1 || n < 1 || B > cfg->max_batch) return 0;
-  int splits;
-  int64_t per;
-  dense_plan(B, cfg->n_kv_heads, n, &splits, &per);
-  const uint64_t part = uint64_t(B) * cfg->n_q_heads * splits * (cfg->d + 2) * 4;
-  return size_t(align256(part));
+  return size_t(align256(dense_part_floats_bound(cfg, B, n) * 4));
 }
 
 int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_t ld, int64_t n, const void* Q,
@@ -443,12 +452,10 @@ int zha_dense_decode(const zha_config* cfg, const void* K, const void* V, int64_
   DenseArgs a;
   std::memset(&a, 0, sizeof(a));
   dense_plan(B, cfg->n_kv_heads, n, &a.splits, &a.per);
-  const uint64_t part = uint64_t(B) * cfg->n_q_heads * a.splits * (cfg->d + 2) * 4;
   a.K = K;
   a.V = V;
   a.Q = Q;
   a.O = O;
-  (void)part;
   a.part = static_cast<float*>(scratch);
   a.ld = ld;
   a.n = n;
@@ -521,8 +528,15 @@ int zha_tree_status(zha_tree* t, void* stream) {
   if (status != 0) {
     const int zero = 0;
     cudaMemcpy(t->dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
-    t->flow_dirty = true;  // a kernel that gave up may have left its flow state and barrier mid-way
-    return fail(status, "a kernel raised an error status (capacity bound exceeded)");
+    t->flow_dirty = true;  // a kernel that gave up may have left the routing state mid-way
+    switch (status) {
+      case ZHA_ERR_CAPACITY:
+        return fail(status, "a kernel raised ZHA_ERR_CAPACITY (a capacity bound would have been exceeded)");
+      case ZHA_ERR_TIMEOUT:
+        return fail(status, "a kernel raised ZHA_ERR_TIMEOUT (a bounded wait on a copy ran out)");
+      default:
+        return fail(status, "a kernel raised an unknown error status");
+    }
   }
   return ZHA_OK;
 }

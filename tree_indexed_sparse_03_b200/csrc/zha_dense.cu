@@ -11,7 +11,8 @@
 // K/V byte is read once for all of them.  Per 16-key tile a warp computes
 // S^T = K Q^T with mma.sync m16n8k16 (keys x heads) and O^T += V^T P with the
 // same instruction (head dim x heads), P moved from the accumulator layout to
-// the operand layout with movmatrix.  K and V are loaded straight from global
+// the operand layout with movmatrix and split into hi + lo bf16 parts (two
+// products, so the weights keep about 16 bits instead of 8).  K and V are loaded straight from global
 // memory into registers with 16-byte loads; the head dimension is permuted
 // consistently between the operands so that every fragment is whole 32-bit
 // words of those loads.  The work is HBM-bound (about 4 flop per byte at 8
@@ -157,8 +158,13 @@ __global__ void __launch_bounds__(kDenseThreads) dense_mma_kernel(DenseArgs a) {
         o[i][2 + hh] *= sc;
       }
     }
-    // P (keys x heads) -> B operand (keys x heads, column-major) via transpose
+    // P (keys x heads) -> B operand (keys x heads, column-major) via transpose, as hi + lo bf16 parts
+    // (two products), so that the rounding of the weights stays near fp32 instead of 2^-8
+    float plo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) plo[i] = p[i] - __bfloat162float(__float2bfloat16_rn(p[i]));
     const uint32_t pb[2] = {movmatrix_trans(pack_bf16(p[0], p[1])), movmatrix_trans(pack_bf16(p[2], p[3]))};
+    const uint32_t pl[2] = {movmatrix_trans(pack_bf16(plo[0], plo[1])), movmatrix_trans(pack_bf16(plo[2], plo[3]))};
     // O^T += V^T P
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
@@ -181,6 +187,7 @@ __global__ void __launch_bounds__(kDenseThreads) dense_mma_kernel(DenseArgs a) {
         af[3] = __byte_perm(word_of(vr[2][0], w1), word_of(vr[3][0], w1), sel);
       }
       mma_bf16_16816(o[i], af, pb);
+      mma_bf16_16816(o[i], af, pl);
     }
   }
   // reduce l over the 8 lanes that share t4
@@ -328,8 +335,10 @@ cudaError_t dense_static_scratch(float** out) {
 }
 
 // ------------------------------------------------------------------ host side
+int dense_target_splits() { return 148 * 4; }  // four CTAs per SM of a B200
+
 void dense_plan(int B, int hkv, int64_t n, int* splits, int64_t* per) {
-  const int target = 148 * 4;  // four CTAs per SM
+  const int target = dense_target_splits();
   int64_t s = (target + int64_t(B) * hkv - 1) / (int64_t(B) * hkv);
   const int64_t max_s = (n + 63) / 64;
   if (s > max_s) s = max_s;

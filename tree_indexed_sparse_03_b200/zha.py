@@ -133,24 +133,6 @@ def tree_layout_fp4(cfg: ZhaConfig, level: int) -> Tuple[int, int]:
     return ro.value, rb.value
 
 
-E2M1_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
-
-
-def e2m1_value(codes: torch.Tensor) -> torch.Tensor:
-    """Values of 4-bit e2m1 codes (uint8 tensor of codes 0..15), fp32."""
-    tab = torch.tensor(E2M1_VALUES, dtype=torch.float32, device=codes.device)
-    v = tab[(codes & 7).long()]
-    return torch.where((codes & 8) != 0, -v, v)
-
-
-def e4m3_value(bits: torch.Tensor) -> torch.Tensor:
-    """Values of e4m3 bytes (finite encodings), fp32."""
-    b = bits.long()
-    e, m = (b >> 3) & 15, (b & 7).to(torch.float32)
-    mag = torch.where(e == 0, torch.ldexp(m, torch.full_like(e, -9)), torch.ldexp(1.0 + m / 8.0, e - 7))
-    return torch.where((b & 128) != 0, -mag, mag)
-
-
 class ZhaTree:
     """A tree over a caller-owned KV cache K, V [Hkv, capacity, d] (CUDA tensors)."""
 
@@ -282,16 +264,6 @@ class ZhaTree:
         b0 = R * (D // 2 + D // 16)
         bias = rec[..., b0: b0 + 4 * R].contiguous().view(torch.float32)
         return codes, scales, bias
-
-    def router_planes(self, level: int):
-        """The planes the routing steps read: (mu [Hkv, cap, R, d], bias [Hkv, cap, R] fp32); for FP4 router
-        planes mu = code * scale (exact)."""
-        if self.cfg.planes != ZHA_PLANES_FP4:
-            mu, bias, _ = self.level_planes(level)
-            return mu, bias
-        codes, scales, bias = self.fp4_records(level)
-        sc = e4m3_value(scales).repeat_interleave(16, dim=-1)
-        return e2m1_value(codes) * sc, bias
 
 
 def launch_count() -> int:
