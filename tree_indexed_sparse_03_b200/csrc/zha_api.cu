@@ -381,6 +381,7 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
   DecodeArgs a;
   fill_decode_args(t, Q, O, kept, kept_cnt, stats, scored, scored_cap, &a);
   a.nheads = B * t->cfg.n_q_heads;
+  a.max_heads = t->cfg.max_batch * t->cfg.n_q_heads;
   cudaError_t e = launch_decode(a, t->cfg.dtype, st);
   if (e != cudaSuccess) {
     tm->flow_dirty = true;

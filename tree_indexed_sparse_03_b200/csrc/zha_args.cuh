@@ -13,7 +13,8 @@ struct DecodeArgs {
   int64_t n_tokens;
   int64_t nl[kMaxLevels + 1];   // complete nodes per level (nl[0] = tokens)
   int n_roots, n_steps;
-  int nheads;                   // sequences x query heads
+  int nheads;                   // sequences x query heads of this call
+  int max_heads;                // max_batch x query heads: the layout of the per-head scratch regions
   char* ws;                     // per-head workspaces, ws_per_bh bytes each
   uint64_t ws_per_bh;
   int64_t cap_sel;              // entries per step buffer (and kept parents)

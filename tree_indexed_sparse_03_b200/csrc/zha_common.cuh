@@ -12,6 +12,7 @@ namespace zha {
 
 constexpr int kMaxLevels = 20;   // b >= 2 and capacity < 2^31 keep L well below this
 constexpr int kMaxRefs = 32;
+constexpr int kMaxDevices = 128;  // CUDA devices a process can address (per-device state of the library)
 
 // ---------------------------------------------------------------- element types
 template <typename T> struct Elem;

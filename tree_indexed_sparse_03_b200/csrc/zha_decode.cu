@@ -42,6 +42,7 @@
 //           writes a head's last partial combines the head's partials -> O.
 // The only waits inside a kernel are a scoring warp's waits for its own bulk
 // copies; they are bounded (on running out the kernel raises ZHA_ERR_TIMEOUT).
+#include <mutex>
 #include <type_traits>
 
 #include "zha_args.cuh"
@@ -63,7 +64,7 @@ constexpr int kBins = 1024;
 constexpr float kBinScale = 32.f;
 constexpr int kMaxHeads = 1024;                    // sequences x query heads per call
 constexpr int kMaxSlots = 8;                       // score ring slots per warp
-constexpr long long kDrainLimit = 1ll << 22;       // bound of the wait for copies in flight after a timeout
+constexpr long long kDrainLimit = 1ll << 30;       // bound of the wait for copies in flight after a timeout
 constexpr int kAttThreads = 256;                   // threads of an attention CTA
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttItems = 32;                      // attend chunks a CTA owns at most
@@ -217,6 +218,22 @@ __device__ __forceinline__ unsigned long long entry_mass(float m, uint32_t key) 
   return __float2ull_rn(w * 1099511627776.0f);  // 2^40
 }
 
+// Shared-memory atomics addressed in the shared window.  The select code
+// reaches its shared arrays through references, which the compiler treats as
+// generic addresses; a generic 64-bit atomic that collides takes a very slow
+// path, so the shared-space forms are issued explicitly.
+__device__ __forceinline__ void smem_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(unsigned(__cvta_generic_to_shared(p))), "l"(v) : "memory");
+}
+__device__ __forceinline__ int smem_inc(int* p) {
+  int r;
+  asm volatile("atom.shared.add.u32 %0, [%1], 1;" : "=r"(r) : "r"(unsigned(__cvta_generic_to_shared(p))) : "memory");
+  return r;
+}
+__device__ __forceinline__ void smem_max_s32(int* p, int v) {
+  asm volatile("red.shared.max.s32 [%0], %1;" ::"r"(unsigned(__cvta_generic_to_shared(p))), "r"(v) : "memory");
+}
+
 // Add mass w to shared-memory histogram bin `bin` for every lane of
 // the warp (bin < 0: nothing).  Lanes holding consecutive entries usually share
 // a bin (siblings sit next to each other in a step's candidate list), so the
@@ -232,13 +249,13 @@ __device__ __forceinline__ void hist_add_warp(unsigned long long* hist, int bin,
   const unsigned lo = unsigned(w & 0xfffffull), hi = unsigned(w >> 20);
   const unsigned lo0 = __reduce_add_sync(0xffffffffu, in0 ? lo : 0u);
   const unsigned hi0 = __reduce_add_sync(0xffffffffu, in0 ? hi : 0u);
-  if (lane == 0 && b0 >= 0) atomicAdd(&hist[b0], (unsigned long long)lo0 + ((unsigned long long)hi0 << 20));
+  if (lane == 0 && b0 >= 0) smem_add_u64(&hist[b0], (unsigned long long)lo0 + ((unsigned long long)hi0 << 20));
   if (b1 != b0) {
     const unsigned lo1 = __reduce_add_sync(0xffffffffu, in1 ? lo : 0u);
     const unsigned hi1 = __reduce_add_sync(0xffffffffu, in1 ? hi : 0u);
-    if (lane == 31 && b1 >= 0) atomicAdd(&hist[b1], (unsigned long long)lo1 + ((unsigned long long)hi1 << 20));
+    if (lane == 31 && b1 >= 0) smem_add_u64(&hist[b1], (unsigned long long)lo1 + ((unsigned long long)hi1 << 20));
   }
-  if (!in0 && !in1 && bin >= 0) atomicAdd(&hist[bin], w);
+  if (!in0 && !in1 && bin >= 0) smem_add_u64(&hist[bin], w);
 }
 
 // Over kBins mass bins (shared memory), find the bin where the running mass,
@@ -428,7 +445,7 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   for (int i = tid; i < n32; i += kDecThreads) {
     const uint32_t k = E.key(i);
     if (in_cut(k)) {
-      const int s = atomicAdd(&sm.bcast32[1], 1);
+      const int s = smem_inc(&sm.bcast32[1]);
       if (s < 32) {
         sm.cut_key[s] = entry_key64(a, Entry{k, E.code(i)});
         sm.cut_w[s] = entry_mass(m, k);
@@ -481,7 +498,7 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
       if (!in_cut(k)) continue;
       const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
-      atomicAdd(&sm.hist[(k64 >> shift) & 255], entry_mass(m, k));
+      smem_add_u64(&sm.hist[(k64 >> shift) & 255], entry_mass(m, k));
     }
     __syncthreads();
     if (tid < 32) {
@@ -694,17 +711,20 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
       for (int u = 0; u < 4; ++u) k[u] = i0 + u < n32 ? E.key(i0 + u) : 0xffffffffu;
     }
   };
-  for (int i0 = 4 * tid; i0 < n32; i0 += 4 * kDecThreads) {
+  for (int b0 = 0; b0 < n32; b0 += 4 * kDecThreads) {  // every lane of a warp takes part in each round
+    const int i0 = b0 + 4 * tid;
     uint32_t k[4];
     keys4(i0, k);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
+      int fb = -1;
+      unsigned long long w = 0;
       if (k[u] >= klo && k[u] < khi) {
-        unsigned long long w;
         float t;
         anchored_bin(r, k[u], &w, &t);
-        atomicAdd(&sm.hist[anchored_fine(t)], w);
+        fb = anchored_fine(t);
       }
+      hist_add_warp(sm.hist, fb, w);
     }
   }
   __syncthreads();
@@ -723,7 +743,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     if (tid == 0) sm.bcast32[2] = -1;
     __syncthreads();
     for (int k = 0; k < BPT; ++k)
-      if (sm.hist[tid * BPT + k] != 0ull) atomicMax(&sm.bcast32[2], tid * BPT + k);
+      if (sm.hist[tid * BPT + k] != 0ull) smem_max_s32(&sm.bcast32[2], tid * BPT + k);
     __syncthreads();
     fbin = sm.bcast32[2];
     if (fbin < 0) return ~0ull;
@@ -752,7 +772,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
         unsigned long long w;
         float t;
         anchored_bin(r, k[u], &w, &t);
-        const int sl = atomicAdd(&sm.bcast32[1], 1);
+        const int sl = smem_inc(&sm.bcast32[1]);
         if (sl < 32) {
           sm.cut_key[sl] = entry_key64(a, Entry{k[u], E.code(i0 + u)});
           sm.cut_w[sl] = w;
@@ -810,7 +830,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
       anchored_bin(r, k, &w, &t);
       const unsigned long long k64 = entry_key64(a, Entry{k, E.code(i)});
       if (pass > 0 && (k64 >> (shift + 8)) != (prefix >> (shift + 8))) continue;
-      atomicAdd(&sm.hist[(k64 >> shift) & 255], w);
+      smem_add_u64(&sm.hist[(k64 >> shift) & 255], w);
     }
     __syncthreads();
     if (tid < 32) {
@@ -1144,10 +1164,12 @@ __device__ __forceinline__ void pdl_wait_and_release() {
 template <typename T, int D>
 struct Ctx {
   const DecodeArgs& a;
-  int nh;
+  int nh;  // heads of this call
+  int mh;  // heads the scratch is laid out for (every call uses the same offsets)
   int64_t cap4, bm_words;
   __device__ explicit Ctx(const DecodeArgs& args)
-      : a(args), nh(args.nheads), cap4((args.cap_sel + 3) & ~int64_t(3)), bm_words(decode_bitmap_words(args.cap_sel)) {}
+      : a(args), nh(args.nheads), mh(args.max_heads), cap4((args.cap_sel + 3) & ~int64_t(3)),
+        bm_words(decode_bitmap_words(args.cap_sel)) {}
   // per-head workspace: step keys [2][cap4], step codes [2][cap4] (parity buffers: step s in s & 1),
   // anchored histograms [2][kBins], units of the next scoring phase [cap4], kept leaves [cap_list]
   __device__ char* ws(int h) const { return a.ws + uint64_t(h) * a.ws_per_bh; }
@@ -1165,7 +1187,7 @@ struct Ctx {
   // head states, then one leaf bitmap per head (one region, zero between calls)
   __device__ HeadState* hstate(int h) const { return reinterpret_cast<HeadState*>(a.flow) + h; }
   __device__ uint32_t* bitmap(int h) const {
-    return reinterpret_cast<uint32_t*>(a.flow + size_t(nh) * sizeof(HeadState)) + h * bm_words;
+    return reinterpret_cast<uint32_t*>(a.flow + size_t(mh) * sizeof(HeadState)) + h * bm_words;
   }
   // the lane's q slice for the FMA estimates: elements [cl*EPC, cl*EPC+EPC), cl = lane % CPR
   __device__ void q_slice(int h, float* qs) const {
@@ -1523,8 +1545,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
       const int sl = slot_d;
       const unsigned parity = phase_d;
       {
-        // bounded wait; on running out: report, wait (again bounded) for the
-        // copies in flight, and stop this warp
+        // bounded wait; on running out: report, wait for the copies in flight
+        // (they read valid node records, so they land within microseconds; the
+        // second bound, far above that, only guarantees termination), and stop
+        // this warp
         long long it = 0;
         bool out = false;
         while (true) {
@@ -2151,20 +2175,33 @@ static void launch_pdl(void (*kern)(Args...), unsigned grid, unsigned block, siz
   cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// The large dynamic shared memory of the decode kernels is an attribute of each
+// kernel on each device: set once per (kernel instance, device), under a lock.
+template <typename T, int D>
+static cudaError_t configure_decode_t() {
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(score_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(ScoreSmem)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(select_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(DecSmem)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attend_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(AttSmem)));
+  if (e != cudaSuccess) return e;
+  done[dev] = true;
+  return cudaSuccess;
+}
+
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(score_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(sizeof(ScoreSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(select_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(sizeof(DecSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(sizeof(AttSmem)));
+  {
+    const cudaError_t e = configure_decode_t<T, D>();
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   const int sms = device_sms();
   const unsigned nh = unsigned(a.nheads);

@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256) dense_combine_kernel(DenseArgs a) {
 
 // ------------------------------------------------------------------ bf16, tensor-core path
 template <int D>
-__global__ void __launch_bounds__(kDenseThreads) dense_mma_kernel(DenseArgs a) {
+__global__ void __launch_bounds__(kDenseThreads, 4) dense_mma_kernel(DenseArgs a) {
   constexpr int NV = D / 32;  // 16-byte Q/K vectors per thread per row
   constexpr int MT = D / 16;  // m-tiles of O^T
   const int split = blockIdx.x, kvh = blockIdx.y, bb = blockIdx.z;
@@ -318,11 +318,11 @@ size_t dense_static_floats() { return kDenseStaticFloats; }
 // per device (with that device current) and cached.
 cudaError_t dense_static_scratch(float** out) {
   static std::mutex mu;
-  static float* addr[128] = {};
+  static float* addr[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
