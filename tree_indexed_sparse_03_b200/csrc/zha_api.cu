@@ -16,6 +16,9 @@ namespace zha {
 cudaError_t launch_tree_update(const TreeDev& t, int dtype, int64_t n_old, int64_t n_new, cudaStream_t st);
 cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
                                cudaStream_t st);
+bool append_fast_ok(const TreeDev& t, int64_t n, int64_t m);
+cudaError_t launch_append_fast(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
+                               cudaStream_t st);
 size_t chunk_smem_bytes(int dtype, int d, int block, int chunk_level, int R);
 size_t decode_flow_bytes(int nheads, int64_t cap_sel);
 uint64_t decode_ws_bytes(int64_t cap_sel, int64_t cap_list);
@@ -307,6 +310,12 @@ int zha_tree_append(zha_tree* t, const void* K_new, const void* V_new, int64_t m
     return fail(ZHA_ERR_INVALID, "K_new and V_new must be 16-byte aligned");
   if (t->n + m > t->cfg.capacity) return fail(ZHA_ERR_CAPACITY, "append exceeds capacity");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (append_fast_ok(t->dev, t->n, m)) {  // no node of levels 2..S completes: copy and new leaves in one kernel
+    cudaError_t e = launch_append_fast(t->dev, t->cfg.dtype, K_new, V_new, t->n, m, st);
+    if (e != cudaSuccess) return fail_cuda(e, "zha_tree_append: fast path");
+    t->n += m;
+    return ZHA_OK;
+  }
   cudaError_t e = launch_append_copy(t->dev, t->cfg.dtype, K_new, V_new, t->n, m, st);
   if (e != cudaSuccess) return fail_cuda(e, "zha_tree_append: copy");
   e = launch_tree_update(t->dev, t->cfg.dtype, t->n, t->n + m, st);

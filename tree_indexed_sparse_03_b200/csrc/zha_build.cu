@@ -23,7 +23,9 @@
 // above are kept in fp32 as well, and levels S+1..L are merged from them by
 // upper_kernel.  An append recomputes the chunks that gain complete leaves
 // and writes only the nodes that became complete, so build(n) followed by
-// append(m) stores exactly the same bits as build(n + m).
+// append(m) stores exactly the same bits as build(n + m); an append that
+// completes no node of levels 2..S (most single tokens) computes only its new
+// leaves, in one kernel that also copies the rows.
 #include "zha_args.cuh"
 
 namespace zha {
@@ -332,6 +334,104 @@ __global__ void quant4_kernel(TreeDev t, int level, int64_t first) {
   for (int j = threadIdx.x; j < padded; j += blockDim.x) bdst[j] = j < R ? bsrc[j] : 0.f;
 }
 
+
+// Appends that complete no node of levels 2..S (most single tokens): one CTA
+// per KV head copies the new rows and computes only the newly completed leaves,
+// with the chunk kernel's arithmetic in the same order (sequential fma over the
+// dimensions for each score, the leaf's softmax over its keys in key order),
+// so the stored bits equal those of a full build.  Levels above the chunk
+// level are merged afterwards by upper_kernel as usual.
+constexpr int kAppendThreads = 256;
+constexpr int kAppendMaxBlock = 64;  // keys per leaf the fast path stages
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kAppendThreads) append_fast_kernel(TreeDev t, const T* Knew, const T* Vnew,
+                                                                     int64_t n_old, int64_t m) {
+  using E = Elem<T>;
+  constexpr int VPR = D * sizeof(T) / 16;
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const int b = t.block, R = t.refs;
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* refs = reinterpret_cast<float*>(smem);                      // [R][D + 1]
+  float* sc = refs + size_t(R) * (D + 1);                             // [b][R] scores, then weights
+  float* fg = sc + size_t(kAppendMaxBlock) * kMaxRefs;                // [R] f, [R] g
+  T* keys = reinterpret_cast<T*>(fg + 2 * kMaxRefs);                   // [b][D]
+  // the new rows of this head (rows are [Hkv][m][d]: head h's rows are contiguous)
+  for (int64_t i = tid; i < m * VPR; i += blockDim.x) {
+    const int64_t r = i / VPR, v = i % VPR;
+    const size_t src = (size_t(h) * m + r) * D + v * (16 / sizeof(T));
+    const size_t dst = (size_t(h) * t.capacity + n_old + r) * D + v * (16 / sizeof(T));
+    *reinterpret_cast<uint4*>(static_cast<T*>(t.K) + dst) = *reinterpret_cast<const uint4*>(Knew + src);
+    *reinterpret_cast<uint4*>(static_cast<T*>(t.V) + dst) = *reinterpret_cast<const uint4*>(Vnew + src);
+  }
+  const int64_t l0 = n_old / b, l1 = (n_old + m) / b;
+  if (l1 == l0) return;
+  const T* Rh = static_cast<const T*>(t.refsp) + size_t(h) * R * D;
+  for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+  const bool keep32 = t.chunk_level == 1 && t.levels > 1;  // level 1 is the chunk level: keep fp32 values
+  __syncthreads();
+  const T* Kh = static_cast<const T*>(t.K) + size_t(h) * t.capacity * D;
+  for (int64_t leaf = l0; leaf < l1; ++leaf) {
+    for (int i = tid; i < b * D; i += blockDim.x) keys[i] = Kh[size_t(leaf) * b * D + i];
+    __syncthreads();
+    // scores s[k][j] = (r_j . k) / sqrt(d): sequential fma over the dimensions
+    for (int i = tid; i < b * R; i += blockDim.x) {
+      const int k = i / R, j = i % R;
+      const T* kr = keys + size_t(k) * D;
+      const float* rr = refs + j * (D + 1);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < D; ++e) acc = __fmaf_rn(E::to_f(kr[e]), rr[e], acc);
+      sc[k * kMaxRefs + j] = __fmul_rn(acc, t.inv_sqrt_d);
+    }
+    __syncthreads();
+    // value, projected mean score and softmax weights of each reference query
+    for (int j = tid; j < R; j += blockDim.x) {
+      float mx = -INFINITY;
+      for (int k = 0; k < b; ++k) mx = fmaxf(mx, sc[k * kMaxRefs + j]);
+      float Z = 0.f;
+      for (int k = 0; k < b; ++k) Z = __fadd_rn(Z, expf(__fsub_rn(sc[k * kMaxRefs + j], mx)));
+      const float f = __fadd_rn(mx, logf(Z));
+      float g = 0.f;
+      for (int k = 0; k < b; ++k) {
+        const float wk = __fdiv_rn(expf(__fsub_rn(sc[k * kMaxRefs + j], mx)), Z);
+        g = __fmaf_rn(wk, sc[k * kMaxRefs + j], g);
+        sc[k * kMaxRefs + j] = wk;
+      }
+      fg[j] = f;
+      fg[kMaxRefs + j] = g;
+    }
+    __syncthreads();
+    // slopes mu, the record (mu in the element type, intercepts), f, and the fp32 copy at the chunk level
+    T* rec = reinterpret_cast<T*>(t.rec(1, h, leaf));
+    for (int i = tid; i < R * D; i += blockDim.x) {
+      const int j = i / D, e = i % D;
+      float acc = 0.f;
+      for (int k = 0; k < b; ++k) acc = __fmaf_rn(sc[k * kMaxRefs + j], E::to_f(keys[size_t(k) * D + e]), acc);
+      rec[size_t(j) * D + e] = E::from_f(acc);
+      if (keep32) t.up(1, h, leaf)[size_t(j) * D + e] = acc;
+    }
+    float* bias = reinterpret_cast<float*>(t.rec(1, h, leaf) + size_t(R) * D * sizeof(T));
+    const int padded = int((t.rec_bytes - size_t(R) * D * sizeof(T)) / 4);
+    for (int j = tid; j < padded; j += blockDim.x) bias[j] = j < R ? __fsub_rn(fg[j], fg[kMaxRefs + j]) : 0.f;
+    for (int j = tid; j < R; j += blockDim.x) {
+      t.fval(1, h, leaf)[j] = fg[j];
+      if (keep32) {
+        float* u = t.up(1, h, leaf);
+        u[size_t(R) * D + j] = fg[j];
+        u[size_t(R) * D + R + j] = fg[kMaxRefs + j];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T, int D>
+size_t append_fast_smem() {
+  return (size_t(kMaxRefs) * (D + 1) + size_t(kAppendMaxBlock) * kMaxRefs + 2 * kMaxRefs) * 4 +
+         size_t(kAppendMaxBlock) * D * sizeof(T);
+}
+
 // Copy m new tokens ([Hkv][m][d] rows) into the cache at positions [n, n+m).
 template <typename T, int D>
 __global__ void append_copy_kernel(TreeDev t, const T* Knew, const T* Vnew, int64_t n, int64_t m) {
@@ -350,11 +450,12 @@ __global__ void append_copy_kernel(TreeDev t, const T* Knew, const T* Vnew, int6
 
 // ------------------------------------------------------------------ host launchers
 template <typename T, int D>
-static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_new, cudaStream_t st) {
+static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_new, cudaStream_t st,
+                                   bool skip_chunk = false) {
   const int b = t.block, S = t.chunk_level;
   const int64_t CK = t.pow_b[S];
   const int64_t n1_old = n_old / b, n1_new = n_new / b;
-  if (n1_new > n1_old) {
+  if (n1_new > n1_old && !skip_chunk) {
     const int64_t c0 = (n1_old * b) / CK;
     const int64_t c1 = (n1_new * b - 1) / CK;
     const ChunkSmem L = chunk_smem_layout<T, D>(b, S, t.refs);
@@ -399,6 +500,42 @@ cudaError_t launch_tree_update(const TreeDev& t, int dtype, int64_t n_old, int64
                       : launch_update_t<__nv_bfloat16, 64>(t, n_old, n_new, st);
   }
   return t.d == 128 ? launch_update_t<float, 128>(t, n_old, n_new, st) : launch_update_t<float, 64>(t, n_old, n_new, st);
+}
+
+// Whether an append of m tokens at n can take append_fast_kernel: no node of levels 2..S completes, the
+// leaves fit its staging, and the copy is small.
+bool append_fast_ok(const TreeDev& t, int64_t n, int64_t m) {
+  if (t.block > kAppendMaxBlock || m > 64) return false;
+  for (int level = 2; level <= t.chunk_level; ++level)
+    if ((n + m) / t.pow_b[level] != n / t.pow_b[level]) return false;
+  return true;
+}
+
+template <typename T, int D>
+static cudaError_t launch_update_t(const TreeDev& t, int64_t n_old, int64_t n_new, cudaStream_t st, bool skip_chunk);
+
+template <typename T, int D>
+static cudaError_t launch_append_fast_t(const TreeDev& t, const void* Kn, const void* Vn, int64_t n, int64_t m,
+                                        cudaStream_t st) {
+  const size_t sm = append_fast_smem<T, D>();
+  cudaError_t e = cudaFuncSetAttribute(append_fast_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  append_fast_kernel<T, D><<<unsigned(t.hkv), kAppendThreads, sm, st>>>(t, static_cast<const T*>(Kn),
+                                                                         static_cast<const T*>(Vn), n, m);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // levels above the chunk level that the new leaves complete, and FP4 router copies
+  return launch_update_t<T, D>(t, n, n + m, st, /*skip_chunk=*/true);
+}
+
+cudaError_t launch_append_fast(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
+                               cudaStream_t st) {
+  if (dtype == ZHA_BF16)
+    return t.d == 128 ? launch_append_fast_t<__nv_bfloat16, 128>(t, Kn, Vn, n, m, st)
+                      : launch_append_fast_t<__nv_bfloat16, 64>(t, Kn, Vn, n, m, st);
+  return t.d == 128 ? launch_append_fast_t<float, 128>(t, Kn, Vn, n, m, st)
+                    : launch_append_fast_t<float, 64>(t, Kn, Vn, n, m, st);
 }
 
 cudaError_t launch_append_copy(const TreeDev& t, int dtype, const void* Kn, const void* Vn, int64_t n, int64_t m,
