@@ -101,24 +101,39 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
   }
   __syncthreads();
 
-  // node slot of (level, index-in-chunk) inside the per-chunk arrays
-  auto slot = [&](int level, int i) {
+  // node slot of (level, index-in-chunk) inside the per-chunk arrays: level l starts at slot_off[l]
+  int slot_off[kMaxLevels + 1];
+  {
     int off = 0, wdt = CK;
-    for (int l = 1; l < level; ++l) { wdt /= b; off += wdt; }
-    return off + i;
-  };
+    for (int l = 1; l <= S; ++l) {
+      slot_off[l] = off;
+      wdt /= b;
+      off += wdt;
+    }
+  }
+  auto slot = [&](int level, int i) { return slot_off[level] + i; };
+  // loops over (node, reference query) rows of D values: thread tid takes element e of rows
+  // tid / D, tid / D + RPI, ... (one division per row, none per element)
+  constexpr int RPI = kBuildThreads / D;
+  const int e_t = tid % D;
 
   int64_t pw = 1;
   for (int j0 = 0; j0 < R; j0 += RG) {
     const int rg = min(RG, R - j0);
-    // scores s[k][jj]
+    // scores s[k][jj]: sequential fma over the dimensions (keys read as 16-byte vectors)
     for (int i = tid; i < nkeys * rg; i += blockDim.x) {
-      const int k = i / rg, jj = i % rg;
+      const int k = i / rg, jj = i - (i / rg) * rg;
       const T* kr = keys + size_t(k) * KS;
       const float* rr = refs + (j0 + jj) * (D + 1);
+      constexpr int EPV = 16 / sizeof(T);
       float acc = 0.f;
-#pragma unroll 8
-      for (int e = 0; e < D; ++e) acc = __fmaf_rn(E::to_f(kr[e]), rr[e], acc);
+#pragma unroll 2
+      for (int e0 = 0; e0 < D; e0 += EPV) {
+        float x[EPV];
+        unpack16<T>(*reinterpret_cast<const uint4*>(kr + e0), x);
+#pragma unroll
+        for (int q = 0; q < EPV; ++q) acc = __fmaf_rn(x[q], rr[e0 + q], acc);
+      }
       w[k * RG + jj] = __fmul_rn(acc, t.inv_sqrt_d);
     }
     __syncthreads();
@@ -142,8 +157,8 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
     }
     __syncthreads();
     // leaf slopes mu
-    for (int i = tid; i < nleaves * rg * D; i += blockDim.x) {
-      const int e = i % D, jj = (i / D) % rg, li = i / (D * rg);
+    for (int row = tid / D; row < nleaves * rg; row += RPI) {
+      const int li = row / rg, jj = row - li * rg, e = e_t;
       float acc = 0.f;
       for (int k = 0; k < b; ++k)
         acc = __fmaf_rn(w[(li * b + k) * RG + jj], E::to_f(keys[size_t(li * b + k) * KS + e]), acc);
@@ -175,8 +190,8 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
           gs[slot(level, ni) * RG + jj] = g;
         }
         __syncthreads();
-        for (int i = tid; i < nval * rg * D; i += blockDim.x) {
-          const int e = i % D, jj = (i / D) % rg, ni = i / (D * rg);
+        for (int row = tid / D; row < nval * rg; row += RPI) {
+          const int ni = row / rg, jj = row - ni * rg, e = e_t;
           const int c0 = slot(level - 1, ni * b);
           float acc = 0.f;
           for (int c = 0; c < b; ++c)
@@ -195,8 +210,8 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
       const int nval = int(min64(per_chunk, n_tokens / pw - base));
       const int64_t first_new = n_old / pw;
       const bool keep32 = (level == S) && (S < t.levels);
-      for (int i = tid; i < nval * rg * D; i += blockDim.x) {
-        const int e = i % D, jj = (i / D) % rg, ni = i / (D * rg);
+      for (int row = tid / D; row < nval * rg; row += RPI) {
+        const int ni = row / rg, jj = row - ni * rg, e = e_t;
         const int64_t gi = base + ni;
         if (gi < first_new) continue;
         const float v = mu[(size_t(slot(level, ni)) * RG + jj) * D + e];
