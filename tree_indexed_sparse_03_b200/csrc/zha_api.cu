@@ -115,7 +115,7 @@ int make_layout(const zha_config* c, Layout* L) {
   if (chunk_smem_bytes(c->dtype, c->d, c->block, L->S, c->n_refs) > 200 * 1024)
     return fail(ZHA_ERR_UNSUPPORTED, "block too large for the build kernel's shared memory");
   L->rec_bytes = uint64_t(c->n_refs) * c->d * es + ((uint64_t(c->n_refs) * 4 + 15) & ~uint64_t(15));
-  L->up_bytes = uint64_t(c->n_refs) * (c->d + 2) * 4;
+  L->up_bytes = (uint64_t(c->n_refs) * (c->d + 2) * 4 + 15) & ~uint64_t(15);  // 16-byte rows for vector stores
   uint64_t off = 0;
   int64_t pw = 1;
   L->pow_b[0] = 1;

@@ -26,6 +26,8 @@
 // append(m) stores exactly the same bits as build(n + m); an append that
 // completes no node of levels 2..S (most single tokens) computes only its new
 // leaves, in one kernel that also copies the rows.
+#include <type_traits>
+
 #include "zha_args.cuh"
 
 namespace zha {
@@ -34,7 +36,7 @@ constexpr int kBuildThreads = 256;
 
 struct ChunkSmem {
   int CK, KS, RG, NN;
-  size_t keys, refs, w, mu, fs, gs, total;
+  size_t keys, refs, refb, w, wa, mu, fs, gs, total;
 };
 
 template <typename T, int D>
@@ -45,26 +47,136 @@ __host__ __device__ inline ChunkSmem chunk_smem_layout(int block, int chunk_leve
   L.CK = CK;
   L.KS = D + 16 / int(sizeof(T));  // key row stride in elements (16-byte pad)
   L.RG = R < 4 ? R : 4;
-  int nn = 0, w = CK;
-  for (int l = 1; l <= chunk_level; ++l) { w /= block; nn += w; }
+  int nn = 0, w = CK, na = 0;
+  for (int l = 1; l <= chunk_level; ++l) {
+    w /= block;
+    nn += w;
+    if (l >= 2) na += w * block;  // children of the level-l nodes
+  }
   L.NN = nn;
   size_t off = 0;
   L.keys = off; off += size_t(CK) * L.KS * sizeof(T); off = (off + 15) & ~size_t(15);
-  L.refs = off; off += size_t(R) * (D + 1) * 4;
-  L.w = off;    off += size_t(CK) * L.RG * 4;
-  L.mu = off;   off += size_t(nn) * L.RG * D * 4;
-  L.fs = off;   off += size_t(nn) * L.RG * 4;
-  L.gs = off;   off += size_t(nn) * L.RG * 4;
+  L.refs = off; off += size_t(R) * (D + 1) * 4;                     // fp32 refs (scalar scores)
+  off = (off + 15) & ~size_t(15);
+  L.refb = off; off += size_t(R) * D * 2;                           // bf16 refs (tensor-core scores)
+  L.w = off;    off += size_t(CK) * R * 4;                          // leaf scores, then softmax weights
+  L.wa = off;   off += size_t(na > 0 ? na : 1) * R * 4;             // merge weights of the children
+  off = (off + 15) & ~size_t(15);
+  L.mu = off;   off += size_t(nn) * L.RG * D * 4;                   // fp32 slopes of one group of refs
+  L.fs = off;   off += size_t(nn) * R * 4;
+  L.gs = off;   off += size_t(nn) * R * 4;
   L.total = (off + 15) & ~size_t(15);
   return L;
 }
 
+// Scores s[k][j] = (r_j . key_k) / sqrt(d) of nkeys keys (rows of `keys`, stride KS elements) and R bf16
+// reference rows (`refb`, [R][D]) on the tensor cores: mma.sync m16n8k16, 16 keys x 8 refs per tile, the D
+// dimensions in 16-wide steps accumulated in order from zero.  Each score depends only on its key, its
+// reference query and this fixed sequence, so every caller (build, append) gets the same bits.  Warps take
+// tiles in turn; scores go to sc[k * R + j].
+template <int D>
+__device__ __forceinline__ void scores_mma(const __nv_bfloat16* keys, int KS, int nkeys,
+                                           const __nv_bfloat16* refb, int R, float inv_sqrt_d, float* sc,
+                                           int warp, int nwarps) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+  const int mt = (nkeys + 15) / 16, nt = (R + 7) / 8;
+  for (int tile = warp; tile < mt * nt; tile += nwarps) {
+    const int m0 = (tile / nt) * 16, n0 = (tile % nt) * 8;
+    const int r0 = min(m0 + g, nkeys - 1), r1 = min(m0 + g + 8, nkeys - 1);  // rows past nkeys: masked
+    const int c = min(n0 + g, R - 1);
+    const __nv_bfloat16* a0p = keys + size_t(r0) * KS + 2 * t4;
+    const __nv_bfloat16* a1p = keys + size_t(r1) * KS + 2 * t4;
+    const __nv_bfloat16* bp = refb + size_t(c) * D + 2 * t4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k0 = 0; k0 < D; k0 += 16) {
+      const uint32_t a[4] = {*reinterpret_cast<const uint32_t*>(a0p + k0), *reinterpret_cast<const uint32_t*>(a1p + k0),
+                             *reinterpret_cast<const uint32_t*>(a0p + k0 + 8),
+                             *reinterpret_cast<const uint32_t*>(a1p + k0 + 8)};
+      const uint32_t bb[2] = {*reinterpret_cast<const uint32_t*>(bp + k0), *reinterpret_cast<const uint32_t*>(bp + k0 + 8)};
+      mma_bf16_16816(acc, a, bb);
+    }
+    const int row0 = m0 + g, row1 = m0 + g + 8, col = n0 + 2 * t4;
+    if (row0 < nkeys) {
+      if (col < R) sc[row0 * R + col] = __fmul_rn(acc[0], inv_sqrt_d);
+      if (col + 1 < R) sc[row0 * R + col + 1] = __fmul_rn(acc[1], inv_sqrt_d);
+    }
+    if (row1 < nkeys) {
+      if (col < R) sc[row1 * R + col] = __fmul_rn(acc[2], inv_sqrt_d);
+      if (col + 1 < R) sc[row1 * R + col + 1] = __fmul_rn(acc[3], inv_sqrt_d);
+    }
+  }
+}
+
+// Scores of the fp32 configurations: sequential fma over the dimensions.
+template <typename T, int D>
+__device__ __forceinline__ void scores_fma(const T* keys, int KS, int nkeys, const float* refs, int R,
+                                           float inv_sqrt_d, float* sc) {
+  using E = Elem<T>;
+  for (int i = threadIdx.x; i < nkeys * R; i += blockDim.x) {
+    const int k = i / R, j = i - (i / R) * R;
+    const T* kr = keys + size_t(k) * KS;
+    const float* rr = refs + j * (D + 1);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) acc = __fmaf_rn(E::to_f(kr[e]), rr[e], acc);
+    sc[k * R + j] = __fmul_rn(acc, inv_sqrt_d);
+  }
+}
+
+// Leaf value, projected mean score and softmax weights of (leaf li, ref j): m = max s, Z = sum exp(s - m),
+// f = m + log Z, w_k = exp(s_k - m) / Z (written over the scores), g = sum_k w_k s_k.
+__device__ __forceinline__ void leaf_softmax(float* s, int stride, int b, float* f_out, float* g_out) {
+  float m = -INFINITY;
+  for (int k = 0; k < b; ++k) m = fmaxf(m, s[k * stride]);
+  float Z = 0.f;
+  for (int k = 0; k < b; ++k) Z = __fadd_rn(Z, expf(__fsub_rn(s[k * stride], m)));
+  const float f = __fadd_rn(m, logf(Z));
+  float g = 0.f;
+  for (int k = 0; k < b; ++k) {
+    const float wk = __fdiv_rn(expf(__fsub_rn(s[k * stride], m)), Z);
+    g = __fmaf_rn(wk, s[k * stride], g);
+    s[k * stride] = wk;
+  }
+  *f_out = f;
+  *g_out = g;
+}
+
+// Eight consecutive values of a row (fp32) -> the element type, stored as one or two 16-byte vectors.
+template <typename T>
+__device__ __forceinline__ void store8(T* dst, const float (&v)[8]);
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[8]) {
+  uint4 o;
+  o.x = pack_bf16(v[0], v[1]);
+  o.y = pack_bf16(v[2], v[3]);
+  o.z = pack_bf16(v[4], v[5]);
+  o.w = pack_bf16(v[6], v[7]);
+  *reinterpret_cast<uint4*>(dst) = o;
+}
+template <>
+__device__ __forceinline__ void store8<float>(float* dst, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8f(float* dst, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
 // One CTA per (chunk, KV head).  Computes every complete node of levels
 // 1..S inside the chunk and writes those with index >= the previous count.
+// Scores of all keys and reference queries first (tensor cores for bf16),
+// then the softmax weights of the leaves and of every merge (all reference
+// queries), then per group of RG reference queries the fp32 slopes, level by
+// level, each thread producing eight consecutive dimensions of a row (the
+// same arithmetic per value: children in order), written to the records as
+// 16-byte vectors.
 template <typename T, int D>
 __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t n_tokens,
                                                               int64_t n_old, int64_t chunk0) {
   using E = Elem<T>;
+  constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
   const int h = blockIdx.y;
   const int64_t chunk = chunk0 + blockIdx.x;
   const int b = t.block, S = t.chunk_level, R = t.refs;
@@ -77,17 +189,19 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
   if (nleaves <= 0) return;
   const int nkeys = nleaves * b;
   const int64_t key0 = chunk * CK;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5;
 
   extern __shared__ __align__(16) unsigned char smem[];
   T* keys = reinterpret_cast<T*>(smem + L.keys);
   float* refs = reinterpret_cast<float*>(smem + L.refs);
+  __nv_bfloat16* refb = reinterpret_cast<__nv_bfloat16*>(smem + L.refb);
   float* w = reinterpret_cast<float*>(smem + L.w);
+  float* wa = reinterpret_cast<float*>(smem + L.wa);
   float* mu = reinterpret_cast<float*>(smem + L.mu);
   float* fs = reinterpret_cast<float*>(smem + L.fs);
   float* gs = reinterpret_cast<float*>(smem + L.gs);
 
-  // Stage the chunk's complete keys (16-byte vectors) and the fp32 refs.
+  // Stage the chunk's complete keys (16-byte vectors) and the refs.
   {
     constexpr int VPR = D * sizeof(T) / 16;  // vectors per key row
     const T* Kh = static_cast<const T*>(t.K) + (size_t(h) * t.capacity + key0) * D;
@@ -97,161 +211,141 @@ __global__ void __launch_bounds__(kBuildThreads) chunk_kernel(TreeDev t, int64_t
       *reinterpret_cast<uint4*>(keys + size_t(k) * KS + v * (16 / sizeof(T))) = x;
     }
     const T* Rh = static_cast<const T*>(t.refsp) + size_t(h) * R * D;
-    for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+    if constexpr (kMma) {
+      for (int i = tid; i < R * D; i += blockDim.x) refb[i] = Rh[i];
+    } else {
+      for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+    }
   }
   __syncthreads();
 
-  // node slot of (level, index-in-chunk) inside the per-chunk arrays: level l starts at slot_off[l]
-  int slot_off[kMaxLevels + 1];
+  // node slot of (level, index-in-chunk) inside the per-chunk arrays, and the first merge weight of each level
+  int slot_off[kMaxLevels + 1], wa_off[kMaxLevels + 1];
   {
-    int off = 0, wdt = CK;
+    int off = 0, aoff = 0, wdt = CK;
     for (int l = 1; l <= S; ++l) {
       slot_off[l] = off;
+      wa_off[l] = aoff;
       wdt /= b;
       off += wdt;
+      if (l >= 2) aoff += wdt * b;
     }
   }
   auto slot = [&](int level, int i) { return slot_off[level] + i; };
-  // loops over (node, reference query) rows of D values: thread tid takes element e of rows
-  // tid / D, tid / D + RPI, ... (one division per row, none per element)
-  constexpr int RPI = kBuildThreads / D;
-  const int e_t = tid % D;
+  auto nval_of = [&](int level) {
+    const int64_t pw = t.pow_b[level], per_chunk = CK / pw;
+    return int(min64(per_chunk, n_tokens / pw - chunk * per_chunk));
+  };
 
-  int64_t pw = 1;
-  for (int j0 = 0; j0 < R; j0 += RG) {
-    const int rg = min(RG, R - j0);
-    // scores s[k][jj]: sequential fma over the dimensions (keys read as 16-byte vectors)
-    for (int i = tid; i < nkeys * rg; i += blockDim.x) {
-      const int k = i / rg, jj = i - (i / rg) * rg;
-      const T* kr = keys + size_t(k) * KS;
-      const float* rr = refs + (j0 + jj) * (D + 1);
-      constexpr int EPV = 16 / sizeof(T);
-      float acc = 0.f;
-#pragma unroll 2
-      for (int e0 = 0; e0 < D; e0 += EPV) {
-        float x[EPV];
-        unpack16<T>(*reinterpret_cast<const uint4*>(kr + e0), x);
-#pragma unroll
-        for (int q = 0; q < EPV; ++q) acc = __fmaf_rn(x[q], rr[e0 + q], acc);
-      }
-      w[k * RG + jj] = __fmul_rn(acc, t.inv_sqrt_d);
-    }
-    __syncthreads();
-    // leaf value, projected mean score and softmax weights
-    for (int i = tid; i < nleaves * rg; i += blockDim.x) {
-      const int li = i / rg, jj = i % rg;
-      float* s = w + (li * b) * RG + jj;
+  // scores of every key and reference query
+  if constexpr (kMma) scores_mma<D>(keys, KS, nkeys, refb, R, t.inv_sqrt_d, w, warp, kBuildThreads / 32);
+  else scores_fma<T, D>(keys, KS, nkeys, refs, R, t.inv_sqrt_d, w);
+  __syncthreads();
+  // leaf values and weights, all reference queries
+  for (int i = tid; i < nleaves * R; i += blockDim.x) {
+    const int li = i / R, j = i - li * R;
+    leaf_softmax(w + (li * b) * R + j, R, b, &fs[slot(1, li) * R + j], &gs[slot(1, li) * R + j]);
+  }
+  __syncthreads();
+  // merge values and weights of levels 2..S, all reference queries
+  for (int level = 2; level <= S; ++level) {
+    const int nval = nval_of(level);
+    for (int i = tid; i < nval * R; i += blockDim.x) {
+      const int ni = i / R, j = i - ni * R;
+      const int c0 = slot(level - 1, ni * b);
       float m = -INFINITY;
-      for (int k = 0; k < b; ++k) m = fmaxf(m, s[k * RG]);
+      for (int c = 0; c < b; ++c) m = fmaxf(m, fs[(c0 + c) * R + j]);
       float Z = 0.f;
-      for (int k = 0; k < b; ++k) Z = __fadd_rn(Z, expf(__fsub_rn(s[k * RG], m)));
+      for (int c = 0; c < b; ++c) Z = __fadd_rn(Z, expf(__fsub_rn(fs[(c0 + c) * R + j], m)));
       const float f = __fadd_rn(m, logf(Z));
       float g = 0.f;
-      for (int k = 0; k < b; ++k) {
-        const float wk = __fdiv_rn(expf(__fsub_rn(s[k * RG], m)), Z);
-        g = __fmaf_rn(wk, s[k * RG], g);
-        s[k * RG] = wk;
+      for (int c = 0; c < b; ++c) {
+        const float a = __fdiv_rn(expf(__fsub_rn(fs[(c0 + c) * R + j], m)), Z);
+        wa[(wa_off[level] + ni * b + c) * R + j] = a;
+        g = __fmaf_rn(a, gs[(c0 + c) * R + j], g);
       }
-      fs[slot(1, li) * RG + jj] = f;
-      gs[slot(1, li) * RG + jj] = g;
+      fs[slot(level, ni) * R + j] = f;
+      gs[slot(level, ni) * R + j] = g;
     }
     __syncthreads();
-    // leaf slopes mu
-    for (int row = tid / D; row < nleaves * rg; row += RPI) {
-      const int li = row / rg, jj = row - li * rg, e = e_t;
-      float acc = 0.f;
-      for (int k = 0; k < b; ++k)
-        acc = __fmaf_rn(w[(li * b + k) * RG + jj], E::to_f(keys[size_t(li * b + k) * KS + e]), acc);
-      mu[(size_t(slot(1, li)) * RG + jj) * D + e] = acc;
-    }
-    __syncthreads();
-    // exact merges of levels 2..S inside the chunk
-    int64_t bl = b;  // b^(level-1)
-    for (int level = 2; level <= S; ++level) {
-      bl *= b;
-      const int64_t per_chunk = CK / bl;
-      const int nval = int(min64(per_chunk, n_tokens / bl - chunk * per_chunk));
-      if (nval > 0) {
-        for (int i = tid; i < nval * rg; i += blockDim.x) {
-          const int ni = i / rg, jj = i % rg;
-          const int c0 = slot(level - 1, ni * b);
-          float m = -INFINITY;
-          for (int c = 0; c < b; ++c) m = fmaxf(m, fs[(c0 + c) * RG + jj]);
-          float Z = 0.f;
-          for (int c = 0; c < b; ++c) Z = __fadd_rn(Z, expf(__fsub_rn(fs[(c0 + c) * RG + jj], m)));
-          const float f = __fadd_rn(m, logf(Z));
-          float g = 0.f;
-          for (int c = 0; c < b; ++c) {
-            const float a = __fdiv_rn(expf(__fsub_rn(fs[(c0 + c) * RG + jj], m)), Z);
-            w[(ni * b + c) * RG + jj] = a;
-            g = __fmaf_rn(a, gs[(c0 + c) * RG + jj], g);
+  }
+
+  // slopes: rows (node, ref of the group) of D values, 8 consecutive values per thread
+  constexpr int VEC = 8, TPR = D / VEC, RPI = kBuildThreads / TPR;
+  const int e0 = (tid % TPR) * VEC;
+  for (int j0 = 0; j0 < R; j0 += RG) {
+    const int rg = min(RG, R - j0);
+    for (int level = 1; level <= S; ++level) {
+      const int64_t pw = t.pow_b[level];
+      const int64_t base = chunk * (CK / pw);
+      const int nval = nval_of(level);
+      const int64_t first_new = n_old / pw;
+      const bool keep32 = (level == S) && (S < t.levels);
+      for (int row = tid / TPR; row < nval * rg; row += RPI) {
+        const int ni = row / rg, jj = row - ni * rg, j = j0 + jj;
+        float acc[VEC];
+#pragma unroll
+        for (int q = 0; q < VEC; ++q) acc[q] = 0.f;
+        if (level == 1) {
+          for (int k = 0; k < b; ++k) {
+            const float wk = w[(ni * b + k) * R + j];
+            float x[VEC];
+            if constexpr (sizeof(T) == 2) {
+              unpack16<T>(*reinterpret_cast<const uint4*>(keys + size_t(ni * b + k) * KS + e0), x);
+            } else {
+              unpack16<T>(*reinterpret_cast<const uint4*>(keys + size_t(ni * b + k) * KS + e0), x);
+              unpack16<T>(*reinterpret_cast<const uint4*>(keys + size_t(ni * b + k) * KS + e0 + 4), x + 4);
+            }
+#pragma unroll
+            for (int q = 0; q < VEC; ++q) acc[q] = __fmaf_rn(wk, x[q], acc[q]);
           }
-          fs[slot(level, ni) * RG + jj] = f;
-          gs[slot(level, ni) * RG + jj] = g;
-        }
-        __syncthreads();
-        for (int row = tid / D; row < nval * rg; row += RPI) {
-          const int ni = row / rg, jj = row - ni * rg, e = e_t;
+        } else {
           const int c0 = slot(level - 1, ni * b);
-          float acc = 0.f;
-          for (int c = 0; c < b; ++c)
-            acc = __fmaf_rn(w[(ni * b + c) * RG + jj], mu[(size_t(c0 + c) * RG + jj) * D + e], acc);
-          mu[(size_t(slot(level, ni)) * RG + jj) * D + e] = acc;
+          for (int c = 0; c < b; ++c) {
+            const float a = wa[(wa_off[level] + ni * b + c) * R + j];
+            const float* src = mu + (size_t(c0 + c) * RG + jj) * D + e0;
+            const float4 u0 = *reinterpret_cast<const float4*>(src), u1 = *reinterpret_cast<const float4*>(src + 4);
+            const float x[VEC] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int q = 0; q < VEC; ++q) acc[q] = __fmaf_rn(a, x[q], acc[q]);
+          }
+        }
+        store8f(mu + (size_t(slot(level, ni)) * RG + jj) * D + e0, acc);
+        const int64_t gi = base + ni;
+        if (gi >= first_new) {
+          store8<T>(reinterpret_cast<T*>(t.rec(level, h, gi)) + size_t(j) * D + e0, acc);
+          if (keep32) store8f(t.up(level, h, gi) + size_t(j) * D + e0, acc);
         }
       }
       __syncthreads();
     }
-    // write the nodes that are new in this call
-    pw = 1;
-    for (int level = 1; level <= S; ++level) {
-      pw *= b;
-      const int64_t per_chunk = CK / pw;
-      const int64_t base = chunk * per_chunk;
-      const int nval = int(min64(per_chunk, n_tokens / pw - base));
-      const int64_t first_new = n_old / pw;
-      const bool keep32 = (level == S) && (S < t.levels);
-      for (int row = tid / D; row < nval * rg; row += RPI) {
-        const int ni = row / rg, jj = row - ni * rg, e = e_t;
-        const int64_t gi = base + ni;
-        if (gi < first_new) continue;
-        const float v = mu[(size_t(slot(level, ni)) * RG + jj) * D + e];
-        T* rec = reinterpret_cast<T*>(t.rec(level, h, gi));
-        rec[size_t(j0 + jj) * D + e] = E::from_f(v);
-        if (keep32) t.up(level, h, gi)[size_t(j0 + jj) * D + e] = v;
-      }
-      for (int i = tid; i < nval * rg; i += blockDim.x) {
-        const int jj = i % rg, ni = i / rg;
-        const int64_t gi = base + ni;
-        if (gi < first_new) continue;
-        const float f = fs[slot(level, ni) * RG + jj];
-        const float g = gs[slot(level, ni) * RG + jj];
-        float* bias = reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T));
-        bias[j0 + jj] = __fsub_rn(f, g);
-        t.fval(level, h, gi)[j0 + jj] = f;
-        if (keep32) {
-          float* u = t.up(level, h, gi);
-          u[size_t(R) * D + j0 + jj] = f;
-          u[size_t(R) * D + R + j0 + jj] = g;
-        }
-      }
-    }
-    __syncthreads();
   }
-  // zero the padding after bias[R] once per new node so records are fully defined
-  {
-    pw = 1;
-    const int pad = int((t.rec_bytes - size_t(R) * D * sizeof(T)) / 4) - R;
-    if (pad > 0) {
-      for (int level = 1; level <= S; ++level) {
-        pw *= b;
-        const int64_t per_chunk = CK / pw, base = chunk * per_chunk;
-        const int nval = int(min64(per_chunk, n_tokens / pw - base));
-        const int64_t first_new = n_old / pw;
-        for (int i = tid; i < nval * pad; i += blockDim.x) {
-          const int64_t gi = base + i / pad;
-          if (gi < first_new) continue;
-          reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T))[R + i % pad] = 0.f;
-        }
+  // intercepts and values of the nodes that are new in this call (and their fp32 copies at the chunk level),
+  // the padding after bias[R] zeroed
+  const int padded = int((t.rec_bytes - size_t(R) * D * sizeof(T)) / 4);
+  for (int level = 1; level <= S; ++level) {
+    const int64_t pw = t.pow_b[level];
+    const int64_t base = chunk * (CK / pw);
+    const int nval = nval_of(level);
+    const int64_t first_new = n_old / pw;
+    const bool keep32 = (level == S) && (S < t.levels);
+    for (int i = tid; i < nval * padded; i += blockDim.x) {
+      const int ni = i / padded, j = i - ni * padded;
+      const int64_t gi = base + ni;
+      if (gi < first_new) continue;
+      float* bias = reinterpret_cast<float*>(t.rec(level, h, gi) + size_t(R) * D * sizeof(T));
+      if (j >= R) {
+        bias[j] = 0.f;
+        continue;
+      }
+      const float f = fs[slot(level, ni) * R + j];
+      const float g = gs[slot(level, ni) * R + j];
+      bias[j] = __fsub_rn(f, g);
+      t.fval(level, h, gi)[j] = f;
+      if (keep32) {
+        float* u = t.up(level, h, gi);
+        u[size_t(R) * D + j] = f;
+        u[size_t(R) * D + R + j] = g;
       }
     }
   }
@@ -363,14 +457,16 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kAppendThreads) append_fast_kernel(TreeDev t, const T* Knew, const T* Vnew,
                                                                      int64_t n_old, int64_t m) {
   using E = Elem<T>;
+  constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
   constexpr int VPR = D * sizeof(T) / 16;
   const int h = blockIdx.x, tid = threadIdx.x;
   const int b = t.block, R = t.refs;
   extern __shared__ __align__(16) unsigned char smem[];
-  float* refs = reinterpret_cast<float*>(smem);                      // [R][D + 1]
-  float* sc = refs + size_t(R) * (D + 1);                             // [b][R] scores, then weights
-  float* fg = sc + size_t(kAppendMaxBlock) * kMaxRefs;                // [R] f, [R] g
-  T* keys = reinterpret_cast<T*>(fg + 2 * kMaxRefs);                   // [b][D]
+  T* keys = reinterpret_cast<T*>(smem);                                              // [b][D]
+  float* refs = reinterpret_cast<float*>(smem + size_t(kAppendMaxBlock) * D * sizeof(T));  // [R][D + 1]
+  __nv_bfloat16* refb = reinterpret_cast<__nv_bfloat16*>(refs + size_t(kMaxRefs) * (D + 1));  // [R][D]
+  float* sc = reinterpret_cast<float*>(refb + size_t(kMaxRefs) * D);                 // [b][R]
+  float* fg = sc + size_t(kAppendMaxBlock) * kMaxRefs;                                // [R] f, [R] g
   // the new rows of this head (rows are [Hkv][m][d]: head h's rows are contiguous)
   for (int64_t i = tid; i < m * VPR; i += blockDim.x) {
     const int64_t r = i / VPR, v = i % VPR;
@@ -382,47 +478,29 @@ __global__ void __launch_bounds__(kAppendThreads) append_fast_kernel(TreeDev t, 
   const int64_t l0 = n_old / b, l1 = (n_old + m) / b;
   if (l1 == l0) return;
   const T* Rh = static_cast<const T*>(t.refsp) + size_t(h) * R * D;
-  for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+  if constexpr (kMma) {
+    for (int i = tid; i < R * D; i += blockDim.x) refb[i] = Rh[i];
+  } else {
+    for (int i = tid; i < R * D; i += blockDim.x) refs[(i / D) * (D + 1) + i % D] = E::to_f(Rh[i]);
+  }
   const bool keep32 = t.chunk_level == 1 && t.levels > 1;  // level 1 is the chunk level: keep fp32 values
   __syncthreads();
   const T* Kh = static_cast<const T*>(t.K) + size_t(h) * t.capacity * D;
   for (int64_t leaf = l0; leaf < l1; ++leaf) {
-    for (int i = tid; i < b * D; i += blockDim.x) keys[i] = Kh[size_t(leaf) * b * D + i];
+    for (int i = tid; i < b * VPR; i += blockDim.x)
+      reinterpret_cast<uint4*>(keys)[i] = *reinterpret_cast<const uint4*>(Kh + size_t(leaf) * b * D + size_t(i) * (16 / sizeof(T)));
     __syncthreads();
-    // scores s[k][j] = (r_j . k) / sqrt(d): sequential fma over the dimensions
-    for (int i = tid; i < b * R; i += blockDim.x) {
-      const int k = i / R, j = i % R;
-      const T* kr = keys + size_t(k) * D;
-      const float* rr = refs + j * (D + 1);
-      float acc = 0.f;
-#pragma unroll 8
-      for (int e = 0; e < D; ++e) acc = __fmaf_rn(E::to_f(kr[e]), rr[e], acc);
-      sc[k * kMaxRefs + j] = __fmul_rn(acc, t.inv_sqrt_d);
-    }
+    // the scores, the weights and the slopes exactly as the chunk kernel computes them
+    if constexpr (kMma) scores_mma<D>(keys, D, b, refb, R, t.inv_sqrt_d, sc, tid >> 5, kAppendThreads / 32);
+    else scores_fma<T, D>(keys, D, b, refs, R, t.inv_sqrt_d, sc);
     __syncthreads();
-    // value, projected mean score and softmax weights of each reference query
-    for (int j = tid; j < R; j += blockDim.x) {
-      float mx = -INFINITY;
-      for (int k = 0; k < b; ++k) mx = fmaxf(mx, sc[k * kMaxRefs + j]);
-      float Z = 0.f;
-      for (int k = 0; k < b; ++k) Z = __fadd_rn(Z, expf(__fsub_rn(sc[k * kMaxRefs + j], mx)));
-      const float f = __fadd_rn(mx, logf(Z));
-      float g = 0.f;
-      for (int k = 0; k < b; ++k) {
-        const float wk = __fdiv_rn(expf(__fsub_rn(sc[k * kMaxRefs + j], mx)), Z);
-        g = __fmaf_rn(wk, sc[k * kMaxRefs + j], g);
-        sc[k * kMaxRefs + j] = wk;
-      }
-      fg[j] = f;
-      fg[kMaxRefs + j] = g;
-    }
+    for (int j = tid; j < R; j += blockDim.x) leaf_softmax(sc + j, R, b, &fg[j], &fg[kMaxRefs + j]);
     __syncthreads();
-    // slopes mu, the record (mu in the element type, intercepts), f, and the fp32 copy at the chunk level
     T* rec = reinterpret_cast<T*>(t.rec(1, h, leaf));
     for (int i = tid; i < R * D; i += blockDim.x) {
       const int j = i / D, e = i % D;
       float acc = 0.f;
-      for (int k = 0; k < b; ++k) acc = __fmaf_rn(sc[k * kMaxRefs + j], E::to_f(keys[size_t(k) * D + e]), acc);
+      for (int k = 0; k < b; ++k) acc = __fmaf_rn(sc[k * R + j], E::to_f(keys[size_t(k) * D + e]), acc);
       rec[size_t(j) * D + e] = E::from_f(acc);
       if (keep32) t.up(1, h, leaf)[size_t(j) * D + e] = acc;
     }
@@ -443,9 +521,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_fast_kernel(TreeDev t, 
 
 template <typename T, int D>
 size_t append_fast_smem() {
-  return (size_t(kMaxRefs) * (D + 1) + size_t(kAppendMaxBlock) * kMaxRefs + 2 * kMaxRefs) * 4 +
-         size_t(kAppendMaxBlock) * D * sizeof(T);
+  return size_t(kAppendMaxBlock) * D * sizeof(T) + size_t(kMaxRefs) * (D + 1) * 4 + size_t(kMaxRefs) * D * 2 +
+         (size_t(kAppendMaxBlock) * kMaxRefs + 2 * kMaxRefs) * 4;
 }
+
 
 // Copy m new tokens ([Hkv][m][d] rows) into the cache at positions [n, n+m).
 template <typename T, int D>
