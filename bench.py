@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="build the workload's tree, run --warmup + --steps decodes untimed, exit (for ncu)")
+    ap.add_argument("--multi", type=int, default=0,
+                    help="with --profile: route --multi queries at once (zha_route_multi) instead of decoding; "
+                         "without: time it and print one line")
     ap.add_argument("--sweep", nargs="?", const="32768,65536,131072,262144,524288,1048576,2097152,4194304",
                     default=None, help="run the light sweep workload at these context lengths (one process each) "
                                        "and print one line per N plus the measured dense/ZHA crossover")
@@ -341,6 +344,15 @@ def run_profile(args):
     tree = z.ZhaTree(cfg, inp.K.to(dev), inp.V.to(dev), inp.refs.to(dev))
     tree.build(n)
     Qs = inp.Q.to(dev)
+    if args.multi:
+        from synth.workloads import random_queries
+        Qm = random_queries(1, args.multi, w.n_q_heads, w.d, w.dtype, topics_from=inp).to(dev)
+        for i in range(args.warmup + args.steps):
+            tree.route_multi(Qm)
+        torch.cuda.synchronize(dev)
+        tree.status()
+        log(f"[bench] profile mode: {args.warmup + args.steps} multi-query routes of {args.multi} queries")
+        return
     for i in range(args.warmup + args.steps):
         tree.decode(Qs[i % w.n_query_sets])
     torch.cuda.synchronize(dev)
@@ -582,6 +594,52 @@ def run_zha(args, world, rank, local):
     del tree
 
 
+def run_multi(args):
+    """Multi-query routing (zha_route_multi) of --multi queries on the workload's tree: time per call and per
+    query against the same queries through zha_decode in groups of max_batch, one JSON line (not the
+    decode metric)."""
+    import tree_indexed_sparse_03_b200 as z
+    from synth.workloads import generate, random_queries
+
+    w = load_workload(args)
+    dev = torch.device("cuda", 0)
+    inp = generate(w)
+    n = w.n_tokens
+    mb = max(1, 1024 // w.n_q_heads)
+    cfg = z.make_config(d=w.d, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, block=w.block, levels=w.levels,
+                        n_refs=w.n_refs, p=w.p, dtype=w.dtype, capacity=n, max_batch=mb, planes=w.planes)
+    tree = z.ZhaTree(cfg, inp.K.to(dev), inp.V.to(dev), inp.refs.to(dev))
+    tree.build(n)
+    Qm = random_queries(1, args.multi, w.n_q_heads, w.d, w.dtype, topics_from=inp).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps * 1000
+
+    def per_decode():
+        for q0 in range(0, args.multi, mb):
+            tree.decode(Qm[q0:q0 + mb])
+
+    reps = max(1, args.steps)
+    us_multi = timed(lambda: tree.route_multi(Qm), reps)
+    us_dec = timed(per_decode, reps)
+    tree.status()
+    print(json.dumps({"metric": "multi-query routing (route + attend of m queries of one context)",
+                      "workload": w.name, "n_tokens": n, "queries": args.multi, "max_batch": mb,
+                      "route_multi_us": round(us_multi, 2), "us_per_query": round(us_multi / args.multi, 3),
+                      "decode_groups_us": round(us_dec, 2),
+                      "speedup_first_step_contraction": round(us_dec / us_multi, 3)}), flush=True)
+
+
 def run_sweep(args):
     """The light sweep: one bench process per context length, then the dense/ZHA crossover."""
     lines = []
@@ -630,6 +688,8 @@ def main():
             run_reference(args, world, rank)
         elif args.profile:
             run_profile(args)
+        elif args.multi:
+            run_multi(args)
         else:
             run_zha(args, world, rank, local)
     finally:

@@ -194,6 +194,30 @@ ZHA_API int zha_decode(const zha_tree* tree, const void* Q, float* O, int32_t B,
                int32_t* kept_cnt, int64_t* stats, int32_t* scored, int64_t scored_cap, void* stream);
 
 /*
+ * zha_route_multi: route and attend m queries of the same context at once,
+ * e.g. the queries of a prefill chunk against the cached context before it.
+ * Each query head is routed exactly as in zha_decode (the top-down top-p
+ * descent of "Zyphra Hierarchical Attention", Zyphra blog, section "Routing
+ * in the tree"; tanhow.com summary, section "How does top-p routing choose
+ * tokens?"), and attends to its kept blocks, the sink and the tail; the
+ * pages model the speed of decode only (summary, section "ZHA 有多快？"),
+ * and a query's attention to the other queries of its own chunk is not part
+ * of this call.  Every query starts from the same candidates, the forest
+ * roots, so the first routing step of all queries is one contraction of the
+ * roots' slope rows with the queries on the tensor cores (bf16
+ * configurations; fp32 ones score it per query); the later steps run as in
+ * zha_decode, max_batch queries at a time.
+ *   Q        - [m][Hq][d] element type, device;  O - [m][Hq][d] fp32, device.
+ *   kept     - optional [m][Hq][cap_leaves] int32 with kept_cnt [m][Hq] int32
+ *              (as in zha_decode); both NULL or both non-NULL.
+ *   m >= 1 (any size; the queries are processed in groups of max_batch).
+ * Asynchronous on `stream`; shares the tree's scratch with zha_decode (calls
+ * on one tree must be issued in order on one stream).  Errors as zha_decode.
+ */
+ZHA_API int zha_route_multi(zha_tree* tree, const void* Q, float* O, int32_t m, int32_t* kept, int32_t* kept_cnt,
+                    void* stream);
+
+/*
  * zha_decode_step_host: one decode step from host memory - copies the new
  * token's K/V (host [Hkv][d] each) and the queries (host [B][Hq][d]) to the
  * device, appends the token, decodes, and copies O back to host o_host

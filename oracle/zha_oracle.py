@@ -356,6 +356,15 @@ def route(planes: PlanesFn, q: np.ndarray, p, n_tokens: int, block: int,
     return trace
 
 
+def route_multi(planes: PlanesFn, Qm: np.ndarray, p, n_tokens: int, block: int,
+                levels: int) -> List[RouteTrace]:
+    """Routing of m queries of one context (e.g. the queries of a prefill chunk): each query head is routed
+    on its own, exactly as a decode query ([blog] "Routing in the tree"); the queries share only the tree.
+    The pages model decode only ([summary] "ZHA 有多快？"); sharing the first step's scoring between the
+    queries is a question of how it is computed, not of what."""
+    return [route(planes, q, p, n_tokens, block, levels) for q in Qm]
+
+
 def tree_planes_fn(tree: Dict[int, Planes]) -> PlanesFn:
     return lambda level, idx: (tree[level].mu[idx], tree[level].bias[idx])
 

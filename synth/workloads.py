@@ -249,3 +249,17 @@ def random_tree_case(seed: int, *, n_tokens: int, d: int, n_q_heads: int, n_kv_h
     Q = torch.randn(batch, n_q_heads, d, generator=g, device=device, dtype=f32) * 1.5
     dt = DTYPES[dtype]
     return K.to(dt), V.to(dt), refs.to(dt), Q.to(dt)
+
+
+def random_queries(seed: int, m: int, n_q_heads: int, d: int, dtype: str, topics_from: Optional[Inputs] = None):
+    """m seeded query sets [m, Hq, d]: Gaussian, or, given a generated workload, drawn around its own query sets
+    (a random one of them plus Gaussian noise of a quarter of their scale), so that routing stays selective."""
+    g = torch.Generator()
+    g.manual_seed(seed)
+    if topics_from is None:
+        Q = torch.randn(m, n_q_heads, d, generator=g) * 1.5
+    else:
+        base = topics_from.Q.reshape(-1, n_q_heads, d).float()
+        pick = torch.randint(0, base.shape[0], (m,), generator=g)
+        Q = base[pick] + 0.25 * base.std() * torch.randn(m, n_q_heads, d, generator=g)
+    return Q.to(DTYPES[dtype])

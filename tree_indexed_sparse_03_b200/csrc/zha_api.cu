@@ -399,6 +399,41 @@ int zha_decode(const zha_tree* t, const void* Q, float* O, int32_t B, int32_t* k
   return ZHA_OK;
 }
 
+int zha_route_multi(zha_tree* t, const void* Q, float* O, int32_t m, int32_t* kept, int32_t* kept_cnt,
+                    void* stream) {
+  if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+  if (!Q || !O) return fail(ZHA_ERR_INVALID, "Q / O is NULL");
+  if ((kept == nullptr) != (kept_cnt == nullptr)) return fail(ZHA_ERR_INVALID, "kept and kept_cnt go together");
+  if (m < 1) return fail(ZHA_ERR_INVALID, "m must be >= 1");
+  if (t->n < 1) return fail(ZHA_ERR_INVALID, "routing needs at least one cached token");
+  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)
+    return fail(ZHA_ERR_INVALID, "Q and O must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int hq = t->cfg.n_q_heads, d = t->cfg.d, es = elem_size(t->cfg.dtype);
+  const int64_t cap1 = t->L.cap_nodes[1];
+  for (int64_t q0 = 0; q0 < m; q0 += t->cfg.max_batch) {
+    const int B = int(min64(t->cfg.max_batch, m - q0));
+    if (t->flow_dirty) {
+      cudaError_t e = cudaMemsetAsync(t->scratch + t->L.flow_off, 0, t->L.flow_bytes, st);
+      if (e != cudaSuccess) return fail_cuda(e, "zha_route_multi: clearing the routing state");
+      t->flow_dirty = false;
+    }
+    DecodeArgs a;
+    fill_decode_args(t, static_cast<const char*>(Q) + size_t(q0) * hq * d * es, O + size_t(q0) * hq * d,
+                     kept ? kept + size_t(q0) * hq * cap1 : nullptr, kept_cnt ? kept_cnt + size_t(q0) * hq : nullptr,
+                     nullptr, nullptr, 0, &a);
+    a.nheads = B * hq;
+    a.max_heads = t->cfg.max_batch * hq;
+    a.root_gemm = t->cfg.dtype == ZHA_BF16 ? 1 : 0;
+    cudaError_t e = launch_decode(a, t->cfg.dtype, st);
+    if (e != cudaSuccess) {
+      t->flow_dirty = true;
+      return fail_cuda(e, "zha_route_multi");
+    }
+  }
+  return ZHA_OK;
+}
+
 int zha_decode_step_host(zha_tree* t, const void* k_host, const void* v_host, const void* q_host, float* o_host,
                          int32_t B, void* stream) {
   if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");

@@ -33,6 +33,7 @@ struct DecodeArgs {
   uint32_t p_mant[kMaxLevels];
   int p_shift[kMaxLevels];
   int p_all[kMaxLevels];
+  int root_gemm;                // the first routing step (the roots, shared by every query) as one contraction
 };
 
 struct DenseArgs {

@@ -2150,6 +2150,91 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
   }
 }
 
+// ---------------------------------------------------------------- multi-query first step
+// Every query head starts from the same candidates, the forest roots, so the
+// first routing step of many queries is one dense contraction: the slope rows
+// of each root (R x d, bf16) times the queries of its KV head (d x queries) on
+// the tensor cores (mma.sync m16n8k16: 16 slope rows x 8 query heads, d in
+// 16-wide steps), e = max_j (b_j + q.mu_j / sqrt d) taken over the rows of the
+// accumulator tiles.  One CTA per (root, KV head, block of sequences): the
+// root's record is staged in shared memory once and each warp serves eight
+// query heads of one sequence's GQA group at a time (one n-tile).  The entries go where
+// the scoring kernel puts step 0's (root i at position i of the head's step
+// buffer, with its largest estimate), so the select of step 0 and the later
+// steps run unchanged.  bf16 configurations.
+constexpr int kRootWarps = 8;
+template <int D>
+__global__ void __launch_bounds__(kRootWarps * 32) root_gemm_kernel(const __grid_constant__ DecodeArgs a) {
+  pdl_wait_and_release();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int root = blockIdx.x, kvh = blockIdx.y;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, g = lane >> 2, t4 = lane & 3;
+  const int R = a.t.refs, hq = a.t.hq, G = a.t.group;
+  const int B = a.nheads / hq;
+  const Ctx<__nv_bfloat16, D> c(a);
+  const uint32_t code = root_code(a, root);
+  if (!valid_code(a, code)) return;
+  // the root's record: R slope rows of D bf16, then R fp32 intercepts
+  const unsigned char* rec = reinterpret_cast<const unsigned char*>(a.t.rec(code_level(code), kvh, code_index(code)));
+  const int rec_words = int(a.t.rec_bytes / 16);
+  for (int i = threadIdx.x; i < rec_words; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem_raw)[i] = *reinterpret_cast<const uint4*>(rec + size_t(i) * 16);
+  __syncthreads();
+  const __nv_bfloat16* mu = reinterpret_cast<const __nv_bfloat16*>(smem_raw);
+  const float* bias = reinterpret_cast<const float*>(smem_raw + size_t(R) * D * 2);
+  const int ntiles = (G + 7) / 8;
+  for (int item = blockIdx.z * kRootWarps + wid; item < B * ntiles; item += gridDim.z * kRootWarps) {
+    const int bb = item / ntiles, n0 = (item - bb * ntiles) * 8;
+    // query head of column g of this n-tile: head n0 + g of the KV head's group in sequence bb (columns past
+    // the group read its last head; their results are dropped)
+    const int hcol = bb * hq + kvh * G + min(n0 + g, G - 1);
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.Q) + size_t(hcol) * D + 2 * t4;
+    float best0 = -INFINITY, best1 = -INFINITY;  // columns 2 t4 and 2 t4 + 1
+    for (int m0 = 0; m0 < R; m0 += 16) {
+      const int r0 = min(m0 + g, R - 1), r1 = min(m0 + g + 8, R - 1);
+      const __nv_bfloat16* a0p = mu + size_t(r0) * D + 2 * t4;
+      const __nv_bfloat16* a1p = mu + size_t(r1) * D + 2 * t4;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k0 = 0; k0 < D; k0 += 16) {
+        const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(a0p + k0), *reinterpret_cast<const uint32_t*>(a1p + k0),
+                                *reinterpret_cast<const uint32_t*>(a0p + k0 + 8),
+                                *reinterpret_cast<const uint32_t*>(a1p + k0 + 8)};
+        const uint32_t bf[2] = {*reinterpret_cast<const uint32_t*>(qp + k0), *reinterpret_cast<const uint32_t*>(qp + k0 + 8)};
+        mma_bf16_16816(acc, af, bf);
+      }
+      // rows m0 + g and m0 + g + 8 of columns 2 t4, 2 t4 + 1
+      const int j0 = m0 + g, j1 = m0 + g + 8;
+      if (j0 < R) {
+        best0 = fmaxf(best0, fmaf(acc[0], a.t.inv_sqrt_d, bias[j0]));
+        best1 = fmaxf(best1, fmaf(acc[1], a.t.inv_sqrt_d, bias[j0]));
+      }
+      if (j1 < R) {
+        best0 = fmaxf(best0, fmaf(acc[2], a.t.inv_sqrt_d, bias[j1]));
+        best1 = fmaxf(best1, fmaf(acc[3], a.t.inv_sqrt_d, bias[j1]));
+      }
+    }
+    // the maximum over the rows: lanes with the same t4 (xor over g)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      best0 = fmaxf(best0, __shfl_xor_sync(0xffffffffu, best0, off));
+      best1 = fmaxf(best1, __shfl_xor_sync(0xffffffffu, best1, off));
+    }
+    if (g == 0) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int col = n0 + 2 * t4 + u;
+        if (col >= G) continue;
+        const int h = bb * hq + kvh * G + col;
+        const uint32_t key = desc_key(u == 0 ? best0 : best1);
+        c.keysP(h, 0)[root] = key;
+        c.codesP(h, 0)[root] = code;
+        atomicMax(&c.hstate(h)->kinv[0], ~key);
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host launcher
 static int device_sms() {
   int dev = 0, sms = 0;
@@ -2160,10 +2245,10 @@ static int device_sms() {
 
 // Launch with programmatic stream serialization (see pdl_wait_and_release).
 template <typename... Args>
-static void launch_pdl(void (*kern)(Args...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+static void launch_pdl(void (*kern)(Args...), dim3 grid, unsigned block, size_t smem, cudaStream_t st,
                        Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -2209,6 +2294,17 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   int launches = 0;
   if (routed) {
     for (int s = 0; s < a.n_steps; ++s) {
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (s == 0 && a.root_gemm) {  // the shared first step as one tensor-core contraction
+          const int items = (a.nheads / a.t.hq) * ((a.t.group + 7) / 8);
+          const unsigned zb = unsigned((items + 8 * kRootWarps - 1) / (8 * kRootWarps));
+          launch_pdl(root_gemm_kernel<D>, dim3(unsigned(a.n_roots), unsigned(a.t.hkv), zb), kRootWarps * 32,
+                     size_t(a.t.rec_bytes), st, a);
+          launch_pdl(select_kernel<T, D>, nh, kDecThreads, sizeof(DecSmem), st, a, s);
+          launches += 2;
+          continue;
+        }
+      }
       launch_pdl(score_kernel<T, D>, unsigned(sms), kDecThreads, sizeof(ScoreSmem), st, a, s);
       launch_pdl(select_kernel<T, D>, nh, kDecThreads, sizeof(DecSmem), st, a, s);
       launches += 2;

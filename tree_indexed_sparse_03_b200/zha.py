@@ -39,6 +39,8 @@ _SIGS = {
     "zha_tree_size": (_c.c_int64, [_c.c_void_p]),
     "zha_decode": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_void_p,
                               _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p]),
+    "zha_route_multi": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_void_p,
+                                   _c.c_void_p]),
     "zha_decode_step_host": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                         _c.c_int32, _c.c_void_p]),
     "zha_dense_scratch_bytes": (_c.c_size_t, [_c.c_void_p, _c.c_int32, _c.c_int64]),
@@ -217,6 +219,22 @@ class ZhaTree:
         if scored is not None:
             res.append(scored)
         return tuple(res)
+
+    def route_multi(self, Q: torch.Tensor, *, want_kept: bool = False, stream=None):
+        """Route and attend m queries Q [m, Hq, d] of this context (zha_route_multi).  Returns O [m, Hq, d] fp32
+        (and (kept, kept_cnt) when asked)."""
+        c = self.cfg
+        if Q.dim() != 3 or tuple(Q.shape[1:]) != (c.n_q_heads, c.d) or Q.dtype != TORCH_DTYPE[c.dtype] or not Q.is_cuda:
+            raise ValueError(f"Q must be a CUDA {TORCH_DTYPE[c.dtype]} tensor [m, {c.n_q_heads}, {c.d}]")
+        m = Q.shape[0]
+        Q = Q.contiguous()
+        O = torch.empty(m, c.n_q_heads, c.d, dtype=torch.float32, device=Q.device)
+        kept = cnt = None
+        if want_kept:
+            kept = torch.full((m, c.n_q_heads, max(1, c.capacity // c.block)), -1, dtype=torch.int32, device=Q.device)
+            cnt = torch.zeros(m, c.n_q_heads, dtype=torch.int32, device=Q.device)
+        _check(lib().zha_route_multi(self._h, Q.data_ptr(), O.data_ptr(), m, _ptr(kept), _ptr(cnt), _stream(stream)))
+        return (O, (kept, cnt)) if want_kept else O
 
     def decode_step_host(self, k_host: Optional[torch.Tensor], v_host: Optional[torch.Tensor], q_host: torch.Tensor,
                          o_host: torch.Tensor, stream=None) -> None:
