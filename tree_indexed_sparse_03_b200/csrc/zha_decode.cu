@@ -42,6 +42,7 @@
 //           writes a head's last partial combines the head's partials -> O.
 // The only waits inside a kernel are a scoring warp's waits for its own bulk
 // copies; they are bounded (on running out the kernel raises ZHA_ERR_TIMEOUT).
+#include <cstddef>
 #include <mutex>
 #include <type_traits>
 
@@ -80,17 +81,16 @@ struct HeadState {  // per (sequence, query head)
   float anchor;            // histogram anchor of the step being built (max e of the step before)
   int steps;               // selects done
   int leaf0;               // leaf block 0 kept (token 0 already attended)
-  int ticket;              // attention chunks of the head merged in group results so far
-  int gticket[32];         // per group of attention CTAs: chunks of the head written so far
+  int reserved[33];
   long long pad[7];
 };
 static_assert(sizeof(HeadState) == 256, "HeadState layout");
 
 // Per-head routing state and leaf bitmaps live in one scratch region.  The
 // first select of a decode starts the head's counters from zero, the last
-// one leaves both parities' step extremes cleared, the combining warps reset
-// the tickets and the export clears the bitmap, so a decode leaves the region
-// ready for the next one (after an error status the host zeroes it).
+// one leaves both parities' step extremes cleared and the export clears the
+// bitmap, so a decode leaves the region ready for the next one (after an
+// error status the host zeroes it).
 
 // 32-bit words of a head's leaf bitmap (one bit per level-1 block), a multiple of 4.
 __host__ __device__ __forceinline__ int64_t decode_bitmap_words(int64_t cap_sel) {
@@ -106,7 +106,10 @@ struct __align__(16) DecSmem {
   uint32_t red32[kDecWarps * 2];
   unsigned long long bcast64[4];
   int bcast32[8];
+  DecodeArgs args;  // the kernel arguments, staged (stage_args); last, so that the arrays above keep
+                    // their 16-byte alignment (the argument block is 8 mod 16 bytes long)
 };
+static_assert(offsetof(DecSmem, u) % 16 == 0 && offsetof(DecSmem, hist) % 16 == 0, "16-byte shared accesses");
 
 // Division of 32-bit values by a fixed divisor d >= 2 with a multiply-high and
 // one correction step (m = floor(2^32 / d) underestimates x / d by less than 1).
@@ -294,7 +297,7 @@ __device__ __forceinline__ int find_cut_bin(DecSmem& sm, unsigned long long base
 // within a warp by shuffles), the masses scanned in sorted order, and the cut
 // is the first entry whose running mass reaches T.
 template <class View>
-__device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View& E, int64_t n, float m,
+__device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a, const View E, int64_t n, float m,
                                                             DecSmem& sm, int step) {
   const int tid = threadIdx.x;
   unsigned long long* ks = sm.hist;  // [np] order keys
@@ -355,7 +358,7 @@ __device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, in
 // asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
 // Every thread returns the same value.
 template <class View>
-__device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const View& E, int64_t n, uint32_t kmin,
+__device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const View E, int64_t n, uint32_t kmin,
                                          DecSmem& sm, int h, int step) {
   const int tid = threadIdx.x, lane = tid & 31;
   if (a.p_all[step]) return ~0ull;
@@ -666,7 +669,7 @@ __device__ __forceinline__ unsigned long long warp_first_key(unsigned long long 
 // keys per lane and do real work only for members.  Every thread returns the
 // same value.
 template <class View>
-__device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs& a, const View& E, int64_t n,
+__device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs& a, const View E, int64_t n,
                                                                float r, const unsigned long long* ghist,
                                                                DecSmem& sm, int h, int step) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -972,18 +975,27 @@ __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.
 // The q operand of the estimate, as B fragments of m16n8k16 (column 0 = q, the
 // other columns zero).  The k order of each k-step is a permutation of the
 // dimensions chosen so that a lane's A words are whole 16-byte chunks of a
-// record row: lane (g = lane/4, t = lane%4) reads chunks t*CPL .. t*CPL+CPL-1
-// of its rows; chunk c (8 dims) feeds k-steps 2c' and 2c'+1 (c' = c - t*CPL),
+// record row: lane (g = lane/4, t = lane%4) takes chunk q_chunk(t, c) of its
+// rows as its c-th chunk (c < CPL = D/32), which feeds k-steps 2c and 2c+1,
 // dims 0-3 the first and 4-7 the second, as (k 2t, 2t+1) and (k 2t+8, 2t+9).
-// The same permutation applied to q leaves the dot product unchanged.
-template <int D>
+// The same permutation applied to q leaves the dot product unchanged.  Two
+// chunk orders: interleaved (chunk c*4 + t: the four lanes of a row read 64
+// contiguous bytes, so the two rows of a quarter-warp meet in at most two-way
+// shared-memory bank conflicts), used for the bf16 slope rows; blocked (chunk
+// t*CPL + c: a lane's chunks contiguous), used for the FP4 router rows, whose
+// packed codes a lane reads as one 16-byte word.
+template <int D, bool kInterleave>
+__device__ __forceinline__ int q_chunk(int t, int c) {
+  return kInterleave ? c * 4 + t : t * (D / 32) + c;
+}
+template <int D, bool kInterleave = true>
 __device__ __forceinline__ void q_fragments(const __nv_bfloat16* q, uint32_t (&qf)[D / 16][2], int lane) {
   constexpr int CPL = D / 32;
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int c = 0; c < CPL; ++c) {
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (g == 0) v = *reinterpret_cast<const uint4*>(q + (t * CPL + c) * 8);
+    if (g == 0) v = *reinterpret_cast<const uint4*>(q + q_chunk<D, kInterleave>(t, c) * 8);
     qf[2 * c][0] = v.x;
     qf[2 * c][1] = v.y;
     qf[2 * c + 1][0] = v.z;
@@ -1003,13 +1015,13 @@ __device__ __forceinline__ float score_record_mma(const unsigned char* rec, int 
   float best = -INFINITY;
   for (int m0 = 0; m0 < R; m0 += 16) {
     const int r0 = min(m0 + g, R - 1), r1 = min(m0 + g + 8, R - 1);  // rows past R: any valid row, masked below
-    const unsigned char* p0 = rec + size_t(r0) * D * 2 + t * CPL * 16;
-    const unsigned char* p1 = rec + size_t(r1) * D * 2 + t * CPL * 16;
+    const unsigned char* p0 = rec + size_t(r0) * D * 2 + t * 16;
+    const unsigned char* p1 = rec + size_t(r1) * D * 2 + t * 16;
     float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const uint4 x0 = *reinterpret_cast<const uint4*>(p0 + c * 16);
-      const uint4 x1 = *reinterpret_cast<const uint4*>(p1 + c * 16);
+    for (int c = 0; c < CPL; ++c) {  // chunk q_chunk<D, true>(t, c) = c*4 + t
+      const uint4 x0 = *reinterpret_cast<const uint4*>(p0 + c * 64);
+      const uint4 x1 = *reinterpret_cast<const uint4*>(p1 + c * 64);
       const uint32_t a0[4] = {x0.x, x1.x, x0.y, x1.y};
       const uint32_t a1[4] = {x0.z, x1.z, x0.w, x1.w};
       mma_bf16_16816(c0, a0, qf[2 * c]);
@@ -1026,11 +1038,11 @@ __device__ __forceinline__ float score_record_mma(const unsigned char* rec, int 
   return best;
 }
 
-// The q operand for FP4 router records: the bf16 fragments of q_fragments
-// converted to f16 (exact for the normal f16 range).
+// The q operand for FP4 router records: the bf16 fragments of q_fragments in
+// the blocked chunk order, converted to f16 (exact for the normal f16 range).
 template <int D>
 __device__ __forceinline__ void q_fragments_f16(const __nv_bfloat16* q, uint32_t (&qf)[D / 16][2], int lane) {
-  q_fragments<D>(q, qf, lane);
+  q_fragments<D, false>(q, qf, lane);
 #pragma unroll
   for (int k = 0; k < D / 16; ++k)
 #pragma unroll
@@ -1159,6 +1171,19 @@ __device__ __forceinline__ void pdl_wait_and_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The kernel arguments copied into shared memory by the whole CTA (ends with
+// a CTA barrier).  The select code runs in non-inlined functions that reach
+// the arguments through a reference: with the copy, that reference points to
+// shared memory rather than into the parameter space, and the per-call
+// context each function builds from it stays in registers (no stack frame).
+__device__ __forceinline__ void stage_args(const DecodeArgs& src, DecodeArgs* dst) {
+  static_assert(sizeof(DecodeArgs) % 4 == 0, "argument block of whole words");
+  const uint32_t* from = reinterpret_cast<const uint32_t*>(&src);
+  uint32_t* to = reinterpret_cast<uint32_t*>(dst);
+  for (int i = threadIdx.x; i < int(sizeof(DecodeArgs) / 4); i += blockDim.x) to[i] = from[i];
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- per-call context
 // The scratch regions of one decode call and the views of them every phase uses.
 template <typename T, int D>
@@ -1207,10 +1232,11 @@ struct Ctx {
 // first kSpecEnt keys and codes are fetched together; a larger step's other
 // keys and codes follow once its size is known.
 template <typename T, int D>
-__device__ __noinline__ void export_kept(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h);
+__device__ __noinline__ void export_kept(const DecodeArgs& a, uint32_t* red32, int h);
 
 template <typename T, int D>
-__device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c, DecSmem& sm, int h, int s) {
+__device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h, int s) {
+  const Ctx<T, D> c(a);
   const int tid = threadIdx.x;
   const int par = s & 1;
   const bool last = s + 1 == a.n_steps;
@@ -1346,7 +1372,7 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c
   if (last && a.kept) {
     __threadfence();
     __syncthreads();
-    export_kept(a, c, sm.red32, h);
+    export_kept<T, D>(a, sm.red32, h);
   }
 }
 
@@ -1356,7 +1382,8 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, const Ctx<T, D>& c
 // which it leaves zeroed.  Each warp owns a contiguous run of words: counts,
 // one scan over warps, then writes.
 template <typename T, int D>
-__device__ __noinline__ void export_kept(const DecodeArgs& a, const Ctx<T, D>& c, uint32_t* red32, int h) {
+__device__ __noinline__ void export_kept(const DecodeArgs& a, uint32_t* red32, int h) {
+  const Ctx<T, D> c(a);
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   uint32_t* bm = c.bitmap(h);
   const long long nw = min64((a.nl[1] + 31) / 32, c.bm_words);
@@ -1397,13 +1424,14 @@ __device__ __noinline__ void export_kept(const DecodeArgs& a, const Ctx<T, D>& c
 
 // One CTA per head.
 template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_constant__ DecodeArgs a, int s) {
+__global__ void __launch_bounds__(kDecThreads, 1) select_kernel(const __grid_constant__ DecodeArgs a_param, int s) {
   pdl_wait_and_release();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
-  const Ctx<T, D> c(a);
+  stage_args(a_param, &sm.args);
+  const DecodeArgs& a = sm.args;
   for (int h = blockIdx.x; h < a.nheads; h += gridDim.x) {
-    select_head<T, D>(a, c, sm, h, s);
+    select_head<T, D>(a, sm, h, s);
     __syncthreads();
   }
 }
@@ -1467,9 +1495,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
   const long long total = build_prefix<kDecThreads>(sp.pref, sp.red64, nh);
   const long long u0 = gwarp < 0 ? 0 : total * gwarp / nwarps;
   const long long u1 = gwarp < 0 ? 0 : total * (gwarp + 1) / nwarps;
-  int cur_h = -1;           // lane 0: head of the pending min-key update
-  uint32_t cur_kmin = 0xffffffffu;
-  int cur_ovf = 0;
   for (long long ub = u0; ub < u1; ub += 32) {
     // one record per lane: its head, its position in the head's step buffer
     // (child c of unit u at u*b + c), its node code
@@ -1505,14 +1530,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
     };
     struct Item {
       int h;
-      long long pos;
+      int src;  // the lane holding the record
       uint32_t code;
     };
     auto next_item = [&](Cursor& cur) -> Item {  // the whole warp calls it, in item order
       const int pl = __ffs(cur.rem) - 1;
       Item it;
       it.h = __shfl_sync(0xffffffffu, uh, pl);
-      it.pos = __shfl_sync(0xffffffffu, upos, pl);
+      it.src = pl;
       it.code = __shfl_sync(0xffffffffu, ucode, pl);
       if (++cur.child == per) {
         cur.child = 0;
@@ -1523,6 +1548,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
     Cursor cur_i{mhas, 0};
     Item slot_item[kMaxSlots];
     int issued = 0, done = 0;
+    float my_e = -INFINITY;  // the estimate of this lane's record
     while (done < items) {
       while (issued < items && issued - done < nslot) {
         const Item it = next_item(cur_i);
@@ -1594,28 +1620,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
       if constexpr (kMma) e = fp4 ? score_record_fp4<D>(rec, R, a.t.inv_sqrt_d, qf, lane)
                                   : score_record_mma<D>(rec, R, a.t.inv_sqrt_d, qf, lane);
       else e = score_record_smem<T, D>(rec, R, a.t.inv_sqrt_d, qs, lane);
-      if (lane == 0) {
-        const uint32_t key = desc_key(e);
-        c.keysP(it.h, par)[it.pos] = key;
-        c.codesP(it.h, par)[it.pos] = it.code;
-        if (it.h != cur_h) {  // flush the previous head's min key and overflow flag
-          if (cur_h >= 0) {
-            atomicMax(&c.hstate(cur_h)->kinv[par], ~cur_kmin);
-            if (cur_ovf) atomicOr(&c.hstate(cur_h)->ovf[par], 1);
-          }
-          cur_h = it.h;
-          cur_kmin = 0xffffffffu;
-          cur_ovf = 0;
-        }
-        cur_kmin = min(cur_kmin, key);
-        if (s >= 1) {
-          unsigned long long w;
-          float t;
-          const int bin = anchored_bin(sp.anchor[it.h], key, &w, &t);
-          if (bin < 0) cur_ovf = 1;
-          else atomicAdd(c.histP(it.h, par) + bin, w);
-        }
-      }
+      if (lane == it.src) my_e = e;
       __syncwarp();
       ++done;
       --in_flight;
@@ -1625,10 +1630,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) score_kernel(const __grid_cons
       }
     }
     if (failed) break;
-  }
-  if (lane == 0 && cur_h >= 0) {
-    atomicMax(&c.hstate(cur_h)->kinv[par], ~cur_kmin);
-    if (cur_ovf) atomicOr(&c.hstate(cur_h)->ovf[par], 1);
+    // the batch's entries, one per lane and all lanes at once: (key, code) at
+    // the entry's position, its mass in the head's anchored histogram
+    const uint32_t key = has ? desc_key(my_e) : 0xffffffffu;
+    if (has) {
+      c.keysP(uh, par)[upos] = key;
+      c.codesP(uh, par)[upos] = ucode;
+      if (s >= 1) {
+        unsigned long long w;
+        float t;
+        const int bin = anchored_bin(sp.anchor[uh], key, &w, &t);
+        if (bin < 0) atomicOr(&c.hstate(uh)->ovf[par], 1);
+        else atomicAdd(c.histP(uh, par) + bin, w);
+      }
+    }
+    // the step's smallest key per head (the batch's lanes hold runs of heads;
+    // usually one head)
+    const int h0 = __shfl_sync(0xffffffffu, uh, __ffs(mhas) - 1);
+    if (__all_sync(0xffffffffu, !has || uh == h0)) {
+      const uint32_t km = __reduce_min_sync(0xffffffffu, key);
+      if (lane == 0) atomicMax(&c.hstate(h0)->kinv[par], ~km);
+    } else if (has) {
+      atomicMax(&c.hstate(uh)->kinv[par], ~key);
+    }
   }
 }
 
@@ -1652,24 +1676,27 @@ __device__ __forceinline__ long long att_head_keys(const Ctx<T, D>& c, int h, lo
 
 // The chunk partition of all heads' attended keys over `grid` CTAs: chunk size (>= 32 keys, so that a CTA
 // owns at most about kAttItems chunks), and per-head chunk prefix in pref[0..nh].
+// Each head's attended-key count, kept-leaf count and sink flag are read once
+// and kept in hkeys / hnl / hsink for the chunk loop.
 template <typename T, int D, int NT>
 __device__ __forceinline__ void att_partition(const Ctx<T, D>& c, long long* pref, unsigned long long* red64,
-                                              int grid, long long* chunk_out, long long* total_out) {
+                                              long long* hkeys, int* hnl, unsigned char* hsink, int grid,
+                                              long long* chunk_out, long long* total_out) {
   const int nh = c.nh;
   for (int i = threadIdx.x; i < nh; i += NT) {
     long long nl;
     bool sink;
-    pref[1 + i] = att_head_keys<T, D>(c, i, &nl, &sink);
+    const long long k = att_head_keys<T, D>(c, i, &nl, &sink);
+    hkeys[i] = k;
+    hnl[i] = int(nl);
+    hsink[i] = sink ? 1 : 0;
+    pref[1 + i] = k;
   }
   __syncthreads();
   const long long total_keys = build_prefix<NT>(pref, red64, nh);
   long long chunk = (total_keys + (long long)grid * kAttItems - 1) / ((long long)grid * kAttItems);
   chunk = max64(32, chunk);
-  for (int i = threadIdx.x; i < nh; i += NT) {
-    long long nl;
-    bool sink;
-    pref[1 + i] = (att_head_keys<T, D>(c, i, &nl, &sink) + chunk - 1) / chunk;
-  }
+  for (int i = threadIdx.x; i < nh; i += NT) pref[1 + i] = (hkeys[i] + chunk - 1) / chunk;
   __syncthreads();
   *total_out = build_prefix<NT>(pref, red64, nh);
   *chunk_out = chunk;
@@ -1680,157 +1707,21 @@ __device__ __forceinline__ void att_partition(const Ctx<T, D>& c, long long* pre
 // time (batches of keys: scores first, then one rescale of the running sums),
 // and each CTA merges its chunks per head into one partial.
 constexpr int kAttSlots = kAttItems + 16;  // partial slots of a CTA (per-head rounding adds up to one per head)
+// The attention CTAs' partition of the chunks, written by CTA 0 after the
+// items of the partial slots: [0] the chunk count, [1] the attention grid,
+// [2 + h] the first chunk of head h (h = 0 .. nheads).
+__device__ __forceinline__ long long* att_meta(const DecodeArgs& a, int D) {
+  return reinterpret_cast<long long*>(a.attn_part + size_t(kMaxAttGrid) * kAttSlots * (2 + D));
+}
+
 struct __align__(16) AttSmem {
   float part[kAttSlots][2 + 128];
   long long pref[kMaxHeads + 1];
+  long long hkeys[kMaxHeads];       // attended keys per head
   unsigned long long red64[kAttWarps];
+  int hnl[kMaxHeads];               // kept level-1 blocks per head
+  unsigned char hsink[kMaxHeads];   // token 0 attended as the sink (leaf block 0 not kept)
 };
-
-// ---------------------------------------------------------------- combine
-// Partials (m, l, o[D]) are merged by rescaling to their common max:
-// M = max m_j, L = sum e^(m_j - M) l_j, o = sum e^(m_j - M) o_j, in slot order
-// (deterministic).  One warp; lane owns elements q*32 + lane.  cnt <= 32
-// partials, slot_of(j) their slots (-1: none).
-template <int D, class SlotFn>
-__device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotFn slot_of, float& M, float& L,
-                                               float (&acc)[(D + 31) / 32]) {
-  const int lane = threadIdx.x & 31;
-  constexpr int NQ = (D + 31) / 32;
-  const long long sl = lane < cnt ? slot_of(lane) : -1;
-  const float mj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D)) : -INFINITY;
-  const float lj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D) + 1) : 0.f;
-  M = mj;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  const float sc = (sl >= 0 && mj != -INFINITY) ? expf(mj - M) : 0.f;
-  L = sc * lj;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
-  for (int t0 = 0; t0 < cnt; t0 += 8) {  // 8 partials' loads in flight per lane
-    float x[8][NQ], w[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const long long st = __shfl_sync(0xffffffffu, sl, (t0 + u) & 31);
-      w[u] = __shfl_sync(0xffffffffu, sc, (t0 + u) & 31);
-      const bool ok = t0 + u < cnt && st >= 0;
-#pragma unroll
-      for (int q = 0; q < NQ; ++q)
-        x[u][q] = (ok && q * 32 + lane < D) ? __ldcg(part + size_t(st) * (2 + D) + 2 + q * 32 + lane) : 0.f;
-      if (!ok) w[u] = 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
-  }
-}
-
-// Combine of head h, whose chunks [P0, P1) were spread over attention CTAs in
-// contiguous chunk ranges (CTA cc starts at range_start(cc)).  CTAs form
-// groups of kCombGroup; the warp that writes the last partial of the head in
-// a group merges that group's partials (at most kCombGroup) into the slot of
-// the group's first chunk of the head; the warp that completes the last group
-// merges the group results (at most 32) -> O, the head's statistics and kept
-// count, and resets the head's tickets.  Called by the warp that wrote CTA
-// blockIdx.x's partial of the head, `mine` chunks at slot `seg`.
-constexpr int kCombGroup = 16;
-static_assert(kMaxAttGrid / kCombGroup <= 32, "group results merge in one pass of 32 lanes");
-template <typename T, int D>
-__device__ __noinline__ void combine_head(const DecodeArgs& a, const Ctx<T, D>& c, int h, long long P0, long long P1,
-                                          long long seg, long long mine, long long total_items, int grid) {
-  const int lane = threadIdx.x & 31;
-  constexpr int NQ = (D + 31) / 32;
-  HeadState* hs = c.hstate(h);
-  auto range_start = [&](long long cc) { return cc >= grid ? total_items : (cc * total_items) / (long long)grid; };
-  const int g = int(blockIdx.x) / kCombGroup;
-  const long long g0 = max64(P0, range_start((long long)g * kCombGroup));
-  const long long g1 = min64(P1, range_start((long long)(g + 1) * kCombGroup));
-  // level 1: this group's chunks of the head
-  int done = 0;
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) {
-    const int prev = atomicAdd(&hs->gticket[g], int(mine));
-    done = prev + int(mine) == int(g1 - g0) ? 1 : 0;
-  }
-  if (!__shfl_sync(0xffffffffu, done, 0)) return;
-  __threadfence();
-  const bool one_group = g0 == P0 && g1 == P1;
-  float M, L, acc[NQ];
-  {
-    // partials of the group's CTAs: slot max(P0, start) for each CTA whose range meets [g0, g1)
-    const long long cbase = (long long)g * kCombGroup;
-    auto slot_of = [&](int j) -> long long {
-      const long long cc = cbase + j;
-      if (cc >= grid) return -1;
-      const long long cs = max64(g0, range_start(cc));
-      return (cs < g1 && cs < range_start(cc + 1)) ? cs : -1;
-    };
-    merge_partials<D>(a.attn_part, kCombGroup, slot_of, M, L, acc);
-  }
-  if (!one_group) {
-    float* G = a.attn_part + size_t(g0) * (2 + D);  // the group result replaces its first partial
-    if (lane == 0) {
-      G[0] = M;
-      G[1] = L;
-      hs->gticket[g] = 0;
-    }
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-      if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
-    // level 2: the head's chunks over all groups
-    __threadfence();
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      const int prev = atomicAdd(&hs->ticket, int(g1 - g0));
-      last = prev + int(g1 - g0) == int(P1 - P0) ? 1 : 0;
-    }
-    if (!__shfl_sync(0xffffffffu, last, 0)) return;
-    __threadfence();
-    // groups meeting [P0, P1): the first is the group of the CTA holding chunk P0
-    long long cfirst = (P0 * grid) / max64(total_items, 1);
-    while (cfirst > 0 && range_start(cfirst) > P0) --cfirst;
-    while (cfirst + 1 < grid && range_start(cfirst + 1) <= P0) ++cfirst;
-    const int gfirst = int(cfirst / kCombGroup);
-    const int ngroups = (grid + kCombGroup - 1) / kCombGroup;
-    auto gslot_of = [&](int j) -> long long {
-      const int gg = gfirst + j;
-      if (gg >= ngroups) return -1;
-      const long long s0 = max64(P0, range_start((long long)gg * kCombGroup));
-      const long long s1 = min64(P1, range_start((long long)(gg + 1) * kCombGroup));
-      return s0 < s1 ? s0 : -1;
-    };
-    merge_partials<D>(a.attn_part, min(32, ngroups - gfirst), gslot_of, M, L, acc);
-  }
-#pragma unroll
-  for (int q = 0; q < NQ; ++q)
-    if (q * 32 + lane < D) a.O[size_t(h) * D + q * 32 + lane] = acc[q] / L;
-  if (lane == 0) {
-    const long long n1 = a.nl[1], b = a.t.block;
-    const long long tail = a.n_tokens - n1 * b;
-    long long nl = 0, scored = 0;
-    int l0 = 0, steps = 0;
-    if (a.n_steps > 0 && a.n_roots > 0) {
-      nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
-      l0 = __ldcg(&hs->leaf0);
-      scored = __ldcg(&hs->scored);
-      steps = __ldcg(&hs->steps);
-    }
-    hs->ticket = 0;
-    hs->gticket[g] = 0;
-    if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
-    if (a.stats) {
-      int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
-      st[ZHA_STAT_NODES_SCORED] = scored;
-      st[ZHA_STAT_LEAVES_KEPT] = nl;
-      st[ZHA_STAT_KEYS] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
-      st[ZHA_STAT_STEPS] = steps;
-    }
-  }
-}
 
 // CTAs per SM the attention kernel is compiled for: two for the tensor-core
 // (bf16) path, whose tiles need up to 128 registers, three for the fp32 path.
@@ -1851,7 +1742,16 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
   const long long n1 = a.nl[1];
   const DivU32 divb{uint32_t(b)};  // key index -> (block, token within it); keys per head < 2^31
   long long chunk, total_items;
-  att_partition<T, D, kAttThreads>(c, sm.pref, sm.red64, int(gridDim.x), &chunk, &total_items);
+  att_partition<T, D, kAttThreads>(c, sm.pref, sm.red64, sm.hkeys, sm.hnl, sm.hsink, int(gridDim.x), &chunk,
+                                   &total_items);
+  if (blockIdx.x == 0) {  // the partition, for the combine kernel
+    long long* meta = att_meta(a, D);
+    for (int i = tid; i <= nh; i += kAttThreads) meta[2 + i] = sm.pref[i];
+    if (tid == 0) {
+      meta[0] = total_items;
+      meta[1] = gridDim.x;
+    }
+  }
   const long long c0 = (long long)blockIdx.x * total_items / gridDim.x;
   const long long c1 = min64((long long)(blockIdx.x + 1) * total_items / gridDim.x, c0 + kAttSlots);
   if (tid == 0 && (long long)(blockIdx.x + 1) * total_items / gridDim.x > c1) raise_status(a.t.status, ZHA_ERR_CAPACITY);
@@ -1863,9 +1763,9 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
       const int h = owner_of(sm.pref, nh, it);
       const long long ci = it - sm.pref[h];
       const int kvh = (h % a.t.hq) / a.t.group;
-      long long nl;
-      bool sink;
-      const long long kh = att_head_keys<T, D>(c, h, &nl, &sink);
+      const long long nl = sm.hnl[h];
+      const bool sink = sm.hsink[h] != 0;
+      const long long kh = sm.hkeys[h];
       const long long leaf_keys = nl * b;
       const long long k0 = ci * chunk, k1 = min64(kh, k0 + chunk);
       float qs[EPC];
@@ -2146,7 +2046,143 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
 #pragma unroll
     for (int q = 0; q < (D + 31) / 32; ++q)
       if (q * 32 + lane < D) G[2 + q * 32 + lane] = acc[q];
-    combine_head<T, D>(a, c, h, sm.pref[h], sm.pref[h + 1], seg, send - seg, total_items, int(gridDim.x));
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// Partials (m, l, o[D]) are merged by rescaling to their common max:
+// M = max m_j, L = sum e^(m_j - M) l_j, o = sum e^(m_j - M) o_j, in slot order
+// (deterministic).  One warp; lane owns elements q*32 + lane.  cnt <= 32
+// partials, slot_of(j) their slots (-1: none).
+template <int D, class SlotFn>
+__device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotFn slot_of, float& M, float& L,
+                                               float (&acc)[(D + 31) / 32]) {
+  const int lane = threadIdx.x & 31;
+  constexpr int NQ = (D + 31) / 32;
+  const long long sl = lane < cnt ? slot_of(lane) : -1;
+  const float mj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D)) : -INFINITY;
+  const float lj = sl >= 0 ? __ldcg(part + size_t(sl) * (2 + D) + 1) : 0.f;
+  M = mj;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float sc = (sl >= 0 && mj != -INFINITY) ? expf(mj - M) : 0.f;
+  L = sc * lj;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+  for (int t0 = 0; t0 < cnt; t0 += 8) {  // 8 partials' loads in flight per lane
+    float x[8][NQ], w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const long long st = __shfl_sync(0xffffffffu, sl, (t0 + u) & 31);
+      w[u] = __shfl_sync(0xffffffffu, sc, (t0 + u) & 31);
+      const bool ok = t0 + u < cnt && st >= 0;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        x[u][q] = (ok && q * 32 + lane < D) ? __ldcg(part + size_t(st) * (2 + D) + 2 + q * 32 + lane) : 0.f;
+      if (!ok) w[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
+  }
+}
+
+// Running merge of (M2, L2, acc2) into (M, L, acc) (one warp, same lanes).
+template <int D>
+__device__ __forceinline__ void merge_into(float& M, float& L, float (&acc)[(D + 31) / 32], float M2, float L2,
+                                           const float (&acc2)[(D + 31) / 32]) {
+  constexpr int NQ = (D + 31) / 32;
+  const float Mn = fmaxf(M, M2);
+  const float s1 = M == -INFINITY ? 0.f : expf(M - Mn), s2 = M2 == -INFINITY ? 0.f : expf(M2 - Mn);
+  L = L * s1 + L2 * s2;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = acc[q] * s1 + acc2[q] * s2;
+  M = Mn;
+}
+
+// One CTA per head, after the attention kernel.  The head's chunks [P0, P1)
+// were spread over attention CTAs in contiguous chunk ranges (CTA cc starts at
+// range_start(cc)); every CTA whose range meets them wrote one partial, at the
+// slot max(P0, range_start(cc)).  Warp w merges the partials of CTAs
+// cfirst + w*32 .. (in blocks of 32, every kCombWarps-th block), then warp 0
+// merges the warps' results in warp order -> O, and writes the head's kept
+// count and statistics.  The order of every sum is fixed (deterministic).
+constexpr int kCombWarps = 8;
+template <typename T, int D>
+__global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const __grid_constant__ DecodeArgs a) {
+  pdl_wait_and_release();
+  constexpr int NQ = (D + 31) / 32;
+  __shared__ float wres[kCombWarps][2 + D];
+  const Ctx<T, D> c(a);
+  const int h = blockIdx.x, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const long long* meta = att_meta(a, D);
+  const long long total_items = __ldcg(meta), grid = max64(__ldcg(meta + 1), 1);
+  const long long P0 = __ldcg(meta + 2 + h), P1 = __ldcg(meta + 3 + h);
+  auto range_start = [&](long long cc) { return cc >= grid ? total_items : (cc * total_items) / grid; };
+  // attention CTAs holding chunk P0 and chunk P1 - 1
+  auto cta_of = [&](long long item) {
+    long long cc = (item * grid) / max64(total_items, 1);
+    while (cc > 0 && range_start(cc) > item) --cc;
+    while (cc + 1 < grid && range_start(cc + 1) <= item) ++cc;
+    return cc;
+  };
+  const long long cfirst = P1 > P0 ? cta_of(P0) : 0, clast = P1 > P0 ? cta_of(P1 - 1) : -1;
+  const int S = int(clast - cfirst + 1);  // partials of the head (<= grid)
+  auto slot_of = [&](long long cc) -> long long {
+    const long long s0 = max64(P0, range_start(cc)), s1 = min64(P1, range_start(cc + 1));
+    return s0 < s1 ? s0 : -1;
+  };
+  float M = -INFINITY, L = 0.f, acc[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+  for (int base = wid * 32; base < S; base += kCombWarps * 32) {
+    float M2, L2, acc2[NQ];
+    merge_partials<D>(a.attn_part, min(32, S - base), [&](int j) { return slot_of(cfirst + base + j); }, M2, L2,
+                      acc2);
+    merge_into<D>(M, L, acc, M2, L2, acc2);
+  }
+  if (lane == 0) {
+    wres[wid][0] = M;
+    wres[wid][1] = L;
+  }
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+    if (q * 32 + lane < D) wres[wid][2 + q * 32 + lane] = acc[q];
+  __syncthreads();
+  if (wid != 0) return;
+  for (int w = 1; w < kCombWarps; ++w) {
+    float acc2[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) acc2[q] = q * 32 + lane < D ? wres[w][2 + q * 32 + lane] : 0.f;
+    merge_into<D>(M, L, acc, wres[w][0], wres[w][1], acc2);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;  // (a head always attends a key; guard the empty case)
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+    if (q * 32 + lane < D) a.O[size_t(h) * D + q * 32 + lane] = acc[q] * inv;
+  if (lane == 0) {
+    HeadState* hs = c.hstate(h);
+    const long long n1 = a.nl[1], b = a.t.block;
+    const long long tail = a.n_tokens - n1 * b;
+    long long nl = 0, scored = 0;
+    int l0 = 0, steps = 0;
+    if (a.n_steps > 0 && a.n_roots > 0) {
+      nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
+      l0 = __ldcg(&hs->leaf0);
+      scored = __ldcg(&hs->scored);
+      steps = __ldcg(&hs->steps);
+    }
+    if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
+    if (a.stats) {
+      int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
+      st[ZHA_STAT_NODES_SCORED] = scored;
+      st[ZHA_STAT_LEAVES_KEPT] = nl;
+      st[ZHA_STAT_KEYS] = nl * b + ((n1 > 0 && !l0) ? 1 : 0) + tail;
+      st[ZHA_STAT_STEPS] = steps;
+    }
   }
 }
 
@@ -2312,7 +2348,8 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
   }
   const int att_grid = min(kMaxAttGrid, att_ctas_per_sm<T>() * sms);  // one wave
   launch_pdl(attend_kernel<T, D>, unsigned(att_grid), kAttThreads, sizeof(AttSmem), st, a);
-  launches += 1;
+  launch_pdl(combine_kernel<T, D>, nh, kCombWarps * 32, 0, st, a);
+  launches += 2;
   count_launches(launches);
   return cudaGetLastError();
 }
