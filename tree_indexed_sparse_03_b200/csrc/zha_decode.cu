@@ -340,21 +340,6 @@ __device__ __noinline__ unsigned long long select_cut_small(const DecodeArgs& a,
 }
 
 // The cut of one routing step: the largest 64-bit order key (e desc, start
-// asc) that is kept.  Every thread returns the same value.
-// Smallest key in [lo, 2^32) whose bin (a monotone non-decreasing function of
-// the key over the keys that occur) is >= target; 2^32 if none.  Every thread
-// computes it (32 steps), so no broadcast is needed.
-template <typename BinFn>
-__device__ __forceinline__ unsigned long long first_key_at_least(uint32_t lo, int target, BinFn bin) {
-  unsigned long long L = lo, H = 0x100000000ull;  // answer in [L, H]
-  while (L < H) {
-    const unsigned long long mid = (L + H) >> 1;
-    if (bin(uint32_t(mid)) >= target) H = mid; else L = mid + 1;
-  }
-  return L;
-}
-
-// The cut of one routing step: the largest 64-bit order key (e desc, start
 // asc) that is kept.  kmin is the smallest key (largest estimate) of the step.
 // Every thread returns the same value.
 template <class View>
@@ -402,12 +387,10 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   unsigned long long below;
   const int cb = find_cut_bin(sm, 0ull, T, &below);
   if (cb < 0) return ~0ull;  // cannot happen for 0 < p < 1; keep everything
-  auto cbin = [&](uint32_t k) { return coarse_bin(entry_gap(m, k)); };
-  // keys of coarse bin cb form the contiguous range [klo, khi)
-  const unsigned long long klo = first_key_at_least(kmin, cb, cbin);
-  const unsigned long long khi = cb + 1 < kBins ? first_key_at_least(uint32_t(klo), cb + 1, cbin) : 0x100000000ull;
+  // members of the coarse bin cb (the bin is monotone in the key: one contiguous key range)
+  auto in_cb = [&](uint32_t k) { return coarse_bin(entry_gap(m, k)) == cb; };
 
-  // fine histogram inside the cut coarse bin: the fine cut bin's key range
+  // fine histogram inside the cut coarse bin
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
   __syncthreads();
   for (int base = wlo; base < whi; base += 32 * U) {
@@ -420,7 +403,7 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
       w[u] = 0;
       if (i < whi) {
         const uint32_t k = E.key(i);
-        if (k >= klo && k < khi) {
+        if (in_cb(k)) {
           bin[u] = fine_bin(entry_gap(m, k), cb);
           w[u] = entry_mass(m, k);
         }
@@ -433,14 +416,10 @@ __device__ __noinline__ unsigned long long select_cut(const DecodeArgs& a, const
   unsigned long long below2;
   const int fb = find_cut_bin(sm, below, T, &below2);
   if (fb < 0) return ~0ull;
-  auto fbin = [&](uint32_t k) {
+  auto in_cut = [&](uint32_t k) {  // a member of the cut fine bin
     const float x = entry_gap(m, k);
-    return coarse_bin(x) > cb ? kBins : fine_bin(x, cb);
+    return coarse_bin(x) == cb && fine_bin(x, cb) == fb;
   };
-  const unsigned long long flo = first_key_at_least(uint32_t(klo), fb, fbin);
-  unsigned long long fhi = fb + 1 < kBins ? first_key_at_least(uint32_t(flo), fb + 1, fbin) : khi;
-  if (fhi > khi) fhi = khi;
-  auto in_cut = [&](uint32_t k) { return k >= flo && k < fhi; };
 
   // gather the entries around the cut
   if (tid == 0) sm.bcast32[1] = 0;
@@ -635,44 +614,20 @@ __device__ __forceinline__ long long anchored_code_of(float r, uint32_t key) {
   return (long long)b * kBins + anchored_fine(t);
 }
 
-// Smallest key in [lo, 2^32) whose f(key) >= target, for f monotone
-// non-decreasing over the keys; 2^32 if none.  One warp, 32-ary search: each
-// round the lanes probe 32 keys spread over the remaining interval (7 rounds
-// for 2^32 keys).  Every lane returns the answer.
-template <typename F>
-__device__ __forceinline__ unsigned long long warp_first_key(unsigned long long lo, long long target, F f) {
-  const int lane = threadIdx.x & 31;
-  unsigned long long L = lo, H = 0x100000000ull;  // answer in [L, H]
-  while (L < H) {
-    const unsigned long long span = H - L;
-    const unsigned long long p = L + (span * unsigned(lane)) / 32u;
-    const bool ge = f(uint32_t(p)) >= target;
-    const unsigned m = __ballot_sync(0xffffffffu, ge);
-    if (m == 0u) {
-      L = __shfl_sync(0xffffffffu, p, 31) + 1;  // all probes below: past the last one
-    } else {
-      const int j = __ffs(m) - 1;
-      const unsigned long long pj = __shfl_sync(0xffffffffu, p, j);
-      if (j == 0) return pj;  // the first probe is L itself
-      L = __shfl_sync(0xffffffffu, p, j - 1) + 1;
-      H = pj;
-    }
-  }
-  return L;
-}
 
 // The cut of a step from its anchored histogram (global, kBins sums): the
-// coarse cut bin from the histogram alone; the exact key ranges of that bin
-// and of its sub-bins from warp searches; one pass over the keys for the
-// sub-bin histogram of the bin's members, one more to gather the members of
-// the cut sub-bin, which are ordered by (e desc, start asc).  Passes read four
-// keys per lane and do real work only for members.  Every thread returns the
-// same value.
+// coarse cut bin from the histogram alone; one pass over the keys for the
+// sub-bin histogram of that bin's members, one more to gather the members of
+// the cut sub-bin, which are ordered by (e desc, start asc).  Membership is
+// tested on each key's (bin, sub-bin), both monotone in the key, so the
+// members are exactly the keys of one contiguous key range.  Passes read four
+// keys per lane and do the mass work only for members.  Every thread returns
+// the same value.
 template <class View>
 __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs& a, const View E, int64_t n,
                                                                float r, const unsigned long long* ghist,
                                                                DecSmem& sm, int h, int step) {
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int tid = threadIdx.x;
   constexpr int BPT = kBins / kDecThreads;
   double* red = reinterpret_cast<double*>(sm.red64);
   const double p = ldexp(double(a.p_mant[step]), -a.p_shift[step]);
@@ -690,15 +645,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
   const int cb = find_cut_bin_f64(sm, mb, before, T, &below_c);
   if (cb < 0) return ~0ull;  // rounding kept T out of reach: keep everything
   const double sc = anchored_scale(cb);
-  // key range [klo, khi) of the coarse bin
-  if (wid < 2) {
-    const unsigned long long k =
-        warp_first_key(0ull, cb + wid, [&](uint32_t key) { return (long long)anchored_bin_of(r, key); });
-    if (lane == 0) sm.bcast64[wid] = k;
-  }
   for (int i = tid; i < kBins; i += kDecThreads) sm.hist[i] = 0ull;
-  __syncthreads();
-  const unsigned long long klo = sm.bcast64[0], khi = sm.bcast64[1];
   __syncthreads();
   const int n32 = int(n);
   // sub-bin histogram of the members (exact integer masses), four keys per lane
@@ -722,7 +669,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     for (int u = 0; u < 4; ++u) {
       int fb = -1;
       unsigned long long w = 0;
-      if (k[u] >= klo && k[u] < khi) {
+      if (anchored_bin_of(r, k[u]) == cb) {  // a member of the coarse bin
         float t;
         anchored_bin(r, k[u], &w, &t);
         fb = anchored_fine(t);
@@ -755,15 +702,8 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     below_f = below_c + double(pre) * sc;
     __syncthreads();
   }
-  // key range [flo, fhi) of the cut sub-bin
-  if (wid < 2) {
-    const long long target = (long long)cb * kBins + fbin + wid;
-    const unsigned long long k = warp_first_key(klo, target, [&](uint32_t key) { return anchored_code_of(r, key); });
-    if (lane == 0) sm.bcast64[2 + wid] = min(k, khi);
-  }
+  const long long fcode = (long long)cb * kBins + fbin;  // (coarse bin, sub-bin) of the cut
   if (tid == 0) sm.bcast32[1] = 0;
-  __syncthreads();
-  const unsigned long long flo = sm.bcast64[2], fhi = sm.bcast64[3];
   __syncthreads();
   // gather the members of the cut sub-bin
   for (int i0 = 4 * tid; i0 < n32; i0 += 4 * kDecThreads) {
@@ -771,7 +711,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     keys4(i0, k);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (k[u] >= flo && k[u] < fhi) {
+      if (anchored_code_of(r, k[u]) == fcode) {
         unsigned long long w;
         float t;
         anchored_bin(r, k[u], &w, &t);
@@ -827,7 +767,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
     __syncthreads();
     for (int i = tid; i < n32; i += kDecThreads) {
       const uint32_t k = E.key(i);
-      if (!(k >= flo && k < fhi)) continue;
+      if (anchored_code_of(r, k) != fcode) continue;
       unsigned long long w;
       float t;
       anchored_bin(r, k, &w, &t);
