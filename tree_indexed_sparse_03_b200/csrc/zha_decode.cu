@@ -191,15 +191,17 @@ __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long 
   }
   if (lane == 31) red[wid] = x;
   __syncthreads();
-  unsigned long long base = 0, tot = 0;
-  for (int w = 0; w < NW; ++w) {
-    const unsigned long long s = red[w];
-    if (w < wid) base += s;
-    tot += s;
+  // the warp totals, scanned across lanes (NW <= 32)
+  unsigned long long t = lane < NW ? red[lane] : 0ull;
+#pragma unroll
+  for (int off = 1; off < NW; off <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, t, off);
+    if (lane >= off) t += y;
   }
+  const unsigned long long base = __shfl_sync(0xffffffffu, t, (wid + 31) & 31);
+  *total = __shfl_sync(0xffffffffu, t, NW - 1);
   __syncthreads();
-  *total = tot;
-  return base + x - v;
+  return (wid > 0 ? base : 0ull) + x - v;
 }
 
 
@@ -245,6 +247,7 @@ __device__ __forceinline__ void smem_max_s32(int* p, int v) {
 // them fit 32 bits) and added by one lane; the remaining lanes add their own.
 // Every lane of the warp must call it.
 __device__ __forceinline__ void hist_add_warp(unsigned long long* hist, int bin, unsigned long long w) {
+  if (!__any_sync(0xffffffffu, bin >= 0)) return;
   const int lane = threadIdx.x & 31;
   const int b0 = __shfl_sync(0xffffffffu, bin, 0);
   const int b1 = __shfl_sync(0xffffffffu, bin, 31);
@@ -563,14 +566,17 @@ __device__ __forceinline__ double block_scan_f64(double v, double* red, double* 
   if (lane == 0) ex = 0.0;
   if (lane == 31) red[wid] = x;
   __syncthreads();
-  double base = 0.0, tot = 0.0;
-  for (int w = 0; w < kDecWarps; ++w) {
-    if (w < wid) base += red[w];
-    tot += red[w];
+  // the warp totals, scanned across lanes in warp order
+  double t = lane < kDecWarps ? red[lane] : 0.0;
+#pragma unroll
+  for (int off = 1; off < kDecWarps; off <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, t, off);
+    if (lane >= off) t += y;
   }
+  const double base = __shfl_sync(0xffffffffu, t, (wid + 31) & 31);
+  *total = __shfl_sync(0xffffffffu, t, kDecWarps - 1);
   __syncthreads();
-  *total = tot;
-  return base + ex;
+  return (wid > 0 ? base : 0.0) + ex;
 }
 
 // First of kBins per-thread-blocked bin masses (BPT consecutive bins per
@@ -1994,6 +2000,7 @@ __global__ void __launch_bounds__(kAttThreads, att_ctas_per_sm<T>()) attend_kern
 // M = max m_j, L = sum e^(m_j - M) l_j, o = sum e^(m_j - M) o_j, in slot order
 // (deterministic).  One warp; lane owns elements q*32 + lane.  cnt <= 32
 // partials, slot_of(j) their slots (-1: none).
+constexpr int kMergeBatch = 16;
 template <int D, class SlotFn>
 __device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotFn slot_of, float& M, float& L,
                                                float (&acc)[(D + 31) / 32]) {
@@ -2011,10 +2018,10 @@ __device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotF
   for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
 #pragma unroll
   for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
-  for (int t0 = 0; t0 < cnt; t0 += 8) {  // 8 partials' loads in flight per lane
-    float x[8][NQ], w[8];
+  for (int t0 = 0; t0 < cnt; t0 += kMergeBatch) {  // kMergeBatch partials' loads in flight per lane
+    float x[kMergeBatch][NQ], w[kMergeBatch];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kMergeBatch; ++u) {
       const long long st = __shfl_sync(0xffffffffu, sl, (t0 + u) & 31);
       w[u] = __shfl_sync(0xffffffffu, sc, (t0 + u) & 31);
       const bool ok = t0 + u < cnt && st >= 0;
@@ -2024,7 +2031,7 @@ __device__ __forceinline__ void merge_partials(const float* part, int cnt, SlotF
       if (!ok) w[u] = 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < kMergeBatch; ++u)
 #pragma unroll
       for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w[u], x[u][q], acc[q]);
   }
@@ -2046,11 +2053,12 @@ __device__ __forceinline__ void merge_into(float& M, float& L, float (&acc)[(D +
 // One CTA per head, after the attention kernel.  The head's chunks [P0, P1)
 // were spread over attention CTAs in contiguous chunk ranges (CTA cc starts at
 // range_start(cc)); every CTA whose range meets them wrote one partial, at the
-// slot max(P0, range_start(cc)).  Warp w merges the partials of CTAs
-// cfirst + w*32 .. (in blocks of 32, every kCombWarps-th block), then warp 0
-// merges the warps' results in warp order -> O, and writes the head's kept
-// count and statistics.  The order of every sum is fixed (deterministic).
-constexpr int kCombWarps = 8;
+// slot max(P0, range_start(cc)).  Warp w merges a contiguous block of at most
+// 32 of those partials (kMaxAttGrid / kCombWarps), then warp 0 merges the
+// warps' results in warp order -> O, and writes the head's kept count and
+// statistics.  The order of every sum is fixed (deterministic).
+constexpr int kCombWarps = 16;
+static_assert(kMaxAttGrid <= 32 * kCombWarps, "a warp merges at most 32 partials");
 template <typename T, int D>
 __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const __grid_constant__ DecodeArgs a) {
   pdl_wait_and_release();
@@ -2075,14 +2083,24 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const __grid_c
     const long long s0 = max64(P0, range_start(cc)), s1 = min64(P1, range_start(cc + 1));
     return s0 < s1 ? s0 : -1;
   };
+  // the head's counters, loaded now (they do not depend on the merge)
+  HeadState* hs = c.hstate(h);
+  long long nl = 0, scored = 0;
+  int l0 = 0, steps = 0;
+  if (wid == 0 && lane == 0 && a.n_steps > 0 && a.n_roots > 0) {
+    nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
+    l0 = __ldcg(&hs->leaf0);
+    scored = __ldcg(&hs->scored);
+    steps = __ldcg(&hs->steps);
+  }
   float M = -INFINITY, L = 0.f, acc[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
-  for (int base = wid * 32; base < S; base += kCombWarps * 32) {
-    float M2, L2, acc2[NQ];
-    merge_partials<D>(a.attn_part, min(32, S - base), [&](int j) { return slot_of(cfirst + base + j); }, M2, L2,
-                      acc2);
-    merge_into<D>(M, L, acc, M2, L2, acc2);
+  {
+    const int per = (S + kCombWarps - 1) / kCombWarps;  // <= 32
+    const int j0 = min(S, wid * per), j1 = min(S, j0 + per);
+    if (j1 > j0)
+      merge_partials<D>(a.attn_part, j1 - j0, [&](int j) { return slot_of(cfirst + j0 + j); }, M, L, acc);
   }
   if (lane == 0) {
     wres[wid][0] = M;
@@ -2104,17 +2122,8 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const __grid_c
   for (int q = 0; q < NQ; ++q)
     if (q * 32 + lane < D) a.O[size_t(h) * D + q * 32 + lane] = acc[q] * inv;
   if (lane == 0) {
-    HeadState* hs = c.hstate(h);
     const long long n1 = a.nl[1], b = a.t.block;
     const long long tail = a.n_tokens - n1 * b;
-    long long nl = 0, scored = 0;
-    int l0 = 0, steps = 0;
-    if (a.n_steps > 0 && a.n_roots > 0) {
-      nl = min64(max64(__ldcg(&hs->n_leaf), 0), a.cap_list);
-      l0 = __ldcg(&hs->leaf0);
-      scored = __ldcg(&hs->scored);
-      steps = __ldcg(&hs->steps);
-    }
     if (a.kept_cnt) a.kept_cnt[h] = int32_t(nl);
     if (a.stats) {
       int64_t* st = a.stats + size_t(h) * ZHA_STAT_COUNT;
