@@ -621,7 +621,8 @@ __device__ __forceinline__ long long anchored_code_of(float r, uint32_t key) {
 }
 
 
-// The cut of a step from its anchored histogram (global, kBins sums): the
+// The cut of a step from its anchored histogram (kBins sums; ghist is the
+// caller's shared-memory copy in sm.hist, read before sm.hist is reused): the
 // coarse cut bin from the histogram alone; one pass over the keys for the
 // sub-bin histogram of that bin's members, one more to gather the members of
 // the cut sub-bin, which are ordered by (e desc, start asc).  Membership is
@@ -641,7 +642,7 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
 #pragma unroll
   for (int k = 0; k < BPT; ++k) {
     const int bin = tid * BPT + k;
-    mb[k] = double(__ldcg(ghist + bin)) * anchored_scale(bin);
+    mb[k] = double(ghist[bin]) * anchored_scale(bin);
     loc += mb[k];
   }
   double Z;
@@ -963,20 +964,24 @@ __device__ __forceinline__ float score_record_mma(const unsigned char* rec, int 
     const int r0 = min(m0 + g, R - 1), r1 = min(m0 + g + 8, R - 1);  // rows past R: any valid row, masked below
     const unsigned char* p0 = rec + size_t(r0) * D * 2 + t * 16;
     const unsigned char* p1 = rec + size_t(r1) * D * 2 + t * 16;
-    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    // four independent accumulators: chunk c's two k-steps go to
+    // cc[2 (c & 1)] and cc[2 (c & 1) + 1], chains of CPL / 2 products each
+    float cc[4][4] = {};
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {  // chunk q_chunk<D, true>(t, c) = c*4 + t
       const uint4 x0 = *reinterpret_cast<const uint4*>(p0 + c * 64);
       const uint4 x1 = *reinterpret_cast<const uint4*>(p1 + c * 64);
       const uint32_t a0[4] = {x0.x, x1.x, x0.y, x1.y};
       const uint32_t a1[4] = {x0.z, x1.z, x0.w, x1.w};
-      mma_bf16_16816(c0, a0, qf[2 * c]);
-      mma_bf16_16816(c1, a1, qf[2 * c + 1]);
+      mma_bf16_16816(cc[2 * (c & 1)], a0, qf[2 * c]);
+      mma_bf16_16816(cc[2 * (c & 1) + 1], a1, qf[2 * c + 1]);
     }
     if (t == 0) {
       const int j0 = m0 + g, j1 = m0 + g + 8;
-      if (j0 < R) best = fmaxf(best, fmaf(c0[0] + c1[0], inv_sqrt_d, bias[j0]));
-      if (j1 < R) best = fmaxf(best, fmaf(c0[2] + c1[2], inv_sqrt_d, bias[j1]));
+      const float s0 = (cc[0][0] + cc[1][0]) + (cc[2][0] + cc[3][0]);
+      const float s1 = (cc[0][2] + cc[1][2]) + (cc[2][2] + cc[3][2]);
+      if (j0 < R) best = fmaxf(best, fmaf(s0, inv_sqrt_d, bias[j0]));
+      if (j1 < R) best = fmaxf(best, fmaf(s1, inv_sqrt_d, bias[j1]));
     }
   }
 #pragma unroll
@@ -1197,6 +1202,10 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
     cp_async16(ck + 4 * v, gk + 4 * v);
     cp_async16(cc + 4 * v, gc + 4 * v);
   }
+  if (s >= 1) {  // the step's anchored histogram, for the anchored cut (every other cut rewrites sm.hist)
+    const unsigned long long* gh = c.histP(h, par);
+    for (int v = tid; v < kBins / 2; v += kDecThreads) cp_async16(sm.hist + 2 * v, gh + 2 * v);
+  }
   cp_async_commit();
   // step 0 starts the head's counters afresh
   const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
@@ -1226,7 +1235,7 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
   if (!a.p_all[s] && n > 0) {
     if (n <= kDecThreads) cut = select_cut_small(a, E, n, m, sm, s);
     else if (s >= 1 && !ovf && __fsub_rn(anchor_h, m) <= kAnchorFar)
-      cut = select_cut_anchored(a, E, n, anchor_h, c.histP(h, par), sm, h, s);
+      cut = select_cut_anchored(a, E, n, anchor_h, sm.hist, sm, h, s);
     else cut = select_cut(a, E, n, kmin, sm, h, s);
   }
   // the kept entries (order key <= cut) in entry order, four per thread and
