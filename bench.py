@@ -282,7 +282,7 @@ def parity_sample(w, inp, tree, Qs, runs):
     otree = zo.build_tree(f64(inp.K[0, :n]), f64(inp.refs[0]), n, w.block, w.levels)
     out = {"sample": f"query heads 0-{w.group - 1} (KV head 0), batch element 0, query sets "
                      f"{[r[0] for r in runs]}, N={n}", "heads": 0, "exact": 0, "flagged": 0, "failed": 0}
-    jac, err, err_m, att = [], [], [], 0.0
+    jac, err, err_m, att, kept_mass = [], [], [], 0.0, []
     for qi, O, kept, cnt in runs:
         Q = Qs[qi].cpu()
         rep = compare_route(tree, Q, kept, cnt, p, n, w.block, w.levels, w.group, heads=heads)
@@ -295,6 +295,7 @@ def parity_sample(w, inp, tree, Qs, runs):
         e2e = end_to_end(inp.K, inp.V, inp.refs, Q, O, kept, cnt, n, w.block, w.levels, p, w.group, 0, (0,),
                          oracle_tree=otree)
         jac += e2e.jaccard
+        kept_mass += e2e.retained
         err += e2e.err
         err_m += e2e.err_matched
     out["attend_max_abs_err"] = att
@@ -303,6 +304,11 @@ def parity_sample(w, inp, tree, Qs, runs):
     out["e2e_matched_sets"] = len(err_m)
     out["max_abs_err"] = float(np.max(err)) if err else None
     out["max_abs_err_matched"] = float(np.max(err_m)) if err_m else None
+    # estimated attention mass the oracle's routes keep over the whole descent, against the product of the
+    # step thresholds that bounds it from below
+    out["retained_mass_mean"] = round(float(np.mean(kept_mass)), 5) if kept_mass else None
+    out["retained_mass_min"] = round(float(np.min(kept_mass)), 5) if kept_mass else None
+    out["retained_mass_bound"] = round(p ** w.levels, 5)
     out["seconds"] = round(time.perf_counter() - t0, 1)
     return out
 
@@ -561,8 +567,8 @@ def run_zha(args, world, rank, local):
         "route_bytes": int(statistics.mean(route_b)),
         "attend_bytes": int(statistics.mean(attend_b)),
         "roofline": {"bound": "hbm",
-                     "kernel": "zha_decode call: per routing step a scoring and a select kernel, then one "
-                               "attention kernel",
+                     "kernel": "zha_decode call: per routing step a scoring and a select kernel, then the "
+                               "attention and combine kernels",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_8tbs": round(achieved / 8000.0, 4), "traffic": measured_traffic(w.name),

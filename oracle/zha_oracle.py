@@ -356,6 +356,18 @@ def route(planes: PlanesFn, q: np.ndarray, p, n_tokens: int, block: int,
     return trace
 
 
+def retained_mass(trace: RouteTrace) -> float:
+    """Estimated attention mass a route keeps: the product over its steps of the
+    share of the step's candidate mass (the softmax of their estimates) that the
+    step keeps.  The blog's section on attention becoming too sparse notes that
+    keeping a fixed share of the probability at every level keeps, after the
+    whole descent, a share of the original mass that shrinks with depth; each
+    step keeps at least its threshold, so the product is at least the product
+    of the thresholds of the steps taken (1 when every step keeps everything).
+    """
+    return float(np.prod([st.cum[st.k - 1] if st.k > 0 else 0.0 for st in trace.steps]))
+
+
 def route_multi(planes: PlanesFn, Qm: np.ndarray, p, n_tokens: int, block: int,
                 levels: int) -> List[RouteTrace]:
     """Routing of m queries of one context (e.g. the queries of a prefill chunk): each query head is routed

@@ -260,6 +260,39 @@ def pin_step_thresholds(zo):
                 assert step.k == _brute_top_p(step.ehat, start, ps), (trial, s, step.k)
 
 
+def pin_retained_mass(zo):
+    """The retained estimated mass of a route: every step keeps at least its threshold of its candidates'
+    softmax mass, so the product is at least the product of the thresholds and at most 1; a route with every
+    threshold 1 keeps all of it (up to rounding); with threshold 1 at the roots and x at the next step the retained
+    mass is that second step's kept share, summed here directly over the kept candidates' estimates."""
+    rng = _rng(23)
+    d = 8
+    for trial in range(12):
+        b = int(rng.integers(2, 5))
+        L = int(rng.integers(2, 4))
+        n = int(rng.integers(b ** 2, min(b ** (L + 1) * 2, 60)))
+        K = rng.normal(size=(n, d)) * 2
+        refs = rng.normal(size=(2, d))
+        tree = zo.build_tree(K, refs, n, b, L)
+        pf = zo.tree_planes_fn(tree)
+        q = rng.normal(size=d) * 2
+        sched = [float(x) for x in rng.choice([0.3, 0.6, 0.9, 0.99], size=L)]
+        trace = zo.route(pf, q, sched, n, b, L)
+        r = zo.retained_mass(trace)
+        bound = float(np.prod([st.p for st in trace.steps]))
+        assert bound - 1e-12 <= r <= 1 + 1e-12, (trial, r, bound)
+        assert abs(zo.retained_mass(zo.route(pf, q, 1.0, n, b, L)) - 1.0) <= 1e-12
+        x = float(rng.choice([0.5, 0.8]))
+        tr2 = zo.route(pf, q, [1.0, x], n, b, L)
+        if len(tr2.steps) == 2:  # (two levels: the roots, then the children of the kept top nodes)
+            st = tr2.steps[1]
+            kept = st.order[: st.k]
+            w = np.exp(st.ehat - st.ehat.max())
+            share = w[kept].sum() / w.sum()
+            assert abs(zo.retained_mass(tr2) - share) <= 1e-12, (trial, zo.retained_mass(tr2), share)
+            assert share >= x - 1e-12
+
+
 def pin_e4m3_grid(zo):
     """Every finite non-negative e4m3 encoding decodes to its value and rounds back to itself; the values
     rise strictly from 0 through 2^-9 (smallest subnormal) and 2^-6 (smallest normal) to 448."""

@@ -296,13 +296,16 @@ class EndToEnd:
     jaccard: List[float] = field(default_factory=list)
     err: List[float] = field(default_factory=list)
     err_matched: List[float] = field(default_factory=list)
+    retained: List[float] = field(default_factory=list)  # the oracle route's retained estimated mass per head
 
     def summary(self) -> Dict[str, float]:
         return {"heads": len(self.jaccard), "jaccard_mean": float(np.mean(self.jaccard)) if self.jaccard else 1.0,
                 "jaccard_min": float(np.min(self.jaccard)) if self.jaccard else 1.0,
                 "matched_sets": len(self.err_matched),
                 "max_abs_err_matched": float(np.max(self.err_matched)) if self.err_matched else 0.0,
-                "max_abs_err": float(np.max(self.err)) if self.err else 0.0}
+                "max_abs_err": float(np.max(self.err)) if self.err else 0.0,
+                "retained_mass_mean": float(np.mean(self.retained)) if self.retained else 1.0,
+                "retained_mass_min": float(np.min(self.retained)) if self.retained else 1.0}
 
 
 def end_to_end(K: torch.Tensor, V: torch.Tensor, refs: torch.Tensor, Q: torch.Tensor, O: torch.Tensor,
@@ -319,6 +322,7 @@ def end_to_end(K: torch.Tensor, V: torch.Tensor, refs: torch.Tensor, Q: torch.Te
     for bb in seqs:
         for h in range(kv_head * group, (kv_head + 1) * group):
             o_ref, tr = zo.decode_head(Kh, Vh, pfn, f64(Q[bb, h]), p, n_tokens, block, levels)
+            rep.retained.append(zo.retained_mass(tr))
             g = set(kept[bb, h, : int(cnt[bb, h])].tolist())
             o = set(tr.leaves)
             rep.jaccard.append(len(g & o) / max(1, len(g | o)))

@@ -183,6 +183,14 @@ def _route_ties_high(planes, q, p, n_tokens, block, levels):
     return trace
 
 
+def _retained_without_last(trace):
+    return float(np.prod([st.cum[st.k - 1] for st in trace.steps[:-1]]))
+
+
+def _retained_one_past(trace):
+    return float(np.prod([st.cum[min(st.k, len(st.cum) - 1)] for st in trace.steps]))
+
+
 MUTATIONS = {
     "leaf scores without 1/sqrt(d)": ("leaf_planes", _leaf_no_scale),
     "leaf intercept sign flipped": ("leaf_planes", _leaf_bias_sign),
@@ -205,6 +213,8 @@ MUTATIONS = {
     "step thresholds ignored after the first": ("step_threshold", _step_threshold_first),
     "e2m1 ties away from zero": ("e2m1_code", _e2m1_ties_up),
     "fp4 scale from amax / 4": ("quantize_fp4", _quantize_scale_amax4),
+    "retained mass without the last step": ("retained_mass", _retained_without_last),
+    "retained mass one past the cut": ("retained_mass", _retained_one_past),
 }
 
 
