@@ -37,9 +37,10 @@
 // Then
 //   attend  (two CTAs per SM) every head's attended keys (kept blocks, sink,
 //           tail) are cut into chunks; CTAs own contiguous ranges of chunks,
-//           warps run an online softmax per chunk (tensor cores for bf16), each
-//           CTA merges its chunks per head into one partial, and the warp that
-//           writes a head's last partial combines the head's partials -> O.
+//           warps run an online softmax per chunk (tensor cores for bf16), and
+//           each CTA merges its chunks per head into one partial;
+//   combine (one CTA per head) the head's partials merged in a fixed order
+//           -> O, the head's kept count and statistics.
 // The only waits inside a kernel are a scoring warp's waits for its own bulk
 // copies; they are bounded (on running out the kernel raises ZHA_ERR_TIMEOUT).
 #include <cstddef>
