@@ -1239,61 +1239,80 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
       cut = select_cut_anchored(a, E, n, anchor_h, sm.hist, sm, h, s);
     else cut = select_cut(a, E, n, kmin, sm, h, s);
   }
-  // the kept entries (order key <= cut) in entry order, four per thread and
-  // round; one block scan per round gives both lists' positions (units in the
-  // high half of the packed count, leaves in the low half)
+  // the kept entries (order key <= cut) in entry order.  A round covers two
+  // sub-rounds of 4 * kDecThreads entries, four per thread each (16-byte
+  // loads); one block scan per round of four 16-bit counts packed in 64 bits
+  // (units and leaves of each sub-round) gives every position, so the lists
+  // stay in entry order.  Kept non-leaves go to the units list (the next
+  // scoring step checks each code before it reads a record); a kept level-1
+  // block is listed only if its index lies in the level (it addresses the
+  // bitmap and the attention's key ranges).
   const uint32_t cut32 = uint32_t(cut >> 32);
   const int n32 = int(n);
+  const uint64_t nl1 = uint64_t(a.nl[1]);
   uint32_t* un = c.units(h);
   uint32_t* lv = c.leaves(h);
   uint32_t* bm = c.bitmap(h);
   long long nu = 0, nlf = 0;
   int leaf0 = 0;
-  for (int base = 0; base < n32; base += 4 * kDecThreads) {
-    const int i0 = base + 4 * tid;
-    uint32_t k[4], cd[4];
-    if (i0 + 4 <= ncache) {
-      const uint4 kv = *reinterpret_cast<const uint4*>(ck + i0);
-      const uint4 cv = *reinterpret_cast<const uint4*>(cc + i0);
-      k[0] = kv.x; k[1] = kv.y; k[2] = kv.z; k[3] = kv.w;
-      cd[0] = cv.x; cd[1] = cv.y; cd[2] = cv.z; cd[3] = cv.w;
-    } else {
+  constexpr int kSub = 4 * kDecThreads;  // entries of a sub-round
+  for (int base = 0; base < n32; base += 2 * kSub) {
+    uint32_t k[2][4], cd[2][4];
+    unsigned kb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i0 = base + r * kSub + 4 * tid;
+      if (i0 + 4 <= ncache) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(ck + i0);
+        const uint4 cv = *reinterpret_cast<const uint4*>(cc + i0);
+        k[r][0] = kv.x; k[r][1] = kv.y; k[r][2] = kv.z; k[r][3] = kv.w;
+        cd[r][0] = cv.x; cd[r][1] = cv.y; cd[r][2] = cv.z; cd[r][3] = cv.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          k[r][u] = i0 + u < n32 ? E.key(i0 + u) : 0xffffffffu;
+          cd[r][u] = i0 + u < n32 ? E.code(i0 + u) : 0u;
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        k[u] = i0 + u < n32 ? E.key(i0 + u) : 0xffffffffu;
-        cd[u] = i0 + u < n32 ? E.code(i0 + u) : 0u;
+        const bool kp = i0 + u < n32 &&
+                        (k[r][u] < cut32 || (k[r][u] == cut32 && entry_key64(a, Entry{k[r][u], cd[r][u]}) <= cut));
+        const bool leaf = code_level(cd[r][u]) == 1;
+        if (kp && (!leaf || uint64_t(code_index(cd[r][u])) < nl1)) {
+          kb[r] |= 1u << u;
+          if (leaf) lb[r] |= 1u << u;
+        }
       }
     }
-    unsigned kb = 0, lb = 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool kp = i0 + u < n32 &&
-                      (k[u] < cut32 || (k[u] == cut32 && entry_key64(a, Entry{k[u], cd[u]}) <= cut));
-      if (kp && valid_code(a, cd[u])) {  // (codes come from the scoring kernel; the check guards the writes)
-        kb |= 1u << u;
-        if (code_level(cd[u]) == 1) lb |= 1u << u;
-      }
-    }
+    // packed counts: leaves / units of sub-round 0 in bits 0-15 / 16-31, of sub-round 1 in 32-47 / 48-63
+    const unsigned long long mine = (unsigned long long)__popc(lb[0]) | (unsigned long long)__popc(kb[0] & ~lb[0]) << 16 |
+                                    (unsigned long long)__popc(lb[1]) << 32 |
+                                    (unsigned long long)__popc(kb[1] & ~lb[1]) << 48;
     unsigned long long tot;
-    const unsigned long long ex =
-        block_scan_u64((unsigned long long)__popc(kb & ~lb) << 32 | (unsigned long long)__popc(lb), sm.red64, &tot);
-    long long pu = nu + (long long)(ex >> 32);
-    long long pl = leaves0 + nlf + (long long)(ex & 0xffffffffull);
+    const unsigned long long ex = block_scan_u64(mine, sm.red64, &tot);
+    auto field = [](unsigned long long v, int f) { return (long long)((v >> (16 * f)) & 0xffffull); };
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (!((kb >> u) & 1u)) continue;
-      if ((lb >> u) & 1u) {
-        const uint32_t li = code_index(cd[u]);
-        if (pl < a.cap_list) lv[pl] = li;
-        ++pl;
-        leaf0 |= li == 0u ? 1 : 0;
-        if (a.kept) atomicOr(bm + (li >> 5), 1u << (li & 31u));
-      } else {
-        un[pu++] = cd[u];
+    for (int r = 0; r < 2; ++r) {
+      // sub-round 1 starts after every kept entry of sub-round 0
+      long long pu = nu + field(ex, 2 * r + 1) + (r ? field(tot, 1) : 0);
+      long long pl = leaves0 + nlf + field(ex, 2 * r) + (r ? field(tot, 0) : 0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (!((kb[r] >> u) & 1u)) continue;
+        if ((lb[r] >> u) & 1u) {
+          const uint32_t li = code_index(cd[r][u]);
+          if (pl < a.cap_list) lv[pl] = li;
+          ++pl;
+          leaf0 |= li == 0u ? 1 : 0;
+          if (a.kept) atomicOr(bm + (li >> 5), 1u << (li & 31u));
+        } else {
+          un[pu++] = cd[r][u];
+        }
       }
     }
-    nu += (long long)(tot >> 32);
-    nlf += (long long)(tot & 0xffffffffull);
+    nu += field(tot, 1) + field(tot, 3);
+    nlf += field(tot, 0) + field(tot, 2);
   }
   const int any_leaf0 = __syncthreads_or(leaf0);
   // state for the next step: its histogram cleared, its anchor = this step's max
