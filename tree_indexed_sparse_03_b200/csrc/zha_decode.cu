@@ -1261,6 +1261,7 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
     unsigned kb[2] = {0u, 0u}, lb[2] = {0u, 0u};
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
+      if (r == 1 && base + kSub >= n32) break;  // (uniform) no entry in the second sub-round
       const int i0 = base + r * kSub + 4 * tid;
       if (i0 + 4 <= ncache) {
         const uint4 kv = *reinterpret_cast<const uint4*>(ck + i0);
@@ -1294,6 +1295,7 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
     auto field = [](unsigned long long v, int f) { return (long long)((v >> (16 * f)) & 0xffffull); };
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
+      if (!kb[r]) continue;
       // sub-round 1 starts after every kept entry of sub-round 0
       long long pu = nu + field(ex, 2 * r + 1) + (r ? field(tot, 1) : 0);
       long long pl = leaves0 + nlf + field(ex, 2 * r) + (r ? field(tot, 0) : 0);
