@@ -1208,6 +1208,12 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
     for (int v = tid; v < kBins / 2; v += kDecThreads) cp_async16(sm.hist + 2 * v, gh + 2 * v);
   }
   cp_async_commit();
+  // the next step's histogram cleared while the copies are in flight (step s-1 wrote and read it; step
+  // s+1's scoring writes it after this kernel)
+  if (!last) {
+    unsigned long long* nhist = c.histP(h, par ^ 1);
+    for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
+  }
   // step 0 starts the head's counters afresh
   const long long n = s == 0 ? (long long)a.n_roots : min64(max64(__ldcg(&hs->n[par]), 0), a.cap_sel);
   const uint32_t kmin = ~__ldcg(&hs->kinv[par]);  // smallest key (largest estimate) of the step
@@ -1317,11 +1323,7 @@ __device__ __noinline__ void select_head(const DecodeArgs& a, DecSmem& sm, int h
     nlf += field(tot, 0) + field(tot, 2);
   }
   const int any_leaf0 = __syncthreads_or(leaf0);
-  // state for the next step: its histogram cleared, its anchor = this step's max
-  if (!last) {
-    unsigned long long* nhist = c.histP(h, par ^ 1);
-    for (int i = tid; i < kBins; i += kDecThreads) nhist[i] = 0ull;
-  }
+  // state for the next step: its anchor = this step's max
   if (tid == 0) {
     long long U = nu, NL = leaves0 + nlf;
     if (U * b > a.cap_sel) {
