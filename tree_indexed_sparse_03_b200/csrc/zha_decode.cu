@@ -844,6 +844,22 @@ __device__ __noinline__ unsigned long long select_cut_anchored(const DecodeArgs&
 // threads; returns the total.
 template <int NT>
 __device__ __forceinline__ long long build_prefix(long long* pref, unsigned long long* red64, int nh) {
+  if (nh <= 32) {  // one warp scans with shuffles; one CTA barrier (red64[0] carries the total)
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      long long v = lane < nh ? pref[1 + lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+      }
+      if (lane < nh) pref[1 + lane] = v;
+      if (lane == 0) pref[0] = 0;
+      if (lane == 31) red64[0] = (unsigned long long)v;
+    }
+    __syncthreads();
+    return (long long)red64[0];
+  }
   long long carry = 0;
   for (int base = 0; base < nh; base += NT) {
     const int i = base + threadIdx.x;
