@@ -157,3 +157,31 @@ def test_shards_reproduce_the_single_tree(sharded_results):
         assert union == trace.leaves, (ci, h)
         assert parts[0][2] == parts[1][2]  # every rank holds the merged output
         assert np.abs(np.array(parts[0][2]) - o_ref).max() <= 1e-12
+
+
+def test_top_p_keep_matches_the_oracle_cut():
+    """The exchange's fixed-point cut keeps the same prefix of the same (estimate desc, start asc) order as the
+    oracle's fp64 cut, except where the cumulative mass at the cut lies within rounding of p; p >= 1 keeps all."""
+    sys.path.insert(0, ROOT)
+    from tree_indexed_sparse_03_b200 import sharded as sh
+    import oracle.zha_oracle as zo
+    rng = np.random.default_rng(5)
+    near = 0
+    for trial in range(400):
+        n = int(rng.integers(1, 80))
+        est = rng.normal(size=n) * float(rng.choice([0.5, 2.0, 8.0]))
+        if trial % 4 == 0:
+            est = np.round(est)  # exact ties: the lower start goes first
+        start = rng.permutation(n).astype(np.int64) * 4
+        p = float(rng.choice([0.3, 0.7, 0.95, 0.999, 1.0]))
+        kept = sh.top_p_keep(est, start, p)
+        order = np.lexsort((start, -est))
+        k, cum = zo.top_p_count(est, order, p)
+        assert list(kept) == list(order[: len(kept)])
+        if p >= 1.0:
+            assert len(kept) == n
+        elif len(kept) != k:
+            near += 1
+            j = min(k, len(kept)) - 1
+            assert abs(cum[j] - p) <= 1e-9, (trial, k, len(kept), cum[j], p)
+    assert near <= 4
